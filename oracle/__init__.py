@@ -1,0 +1,204 @@
+"""fp64 CPU oracle for the batch-invariant forward-pass kernels.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports this package:
+only the tests, the smoke check and the benchmark's CPU-baseline leg may call it.
+It shares no code with the CUDA library; inputs come from ``synth`` as exact
+float64 widenings of the bf16 bits the GPU saw.
+
+Every function evaluates the plain mathematical definition in float64, with no
+blocking, splitting or reordering of its own: the batch-invariant GPU kernels
+reach the same mathematical result in one fixed fp32 order, so the definition is
+the reference. Sources (web pages on batch invariance):
+
+* "Defeating Nondeterminism in LLM Inference" technical summary (mobiles-han
+  blog), section 対応策：バッチ不変なカーネル設計, kernel table rows RMSNorm,
+  MatMul and Attention — the three operations and what each must keep fixed.
+* same blog, usage article, section 注意点・補足実装 (FixedAttention sketch) —
+  the cache and the current chunk are joined into one layout before attention.
+* "Greedy Decoding Is Not Precision-Invariant" (arXiv 2609.26621), abstract —
+  the top-2 logit margin at the LM head decides greedy flips; the LM head is
+  recomputed in FP32 only when that margin is below a threshold.
+
+Readings where the pages are silent (each is pinned by a test):
+* RMSNorm: y = x / sqrt(mean(x^2) + eps) * w, eps inside the root.
+* MatMul: C = A @ W^T with W stored [N, K].
+* Attention: softmax(q . k * scale) v with scale = 1/sqrt(D); q-head h reads
+  kv-head h // (Hq/Hkv); a query at absolute position p sees keys 0..p
+  (inclusive); decode queries see keys 0..L-1.
+* LM head: greedy token = argmax of the logits, lowest index on ties; the
+  recompute decision compares the top-2 margin of the bf16-rounded logits,
+  taken in fp32, against the threshold.
+
+Parity pins: every function here is pinned (tests/test_oracle.py).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+PAGE = 16  # tokens per KV page of the unified store
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm — "Defeating Nondeterminism" summary, kernel table, row RMSNorm
+
+
+def rmsnorm(x: np.ndarray, w: np.ndarray, eps: float) -> np.ndarray:
+    """y[m, :] = x[m, :] / sqrt(mean_k x[m, k]^2 + eps) * w, in float64."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * w
+
+
+# ---------------------------------------------------------------------------
+# MatMul — same table, row MatMul
+
+
+def matmul(a: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """C[m, n] = sum_k A[m, k] * W[n, k] (W stored [N, K]), in float64."""
+    return np.asarray(a, dtype=np.float64) @ np.asarray(w, dtype=np.float64).T
+
+
+# ---------------------------------------------------------------------------
+# Attention over the unified paged store — same table, row Attention, and the
+# FixedAttention sketch (cache and current tokens in one layout)
+
+
+def gather_kv(cache: np.ndarray, page_row: np.ndarray, g: int, n_tokens: int) -> np.ndarray:
+    """Tokens 0..n_tokens-1 of kv-head g, read through one page-table row.
+
+    cache is [num_pages, Hkv, PAGE, D]; token t sits in slot t % PAGE of
+    physical page page_row[t // PAGE].
+    """
+    t = np.arange(n_tokens)
+    pages = np.asarray(page_row, dtype=np.int64)[t // PAGE]
+    return np.asarray(cache[pages, g, t % PAGE], dtype=np.float64)
+
+
+def softmax_attend(q: np.ndarray, keys: np.ndarray, vals: np.ndarray, scale: float) -> np.ndarray:
+    """softmax(keys @ q * scale) @ vals for one query vector, max-subtracted, float64."""
+    s = keys @ np.asarray(q, dtype=np.float64) * scale
+    e = np.exp(s - s.max())
+    return (e @ vals) / e.sum()
+
+
+def attention_rows(q, k_cache, v_cache, page_table, row_page, row_len, scale=None):
+    """Attention for a list of query rows.
+
+    q: [R, Hq, D]; row r reads page-table row row_page[r] and sees keys
+    0..row_len[r]-1. Returns [R, Hq, D] float64. A row with no visible key
+    returns zeros.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k_cache = np.asarray(k_cache, dtype=np.float64)
+    v_cache = np.asarray(v_cache, dtype=np.float64)
+    R, Hq, D = q.shape
+    Hkv = k_cache.shape[1]
+    group = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = np.zeros((R, Hq, D), dtype=np.float64)
+    for r in range(R):
+        L = int(row_len[r])
+        if L <= 0:
+            continue
+        prow = np.asarray(page_table[int(row_page[r])])
+        for g in range(Hkv):
+            keys = gather_kv(k_cache, prow, g, L)
+            vals = gather_kv(v_cache, prow, g, L)
+            for j in range(group):
+                h = g * group + j
+                out[r, h] = softmax_attend(q[r, h], keys, vals, scale)
+    return out
+
+
+def attention_decode(q, k_cache, v_cache, page_table, seq_lens, scale=None):
+    """Decode: query b (one new token per sequence) sees keys 0..seq_lens[b]-1."""
+    B = np.asarray(q).shape[0]
+    return attention_rows(q, k_cache, v_cache, page_table, np.arange(B), np.asarray(seq_lens), scale)
+
+
+def attention_prefill(q, q_seq, q_pos, k_cache, v_cache, page_table, scale=None):
+    """Causal prefill: the query at absolute position p of sequence s sees keys 0..p of s."""
+    return attention_rows(q, k_cache, v_cache, page_table, np.asarray(q_seq),
+                          np.asarray(q_pos) + 1, scale)
+
+
+# ---------------------------------------------------------------------------
+# LM head with the margin test — "Greedy Decoding Is Not Precision-Invariant",
+# abstract (selective FP32 LM-head recompute below a margin threshold)
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to bf16 as the GPU epilogue does (fp64 -> fp32 RNE, fp32 -> bf16 RNE).
+
+    Works on the fp32 bit pattern: add 0x7FFF plus the lowest kept bit, then
+    truncate the low 16 bits. NaN/inf are not expected here.
+    """
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    bits = f.view(np.uint32).astype(np.uint64)
+    lsb = (bits >> 16) & 1
+    rounded = ((bits + 0x7FFF + lsb) >> 16) << 16
+    return rounded.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def argmax_lowest(v: np.ndarray) -> int:
+    """Index of the largest value, lowest index among equals."""
+    v = np.asarray(v)
+    return int(np.flatnonzero(v == v.max())[0])
+
+
+def top2(v: np.ndarray):
+    """(top1 value, top1 index, top2 value, top2 index) with lowest-index tie-break."""
+    v = np.asarray(v, dtype=np.float64)
+    i1 = argmax_lowest(v)
+    rest = v.copy()
+    rest[i1] = -np.inf
+    i2 = argmax_lowest(rest)
+    return v[i1], i1, v[i2], i2
+
+
+def lmhead(h: np.ndarray, w: np.ndarray, threshold: float):
+    """Greedy LM head.
+
+    Returns a dict with
+      logits  [M, V] float64 (exact),
+      tokens  [M] int: argmax of the exact logits,
+      margin  [M] float64: exact top1 - top2,
+      margin_bf16 [M] float64: top1 - top2 of the bf16-rounded logits
+                  (the quantity the first pass thresholds),
+      recompute [M] bool: margin_bf16 < threshold,
+      tokens_bf16 [M] int: argmax of the bf16-rounded logits.
+    """
+    logits = matmul(h, w)
+    M = logits.shape[0]
+    tokens = np.empty(M, dtype=np.int64)
+    tokens_bf16 = np.empty(M, dtype=np.int64)
+    margin = np.empty(M)
+    margin_bf16 = np.empty(M)
+    lb = round_to_bf16(logits)
+    for m in range(M):
+        v1, i1, v2, _ = top2(logits[m])
+        tokens[m], margin[m] = i1, v1 - v2
+        b1, j1, b2, _ = top2(lb[m])
+        tokens_bf16[m] = j1
+        margin_bf16[m] = float(np.float32(b1) - np.float32(b2))
+    return dict(logits=logits, tokens=tokens, margin=margin, margin_bf16=margin_bf16,
+                recompute=margin_bf16 < threshold, tokens_bf16=tokens_bf16)
+
+
+# ---------------------------------------------------------------------------
+# Normwise error used by every parity test
+
+
+def normwise_rel_err(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """Per row: max |got - ref| / max |ref| (rows are the leading axes flattened)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    g = got.reshape(-1, got.shape[-1])
+    r = ref.reshape(-1, ref.shape[-1])
+    den = np.abs(r).max(axis=1)
+    den[den == 0] = 1.0
+    return np.abs(g - r).max(axis=1) / den
