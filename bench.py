@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the batch-invariant kernels (one JSON line on rank 0).
+
+Step (the default workload "k4096_m2048"): one batch of M=2048 rows at hidden
+size K=4096 goes through bi_rmsnorm and then bi_matmul against three weights
+with N = 4096, 6144 and 14336 (K=4096): the RMSNorm-then-matmul configuration
+swept by the invariance tests, at its largest batch. `value` is the matmul
+throughput of the whole step (2*M*K*sum(N) FLOPs / step time, the RMSNorm
+included in the time), summed over all GPUs; every GPU runs its own replica
+(rows are independent, nothing is exchanged), so scaling is weak.
+
+Also reported on rank 0 at N=1: the per-kernel roofline of the dominant kernel
+(the tcgen05 matmul), the slowdown against the non-invariant path (cuBLAS via
+torch.matmul + F.rms_norm) on the same box, an end-to-end figure through the
+public API with host buffers, the clocks seen during the timed region, the fp64
+CPU oracle timed on a bounded sample, and (``--rows``, default on) one
+measurement of every other hot-path kernel: RMSNorm bandwidth, decode attention
+bandwidth, causal prefill throughput and the LM head.
+
+``--impl reference`` times the fp64 CPU oracle on the same workload and metric
+(bounded samples per step) and prints the reference line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "bi-matmul TFLOP/s, RMSNorm/attn HBM GB/s, % roofline, slowdown vs non-invariant"
+K_HIDDEN = 4096
+NS = (4096, 6144, 14336)
+EPS = 1e-6
+WORKLOAD = "k4096_m2048"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]), "sm_max_mhz": float(p.get("sm_max_mhz", 1965)),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (timing only; no data-path collective)
+
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        dist.barrier()
+
+
+def aggregate(units: float, ms: float, world: int, device=None):
+    """Whole-job (sum of units, max of elapsed ms) over ranks."""
+    if world <= 1:
+        return units, ms
+    t = torch.tensor([units], dtype=torch.float64, device=device)
+    m = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    dist.all_reduce(m, op=dist.ReduceOp.MAX)
+    return float(t.item()), float(m.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        mhz = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        maxmhz = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        busy = [m for m in mhz if m > 0.5 * maxmhz] or mhz
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": maxmhz, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# the step
+
+
+class Workload:
+    """Resident inputs of the default step (weights + two rotating activation sets)."""
+
+    def __init__(self, M: int, device):
+        self.M = M
+        self.device = device
+        xs = [synth.normal_bf16((M, K_HIDDEN), 100 + i) for i in range(2)]
+        self.x = [x.to(device) for x in xs]
+        self.wn = synth.normal_bf16((K_HIDDEN,), 110, std=0.1, mean=1.0).to(device)
+        self.W = [synth.normal_bf16((n, K_HIDDEN), 120 + j, std=0.02).to(device) for j, n in enumerate(NS)]
+        self.y = torch.empty((M, K_HIDDEN), dtype=torch.bfloat16, device=device)
+        self.C = [torch.empty((M, n), dtype=torch.bfloat16, device=device) for n in NS]
+        self.flops = 2.0 * M * K_HIDDEN * sum(NS)
+        self.rms_bytes = 4.0 * M * K_HIDDEN + 2.0 * K_HIDDEN
+        self.launches_per_step = 1 + len(NS)
+
+
+def step_ours(bi, wl: Workload, i: int, ev=None):
+    """RMSNorm then the three matmuls. ev: optional list of (start, end) event pairs per kernel."""
+    if ev is None:
+        bi.rmsnorm(wl.x[i % 2], wl.wn, EPS, out=wl.y)
+        for W, C in zip(wl.W, wl.C):
+            bi.matmul(wl.y, W, out=C)
+        return
+    ev[0][0].record()
+    bi.rmsnorm(wl.x[i % 2], wl.wn, EPS, out=wl.y)
+    ev[0][1].record()
+    for j, (W, C) in enumerate(zip(wl.W, wl.C)):
+        ev[j + 1][0].record()
+        bi.matmul(wl.y, W, out=C)
+        ev[j + 1][1].record()
+
+
+def step_cublas(wl: Workload, i: int):
+    y = torch.nn.functional.rms_norm(wl.x[i % 2], (K_HIDDEN,), wl.wn, EPS)
+    for W, C in zip(wl.W, wl.C):
+        torch.matmul(y, W.t(), out=C)
+
+
+def time_loop(fn, steps: int, warmup: int, world: int):
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(steps):
+        fn(i)
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return s.elapsed_time(e)
+
+
+def traffic_from_profile():
+    """Per-launch DRAM bytes of the matmul kernel from the committed ncu summary,
+    or None if the kernel source changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "gemm_bf16_kernel_traffic.json")
+    src = os.path.join(ROOT, "invariant_deterministic_04_b200", "csrc", "gemm.cuh")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        with open(src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()
+        if p.get("gemm_cuh_sha256") != h:
+            return None
+        return p
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (bounded sample)
+
+
+def oracle_step_sample(rows: int, seed: int = 0):
+    """fp64 oracle on `rows` rows of the step: RMSNorm then the three matmuls. Returns (flops, seconds)."""
+    import oracle
+
+    x = synth.to_f64(synth.normal_bf16((rows, K_HIDDEN), 100 + seed))
+    wn = synth.to_f64(synth.normal_bf16((K_HIDDEN,), 110, std=0.1, mean=1.0))
+    Ws = [synth.to_f64(synth.normal_bf16((n, K_HIDDEN), 120 + j, std=0.02)) for j, n in enumerate(NS)]
+    t0 = time.perf_counter()
+    y = oracle.rmsnorm(x, wn, EPS)
+    for W in Ws:
+        oracle.matmul(y, W)
+    return 2.0 * rows * K_HIDDEN * sum(NS), time.perf_counter() - t0
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s: float = 10.0):
+    rows = 32
+    flops, t = oracle_step_sample(rows)
+    rows = int(max(32, min(2048, rows * budget_s / max(t, 1e-3))))
+    flops, t = oracle_step_sample(rows, seed=1)
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle: RMSNorm + matmuls (N=4096,6144,14336; K=4096) on {rows} of the "
+                      f"2048 rows, {t:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# other hot-path kernels (one measurement each, rank 0)
+
+
+def _events_ms(fn, iters=10, warmup=3):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(iters):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / iters
+
+
+def other_rows(bi, device, pk):
+    out = {}
+    # RMSNorm bandwidth at a size far above L2 (M = 65536, K = 4096: 1 GiB in + out)
+    M = 65536
+    x = torch.randn((M, K_HIDDEN), device=device, dtype=torch.float32).to(torch.bfloat16)
+    w = synth.normal_bf16((K_HIDDEN,), 110, std=0.1, mean=1.0).to(device)
+    y = torch.empty_like(x)
+    ms = _events_ms(lambda: bi.rmsnorm(x, w, EPS, out=y))
+    ms_ref = _events_ms(lambda: torch.nn.functional.rms_norm(x, (K_HIDDEN,), w, EPS))
+    gbs = (4.0 * M * K_HIDDEN + 2 * K_HIDDEN) / ms / 1e6
+    out["rmsnorm_m65536_k4096"] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3), "ms": round(ms, 4),
+                                   "slowdown_vs_F.rms_norm": round(ms / ms_ref, 3)}
+    del x, y
+
+    # decode attention: B=64 sequences, lengths ~ U[1, 32768], GQA 32/8, D=128
+    B, Lmax = 64, 32768
+    lens = synth.decode_lengths(B, Lmax, seed=50)
+    kv = synth.paged_kv_device(lens, 8, 128, seed=51, max_pages=Lmax // 16, device=device)
+    q = synth.normal_bf16((B, 32, 128), 52).to(device)
+    ws = torch.empty(bi.attention_workspace_size(B, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
+    o = torch.empty_like(q)
+    ms = _events_ms(lambda: bi.attention_decode(q, kv.k_cache, kv.v_cache, kv.page_table, kv.seq_lens, out=o,
+                                                workspace=ws))
+    kv_bytes = 4096.0 * int(lens.sum())  # K and V: L * Hkv * D * 2 bytes * 2
+    gbs = kv_bytes / ms / 1e6
+    out["decode_b64_l32k"] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3), "ms": round(ms, 4),
+                              "kv_bytes": kv_bytes}
+    del kv, ws
+
+    # causal prefill, one sequence of 4096 tokens
+    S = 4096
+    kvp = synth.paged_kv_device([S], 8, 128, seed=60, max_pages=S // 16, device=device)
+    qp = synth.normal_bf16((S, 32, 128), 61).to(device)
+    qs = torch.zeros(S, dtype=torch.int32, device=device)
+    qpos = torch.arange(S, dtype=torch.int32, device=device)
+    wsp = torch.empty(bi.attention_workspace_size(S, 32, 128, kvp.max_pages), dtype=torch.uint8, device=device)
+    op = torch.empty_like(qp)
+    ms = _events_ms(lambda: bi.attention_prefill(qp, qs, qpos, kvp.k_cache, kvp.v_cache, kvp.page_table, out=op,
+                                                 workspace=wsp), iters=3, warmup=1)
+    flops = 2.0 * 32 * 128 * S * (S + 1)  # q.k and p.v over the visible keys
+    alu_peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
+    out["prefill_s4096"] = {"TFLOP/s": round(flops / ms / 1e9, 2), "frac_fp32_alu": round(flops / ms / 1e9 / alu_peak, 3),
+                            "ms": round(ms, 3)}
+    del kvp, wsp
+
+    # LM head: 64 rows, vocabulary 32000, hidden 2048
+    h = synth.normal_bf16((64, 2048), 70).to(device)
+    Wl = synth.normal_bf16((32000, 2048), 71, std=0.02).to(device)
+    tok = torch.empty(64, dtype=torch.int32, device=device)
+    rec = torch.empty(64, dtype=torch.int32, device=device)
+    wsl = torch.empty(bi.lmhead_workspace_size(64, 32000), dtype=torch.uint8, device=device)
+    ms = _events_ms(lambda: bi.lmhead_argmax(h, Wl, 0.5, tokens=tok, recomputed=rec, workspace=wsl))
+    ms_ref = _events_ms(lambda: torch.argmax(torch.matmul(h, Wl.t()), dim=1))
+    out["lmhead_m64_v32000"] = {"ms": round(ms, 4), "recomputed_rows": int(rec.sum()),
+                                "slowdown_vs_cublas_argmax": round(ms / ms_ref, 3)}
+    return out
+
+
+# ---------------------------------------------------------------------------
+
+
+def run_reference(args, rank, world):
+    """The fp64 CPU oracle on the same workload and metric (bounded samples per step)."""
+    if rank != 0:
+        return
+    total = args.steps + args.warmup
+    flops, t = oracle_step_sample(8)
+    per = max(1, min(2048, int(8 * (90.0 / total) / max(t, 1e-3))))
+    for i in range(args.warmup):
+        oracle_step_sample(per, seed=i % 2)
+    fl, tt = 0.0, 0.0
+    for i in range(args.steps):
+        f, s = oracle_step_sample(per, seed=i % 2)
+        fl += f
+        tt += s
+    v = fl / tt / 1e12
+    sample = f"fp64 numpy oracle, {per} of the 2048 rows per step (RMSNorm + matmuls N=4096,6144,14336; K=4096)"
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": 2048, "K": K_HIDDEN, "N": list(NS), "rows_per_step": per},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local):
+    import invariant_deterministic_04_b200 as bi
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    bi.lib()
+    pk = peaks()
+    wl = Workload(args.M, device)
+
+    # device-timed steps, with per-kernel events inside the timed region
+    nk = wl.launches_per_step
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nk)]
+           for _ in range(args.steps)]
+    for i in range(args.warmup):
+        step_ours(bi, wl, i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(args.steps):
+        step_ours(bi, wl, i, evs[i])
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ms_total = s.elapsed_time(e)
+    kernel_ms = [sum(evs[i][j][0].elapsed_time(evs[i][j][1]) for i in range(args.steps)) for j in range(nk)]
+    units, ms_max = aggregate(wl.flops * args.steps, ms_total, world, device)
+    value = units / (ms_max / 1e3) / 1e12
+    gpu_launches = nk * args.steps
+
+    # end to end through the public API: pinned host input in, all outputs back to pinned host memory
+    xh = [wl.x[j].cpu().pin_memory() for j in range(2)]
+    ch = [torch.empty(C.shape, dtype=C.dtype).pin_memory() for C in wl.C]
+    xd = torch.empty_like(wl.x[0])
+    e2e_steps = max(10, min(args.steps, 100))
+
+    def e2e_step(i):
+        xd.copy_(xh[i % 2], non_blocking=True)
+        bi.rmsnorm(xd, wl.wn, EPS, out=wl.y)
+        for W, C, H in zip(wl.W, wl.C, ch):
+            bi.matmul(wl.y, W, out=C)
+            H.copy_(C, non_blocking=True)
+
+    e2e_ms = time_loop(e2e_step, e2e_steps, 3, world)
+    e2e_units, e2e_max = aggregate(wl.flops * e2e_steps, e2e_ms, world, device)
+    h2d = wl.M * K_HIDDEN * 2
+    d2h = sum(wl.M * n * 2 for n in NS)
+
+    # non-invariant path on the same box
+    ref_ms = time_loop(lambda i: step_cublas(wl, i), args.steps, args.warmup, world)
+
+    if rank != 0:
+        return
+    gemm_ms = sum(kernel_ms[1:])
+    gemm_flops = 2.0 * wl.M * K_HIDDEN * sum(NS) * args.steps
+    achieved = gemm_flops / (gemm_ms / 1e3) / 1e12
+    prof = traffic_from_profile()
+    traffic = None
+    if prof:
+        traffic = prof.get("dram_bytes_per_launch")
+    roof = {"bound": "tensor", "kernel": "gemm_bf16_kernel (tcgen05)", "achieved": round(achieved, 1),
+            "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops_sustained"], 3),
+            "peak_kind": f"bf16 sustained ({pk['source']})", "frac_of_burst": round(achieved / pk["bf16_tflops"], 3),
+            "traffic": traffic, "kernel_share": round(gemm_ms / sum(kernel_ms), 3)}
+    rms_ms = kernel_ms[0] / args.steps
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": wl.M, "K": K_HIDDEN, "N": list(NS), "step": "bi_rmsnorm + 3 x bi_matmul",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "working set > L2 (201 MB of weights per step; two activation buffers rotate)"},
+        "roofline": roof,
+        "rmsnorm_in_step": {"GB/s": round(wl.rms_bytes / rms_ms / 1e6, 1), "ms": round(rms_ms, 4),
+                            "note": "16 MiB in + 16 MiB out per launch"},
+        "slowdown_vs_noninvariant": round((ms_total / args.steps) / (ref_ms / args.steps), 3),
+        "noninvariant_ms_per_step": round(ref_ms / args.steps, 4),
+        "e2e": {"value": round(e2e_units / (e2e_max / 1e3) / 1e12, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": gpu_launches,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
+    if world == 1 and args.rows:
+        del wl
+        torch.cuda.empty_cache()
+        line["rows"] = other_rows(bi, device, pk)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--M", type=int, default=2048)
+    ap.add_argument("--rows", dest="rows", action="store_true", default=True)
+    ap.add_argument("--no-rows", dest="rows", action="store_false")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = init_dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

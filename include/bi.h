@@ -1,0 +1,198 @@
+/*
+ * bi.h — batch-invariant forward-pass kernels for transformer inference (B200, sm_100a).
+ *
+ * What "batch-invariant" means here: the bits of any output row depend only on
+ * that row's own inputs. They do not depend on how many rows were batched with it,
+ * on its position in the batch, on the other rows, on how many SMs were free, or
+ * on whether its keys/values were written to the cache earlier or in the current
+ * chunk. Every kernel reduces each row in one fixed order, fixed by the problem's
+ * static shape (K, N, D, head counts) and never by the batch size M, the number of
+ * sequences B or their lengths. Sources:
+ *   - "Defeating Nondeterminism in LLM Inference" technical summary (mobiles-han
+ *     blog), section 対応策：バッチ不変なカーネル設計: the kernel table (RMSNorm uses a
+ *     data-parallel strategy; MatMul uses one kernel configuration for all shapes;
+ *     Attention joins cache and current tokens into one layout and uses fixed-size
+ *     KV splits).
+ *   - Techzine, "Thinking Machines wil AI voorspelbaarder maken": reductions and
+ *     sums always happen in one fixed order, whatever the batch size or load.
+ *   - hakusoku, "LLM推論における非決定性の克服", section カーネル実装と加算順序: no
+ *     atomic adds in the forward pass; tree reductions give deterministic results.
+ *   - "Greedy Decoding Is Not Precision-Invariant" (arXiv 2609.26621), abstract:
+ *     greedy argmax with an FP32 recompute of the LM head only when the top-2
+ *     logit margin is below a threshold.
+ *
+ * Conventions for every call:
+ *   - bf16 tensors are raw bfloat16 bits (bi_bf16). All pointers except the
+ *     workspace-size queries' are DEVICE pointers owned by the caller; the
+ *     library never frees or keeps them.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy default
+ *     stream) and never synchronise. Host validation runs first: on any error
+ *     status nothing is launched.
+ *   - Leading dimensions are in elements. bf16 pointers and leading dimensions
+ *     must give 16-byte aligned rows (pointer % 16 == 0, ld % 8 == 0), else
+ *     BI_ERR_ALIGN.
+ *   - A launch failure returns BI_ERR_CUDA. Conditions only the device can see
+ *     (a page id outside the store, a length beyond the page table, a bounded
+ *     device wait that expired) set a device error word that
+ *     bi_get_device_error() reads; the affected rows are skipped or zeroed.
+ *   - No atomics touch any value; results are bit-identical run to run.
+ *   - The library allocates no device memory: scratch space is a caller-owned
+ *     workspace whose size the *_workspace_size() queries give.
+ */
+#ifndef BI_H_
+#define BI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t bi_bf16; /* raw bfloat16 bits */
+
+typedef enum {
+  BI_OK = 0,
+  BI_ERR_NULL = 1,           /* a required pointer is NULL */
+  BI_ERR_SHAPE = 2,          /* a size is negative, zero where not allowed, or inconsistent */
+  BI_ERR_ALIGN = 3,          /* a pointer or leading dimension breaks the 16-byte rule */
+  BI_ERR_WORKSPACE = 4,      /* workspace NULL or smaller than the size query */
+  BI_ERR_UNSUPPORTED = 5,    /* valid request this build does not implement (e.g. D not 64/128) */
+  BI_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed */
+  BI_ERR_DEVICE_TIMEOUT = 7, /* reported by bi_get_device_error: a bounded device wait expired */
+  BI_ERR_DEVICE_INDEX = 8    /* reported by bi_get_device_error: a page id / seq id / length out of range */
+} bi_status;
+
+/* Human-readable name of a status code. Never NULL. */
+const char* bi_status_string(int status);
+
+/* ABI version of this library (increments on any signature change). */
+int bi_version(void);
+
+/* Compile-time constants of the invariant schedule. */
+#define BI_PAGE_TOKENS 16   /* tokens per KV page */
+#define BI_KV_SPLIT 256     /* tokens per attention split (fixed size, not a fixed count) */
+#define BI_GEMM_BM 128      /* matmul tile rows (tcgen05 M) */
+#define BI_GEMM_BN 256      /* matmul tile columns (tcgen05 N) */
+#define BI_GEMM_BK 64       /* matmul K block; K is summed block by block in ascending order */
+
+/*
+ * RMSNorm. Source: "Defeating Nondeterminism in LLM Inference" summary, kernel
+ * table, row RMSNorm (data-parallel: each row reduced alone, never split across
+ * CTAs at small batch).
+ *   y[m, k] = bf16_rne( x[m, k] * rsqrt( (sum_k x[m, k]^2) / K + eps ) * w[k] )
+ * x: [M, K] bf16 row-major, row stride ldx. w: [K] bf16. y: [M, K] bf16, stride ldy
+ * (y may alias x when ldy == ldx). fp32 accumulation in one fixed order per row
+ * that depends on K only. M == 0 is a no-op. Requires 8 <= K <= 16384, K % 8 == 0.
+ */
+bi_status bi_rmsnorm(const bi_bf16* x, int64_t ldx, const bi_bf16* w, bi_bf16* y, int64_t ldy,
+                     int64_t M, int64_t K, float eps, void* stream);
+
+/*
+ * MatMul, C = A * W^T. Source: same table, row MatMul (one kernel configuration
+ * for every shape; no split-K; no switching between tensor-core and other paths).
+ *   C[m, n] = bf16_rne( sum_k A[m, k] * W[n, k] ),  fp32 accumulation in TMEM
+ * A: [M, K] bf16 row-major (K contiguous), stride lda. W: [N, K] bf16 row-major
+ * (the nn.Linear weight layout), stride ldw. C: [M, N] bf16, stride ldc; must not
+ * overlap A or W. Tile 128 x 256, K summed in 64-wide blocks in ascending order by
+ * tcgen05.mma; the same for every M. M == 0 or N == 0 is a no-op.
+ * Requires K % 64 == 0, K >= 64, N % 8 == 0.
+ */
+bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw, bi_bf16* C,
+                    int64_t ldc, int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * Workspace bytes for bi_attention_decode (rows = B) or bi_attention_prefill
+ * (rows = T). Depends on rows, Hq, D and the page-table width only.
+ */
+size_t bi_attention_workspace_size(int64_t rows, int Hq, int D, int max_pages_per_seq);
+
+/*
+ * Decode attention over the unified paged KV store. Source: same table, row
+ * Attention (cache and current tokens in one layout; fixed-size KV splits), and
+ * the FixedAttention sketch in the usage article, section 注意点・補足実装.
+ *   out[b, h, :] = softmax_j( scale * q[b, h, :] . K_b[j, g, :] ) V_b[j, g, :],
+ *   j = 0 .. seq_lens[b]-1, g = h / (Hq / Hkv).
+ * q: [B, Hq, D] bf16. k_cache, v_cache: [num_pages, Hkv, 16, D] bf16 (a page holds
+ * 16 consecutive tokens of one sequence for every kv-head). page_table: [B,
+ * max_pages_per_seq] int32; token j of sequence b is slot j % 16 of physical page
+ * page_table[b, j / 16]; entries past the last page are never read. seq_lens: [B]
+ * int32. out: [B, Hq, D] bf16. Schedule: tokens are cut into splits at absolute
+ * positions 0, 256, 512, ... (split count grows with the length); each split is
+ * reduced over its 16-token pages in order, then splits are folded in ascending
+ * order. Slots past a sequence's length are never read into the result (stale
+ * pages may hold NaN). A sequence of length 0 yields zeros. D in {64, 128};
+ * Hq % Hkv == 0 and Hq / Hkv in {1, 2, 4, 8}. workspace: >= the size query.
+ */
+bi_status bi_attention_decode(const bi_bf16* q, const bi_bf16* k_cache, const bi_bf16* v_cache,
+                              int64_t num_pages, const int32_t* page_table, int max_pages_per_seq,
+                              const int32_t* seq_lens, bi_bf16* out, int B, int Hq, int Hkv, int D,
+                              float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Causal prefill attention over the same store (chunked or whole). Source: same
+ * table, row Attention (chunked prefill / prefix caching must not change the
+ * path), and the usage article's test list (prefill, decode, cache on or off).
+ * Query row t belongs to sequence q_seq[t] at absolute position q_pos[t] and sees
+ * that sequence's keys 0 .. q_pos[t] (inclusive). The chunk's own K/V must already
+ * be in the store (bi_kv_append), so cached and fresh tokens take one code path.
+ * Each row is computed with exactly the per-row schedule of bi_attention_decode
+ * for length q_pos[t] + 1, so a row's bits do not depend on the chunking, on T,
+ * or on which other rows are present, and equal the decode result at that length.
+ * q: [T, Hq, D] bf16. q_seq, q_pos: [T] int32. page_table: [num_seqs,
+ * max_pages_per_seq] int32. out: [T, Hq, D] bf16. T == 0 is a no-op.
+ */
+bi_status bi_attention_prefill(const bi_bf16* q, const int32_t* q_seq, const int32_t* q_pos,
+                               const bi_bf16* k_cache, const bi_bf16* v_cache, int64_t num_pages,
+                               const int32_t* page_table, int num_seqs, int max_pages_per_seq,
+                               bi_bf16* out, int T, int Hq, int Hkv, int D, float scale,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Glue: write new tokens' K/V into the paged store (the unified layout of the
+ * FixedAttention sketch). Token t of k_new/v_new ([T, Hkv, D] bf16) goes to slot
+ * q_pos[t] % 16 of page page_table[q_seq[t], q_pos[t] / 16]. Pure copies; T == 0
+ * is a no-op. Out-of-range ids set the device error word and skip the token.
+ */
+bi_status bi_kv_append(const bi_bf16* k_new, const bi_bf16* v_new, const int32_t* q_seq,
+                       const int32_t* q_pos, bi_bf16* k_cache, bi_bf16* v_cache, int64_t num_pages,
+                       const int32_t* page_table, int num_seqs, int max_pages_per_seq, int T,
+                       int Hkv, int D, void* stream);
+
+/* Workspace bytes for bi_lmhead_argmax with M rows and vocabulary V. */
+size_t bi_lmhead_workspace_size(int64_t M, int64_t V);
+
+/*
+ * Greedy LM head with selective FP32 recompute. Source: "Greedy Decoding Is Not
+ * Precision-Invariant" (arXiv 2609.26621), abstract.
+ *   1. logits = bi_matmul(h, W) rounded to bf16 (the first, bf16 pass);
+ *   2. per row: top-2 of the bf16 logits (lowest index wins ties; NaN never
+ *      wins), margin = top1 - top2 in fp32;
+ *   3. rows with margin < margin_threshold are recomputed in fp32: operands
+ *      widened from bf16, one fp32 FMA chain per logit in ascending k (no tensor
+ *      cores, no TF32), and the token is the argmax of those fp32 logits;
+ *      other rows keep the first-pass argmax.
+ * h: [M, K] bf16, stride ldh. W: [V, K] bf16 contiguous. tokens: [M] int32 out.
+ * recomputed: [M] int32 out (1 if the row took step 3, else 0). logits_fp32:
+ * optional [M, V] fp32 out (may be NULL): rows that took step 3 receive their fp32
+ * logits, other rows are not written. Requires the bi_matmul rules on K and
+ * V % 8 == 0. M == 0 is a no-op.
+ */
+bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int64_t M, int64_t V,
+                           int64_t K, float margin_threshold, int32_t* tokens, int32_t* recomputed,
+                           float* logits_fp32, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/*
+ * Reads and clears the device error word of the current device (synchronises the
+ * device first). *code receives BI_OK, BI_ERR_DEVICE_TIMEOUT or
+ * BI_ERR_DEVICE_INDEX (the first error recorded since the last read). Returns
+ * BI_ERR_NULL if code is NULL, BI_ERR_CUDA if the read fails.
+ */
+bi_status bi_get_device_error(int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BI_H_ */

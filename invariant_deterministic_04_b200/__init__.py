@@ -1,0 +1,253 @@
+"""Python binding of libbi, the batch-invariant forward-pass kernels for B200.
+
+Argument marshalling only: every step of every operation runs in the CUDA
+kernels behind the C ABI declared in include/bi.h. PyTorch provides device
+memory and the current stream. There is no CPU or library fallback: if
+libbi.so is missing or fails to load, every call raises ``BIError``.
+
+Operations (see include/bi.h for the exact contracts):
+  rmsnorm, matmul, attention_decode, attention_prefill, kv_append,
+  lmhead_argmax, get_device_error.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+from ._build import LIB_PATH, build_library  # noqa: F401
+
+PAGE_TOKENS = 16
+KV_SPLIT = 256
+
+_STATUS = {
+    0: "BI_OK", 1: "BI_ERR_NULL", 2: "BI_ERR_SHAPE", 3: "BI_ERR_ALIGN", 4: "BI_ERR_WORKSPACE",
+    5: "BI_ERR_UNSUPPORTED", 6: "BI_ERR_CUDA", 7: "BI_ERR_DEVICE_TIMEOUT", 8: "BI_ERR_DEVICE_INDEX",
+}
+
+
+class BIError(RuntimeError):
+    def __init__(self, where: str, status: int):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+
+
+_P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+_SIGNATURES = {
+    "bi_status_string": ([_I32], ctypes.c_char_p),
+    "bi_version": ([], _I32),
+    "bi_rmsnorm": ([_P, _I64, _P, _P, _I64, _I64, _I64, _F, _P], _I32),
+    "bi_matmul": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _P], _I32),
+    "bi_attention_workspace_size": ([_I64, _I32, _I32, _I32], _SZ),
+    "bi_attention_decode": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ, _P], _I32),
+    "bi_attention_prefill": ([_P, _P, _P, _P, _P, _I64, _P, _I32, _I32, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ, _P],
+                             _I32),
+    "bi_kv_append": ([_P, _P, _P, _P, _P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P], _I32),
+    "bi_lmhead_workspace_size": ([_I64, _I64], _SZ),
+    "bi_lmhead_argmax": ([_P, _I64, _P, _I64, _I64, _I64, _F, _P, _P, _P, _P, _SZ, _P], _I32),
+    "bi_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], _I32),
+}
+
+_lib = None
+_load_error = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libbi.so (raises BIError-like RuntimeError if it cannot be loaded)."""
+    global _lib, _load_error
+    if _lib is not None:
+        return _lib
+    if _load_error is None:
+        if not os.path.exists(LIB_PATH):
+            _load_error = f"{LIB_PATH} is missing; build it with __graft_entry__.build() (nvcc, sm_100a)"
+        else:
+            try:
+                handle = ctypes.CDLL(LIB_PATH)
+                for name, (args, ret) in _SIGNATURES.items():
+                    fn = getattr(handle, name)
+                    fn.argtypes, fn.restype = args, ret
+                _lib = handle
+                return _lib
+            except OSError as e:  # pragma: no cover
+                _load_error = f"cannot load {LIB_PATH}: {e}"
+    raise RuntimeError(_load_error)
+
+
+def _check(where: str, status: int):
+    if status != 0:
+        raise BIError(where, status)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _req(t: torch.Tensor, dtype, name: str, dims: int | None = None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dims is not None and t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dims, got {tuple(t.shape)}")
+
+
+def _contig(t: torch.Tensor, name: str):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ---------------------------------------------------------------------------
+
+
+def rmsnorm(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, out: torch.Tensor | None = None, stream=None):
+    """y = bf16(x * rsqrt(mean(x^2) + eps) * w), one fixed reduction order per row."""
+    _req(x, torch.bfloat16, "x", 2)
+    _req(w, torch.bfloat16, "w", 1)
+    _contig(w, "w")
+    if x.stride(1) != 1:
+        raise ValueError("x rows must be contiguous")
+    M, K = x.shape
+    y = torch.empty_like(x, memory_format=torch.contiguous_format) if out is None else out
+    _check("bi_rmsnorm", lib().bi_rmsnorm(_ptr(x), x.stride(0), _ptr(w), _ptr(y), y.stride(0), M, K, eps,
+                                         _stream(stream)))
+    return y
+
+
+def matmul(a: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    """C = A W^T with A [M, K], W [N, K] (nn.Linear layout), bf16 out, fixed tile and K order."""
+    _req(a, torch.bfloat16, "a", 2)
+    _req(w, torch.bfloat16, "w", 2)
+    if a.stride(1) != 1 or w.stride(1) != 1:
+        raise ValueError("a and w rows must be contiguous")
+    M, K = a.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError(f"inner dimensions differ: {tuple(a.shape)} x {tuple(w.shape)}^T")
+    c = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else out
+    _check("bi_matmul", lib().bi_matmul(_ptr(a), a.stride(0), _ptr(w), w.stride(0), _ptr(c), c.stride(0), M, N, K,
+                                       _stream(stream)))
+    return c
+
+
+def attention_workspace_size(rows: int, Hq: int, D: int, max_pages_per_seq: int) -> int:
+    return int(lib().bi_attention_workspace_size(rows, Hq, D, max_pages_per_seq))
+
+
+def _workspace(nbytes: int, device, workspace):
+    if workspace is not None:
+        return workspace, workspace.numel() * workspace.element_size()
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device), nbytes
+
+
+def attention_decode(q, k_cache, v_cache, page_table, seq_lens, scale: float | None = None, out=None,
+                     workspace=None, stream=None):
+    """Decode attention over the paged store; q [B, Hq, D] -> out [B, Hq, D]."""
+    _req(q, torch.bfloat16, "q", 3)
+    _req(k_cache, torch.bfloat16, "k_cache", 4)
+    _req(v_cache, torch.bfloat16, "v_cache", 4)
+    _req(page_table, torch.int32, "page_table", 2)
+    _req(seq_lens, torch.int32, "seq_lens", 1)
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (page_table, "page_table"),
+                 (seq_lens, "seq_lens")):
+        _contig(t, n)
+    B, Hq, D = q.shape
+    num_pages, Hkv = k_cache.shape[0], k_cache.shape[1]
+    if k_cache.shape != v_cache.shape or k_cache.shape[2] != PAGE_TOKENS or k_cache.shape[3] != D:
+        raise ValueError("k_cache/v_cache must be [num_pages, Hkv, 16, D]")
+    if page_table.shape[0] < B or seq_lens.shape[0] < B:
+        raise ValueError("page_table and seq_lens need a row per sequence")
+    maxp = page_table.shape[1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out = torch.empty_like(q) if out is None else out
+    ws, nbytes = _workspace(attention_workspace_size(B, Hq, D, maxp), q.device, workspace)
+    _check("bi_attention_decode", lib().bi_attention_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), maxp, _ptr(seq_lens), _ptr(out),
+        B, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def attention_prefill(q, q_seq, q_pos, k_cache, v_cache, page_table, scale: float | None = None, out=None,
+                      workspace=None, stream=None):
+    """Causal prefill; row t of q [T, Hq, D] sees keys 0..q_pos[t] of sequence q_seq[t]."""
+    _req(q, torch.bfloat16, "q", 3)
+    _req(q_seq, torch.int32, "q_seq", 1)
+    _req(q_pos, torch.int32, "q_pos", 1)
+    _req(k_cache, torch.bfloat16, "k_cache", 4)
+    _req(v_cache, torch.bfloat16, "v_cache", 4)
+    _req(page_table, torch.int32, "page_table", 2)
+    for t, n in ((q, "q"), (q_seq, "q_seq"), (q_pos, "q_pos"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                 (page_table, "page_table")):
+        _contig(t, n)
+    T, Hq, D = q.shape
+    num_pages, Hkv = k_cache.shape[0], k_cache.shape[1]
+    if k_cache.shape != v_cache.shape or k_cache.shape[2] != PAGE_TOKENS or k_cache.shape[3] != D:
+        raise ValueError("k_cache/v_cache must be [num_pages, Hkv, 16, D]")
+    if q_seq.shape[0] != T or q_pos.shape[0] != T:
+        raise ValueError("q_seq and q_pos need one entry per query row")
+    num_seqs, maxp = page_table.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out = torch.empty_like(q) if out is None else out
+    ws, nbytes = _workspace(attention_workspace_size(T, Hq, D, maxp), q.device, workspace)
+    _check("bi_attention_prefill", lib().bi_attention_prefill(
+        _ptr(q), _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), num_seqs,
+        maxp, _ptr(out), T, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def kv_append(k_new, v_new, q_seq, q_pos, k_cache, v_cache, page_table, stream=None):
+    """Write k_new/v_new [T, Hkv, D] into the paged store at (q_seq[t], q_pos[t])."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _req(t, torch.bfloat16, n)
+        _contig(t, n)
+    for t, n in ((q_seq, "q_seq"), (q_pos, "q_pos"), (page_table, "page_table")):
+        _req(t, torch.int32, n)
+        _contig(t, n)
+    T, Hkv, D = k_new.shape
+    num_seqs, maxp = page_table.shape
+    _check("bi_kv_append", lib().bi_kv_append(
+        _ptr(k_new), _ptr(v_new), _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
+        _ptr(page_table), num_seqs, maxp, T, Hkv, D, _stream(stream)))
+
+
+def lmhead_workspace_size(M: int, V: int) -> int:
+    return int(lib().bi_lmhead_workspace_size(M, V))
+
+
+def lmhead_argmax(h, w, margin_threshold: float = 0.5, want_logits: bool = False, tokens=None, recomputed=None,
+                  logits_fp32=None, workspace=None, stream=None):
+    """Greedy tokens with the selective FP32 recompute.
+
+    Returns (tokens int32 [M], recomputed int32 [M], logits_fp32 [M, V] or None).
+    """
+    _req(h, torch.bfloat16, "h", 2)
+    _req(w, torch.bfloat16, "w", 2)
+    _contig(w, "w")
+    if h.stride(1) != 1:
+        raise ValueError("h rows must be contiguous")
+    M, K = h.shape
+    V = w.shape[0]
+    dev = h.device
+    tokens = torch.empty(M, dtype=torch.int32, device=dev) if tokens is None else tokens
+    recomputed = torch.empty(M, dtype=torch.int32, device=dev) if recomputed is None else recomputed
+    if want_logits and logits_fp32 is None:
+        logits_fp32 = torch.full((M, V), float("nan"), dtype=torch.float32, device=dev)
+    ws, nbytes = _workspace(lmhead_workspace_size(M, V), dev, workspace)
+    _check("bi_lmhead_argmax", lib().bi_lmhead_argmax(
+        _ptr(h), h.stride(0), _ptr(w), M, V, K, margin_threshold, _ptr(tokens), _ptr(recomputed),
+        _ptr(logits_fp32), _ptr(ws), nbytes, _stream(stream)))
+    return tokens, recomputed, logits_fp32
+
+
+def get_device_error() -> int:
+    """Read and clear the device error word (synchronises the device)."""
+    code = ctypes.c_int32(0)
+    _check("bi_get_device_error", lib().bi_get_device_error(ctypes.byref(code)))
+    return int(code.value)

@@ -1,0 +1,395 @@
+// Batch-invariant attention over a unified paged KV store (decode and causal prefill).
+//
+// Sources: "Defeating Nondeterminism in LLM Inference" technical summary
+// (mobiles-han blog), section 対応策：バッチ不変なカーネル設計, kernel table, row
+// Attention — join the cache and the current tokens into one layout before
+// attending, and cut the KV sequence into splits of a fixed SIZE (not a fixed
+// count chosen from the batch); the usage article, section 注意点・補足実装
+// (FixedAttention sketch: concatenate cache and new keys, fixed chunk size).
+//
+// Per-row schedule (identical for decode and prefill; a function of the row's own
+// visible length L only):
+//   * the visible keys 0..L-1 are cut into splits at absolute positions 0, 256,
+//     512, ...; split s covers pages 16s .. 16s+15 of the row's page-table row;
+//   * one warp reduces one (row, kv-head, split) for the Hq/Hkv query heads that
+//     share the kv-head, page by page in ascending order, with an online softmax
+//     in the base-2 domain (scores pre-multiplied by scale*log2(e));
+//   * inside a page, a token's q.k is an 8-term FMA chain per lane (8 dims)
+//     followed by a fixed xor reduce-scatter tree over the D/8 lanes of the token;
+//     token t of the page is handled by lane group t mod (256/D) and the groups'
+//     partial sums are merged by a fixed xor tree at the end of the split;
+//   * splits are folded in ascending order: M = max_s m_s, then
+//     L = sum_s l_s 2^(m_s - M), O = sum_s o_s 2^(m_s - M) (FMA chains from 0),
+//     out = O / L rounded to bf16.
+// A prefill query at absolute position p is computed as a decode row of length
+// p + 1 reading the same page-table row, so whole and chunked prefill, and decode,
+// give the same bits for the same row. Slots past L are never folded in (stale
+// slots may hold NaN); the copy engine only fetches the valid rows of a page.
+#pragma once
+
+#include "device.cuh"
+
+namespace bi {
+namespace attn {
+
+constexpr int PAGE = BI_PAGE_TOKENS;
+constexpr int SPLIT = BI_KV_SPLIT;
+constexpr int PAGES_PER_SPLIT = SPLIT / PAGE;
+constexpr int kWarps = 8;  // warps per CTA in the split kernel, each with its own page ring
+constexpr int NSTAGE = 3;  // pages in flight per warp
+
+// Where a query row reads its keys: decode rows use (row, seq_lens[row]);
+// prefill rows use (q_seq[row], q_pos[row] + 1).
+struct Rows {
+  const int32_t* seq_lens;
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  int num_pt_rows;
+  int max_pages;
+};
+
+// Returns the row's visible length (0 if its ids are out of range, with the
+// device error recorded) and its page-table row.
+__device__ __forceinline__ int row_len(const Rows& R, int r, int& pt_row) {
+  int len;
+  if (R.q_pos) {
+    pt_row = R.q_seq[r];
+    len = R.q_pos[r] + 1;
+  } else {
+    pt_row = r;
+    len = R.seq_lens[r];
+  }
+  if (pt_row < 0 || pt_row >= R.num_pt_rows || len < 0 || len > R.max_pages * PAGE) {
+    record_error(BI_ERR_DEVICE_INDEX);
+    pt_row = 0;
+    return 0;
+  }
+  return len;
+}
+
+__device__ __forceinline__ int num_splits(const Rows& R, int r) {
+  int pt_row;
+  const int len = row_len(R, r, pt_row);
+  return (len + SPLIT - 1) / SPLIT;
+}
+
+// off[r] = number of splits of rows 0..r-1; off[nrows] = total. One CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) split_offsets_kernel(Rows R, int nrows, int32_t* off) {
+  __shared__ int32_t sums[1024];
+  const int tid = threadIdx.x;
+  const int per = (nrows + 1023) / 1024;
+  const int r0 = tid * per;
+  const int r1 = min(r0 + per, nrows);
+  int local = 0;
+  for (int r = r0; r < r1; ++r) local += num_splits(R, r);
+  sums[tid] = local;
+  __syncthreads();
+  for (int d = 1; d < 1024; d <<= 1) {
+    const int v = tid >= d ? sums[tid - d] : 0;
+    __syncthreads();
+    sums[tid] += v;
+    __syncthreads();
+  }
+  int run = sums[tid] - local;
+  for (int r = r0; r < r1; ++r) {
+    off[r] = run;
+    run += num_splits(R, r);
+  }
+  if (tid == 1023) off[nrows] = sums[1023];
+}
+
+// Reduce-scatter of G per-head partial sums over the LPT lanes of one token
+// (xor butterfly, highest offset first). At each level a lane keeps the half of
+// its heads selected by its lane bit and adds the partner's copy of that half
+// (own + partner); once one head is left the remaining levels are all-reduce
+// steps. Returns the full sum of head dl / (LPT / G).
+template <int G, int LPT>
+__device__ __forceinline__ float reduce_scatter(float (&v)[G], int dl) {
+#pragma unroll
+  for (int off = LPT / 2, n = G; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const bool upper = (dl & off) != 0;
+#pragma unroll
+      for (int i = 0; i < G / 2; ++i) {
+        if (i < n / 2) {
+          const float send = upper ? v[i] : v[i + n / 2];
+          const float keep = upper ? v[i + n / 2] : v[i];
+          v[i] = __fadd_rn(keep, __shfl_xor_sync(kFullMask, send, off));
+        }
+      }
+      n >>= 1;
+    } else {
+      v[0] = __fadd_rn(v[0], __shfl_xor_sync(kFullMask, v[0], off));
+    }
+  }
+  return v[0];
+}
+
+// Inverse of the scatter: every lane of the token receives the G per-head values
+// (head h held by lanes with dl / (LPT / G) == h). Pure data movement.
+template <int G, int LPT>
+__device__ __forceinline__ void all_gather(float x, int dl, float (&out)[G]) {
+  out[0] = x;
+#pragma unroll
+  for (int off = LPT / G, n = 1; off < LPT; off <<= 1, n <<= 1) {
+    const bool upper = (dl & off) != 0;
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i) {
+      if (i < n) {
+        const float other = __shfl_xor_sync(kFullMask, out[i], off);
+        const float mine = out[i];
+        out[i] = upper ? other : mine;
+        out[i + n] = upper ? mine : other;
+      }
+    }
+  }
+}
+
+template <int D>
+constexpr int split_smem_bytes() {
+  return kWarps * NSTAGE * 2 * PAGE * D * 2 + kWarps * NSTAGE * 8;
+}
+
+// One warp per (row, kv-head g, split): writes the split's (m, l) per query head
+// and its unnormalised o[D] per query head into the workspace.
+template <int D, int G>
+__global__ void __launch_bounds__(kWarps * 32, 1)
+    attn_split_kernel(const uint16_t* __restrict__ q, int Hq, int Hkv, const uint16_t* __restrict__ kc,
+                      const uint16_t* __restrict__ vc, int64_t num_pages, const int32_t* __restrict__ pt,
+                      Rows R, int nrows, const int32_t* __restrict__ off, float* __restrict__ po,
+                      float2* __restrict__ pml, float c) {
+  constexpr int LPT = D / 8;        // lanes per token (8 dims per lane)
+  constexpr int TPW = 32 / LPT;     // tokens per warp step
+  constexpr int STEPS = PAGE / TPW;
+  constexpr int HEAD_LANES = LPT / G;
+  constexpr int PAGE_BYTES = PAGE * D * 2;
+  constexpr int STAGE_BYTES = 2 * PAGE_BYTES;
+  static_assert(G >= 1 && G <= LPT, "group size");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tg = lane / LPT, dl = lane % LPT;
+  const int hd = dl / HEAD_LANES;
+  const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * NSTAGE * STAGE_BYTES);
+  const uint32_t bars = smem_u32(smem) + (uint32_t)(kWarps * NSTAGE * STAGE_BYTES + warp * NSTAGE * 8);
+
+  if (lane == 0) {
+    for (int s = 0; s < NSTAGE; ++s) mbar_init(bars + 8 * s, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  const int total = off[nrows] * Hkv;
+  const int64_t kv_head_stride = (int64_t)PAGE * D;
+  uint32_t seq = 0;  // pages this warp has consumed so far
+
+  for (int item = blockIdx.x * kWarps + warp; item < total; item += gridDim.x * kWarps) {
+    const int f = item / Hkv, g = item - (item / Hkv) * Hkv;
+    int lo = 0, hi = nrows;  // off[lo] <= f < off[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (off[mid] <= f) lo = mid;
+      else hi = mid;
+    }
+    const int r = lo, s = f - off[lo];
+    int pt_row;
+    const int len = row_len(R, r, pt_row);
+    const int t0 = s * SPLIT;
+    const int t1 = min(t0 + SPLIT, len);
+    const int np = (t1 - t0 + PAGE - 1) / PAGE;
+    const int32_t* prow = pt + (int64_t)pt_row * R.max_pages + s * PAGES_PER_SPLIT;
+
+    float qf[G][8];
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + ((int64_t)r * Hq + g * G + j) * D + dl * 8));
+      unpack8(qv, qf[j]);
+    }
+
+    // Lane 0 starts the copy of page j of this split into its ring stage.
+    auto issue = [&](int j, uint32_t sq) {
+      const uint32_t st = sq % NSTAGE;
+      const uint32_t bar = bars + 8 * st;
+      const int pg = prow[j];
+      const int nvalid = min(PAGE, t1 - t0 - j * PAGE);
+      if (pg < 0 || pg >= num_pages) {
+        record_error(BI_ERR_DEVICE_INDEX);
+        mbar_arrive_expect_tx(bar, 0);
+        return;
+      }
+      const uint32_t bytes = (uint32_t)(nvalid * D * 2);
+      const int64_t src = ((int64_t)pg * Hkv + g) * kv_head_stride;
+      const uint32_t kdst = ring + st * STAGE_BYTES;
+      mbar_arrive_expect_tx(bar, 2 * bytes);
+      bulk_g2s(kdst, kc + src, bytes, bar);
+      bulk_g2s(kdst + PAGE_BYTES, vc + src, bytes, bar);
+    };
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      for (int j = 0; j < NSTAGE && j < np; ++j) issue(j, seq + j);
+    }
+
+    float m = -INFINITY, l = 0.f;
+    float o[G][8];
+#pragma unroll
+    for (int j = 0; j < G; ++j)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[j][e] = 0.f;
+
+    bool ok = true;
+    for (int j = 0; j < np; ++j, ++seq) {
+      const uint32_t st = seq % NSTAGE;
+      ok = __all_sync(kFullMask, mbar_wait(bars + 8 * st, (seq / NSTAGE) & 1u));
+      if (!ok) break;
+      const int pg = prow[j];
+      const int nvalid = (pg < 0 || pg >= num_pages) ? 0 : min(PAGE, t1 - t0 - j * PAGE);
+      const uint32_t kb = ring + st * STAGE_BYTES, vb = kb + PAGE_BYTES;
+
+      float sc[STEPS];
+#pragma unroll
+      for (int u = 0; u < STEPS; ++u) {
+        const int t = u * TPW + tg;
+        float kf[8];
+        unpack8(ld_shared_v4(kb + (uint32_t)((t * D + dl * 8) * 2)), kf);
+        float part[G];
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          float a = __fmul_rn(qf[i][0], kf[0]);
+#pragma unroll
+          for (int e = 1; e < 8; ++e) a = __fmaf_rn(qf[i][e], kf[e], a);
+          part[i] = a;
+        }
+        const float dot = reduce_scatter<G, LPT>(part, dl);
+        sc[u] = t < nvalid ? __fmul_rn(dot, c) : -INFINITY;
+      }
+      float pm = sc[0];
+#pragma unroll
+      for (int u = 1; u < STEPS; ++u) pm = fmaxf(pm, sc[u]);
+#pragma unroll
+      for (int o2 = LPT; o2 < 32; o2 <<= 1) pm = fmaxf(pm, __shfl_xor_sync(kFullMask, pm, o2));
+      const float m_new = fmaxf(m, pm);
+      const float alpha = m_new == -INFINITY ? 1.f : exp2f(__fsub_rn(m, m_new));
+      l = __fmul_rn(l, alpha);
+      float al[G];
+      all_gather<G, LPT>(alpha, dl, al);
+#pragma unroll
+      for (int i = 0; i < G; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[i][e] = __fmul_rn(o[i][e], al[i]);
+#pragma unroll
+      for (int u = 0; u < STEPS; ++u) {
+        const int t = u * TPW + tg;
+        const bool valid = t < nvalid;
+        const float p = valid ? exp2f(__fsub_rn(sc[u], m_new)) : 0.f;
+        l = __fadd_rn(l, p);
+        float pa[G];
+        all_gather<G, LPT>(p, dl, pa);
+        float vf[8];
+        unpack8(ld_shared_v4(vb + (uint32_t)((t * D + dl * 8) * 2)), vf);
+        if (valid) {
+#pragma unroll
+          for (int i = 0; i < G; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[i][e] = __fmaf_rn(pa[i], vf[e], o[i][e]);
+        }
+      }
+      m = m_new;
+      __syncwarp();
+      if (lane == 0 && j + NSTAGE < np) {
+        fence_proxy_async_smem();
+        issue(j + NSTAGE, seq + NSTAGE);
+      }
+    }
+    if (!ok) return;  // a copy never landed: error recorded, leave the warp
+
+    // Merge the token groups of the warp (fixed xor tree).
+#pragma unroll
+    for (int o2 = LPT; o2 < 32; o2 <<= 1) {
+      l = __fadd_rn(l, __shfl_xor_sync(kFullMask, l, o2));
+#pragma unroll
+      for (int i = 0; i < G; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[i][e] = __fadd_rn(o[i][e], __shfl_xor_sync(kFullMask, o[i][e], o2));
+    }
+    if (tg == 0) {
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        float4* dst = reinterpret_cast<float4*>(po + ((int64_t)f * Hq + g * G + i) * D + dl * 8);
+        dst[0] = make_float4(o[i][0], o[i][1], o[i][2], o[i][3]);
+        dst[1] = make_float4(o[i][4], o[i][5], o[i][6], o[i][7]);
+      }
+      if (dl % HEAD_LANES == 0) pml[(int64_t)f * Hq + g * G + hd] = make_float2(m, l);
+    }
+  }
+}
+
+// One warp per (row, query head): fold the row's splits in ascending order.
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ po,
+                                                           const float2* __restrict__ pml,
+                                                           const int32_t* __restrict__ off, int nrows,
+                                                           int Hq, uint16_t* __restrict__ out) {
+  constexpr int DPL = D / 32;  // dims per lane
+  const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= nrows * Hq) return;
+  const int r = w / Hq, h = w - (w / Hq) * Hq;
+  const int f0 = off[r], n = off[r + 1] - off[r];
+  float O[DPL];
+#pragma unroll
+  for (int d = 0; d < DPL; ++d) O[d] = 0.f;
+  float L = 0.f;
+  float M = -INFINITY;
+  for (int s = 0; s < n; ++s) M = fmaxf(M, pml[(int64_t)(f0 + s) * Hq + h].x);
+  if (M != -INFINITY) {
+    for (int s = 0; s < n; ++s) {
+      const int64_t idx = (int64_t)(f0 + s) * Hq + h;
+      const float2 ml = pml[idx];
+      const float wgt = exp2f(__fsub_rn(ml.x, M));
+      L = __fmaf_rn(ml.y, wgt, L);
+      const float* src = po + idx * D + lane * DPL;
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) O[d] = __fmaf_rn(src[d], wgt, O[d]);
+    }
+  }
+  uint16_t* dst = out + ((int64_t)r * Hq + h) * D + lane * DPL;
+#pragma unroll
+  for (int d = 0; d < DPL; d += 2) {
+    const float a = L > 0.f ? __fdiv_rn(O[d], L) : 0.f;
+    const float b = L > 0.f ? __fdiv_rn(O[d + 1], L) : 0.f;
+    *reinterpret_cast<uint32_t*>(dst + d) = pack_bf16x2(a, b);
+  }
+}
+
+// One warp per (token, kv-head): copy the token's K and V rows into its page slot.
+__global__ void __launch_bounds__(256) kv_append_kernel(const uint16_t* __restrict__ kn,
+                                                        const uint16_t* __restrict__ vn,
+                                                        const int32_t* __restrict__ q_seq,
+                                                        const int32_t* __restrict__ q_pos,
+                                                        uint16_t* __restrict__ kc, uint16_t* __restrict__ vc,
+                                                        int64_t num_pages, const int32_t* __restrict__ pt,
+                                                        int num_seqs, int max_pages, int T, int Hkv, int D) {
+  const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= (int64_t)T * Hkv) return;
+  const int t = (int)(w / Hkv), g = (int)(w - (w / Hkv) * Hkv);
+  const int sq = q_seq[t], pos = q_pos[t];
+  if (sq < 0 || sq >= num_seqs || pos < 0 || pos >= max_pages * PAGE) {
+    if (lane == 0) record_error(BI_ERR_DEVICE_INDEX);
+    return;
+  }
+  const int pg = pt[(int64_t)sq * max_pages + pos / PAGE];
+  if (pg < 0 || pg >= num_pages) {
+    if (lane == 0) record_error(BI_ERR_DEVICE_INDEX);
+    return;
+  }
+  const int64_t dst = (((int64_t)pg * Hkv + g) * PAGE + pos % PAGE) * D;
+  const int64_t src = ((int64_t)t * Hkv + g) * D;
+  for (int i = lane; i < D / 8; i += 32) {
+    reinterpret_cast<uint4*>(kc + dst)[i] = __ldg(reinterpret_cast<const uint4*>(kn + src) + i);
+    reinterpret_cast<uint4*>(vc + dst)[i] = __ldg(reinterpret_cast<const uint4*>(vn + src) + i);
+  }
+}
+
+}  // namespace attn
+}  // namespace bi

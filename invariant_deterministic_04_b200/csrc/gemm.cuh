@@ -1,0 +1,299 @@
+// Batch-invariant bf16 matmul C = A * W^T on 5th-generation tensor cores.
+//
+// Source: "Defeating Nondeterminism in LLM Inference" technical summary
+// (mobiles-han blog), section 対応策：バッチ不変なカーネル設計, kernel table, row
+// MatMul: use one kernel configuration for every shape — fixed tile sizes, no
+// split-K, no switch between tensor-core and non-tensor-core paths — and accept a
+// modest loss of speed.
+//
+// Design (sm_100a):
+//   * one output tile = 128 rows x 256 columns, held as fp32 in tensor memory
+//     (TMEM, 256 columns per accumulator, two accumulators per CTA so the
+//     epilogue of one tile overlaps the main loop of the next);
+//   * K is consumed in 64-wide blocks in ascending order; each block is four
+//     tcgen05.mma.kind::f16 instructions of shape 128x256x16, again in ascending
+//     k. Every output element therefore sees the same sequence of tensor-core
+//     accumulations for every M and every position of its row in the tile;
+//   * A and W tiles are brought into shared memory by TMA (128-byte swizzle,
+//     K-major) through a 4-stage mbarrier ring; out-of-range rows of a ragged tile
+//     are zero-filled by TMA and masked in the epilogue, so they cannot touch other rows;
+//   * warp 0 issues TMA, warp 1 (one thread) issues the MMAs, warps 2-5 drain
+//     TMEM (tcgen05.ld), round to bf16 (nearest even) and store;
+//   * persistent grid of min(#tiles, #SMs) CTAs; tile t goes to CTA t mod grid.
+//     The grid only decides which CTA computes a tile, never how.
+//   * every mbarrier wait is bounded; on expiry the kernel records
+//     BI_ERR_DEVICE_TIMEOUT, all roles leave their loops, TMEM is freed.
+#pragma once
+
+#include <mutex>
+
+#include "device.cuh"
+
+namespace bi {
+namespace gemm {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KiB
+constexpr int B_BYTES = BN * BK * 2;  // 32 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BN;  // two fp32 accumulators
+constexpr int kThreads = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kEpiThreads = 128;
+constexpr int BAR_BYTES = 8 * (2 * STAGES + 4) + 16;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+
+// Instruction descriptor for kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 =
+// 1), B bf16 (bits 10-12 = 1), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+// Shared-memory matrix descriptor for a K-major operand written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart (stride byte
+// offset), version 1, layout SWIZZLE_128B (2). Start address is advanced by 32
+// bytes per 16-element k step inside the atom.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     uint16_t* __restrict__ C, int64_t ldc, int M, int N, int K) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t a_s = base;
+  const uint32_t b_s = base + STAGES * A_BYTES;
+  const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+  // barriers: full[0..S), empty[0..S), tfull[0..2), tempty[0..2)
+#define FULL(s) (bar0 + 8u * (s))
+#define EMPTY(s) (bar0 + 8u * (STAGES + (s)))
+#define TFULL(a) (bar0 + 8u * (2 * STAGES + (a)))
+#define TEMPTY(a) (bar0 + 8u * (2 * STAGES + 2 + (a)))
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 4));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
+  const int tiles = mt * nt;
+  const int nkb = K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(FULL(s), 1);
+      mbar_init(EMPTY(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(TFULL(a), 1);
+      mbar_init(TEMPTY(a), kEpiThreads);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---- TMA producer
+      int s = 0;
+      uint32_t ph = 0;
+      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+        const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(EMPTY(s), ph ^ 1u)) {
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(FULL(s), STAGE_BYTES);
+          tma_load_2d(a_s + s * A_BYTES, &tmA, kb * BK, m0, FULL(s));
+          tma_load_2d(b_s + s * B_BYTES, &tmB, kb * BK, n0, FULL(s));
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---- MMA issuer (single thread)
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+        if (!mbar_wait(TEMPTY(acc), aph ^ 1u)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(FULL(s), ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sw128_desc(a_s + s * A_BYTES + kk * 32);
+            const uint64_t bd = sw128_desc(b_s + s * B_BYTES + kk * 32);
+            tc_mma_f16(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(EMPTY(s));  // frees the stage once these MMAs have read it
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_commit(TFULL(acc));  // accumulator complete
+        acc ^= 1;
+        if (acc == 0) aph ^= 1u;
+      }
+    }
+  } else {  // ---- epilogue: warps 2..5; warp w may read TMEM lanes 32*(w%4) .. +31
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
+      const bool ok = __all_sync(kFullMask, mbar_wait(TFULL(acc), aph));
+      if (!ok || *abort_flag) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int row = m0 + quarter * 32 + lane;
+      uint16_t* crow = C + (int64_t)row * ldc;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();  // tcgen05.ld is .sync.aligned: the warp must be converged
+        tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
+        tmem_wait_ld();
+        const int col = n0 + c * 32;
+        if (row < M && col < N) {
+          if (col + 32 <= N) {
+            uint4* dst = reinterpret_cast<uint4*>(crow + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              dst[v] = o;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (col + e < N) crow[col + e] = to_bf16_bits(__uint_as_float(r[e]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(TEMPTY(acc));
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+  }
+#undef FULL
+#undef EMPTY
+#undef TFULL
+#undef TEMPTY
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] with row stride ld (elements); box = 64 cols x box_rows.
+inline bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int64_t ld,
+                     uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2u};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool smem_set = false;
+};
+
+inline DeviceInfo* device_info(int dev) {
+  static DeviceInfo infos[64];
+  static std::mutex mu;
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceInfo* d = &infos[dev];
+  if (d->sms == 0) {
+    if (cudaDeviceGetAttribute(&d->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+  }
+  if (!d->smem_set) {
+    if (cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+        cudaSuccess)
+      return nullptr;
+    d->smem_set = true;
+  }
+  return d;
+}
+
+inline bi_status launch(const uint16_t* A, int64_t lda, const uint16_t* W, int64_t ldw, uint16_t* C,
+                        int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
+  DeviceInfo* info = device_info(dev);
+  if (!info) return BI_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, lda, BM) || !make_map(&tb, W, N, K, ldw, BN)) return BI_ERR_CUDA;
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = (int)(tiles < info->sms ? tiles : info->sms);
+  gemm_bf16_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(ta, tb, C, ldc, (int)M, (int)N, (int)K);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+}  // namespace gemm
+}  // namespace bi

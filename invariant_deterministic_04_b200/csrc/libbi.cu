@@ -1,0 +1,279 @@
+// libbi: the C ABI of the batch-invariant kernels (declared in include/bi.h).
+//
+// One translation unit: the kernels are included here so that they share the
+// device error word without relocatable device code. Every entry point validates
+// its arguments on the host first and launches nothing on error.
+#include <climits>
+#include <cmath>
+#include <mutex>
+
+#include "device.cuh"
+#include "rmsnorm.cuh"
+#include "gemm.cuh"
+#include "attention.cuh"
+#include "lmhead.cuh"
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool ranges_overlap(const void* a, size_t abytes, const void* b, size_t bbytes) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bbytes && b0 < a0 + abytes;
+}
+
+size_t span_bytes(int64_t rows, int64_t cols, int64_t ld, size_t elem) {
+  return rows <= 0 ? 0 : (size_t)((rows - 1) * ld + cols) * elem;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// ---- attention helpers
+
+int max_splits(int max_pages_per_seq) { return (max_pages_per_seq + bi::attn::PAGES_PER_SPLIT - 1) / bi::attn::PAGES_PER_SPLIT; }
+
+struct AttnWs {
+  int32_t* off;
+  float2* pml;
+  float* po;
+};
+
+size_t attn_ws_size(int64_t rows, int Hq, int D, int max_pages, AttnWs* layout, void* base) {
+  if (rows < 0 || Hq <= 0 || D <= 0 || max_pages <= 0) return 0;
+  const int64_t ms = max_splits(max_pages);
+  const size_t off_b = align256((size_t)(rows + 1) * 4);
+  const size_t pml_b = align256((size_t)rows * ms * Hq * 8);
+  const size_t po_b = align256((size_t)rows * ms * Hq * D * 4);
+  if (layout && base) {
+    uint8_t* p = static_cast<uint8_t*>(base);
+    layout->off = reinterpret_cast<int32_t*>(p);
+    layout->pml = reinterpret_cast<float2*>(p + off_b);
+    layout->po = reinterpret_cast<float*>(p + off_b + pml_b);
+  }
+  return off_b + pml_b + po_b;
+}
+
+template <int D, int G>
+cudaError_t launch_split(int grid_per_sm, const uint16_t* q, int Hq, int Hkv, const uint16_t* kc,
+                         const uint16_t* vc, int64_t num_pages, const int32_t* pt, bi::attn::Rows R, int nrows,
+                         const AttnWs& ws, float c, cudaStream_t st) {
+  constexpr int smem = bi::attn::split_smem_bytes<D>();
+  static std::once_flag once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr = cudaSuccess;
+  std::call_once(once[dev & 63], [&] {
+    attr = cudaFuncSetAttribute(bi::attn::attn_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem);
+  });
+  if (attr != cudaSuccess) return attr;
+  const int grid = device_sms() * grid_per_sm;
+  bi::attn::attn_split_kernel<D, G><<<grid, bi::attn::kWarps * 32, smem, st>>>(q, Hq, Hkv, kc, vc, num_pages, pt,
+                                                                                R, nrows, ws.off, ws.po, ws.pml, c);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_split_g(int G, const uint16_t* q, int Hq, int Hkv, const uint16_t* kc, const uint16_t* vc,
+                           int64_t num_pages, const int32_t* pt, bi::attn::Rows R, int nrows, const AttnWs& ws,
+                           float c, cudaStream_t st) {
+  // D=128 fills ~192 KiB of shared memory per CTA (one CTA per SM); D=64 fits two.
+  const int per_sm = D == 128 ? 1 : 2;
+  switch (G) {
+    case 1: return launch_split<D, 1>(per_sm, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    case 2: return launch_split<D, 2>(per_sm, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    case 4: return launch_split<D, 4>(per_sm, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    default: return launch_split<D, 8>(per_sm, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+  }
+}
+
+bi_status attention_common(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int64_t num_pages,
+                           const int32_t* pt, int max_pages, bi::attn::Rows R, int nrows, uint16_t* out,
+                           int Hq, int Hkv, int D, float scale, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages <= 0 || max_pages <= 0) return BI_ERR_SHAPE;
+  const int G = Hq / Hkv;
+  if ((D != 64 && D != 128) || (G != 1 && G != 2 && G != 4 && G != 8)) return BI_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale)) return BI_ERR_SHAPE;
+  // index arithmetic of the work list is 32-bit
+  if ((int64_t)nrows * max_splits(max_pages) * Hkv >= INT_MAX || (int64_t)nrows * Hq >= INT_MAX / 8)
+    return BI_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(out) || !aligned16(ws)) return BI_ERR_ALIGN;
+  AttnWs lay{};
+  const size_t need = attn_ws_size(nrows, Hq, D, max_pages, &lay, ws);
+  if (ws_bytes < need) return BI_ERR_WORKSPACE;
+  if (nrows == 0) return BI_OK;
+  const float c = (float)((double)scale * 1.4426950408889634);  // scale * log2(e)
+  bi::attn::split_offsets_kernel<<<1, 1024, 0, st>>>(R, nrows, lay.off);
+  if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
+  cudaError_t e = D == 128 ? launch_split_g<128>(G, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st)
+                           : launch_split_g<64>(G, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st);
+  if (e != cudaSuccess) return BI_ERR_CUDA;
+  const int warps = nrows * Hq;
+  const int grid = (warps + 7) / 8;
+  if (D == 128)
+    bi::attn::attn_combine_kernel<128><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+  else
+    bi::attn::attn_combine_kernel<64><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+// ---- LM head workspace: bf16 logits [M, V], fp32 logits [M, V], flagged list [M + 1]
+struct LmWs {
+  uint16_t* logits16;
+  float* logits32;
+  int32_t* list;
+};
+
+size_t lm_ws_size(int64_t M, int64_t V, LmWs* lay, void* base) {
+  if (M < 0 || V <= 0) return 0;
+  const size_t a = align256((size_t)M * V * 2), b = align256((size_t)M * V * 4), c = align256((size_t)(M + 1) * 4);
+  if (lay && base) {
+    uint8_t* p = static_cast<uint8_t*>(base);
+    lay->logits16 = reinterpret_cast<uint16_t*>(p);
+    lay->logits32 = reinterpret_cast<float*>(p + a);
+    lay->list = reinterpret_cast<int32_t*>(p + a + b);
+  }
+  return a + b + c;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bi_status_string(int status) {
+  switch (status) {
+    case BI_OK: return "BI_OK";
+    case BI_ERR_NULL: return "BI_ERR_NULL";
+    case BI_ERR_SHAPE: return "BI_ERR_SHAPE";
+    case BI_ERR_ALIGN: return "BI_ERR_ALIGN";
+    case BI_ERR_WORKSPACE: return "BI_ERR_WORKSPACE";
+    case BI_ERR_UNSUPPORTED: return "BI_ERR_UNSUPPORTED";
+    case BI_ERR_CUDA: return "BI_ERR_CUDA";
+    case BI_ERR_DEVICE_TIMEOUT: return "BI_ERR_DEVICE_TIMEOUT";
+    case BI_ERR_DEVICE_INDEX: return "BI_ERR_DEVICE_INDEX";
+    default: return "BI_ERR_UNKNOWN";
+  }
+}
+
+int bi_version(void) { return 1; }
+
+bi_status bi_rmsnorm(const bi_bf16* x, int64_t ldx, const bi_bf16* w, bi_bf16* y, int64_t ldy, int64_t M,
+                     int64_t K, float eps, void* stream) {
+  if (!x || !w || !y) return BI_ERR_NULL;
+  if (M < 0 || K < 8 || K % 8 != 0 || ldx < K || ldy < K || M > INT_MAX || !std::isfinite(eps) || eps < 0)
+    return BI_ERR_SHAPE;
+  if (K > 16384) return BI_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) || ldx % 8 || ldy % 8) return BI_ERR_ALIGN;
+  if (M == 0) return BI_OK;
+  if (x != y && ranges_overlap(x, span_bytes(M, K, ldx, 2), y, span_bytes(M, K, ldy, 2))) return BI_ERR_SHAPE;
+  return bi::rms::launch(x, ldx, w, y, ldy, M, (int)K, eps, as_stream(stream)) == cudaSuccess ? BI_OK
+                                                                                              : BI_ERR_CUDA;
+}
+
+bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw, bi_bf16* C, int64_t ldc,
+                    int64_t M, int64_t N, int64_t K, void* stream) {
+  if (!A || !W || !C) return BI_ERR_NULL;
+  if (M < 0 || N < 0 || K < 64 || K % 64 != 0 || N % 8 != 0 || M > INT_MAX || N > INT_MAX || K > INT_MAX)
+    return BI_ERR_SHAPE;
+  if (lda < K || ldw < K || ldc < N) return BI_ERR_SHAPE;
+  if (!aligned16(A) || !aligned16(W) || !aligned16(C) || lda % 8 || ldw % 8 || ldc % 8) return BI_ERR_ALIGN;
+  if (M == 0 || N == 0) return BI_OK;
+  const size_t cb = span_bytes(M, N, ldc, 2);
+  if (ranges_overlap(C, cb, A, span_bytes(M, K, lda, 2)) || ranges_overlap(C, cb, W, span_bytes(N, K, ldw, 2)))
+    return BI_ERR_SHAPE;
+  return bi::gemm::launch(A, lda, W, ldw, C, ldc, M, N, K, as_stream(stream));
+}
+
+size_t bi_attention_workspace_size(int64_t rows, int Hq, int D, int max_pages_per_seq) {
+  return attn_ws_size(rows, Hq, D, max_pages_per_seq, nullptr, nullptr);
+}
+
+bi_status bi_attention_decode(const bi_bf16* q, const bi_bf16* k_cache, const bi_bf16* v_cache, int64_t num_pages,
+                              const int32_t* page_table, int max_pages_per_seq, const int32_t* seq_lens,
+                              bi_bf16* out, int B, int Hq, int Hkv, int D, float scale, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out) return BI_ERR_NULL;
+  if (B < 0) return BI_ERR_SHAPE;
+  if (!workspace) return B == 0 ? BI_OK : BI_ERR_WORKSPACE;
+  bi::attn::Rows R{seq_lens, nullptr, nullptr, B, max_pages_per_seq};
+  return attention_common(q, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, B, out, Hq, Hkv, D,
+                          scale, workspace, workspace_bytes, as_stream(stream));
+}
+
+bi_status bi_attention_prefill(const bi_bf16* q, const int32_t* q_seq, const int32_t* q_pos,
+                               const bi_bf16* k_cache, const bi_bf16* v_cache, int64_t num_pages,
+                               const int32_t* page_table, int num_seqs, int max_pages_per_seq, bi_bf16* out,
+                               int T, int Hq, int Hkv, int D, float scale, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (!q || !q_seq || !q_pos || !k_cache || !v_cache || !page_table || !out) return BI_ERR_NULL;
+  if (T < 0 || num_seqs <= 0) return BI_ERR_SHAPE;
+  if (!workspace) return T == 0 ? BI_OK : BI_ERR_WORKSPACE;
+  bi::attn::Rows R{nullptr, q_seq, q_pos, num_seqs, max_pages_per_seq};
+  return attention_common(q, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, T, out, Hq, Hkv, D,
+                          scale, workspace, workspace_bytes, as_stream(stream));
+}
+
+bi_status bi_kv_append(const bi_bf16* k_new, const bi_bf16* v_new, const int32_t* q_seq, const int32_t* q_pos,
+                       bi_bf16* k_cache, bi_bf16* v_cache, int64_t num_pages, const int32_t* page_table,
+                       int num_seqs, int max_pages_per_seq, int T, int Hkv, int D, void* stream) {
+  if (!k_new || !v_new || !q_seq || !q_pos || !k_cache || !v_cache || !page_table) return BI_ERR_NULL;
+  if (T < 0 || num_seqs <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || Hkv <= 0 || D <= 0)
+    return BI_ERR_SHAPE;
+  if (D % 8 != 0) return BI_ERR_UNSUPPORTED;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache)) return BI_ERR_ALIGN;
+  if (T == 0) return BI_OK;
+  const int64_t warps = (int64_t)T * Hkv;
+  if ((warps + 7) / 8 > INT_MAX) return BI_ERR_SHAPE;
+  bi::attn::kv_append_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, as_stream(stream)>>>(
+      k_new, v_new, q_seq, q_pos, k_cache, v_cache, num_pages, page_table, num_seqs, max_pages_per_seq, T, Hkv, D);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+size_t bi_lmhead_workspace_size(int64_t M, int64_t V) { return lm_ws_size(M, V, nullptr, nullptr); }
+
+bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int64_t M, int64_t V, int64_t K,
+                           float margin_threshold, int32_t* tokens, int32_t* recomputed, float* logits_fp32,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!h || !W || !tokens || !recomputed) return BI_ERR_NULL;
+  if (M < 0 || V < 8 || V % 8 != 0 || K < 64 || K % 64 != 0 || ldh < K || M > INT_MAX || V > INT_MAX ||
+      std::isnan(margin_threshold))
+    return BI_ERR_SHAPE;
+  if (!aligned16(h) || !aligned16(W) || ldh % 8 || (logits_fp32 && !aligned16(logits_fp32))) return BI_ERR_ALIGN;
+  if (M == 0) return BI_OK;
+  if (!workspace) return BI_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BI_ERR_ALIGN;
+  if ((M + 31) / 32 > 65535) return BI_ERR_UNSUPPORTED;
+  LmWs lay{};
+  if (workspace_bytes < lm_ws_size(M, V, &lay, workspace)) return BI_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  bi_status s = bi::gemm::launch(h, ldh, W, K, lay.logits16, V, M, V, K, st);
+  if (s != BI_OK) return s;
+  bi::lmhead::top2_kernel<<<(unsigned)M, bi::lmhead::kThreads, 0, st>>>(lay.logits16, V, margin_threshold, tokens,
+                                                                      recomputed);
+  bi::lmhead::compact_kernel<<<1, 1024, 0, st>>>(recomputed, (int)M, lay.list);
+  float* out32 = logits_fp32 ? logits_fp32 : lay.logits32;
+  const dim3 rgrid((unsigned)((V + bi::lmhead::VB - 1) / bi::lmhead::VB), (unsigned)((M + bi::lmhead::RB - 1) / bi::lmhead::RB));
+  bi::lmhead::recompute_kernel<<<rgrid, 256, 0, st>>>(h, ldh, W, V, (int)K, (int)M, lay.list, out32);
+  bi::lmhead::argmax_kernel<<<(unsigned)M, bi::lmhead::kThreads, 0, st>>>(out32, V, recomputed, tokens);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_get_device_error(int32_t* code) {
+  if (!code) return BI_ERR_NULL;
+  if (cudaDeviceSynchronize() != cudaSuccess) return BI_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bi::g_error_word, sizeof(int)) != cudaSuccess) return BI_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(bi::g_error_word, &zero, sizeof(int)) != cudaSuccess) return BI_ERR_CUDA;
+  *code = v;
+  return BI_OK;
+}
+
+}  // extern "C"

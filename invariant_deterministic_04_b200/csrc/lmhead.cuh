@@ -1,0 +1,232 @@
+// Greedy LM head with a selective FP32 recompute.
+//
+// Source: "Greedy Decoding Is Not Precision-Invariant: Cross-Precision Output
+// Divergence in LLM Inference" (arXiv 2609.26621), abstract: whether greedy
+// decoding flips depends mainly on the top-2 logit margin at the LM head; the best
+// low-overhead fix recomputes the LM head in FP32 only when that margin is below a
+// threshold.
+//
+// Pipeline (all on the caller's stream, no host round trip):
+//   1. bf16 logits = bi_matmul(h, W)                         (tensor cores)
+//   2. top2_kernel: per row, top-2 of the bf16 logits (value desc, index asc; NaN
+//      never wins), margin = top1 - top2 in fp32, flag = margin < threshold;
+//      token = top-1 index.
+//   3. compact_kernel: ascending list of flagged rows.
+//   4. recompute_kernel: fp32 logits of the flagged rows from bf16 operands
+//      widened to fp32, each logit one FMA chain over k = 0..K-1 (CUDA cores).
+//   5. argmax_kernel: token of each flagged row = argmax of its fp32 logits.
+// The top-2 and argmax merges are order-independent (a strict total order), and
+// each fp32 logit depends only on its own row, so every row is batch-invariant.
+#pragma once
+
+#include "device.cuh"
+
+namespace bi {
+namespace lmhead {
+
+struct Top2 {
+  float v1;
+  int i1;
+  float v2;
+  int i2;
+};
+
+__device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
+  return a > b || (a == b && ia < ib);
+}
+
+__device__ __forceinline__ void insert(Top2& t, float v, int i) {
+  if (better(v, i, t.v1, t.i1)) {
+    t.v2 = t.v1;
+    t.i2 = t.i1;
+    t.v1 = v;
+    t.i1 = i;
+  } else if (better(v, i, t.v2, t.i2)) {
+    t.v2 = v;
+    t.i2 = i;
+  }
+}
+
+__device__ __forceinline__ float sanitize(float v) { return v != v ? -INFINITY : v; }
+
+constexpr int kThreads = 256;
+
+__global__ void __launch_bounds__(kThreads) top2_kernel(const uint16_t* __restrict__ logits, int64_t V,
+                                                        float threshold, int32_t* __restrict__ tokens,
+                                                        int32_t* __restrict__ flags) {
+  __shared__ Top2 warp_best[kThreads / 32];
+  const int64_t row = blockIdx.x;
+  const uint4* src = reinterpret_cast<const uint4*>(logits + row * V);
+  Top2 t{-INFINITY, 0x7FFFFFFF, -INFINITY, 0x7FFFFFFF};
+  const int64_t nvec = V / 8;
+  for (int64_t j = threadIdx.x; j < nvec; j += kThreads) {
+    float f[8];
+    unpack8(__ldg(src + j), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) insert(t, sanitize(f[e]), (int)(j * 8 + e));
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const float a1 = __shfl_xor_sync(kFullMask, t.v1, o), a2 = __shfl_xor_sync(kFullMask, t.v2, o);
+    const int j1 = __shfl_xor_sync(kFullMask, t.i1, o), j2 = __shfl_xor_sync(kFullMask, t.i2, o);
+    insert(t, a1, j1);
+    insert(t, a2, j2);
+  }
+  if ((threadIdx.x & 31) == 0) warp_best[threadIdx.x >> 5] = t;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Top2 b = warp_best[0];
+    for (int w = 1; w < kThreads / 32; ++w) {
+      insert(b, warp_best[w].v1, warp_best[w].i1);
+      insert(b, warp_best[w].v2, warp_best[w].i2);
+    }
+    const float margin = __fsub_rn(b.v1, b.v2);  // +inf when V == 1
+    tokens[row] = b.i1;
+    flags[row] = (margin < threshold) ? 1 : 0;
+  }
+}
+
+// list[0..count) = indices of flagged rows, ascending; list[M] = count.
+__global__ void __launch_bounds__(1024) compact_kernel(const int32_t* __restrict__ flags, int M,
+                                                       int32_t* __restrict__ list) {
+  __shared__ int32_t sums[1024];
+  const int tid = threadIdx.x;
+  const int per = (M + 1023) / 1024;
+  const int r0 = tid * per, r1 = min(r0 + per, M);
+  int local = 0;
+  for (int r = r0; r < r1; ++r) local += flags[r] != 0;
+  sums[tid] = local;
+  __syncthreads();
+  for (int d = 1; d < 1024; d <<= 1) {
+    const int v = tid >= d ? sums[tid - d] : 0;
+    __syncthreads();
+    sums[tid] += v;
+    __syncthreads();
+  }
+  int run = sums[tid] - local;
+  for (int r = r0; r < r1; ++r)
+    if (flags[r]) list[run++] = r;
+  if (tid == 1023) list[M] = sums[1023];
+}
+
+// fp32 logits of flagged rows: out[row, v] = sum_k h[row, k] * W[v, k], one FMA
+// chain in ascending k per logit. Tile: 32 flagged rows x 128 vocabulary rows,
+// k staged 32 at a time through shared memory; each thread owns 4 x 4 outputs.
+constexpr int RB = 32, VB = 128, KB = 32;
+
+__global__ void __launch_bounds__(256) recompute_kernel(const uint16_t* __restrict__ h, int64_t ldh,
+                                                        const uint16_t* __restrict__ W, int64_t V, int K, int M,
+                                                        const int32_t* __restrict__ list,
+                                                        float* __restrict__ out) {
+  __shared__ __align__(16) float hs[KB][RB];
+  __shared__ __align__(16) float ws[KB][VB];
+  const int count = list[M];
+  const int f0 = blockIdx.y * RB;
+  if (f0 >= count) return;
+  const int64_t v0 = (int64_t)blockIdx.x * VB;
+  const int tid = threadIdx.x;
+  const int tx = tid & 31, ty = tid >> 5;  // vocab 4*tx.., rows 4*ty..
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = 0; k0 < K; k0 += KB) {
+    // h tile: 32 rows x 32 k (bf16 -> fp32), transposed to [k][row]
+    for (int e = tid; e < RB * KB; e += 256) {
+      const int rr = e / KB, kk = e % KB;
+      const int f = f0 + rr;
+      float val = 0.f;
+      if (f < count) {
+        const uint16_t b = h[(int64_t)list[f] * ldh + k0 + kk];
+        val = __uint_as_float((uint32_t)b << 16);
+      }
+      hs[kk][rr] = val;
+    }
+    // W tile: 128 vocab x 32 k, transposed to [k][vocab]
+    for (int e = tid; e < VB * (KB / 8); e += 256) {
+      const int vv = e / (KB / 8), kq = e % (KB / 8);
+      float f[8];
+      if (v0 + vv < V) {
+        unpack8(__ldg(reinterpret_cast<const uint4*>(W + (v0 + vv) * K + k0) + kq), f);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ws[kq * 8 + i][vv] = f[i];
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < KB; ++kk) {
+      const float4 hv = *reinterpret_cast<const float4*>(&hs[kk][ty * 4]);
+      const float4 wv = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+      const float hr[4] = {hv.x, hv.y, hv.z, hv.w};
+      const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(hr[i], wr[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int f = f0 + ty * 4 + i;
+    if (f >= count) continue;
+    float* dst = out + (int64_t)list[f] * V;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t v = v0 + tx * 4 + j;
+      if (v < V) dst[v] = acc[i][j];
+    }
+  }
+}
+
+// Token of each flagged row = argmax of its fp32 logits (lowest index on ties).
+__global__ void __launch_bounds__(kThreads) argmax_kernel(const float* __restrict__ logits, int64_t V,
+                                                          const int32_t* __restrict__ flags,
+                                                          int32_t* __restrict__ tokens) {
+  __shared__ float wv[kThreads / 32];
+  __shared__ int wi[kThreads / 32];
+  const int64_t row = blockIdx.x;
+  if (!flags[row]) return;
+  const float* src = logits + row * V;
+  float best = -INFINITY;
+  int bi_ = 0x7FFFFFFF;
+  for (int64_t j = threadIdx.x; j < V; j += kThreads) {
+    const float v = sanitize(src[j]);
+    if (better(v, (int)j, best, bi_)) {
+      best = v;
+      bi_ = (int)j;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const float v = __shfl_xor_sync(kFullMask, best, o);
+    const int i = __shfl_xor_sync(kFullMask, bi_, o);
+    if (better(v, i, best, bi_)) {
+      best = v;
+      bi_ = i;
+    }
+  }
+  if ((threadIdx.x & 31) == 0) {
+    wv[threadIdx.x >> 5] = best;
+    wi[threadIdx.x >> 5] = bi_;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = wv[0];
+    int bi2 = wi[0];
+    for (int w = 1; w < kThreads / 32; ++w)
+      if (better(wv[w], wi[w], b, bi2)) {
+        b = wv[w];
+        bi2 = wi[w];
+      }
+    tokens[row] = bi2;
+  }
+}
+
+}  // namespace lmhead
+}  // namespace bi

@@ -158,3 +158,53 @@ def lmhead_inputs(M: int, V: int, K: int, seed: int = 0):
 
 def permutation(n: int, seed: int) -> torch.Tensor:
     return torch.randperm(n, generator=generator(seed))
+
+
+# ---------------------------------------------------------------------------
+# Full-size paged stores, generated on the GPU from a seed (the CPU generator
+# would take minutes for tens of GB). Same recipe as paged_kv.
+
+
+def _device_normal_bf16(shape, gen, device, chunk_elems=1 << 28):
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    flat = out.view(-1)
+    for s in range(0, flat.numel(), chunk_elems):
+        e = min(flat.numel(), s + chunk_elems)
+        flat[s:e] = torch.randn(e - s, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+    return out
+
+
+def paged_kv_device(seq_lens, Hkv: int, D: int, seed: int, max_pages: int, device, spare_pages: int = 1) -> PagedKV:
+    lens = [int(v) for v in (seq_lens.tolist() if torch.is_tensor(seq_lens) else seq_lens)]
+    B = len(lens)
+    npages_seq = [math.ceil(L / PAGE) for L in lens]
+    total = sum(npages_seq) + spare_pages
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    k = _device_normal_bf16((total, Hkv, PAGE, D), gen, device)
+    v = _device_normal_bf16((total, Hkv, PAGE, D), gen, device)
+    perm = torch.randperm(total, generator=generator(seed + 2)).to(torch.int32)
+    pt = torch.full((B, max_pages), -1, dtype=torch.int32)
+    pos = 0
+    for b, n in enumerate(npages_seq):
+        pt[b, :n] = perm[pos:pos + n]
+        pos += n
+    # stale data past each sequence's length and in the spare pages
+    nan = float("nan")
+    tails = [(int(pt[b, (L - 1) // PAGE]), L % PAGE) for b, L in enumerate(lens) if L % PAGE]
+    for p, s in tails:
+        k[p, :, s:, :] = nan
+        v[p, :, s:, :] = nan
+    for p in perm[pos:].tolist():
+        k[p] = nan
+        v[p] = nan
+    return PagedKV(k, v, pt.to(device), torch.tensor(lens, dtype=torch.int32, device=device), max_pages)
+
+
+def sequence_pages(kv: PagedKV, b: int, L: int):
+    """CPU copy of one sequence's pages as a private store (pages renumbered 0..n-1)."""
+    n = math.ceil(L / PAGE)
+    pages = kv.page_table[b, :n].to(torch.int64)
+    k = kv.k_cache[pages].cpu()
+    v = kv.v_cache[pages].cpu()
+    return k, v, torch.arange(n, dtype=torch.int32).view(1, n)

@@ -1,0 +1,147 @@
+"""C-ABI checks that need no GPU: the library builds for sm_100a, loads, exports
+every entry point include/bi.h declares, and rejects bad arguments on the host
+(returning the right status and launching nothing)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import invariant_deterministic_04_b200 as bi
+from invariant_deterministic_04_b200._build import build_library
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bi.h")
+
+OK, NULL, SHAPE, ALIGN, WS, UNSUP = 0, 1, 2, 3, 4, 5
+P = 0x10000  # 16-byte aligned stand-in address; host validation never dereferences it
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_library()
+    return bi.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bi_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_hot_path():
+    names = declared_functions()
+    for n in ("bi_rmsnorm", "bi_matmul", "bi_attention_decode", "bi_attention_prefill", "bi_lmhead_argmax",
+              "bi_attention_workspace_size", "bi_lmhead_workspace_size", "bi_get_device_error", "bi_kv_append"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    assert L.bi_status_string(0) == b"BI_OK"
+    assert L.bi_status_string(4) == b"BI_ERR_WORKSPACE"
+    assert L.bi_status_string(99) == b"BI_ERR_UNKNOWN"
+    assert L.bi_version() == 1
+
+
+def test_rmsnorm_validation(L):
+    f = L.bi_rmsnorm
+    assert f(None, 512, P, P, 512, 4, 512, 1e-6, None) == NULL
+    assert f(P, 512, P, P, 512, -1, 512, 1e-6, None) == SHAPE
+    assert f(P, 512, P, P, 512, 4, 500, 1e-6, None) == SHAPE        # K % 8
+    assert f(P, 256, P, P, 512, 4, 512, 1e-6, None) == SHAPE        # ldx < K
+    assert f(P, 512, P, P, 512, 4, 512, float("nan"), None) == SHAPE
+    assert f(P, 32768, P, P, 32768, 4, 32768, 1e-6, None) == UNSUP
+    assert f(P + 2, 512, P, P, 512, 4, 512, 1e-6, None) == ALIGN
+    assert f(P, 516, P, P, 512, 4, 512, 1e-6, None) == ALIGN        # ld % 8
+    assert f(P, 512, P, P, 512, 0, 512, 1e-6, None) == OK           # empty: no-op
+    # partially overlapping input and output rows are rejected (exact aliasing is allowed)
+    assert f(P, 512, P + 0x100000, P + 16, 512, 4, 512, 1e-6, None) == SHAPE
+
+
+def test_matmul_validation(L):
+    f = L.bi_matmul
+    assert f(P, 512, None, 512, P, 64, 4, 64, 512, None) == NULL
+    assert f(P, 500, P, 500, P, 64, 4, 64, 500, None) == SHAPE      # K % 64
+    assert f(P, 512, P, 512, P, 64, 4, 60, 512, None) == SHAPE      # N % 8
+    assert f(P, 512, P, 512, P, 64, 4, 64, 0, None) == SHAPE        # K == 0
+    assert f(P, 256, P, 512, P, 64, 4, 64, 512, None) == SHAPE      # lda < K
+    assert f(P, 512, P + 8, 512, P, 64, 4, 64, 512, None) == ALIGN
+    assert f(P, 512, P, 516, P, 64, 4, 64, 512, None) == ALIGN      # ldw % 8
+    assert f(P, 512, P, 512, P, 64, 0, 64, 512, None) == OK         # M == 0
+    assert f(P, 512, P, 512, P, 64, 4, 0, 512, None) == OK          # N == 0
+    # output overlapping an operand
+    assert f(P, 512, P + 0x1000000, 512, P + 64, 64, 4, 64, 512, None) == SHAPE
+
+
+def test_attention_workspace_size(L):
+    s = L.bi_attention_workspace_size
+    assert s(0, 32, 128, 2048) > 0
+    a, b = s(4, 32, 128, 2048), s(8, 32, 128, 2048)
+    assert b > a
+    # 128 splits of 256 tokens for 32768 tokens; fp32 o[D] + (m, l) per split and head
+    assert s(1, 32, 128, 2048) >= 128 * 32 * (128 * 4 + 8)
+    assert s(-1, 32, 128, 16) == 0 and s(4, 0, 128, 16) == 0
+
+
+def test_attention_validation(L):
+    d = L.bi_attention_decode
+    ws = L.bi_attention_workspace_size(4, 32, 128, 64)
+    args = lambda **k: [k.get("q", P), P, P, k.get("np", 100), P, k.get("maxp", 64), P, P, k.get("B", 4),
+                        k.get("Hq", 32), k.get("Hkv", 8), k.get("D", 128), k.get("scale", 0.088),
+                        k.get("ws", P), k.get("wsb", ws), None]
+    assert d(*args(q=None)) == NULL
+    assert d(*args(B=-1)) == SHAPE
+    assert d(*args(Hq=30)) == SHAPE                  # Hq % Hkv
+    assert d(*args(D=96)) == UNSUP
+    assert d(*args(Hq=48, Hkv=3)) == UNSUP           # group 16
+    assert d(*args(wsb=ws - 1)) == WS
+    assert d(*args(ws=None)) == WS
+    assert d(*args(q=P + 4)) == ALIGN
+    assert d(*args(np=0)) == SHAPE
+    assert d(*args(scale=float("inf"))) == SHAPE
+    assert d(*args(B=0, ws=None, wsb=0)) == OK
+    p = L.bi_attention_prefill
+    wsp = L.bi_attention_workspace_size(10, 32, 64, 8)
+    assert p(P, None, P, P, P, 100, P, 2, 8, P, 10, 32, 8, 64, 0.125, P, wsp, None) == NULL
+    assert p(P, P, P, P, P, 100, P, 0, 8, P, 10, 32, 8, 64, 0.125, P, wsp, None) == SHAPE
+    assert p(P, P, P, P, P, 100, P, 2, 8, P, 10, 32, 8, 64, 0.125, P, wsp - 256, None) == WS
+    assert p(P, P, P, P, P, 100, P, 2, 8, P, 0, 32, 8, 64, 0.125, None, 0, None) == OK
+
+
+def test_kv_append_validation(L):
+    f = L.bi_kv_append
+    assert f(None, P, P, P, P, P, 10, P, 1, 4, 3, 8, 128, None) == NULL
+    assert f(P, P, P, P, P, P, 10, P, 1, 4, -3, 8, 128, None) == SHAPE
+    assert f(P, P, P, P, P, P, 10, P, 1, 4, 3, 8, 100, None) == UNSUP
+    assert f(P + 8, P, P, P, P, P, 10, P, 1, 4, 3, 8, 128, None) == ALIGN
+    assert f(P, P, P, P, P, P, 10, P, 1, 4, 0, 8, 128, None) == OK
+
+
+def test_lmhead_validation(L):
+    f = L.bi_lmhead_argmax
+    ws = L.bi_lmhead_workspace_size(4, 32000)
+    assert ws >= 4 * 32000 * 6
+    assert f(None, 2048, P, 4, 32000, 2048, 0.5, P, P, None, P, ws, None) == NULL
+    assert f(P, 2048, P, 4, 32004, 2048, 0.5, P, P, None, P, ws, None) == SHAPE   # V % 8
+    assert f(P, 2048, P, 4, 32000, 2000, 0.5, P, P, None, P, ws, None) == SHAPE   # K % 64
+    assert f(P, 2048, P, 4, 32000, 2048, float("nan"), P, P, None, P, ws, None) == SHAPE
+    assert f(P, 2048, P, 4, 32000, 2048, 0.5, P, P, None, P, ws - 1, None) == WS
+    assert f(P, 2048, P, 4, 32000, 2048, 0.5, P, P, None, None, ws, None) == WS
+    assert f(P, 2048, P, 4, 32000, 2048, 0.5, P, P, P + 4, P, ws, None) == ALIGN
+    assert f(P, 2048, P, 0, 32000, 2048, 0.5, P, P, None, None, 0, None) == OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import importlib
+
+    mod = importlib.import_module("invariant_deterministic_04_b200")
+    monkeypatch.setattr(mod, "_lib", None)
+    monkeypatch.setattr(mod, "_load_error", None)
+    monkeypatch.setattr(mod, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        mod.lib()

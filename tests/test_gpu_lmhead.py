@@ -1,0 +1,93 @@
+"""bi_lmhead_argmax on the GPU: greedy tokens, recompute flags and fp32 logits
+against the fp64 oracle; planted margins; bit-invariance across batch size;
+thresholds that force or forbid the recompute; full size M=64, V=32000, K=2048."""
+import numpy as np
+import pytest
+import torch
+
+import invariant_deterministic_04_b200 as bi
+import oracle
+import synth
+from gpu_util import TOL_FP32, dev, same_bits
+
+pytestmark = pytest.mark.gpu
+TAU = 0.5
+
+
+def _check_against_oracle(h, w, tau, tokens, rec, logits):
+    r = oracle.lmhead(synth.to_f64(h), synth.to_f64(w), tau)
+    rec = rec.cpu().numpy().astype(bool)
+    tokens = tokens.cpu().numpy()
+    # the recompute decision: compared where the oracle's bf16 margin is clearly on one side
+    # (a 1-ulp difference in a bf16 logit can move the margin by up to 2 bf16 ulps)
+    top = np.abs(r["logits"]).max(axis=1)
+    band = 2 * 2.0 ** (np.floor(np.log2(np.maximum(top, 1e-30))) - 7)
+    clear = np.abs(r["margin_bf16"] - tau) > band
+    assert (rec[clear] == r["recompute"][clear]).all()
+    # recomputed rows: fp32 logits within 1e-5 normwise, token = exact argmax whenever
+    # the exact top-2 margin exceeds the fp32 error bound
+    if rec.any():
+        lg = logits.cpu().numpy()[rec]
+        err = oracle.normwise_rel_err(lg, r["logits"][rec])
+        assert err.max() <= TOL_FP32, err.max()
+        bound = 4 * TOL_FP32 * top[rec]
+        ok = r["margin"][rec] > bound
+        assert (tokens[rec][ok] == r["tokens"][rec][ok]).all()
+    # first-pass rows: token = argmax of the bf16-rounded logits where those have a clear top-1
+    keep = ~rec & clear
+    assert (tokens[keep] == r["tokens_bf16"][keep]).all()
+    return r, rec
+
+
+@pytest.mark.parametrize("M,V,K", [(9, 1000, 256), (1, 32000, 2048), (64, 32000, 2048), (40, 4096, 512)])
+def test_lmhead_matches_oracle(M, V, K):
+    h, w = synth.lmhead_inputs(M, V, K, seed=M + V)
+    tok, rec, lg = bi.lmhead_argmax(h.to(dev()), w.to(dev()), TAU, want_logits=True)
+    _check_against_oracle(h, w, TAU, tok, rec, lg)
+    # rows that were not recomputed are left untouched in logits_fp32
+    norec = ~rec.cpu().bool()
+    assert torch.isnan(lg.cpu()[norec]).all()
+
+
+def test_lmhead_planted_margins():
+    K, V = 128, 512
+    _, w = synth.lmhead_inputs(1, V, K, seed=70)
+    h = torch.zeros((3, K), dtype=torch.bfloat16)
+    h[0, 0] = h[1, 1] = h[2, 2] = 1.0
+    w[:, :3] = w[:, :3].clamp(-1, 1)
+    w[7, 0], w[30, 0] = 3.0, 2.875      # margin 0.125 -> recompute, token 7
+    w[12, 1], w[40, 1] = 8.0, 3.0       # margin 5 -> first pass, token 12
+    w[5, 2], w[6, 2] = 2.0, 2.0         # exact tie -> margin 0, lowest index wins
+    tok, rec, lg = bi.lmhead_argmax(h.to(dev()), w.to(dev()), TAU, want_logits=True)
+    assert tok.cpu().tolist() == [7, 12, 5]
+    assert rec.cpu().tolist() == [1, 0, 1]
+    assert float(lg[0, 7]) == 3.0 and float(lg[0, 30]) == 2.875
+
+
+def test_lmhead_thresholds_force_or_forbid_recompute():
+    h, w = synth.lmhead_inputs(16, 4096, 512, seed=71)
+    hd, wd = h.to(dev()), w.to(dev())
+    _, rec0, _ = bi.lmhead_argmax(hd, wd, 0.0)
+    assert int(rec0.sum()) == 0
+    tok, rec1, lg = bi.lmhead_argmax(hd, wd, float("inf"), want_logits=True)
+    assert int(rec1.sum()) == 16
+    assert (tok.cpu() == torch.argmax(lg.cpu(), dim=1).to(torch.int32)).all()
+
+
+def test_lmhead_batch_invariant():
+    M, V, K = 64, 32000, 2048
+    h, w = synth.lmhead_inputs(M, V, K, seed=72)
+    hd, wd = h.to(dev()), w.to(dev())
+    tok, rec, lg = bi.lmhead_argmax(hd, wd, TAU, want_logits=True)
+    for r in (0, 13, 63):
+        t1, r1, l1 = bi.lmhead_argmax(hd[r:r + 1].contiguous(), wd, TAU, want_logits=True)
+        assert int(t1[0]) == int(tok[r]) and int(r1[0]) == int(rec[r])
+        if int(r1[0]):
+            assert same_bits(l1[0], lg[r])
+    for m in (1, 2, 7, 33):
+        t2, r2, l2 = bi.lmhead_argmax(hd[:m].contiguous(), wd, TAU, want_logits=True)
+        assert torch.equal(t2, tok[:m]) and torch.equal(r2, rec[:m])
+        mask = r2.bool()
+        assert same_bits(l2[mask], lg[:m][mask])
+    t3, r3, _ = bi.lmhead_argmax(hd, wd, TAU)
+    assert torch.equal(t3, tok) and torch.equal(r3, rec)

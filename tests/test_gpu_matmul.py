@@ -1,0 +1,110 @@
+"""bi_matmul on the GPU (tcgen05 + TMA): parity with the fp64 oracle, exact
+small-integer products (pins the shared-memory layout and descriptors),
+row-position independence inside a 128-row tile, bit-invariance across the M
+sweep at K=4096, N in {4096, 6144, 14336}, run-to-run bit-exactness, and the
+RMSNorm -> matmul chain of the 32 x 512 -> 1024 configuration."""
+import numpy as np
+import pytest
+import torch
+
+import invariant_deterministic_04_b200 as bi
+import oracle
+import synth
+from gpu_util import TOL_BF16, dev, max_rel, same_bits
+
+pytestmark = pytest.mark.gpu
+
+M_SWEEP = [1, 2, 3, 4, 7, 8, 13, 16, 32, 33, 64, 127, 128, 255, 256, 257, 512, 1023, 1024, 2047, 2048]
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 520, 512), (1, 256, 64), (128, 256, 128), (129, 264, 192),
+                                   (32, 1024, 512), (5, 8, 64), (257, 4096, 1024)])
+def test_matmul_matches_oracle(M, N, K):
+    a, w = synth.matmul_inputs(M, N, K, seed=M * 7 + N + K)
+    c = bi.matmul(a.to(dev()), w.to(dev()))
+    assert max_rel(c, oracle.matmul(synth.to_f64(a), synth.to_f64(w))) <= TOL_BF16
+
+
+def test_matmul_small_integers_exact():
+    # entries in {-1, 0, 1}: every product and partial sum is an integer below 2^24
+    # and |C| <= K = 192 fits bf16 exactly, so any layout slip shows as a wrong integer.
+    g = synth.generator(21)
+    M, N, K = 200, 520, 192
+    a = torch.randint(-1, 2, (M, K), generator=g).to(torch.bfloat16)
+    w = torch.randint(-1, 2, (N, K), generator=g).to(torch.bfloat16)
+    c = bi.matmul(a.to(dev()), w.to(dev())).cpu()
+    ref = oracle.matmul(synth.to_f64(a), synth.to_f64(w))
+    np.testing.assert_array_equal(synth.to_f64(c), ref)
+
+
+def test_matmul_one_hot_rows_select_weight_columns():
+    N, K = 512, 256
+    _, w = synth.matmul_inputs(1, N, K, seed=22)
+    ks = [0, 1, 63, 64, 100, 255]
+    a = torch.zeros((len(ks), K), dtype=torch.bfloat16)
+    for m, k in enumerate(ks):
+        a[m, k] = 1.0
+    c = bi.matmul(a.to(dev()), w.to(dev())).cpu()
+    for m, k in enumerate(ks):
+        assert same_bits(c[m], w[:, k].contiguous())
+
+
+def test_matmul_row_position_independent():
+    # Each row computed alone (M = 1, tile row 0) equals the same row computed at
+    # tile row r % 128 of a 300-row batch, bit for bit.
+    M, N, K = 300, 512, 1024
+    a, w = synth.matmul_inputs(M, N, K, seed=23)
+    a, w = a.to(dev()), w.to(dev())
+    full = bi.matmul(a, w)
+    for r in range(M):
+        assert same_bits(bi.matmul(a[r:r + 1].contiguous(), w)[0], full[r]), r
+
+
+@pytest.mark.parametrize("N", [4096, 6144, 14336])
+def test_matmul_batch_invariant_over_m_sweep(N):
+    K = 4096
+    a, w = synth.matmul_inputs(2048, N, K, seed=24)
+    a, w = a.to(dev()), w.to(dev())
+    full = bi.matmul(a, w)
+    for m in M_SWEEP:
+        assert same_bits(bi.matmul(a[:m].contiguous(), w), full[:m]), m
+    # rows in a permuted batch and a batch taken from the middle
+    perm = synth.permutation(2048, 25).to(dev())
+    assert same_bits(bi.matmul(a[perm].contiguous(), w), full[perm])
+    assert same_bits(bi.matmul(a[1000:1037].contiguous(), w), full[1000:1037])
+    # full-size parity on sampled rows
+    rows = [0, 1, 127, 128, 1023, 2047]
+    ref = oracle.matmul(synth.to_f64(a[rows].cpu()), synth.to_f64(w.cpu()))
+    assert max_rel(full[rows], ref) <= TOL_BF16
+
+
+def test_matmul_run_to_run():
+    a, w = synth.matmul_inputs(2048, 6144, 4096, seed=26)
+    a, w = a.to(dev()), w.to(dev())
+    first = bi.matmul(a, w)
+    for _ in range(3):
+        assert same_bits(bi.matmul(a, w), first)
+
+
+def test_matmul_strided_operands_and_output():
+    a, w = synth.matmul_inputs(100, 512, 1024, seed=27)
+    a, w = a.to(dev()), w.to(dev())
+    out = torch.zeros((100, 1024), dtype=torch.bfloat16, device=dev())
+    bi.matmul(a[:, :512], w[:, :512], out=out[:, 256:768])
+    ref = bi.matmul(a[:, :512].contiguous(), w[:, :512].contiguous())
+    assert same_bits(out[:, 256:768], ref)
+    assert int(out[:, :256].abs().sum()) == 0 and int(out[:, 768:].abs().sum()) == 0
+
+
+def test_rmsnorm_matmul_chain_32x512x1024():
+    x, wn = synth.rmsnorm_inputs(32, 512, seed=0)
+    _, W = synth.matmul_inputs(32, 1024, 512, seed=2)
+    xd, wnd, Wd = x.to(dev()), wn.to(dev()), W.to(dev())
+    c = bi.matmul(bi.rmsnorm(xd, wnd, 1e-6), Wd)
+    for m in (1, 2, 7, 16):
+        for start in (0, 32 - m):
+            sub = bi.matmul(bi.rmsnorm(xd[start:start + m].contiguous(), wnd, 1e-6), Wd)
+            assert same_bits(sub, c[start:start + m])
+    # the chain in double, no bf16 intermediate
+    ref = oracle.matmul(oracle.rmsnorm(synth.to_f64(x), synth.to_f64(wn), 1e-6), synth.to_f64(W))
+    assert max_rel(c, ref) <= TOL_BF16
