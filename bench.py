@@ -276,9 +276,23 @@ def _events_ms(fn, iters=10, warmup=3):
     return s.elapsed_time(e) / iters
 
 
-def other_rows(bi, device, pk):
+def other_rows(bi, device, pk, only=None):
     out = {}
+    want = (lambda name: only is None or only == name)
     # RMSNorm bandwidth at a size far above L2 (M = 65536, K = 4096: 1 GiB in + out)
+    if want("rmsnorm"):
+        out.update(_row_rmsnorm(bi, device, pk))
+    if want("decode"):
+        out.update(_row_decode(bi, device, pk))
+    if want("prefill"):
+        out.update(_row_prefill(bi, device, pk))
+    if want("lmhead"):
+        out.update(_row_lmhead(bi, device, pk))
+    return out
+
+
+def _row_rmsnorm(bi, device, pk):
+    out = {}
     M = 65536
     x = torch.randn((M, K_HIDDEN), device=device, dtype=torch.float32).to(torch.bfloat16)
     w = synth.normal_bf16((K_HIDDEN,), 110, std=0.1, mean=1.0).to(device)
@@ -288,8 +302,11 @@ def other_rows(bi, device, pk):
     gbs = (4.0 * M * K_HIDDEN + 2 * K_HIDDEN) / ms / 1e6
     out["rmsnorm_m65536_k4096"] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3), "ms": round(ms, 4),
                                    "slowdown_vs_F.rms_norm": round(ms / ms_ref, 3)}
-    del x, y
+    return out
 
+
+def _row_decode(bi, device, pk):
+    out = {}
     # decode attention: B=64 sequences, lengths ~ U[1, 32768], GQA 32/8, D=128
     B, Lmax = 64, 32768
     lens = synth.decode_lengths(B, Lmax, seed=50)
@@ -303,8 +320,11 @@ def other_rows(bi, device, pk):
     gbs = kv_bytes / ms / 1e6
     out["decode_b64_l32k"] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3), "ms": round(ms, 4),
                               "kv_bytes": kv_bytes}
-    del kv, ws
+    return out
 
+
+def _row_prefill(bi, device, pk):
+    out = {}
     # causal prefill, one sequence of 4096 tokens
     S = 4096
     kvp = synth.paged_kv_device([S], 8, 128, seed=60, max_pages=S // 16, device=device)
@@ -319,8 +339,11 @@ def other_rows(bi, device, pk):
     alu_peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
     out["prefill_s4096"] = {"TFLOP/s": round(flops / ms / 1e9, 2), "frac_fp32_alu": round(flops / ms / 1e9 / alu_peak, 3),
                             "ms": round(ms, 3)}
-    del kvp, wsp
+    return out
 
+
+def _row_lmhead(bi, device, pk):
+    out = {}
     # LM head: 64 rows, vocabulary 32000, hidden 2048
     h = synth.normal_bf16((64, 2048), 70).to(device)
     Wl = synth.normal_bf16((32000, 2048), 71, std=0.02).to(device)
@@ -468,13 +491,20 @@ def main():
     ap.add_argument("--rows", dest="rows", action="store_true", default=True)
     ap.add_argument("--no-rows", dest="rows", action="store_false")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--row", choices=["rmsnorm", "decode", "prefill", "lmhead"], default=None,
+                    help="measure only this hot-path kernel (for profiling) and print its line")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     rank, world, local = init_dist()
     try:
-        if args.impl == "reference":
+        if args.row is not None:
+            import invariant_deterministic_04_b200 as bi
+
+            torch.cuda.set_device(local)
+            print(json.dumps({"row": args.row, **other_rows(bi, torch.device("cuda", local), peaks(), only=args.row)}))
+        elif args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_ours(args, rank, world, local)
