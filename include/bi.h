@@ -130,6 +130,35 @@ bi_status bi_attention_decode(const bi_bf16* q, const bi_bf16* k_cache, const bi
                               float scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Decode attention for callers that cannot allocate device memory. The pages have
+ * no counterpart for this call; it exists for code that may not call cudaMalloc or
+ * hold an allocator: for example a plugin or callback running inside another
+ * framework that owns every byte of device memory and forbids allocation there, or a
+ * latency-critical path where cudaMalloc's implicit device-wide synchronisation is
+ * not allowed.
+ * Same arguments, result and schedule as bi_attention_decode (bit-identical
+ * output), minus the workspace: the scratch is a fixed array of
+ * BI_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits. A request whose workspace size
+ * (bi_attention_workspace_size(B, Hq, D, max_pages_per_seq)) exceeds it returns
+ * BI_ERR_WORKSPACE and launches nothing.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - All calls share the one array and it keeps the previous call's contents.
+ *     Nothing in it needs to start at zero: every byte a call reads was written
+ *     earlier in the same call. Calls that overlap on the GPU (different streams,
+ *     or different host threads on the same device) race on the array and must be
+ *     serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define BI_STATIC_SCRATCH_BYTES ((size_t)32 << 20) /* 32 MiB */
+bi_status bi_attention_decode_static(const bi_bf16* q, const bi_bf16* k_cache, const bi_bf16* v_cache,
+                                     int64_t num_pages, const int32_t* page_table, int max_pages_per_seq,
+                                     const int32_t* seq_lens, bi_bf16* out, int B, int Hq, int Hkv, int D,
+                                     float scale, void* stream);
+
+/*
  * Causal prefill attention over the same store (chunked or whole). Source: same
  * table, row Attention (chunked prefill / prefix caching must not change the
  * path), and the usage article's test list (prefill, decode, cache on or off).

@@ -43,6 +43,7 @@ _SIGNATURES = {
     "bi_matmul": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _P], _I32),
     "bi_attention_workspace_size": ([_I64, _I32, _I32, _I32], _SZ),
     "bi_attention_decode": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ, _P], _I32),
+    "bi_attention_decode_static": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P], _I32),
     "bi_attention_prefill": ([_P, _P, _P, _P, _P, _I64, _P, _I32, _I32, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ, _P],
                              _I32),
     "bi_kv_append": ([_P, _P, _P, _P, _P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P], _I32),
@@ -171,6 +172,36 @@ def attention_decode(q, k_cache, v_cache, page_table, seq_lens, scale: float | N
     _check("bi_attention_decode", lib().bi_attention_decode(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), maxp, _ptr(seq_lens), _ptr(out),
         B, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def attention_decode_static(q, k_cache, v_cache, page_table, seq_lens, scale: float | None = None, out=None,
+                            stream=None):
+    """Decode attention that allocates nothing: its scratch is a fixed 32 MiB array inside
+    libbi (for callers that cannot allocate device memory). Same result as attention_decode.
+    Calls that overlap on the GPU share that array and must be serialised by the caller."""
+    _req(q, torch.bfloat16, "q", 3)
+    _req(k_cache, torch.bfloat16, "k_cache", 4)
+    _req(v_cache, torch.bfloat16, "v_cache", 4)
+    _req(page_table, torch.int32, "page_table", 2)
+    _req(seq_lens, torch.int32, "seq_lens", 1)
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (page_table, "page_table"),
+                 (seq_lens, "seq_lens")):
+        _contig(t, n)
+    B, Hq, D = q.shape
+    num_pages, Hkv = k_cache.shape[0], k_cache.shape[1]
+    if k_cache.shape != v_cache.shape or k_cache.shape[2] != PAGE_TOKENS or k_cache.shape[3] != D:
+        raise ValueError("k_cache/v_cache must be [num_pages, Hkv, 16, D]")
+    if page_table.shape[0] < B or seq_lens.shape[0] < B:
+        raise ValueError("page_table and seq_lens need a row per sequence")
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out = torch.empty_like(q) if out is None else out
+    _check("bi_attention_decode_static", lib().bi_attention_decode_static(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), page_table.shape[1], _ptr(seq_lens),
+        _ptr(out), B, Hq, Hkv, D, scale, _stream(stream)))
     return out
 
 

@@ -145,6 +145,35 @@ size_t lm_ws_size(int64_t M, int64_t V, LmWs* lay, void* base) {
 
 }  // namespace
 
+// Scratch of bi_attention_decode_static: a fixed array instead of a caller
+// workspace, for callers that cannot allocate device memory. Every GPU that loads
+// the library holds it until the process exits. Host code may not pass the
+// symbol itself to a kernel (on the host it names a stand-in, not device memory):
+// its device address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_decode_scratch[BI_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {};
+
+// Device address of g_decode_scratch on the current device (looked up on first use).
+bi_status decode_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return BI_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return BI_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return BI_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* bi_status_string(int status) {
@@ -205,6 +234,22 @@ bi_status bi_attention_decode(const bi_bf16* q, const bi_bf16* k_cache, const bi
   bi::attn::Rows R{seq_lens, nullptr, nullptr, B, max_pages_per_seq};
   return attention_common(q, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, B, out, Hq, Hkv, D,
                           scale, workspace, workspace_bytes, as_stream(stream));
+}
+
+bi_status bi_attention_decode_static(const bi_bf16* q, const bi_bf16* k_cache, const bi_bf16* v_cache,
+                                     int64_t num_pages, const int32_t* page_table, int max_pages_per_seq,
+                                     const int32_t* seq_lens, bi_bf16* out, int B, int Hq, int Hkv, int D,
+                                     float scale, void* stream) {
+  if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out) return BI_ERR_NULL;
+  if (B < 0) return BI_ERR_SHAPE;
+  if (B == 0) return BI_OK;
+  if (attn_ws_size(B, Hq, D, max_pages_per_seq, nullptr, nullptr) > BI_STATIC_SCRATCH_BYTES) return BI_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const bi_status s = decode_scratch_address(&scratch);
+  if (s != BI_OK) return s;
+  bi::attn::Rows R{seq_lens, nullptr, nullptr, B, max_pages_per_seq};
+  return attention_common(q, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, B, out, Hq, Hkv, D,
+                          scale, scratch, BI_STATIC_SCRATCH_BYTES, as_stream(stream));
 }
 
 bi_status bi_attention_prefill(const bi_bf16* q, const int32_t* q_seq, const int32_t* q_pos,
