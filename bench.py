@@ -203,18 +203,22 @@ def time_loop(fn, steps: int, warmup: int, world: int):
 
 
 def traffic_from_profile():
-    """Per-launch DRAM bytes of the matmul kernel from the committed ncu summary,
-    or None if the kernel source changed since it was captured."""
-    path = os.path.join(ROOT, "profiles", "gemm_bf16_kernel_traffic.json")
+    """Per-launch DRAM bytes of the N=14336 matmul launch from the committed ncu
+    summary, or None if gemm.cuh changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "gemm_bf16_kernel_traffic.txt")
     src = os.path.join(ROOT, "invariant_deterministic_04_b200", "csrc", "gemm.cuh")
     try:
+        rec = {}
         with open(path) as f:
-            p = json.load(f)
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    rec[k.strip()] = v.strip()
         with open(src, "rb") as f:
             h = hashlib.sha256(f.read()).hexdigest()
-        if p.get("gemm_cuh_sha256") != h:
+        if rec.get("gemm_cuh_sha256") != h:
             return None
-        return p
+        return int(rec["dram_bytes_per_launch"])
     except Exception:
         return None
 
@@ -443,17 +447,22 @@ def run_ours(args, rank, world, local):
 
     if rank != 0:
         return
+    # roofline of the dominant kernel: the tcgen05 matmul, on its N=14336 launch
+    # (the largest of the step; the one the committed ncu capture covers)
+    big = len(NS)  # kernel index of the N=14336 launch
+    big_flops = 2.0 * wl.M * K_HIDDEN * NS[-1]
+    big_ms = kernel_ms[big] / args.steps
+    achieved = big_flops / (big_ms / 1e3) / 1e12
     gemm_ms = sum(kernel_ms[1:])
-    gemm_flops = 2.0 * wl.M * K_HIDDEN * sum(NS) * args.steps
-    achieved = gemm_flops / (gemm_ms / 1e3) / 1e12
-    prof = traffic_from_profile()
-    traffic = None
-    if prof:
-        traffic = prof.get("dram_bytes_per_launch")
-    roof = {"bound": "tensor", "kernel": "gemm_bf16_kernel (tcgen05)", "achieved": round(achieved, 1),
-            "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops_sustained"], 3),
-            "peak_kind": f"bf16 sustained ({pk['source']})", "frac_of_burst": round(achieved / pk["bf16_tflops"], 3),
-            "traffic": traffic, "kernel_share": round(gemm_ms / sum(kernel_ms), 3)}
+    step_gemm_tflops = 2.0 * wl.M * K_HIDDEN * sum(NS) * args.steps / (gemm_ms / 1e3) / 1e12
+    roof = {"bound": "tensor", "kernel": "gemm_bf16_kernel (tcgen05), M=2048 N=14336 K=4096 launch",
+            "achieved": round(achieved, 1), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+            "frac": round(achieved / pk["bf16_tflops_sustained"], 3),
+            "peak_kind": f"bf16 sustained ({pk['source']}); the step runs back to back for the whole timed region",
+            "frac_of_burst": round(achieved / pk["bf16_tflops"], 3), "traffic": traffic_from_profile(),
+            "algorithmic_bytes_per_launch": 2 * (wl.M * K_HIDDEN + NS[-1] * K_HIDDEN + wl.M * NS[-1]),
+            "launch_ms": round(big_ms, 4), "all_matmul_launches_tflops": round(step_gemm_tflops, 1),
+            "kernel_share": round(gemm_ms / sum(kernel_ms), 3)}
     rms_ms = kernel_ms[0] / args.steps
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
