@@ -362,6 +362,60 @@ def _row_lmhead(bi, device, pk):
 
 
 # ---------------------------------------------------------------------------
+# the K=4096 sweep (one JSON line per (M, N)): bi_matmul vs cuBLAS, W warm and W cold
+
+
+M_SWEEP = [1, 2, 3, 4, 7, 8, 13, 16, 32, 33, 64, 127, 128, 255, 256, 257, 512, 1023, 1024, 2047, 2048]
+
+
+def run_sweep(bi, device, pk, iters=20):
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)  # > L2 (126 MB)
+    A = synth.normal_bf16((2048, K_HIDDEN), 100).to(device)
+    wn = synth.normal_bf16((K_HIDDEN,), 110, std=0.1, mean=1.0).to(device)
+
+    def timed(fn, cold):
+        ts = []
+        for i in range(iters + 3):
+            if cold:
+                flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(s.elapsed_time(e))
+        return statistics.median(ts)
+
+    for j, n in enumerate(NS):
+        W = synth.normal_bf16((n, K_HIDDEN), 120 + j, std=0.02).to(device)
+        C = torch.empty((2048, n), dtype=torch.bfloat16, device=device)
+        for m in M_SWEEP:
+            a, c = A[:m], C[:m]
+            flops = 2.0 * m * n * K_HIDDEN
+            byts = 2.0 * (m * K_HIDDEN + n * K_HIDDEN + m * n)
+            rec = {"sweep": "matmul", "M": m, "N": n, "K": K_HIDDEN}
+            for cold in (False, True):
+                ms = timed(lambda: bi.matmul(a, W, out=c), cold)
+                ref = timed(lambda: torch.matmul(a, W.t(), out=c), cold)
+                roof_ms = max(flops / pk["bf16_tflops"] / 1e9, byts / pk["hbm_gbs"] / 1e6)
+                key = "cold" if cold else "warm"
+                rec[key] = {"ms": round(ms, 5), "TFLOP/s": round(flops / ms / 1e9, 1),
+                            "frac_tensor_peak": round(flops / ms / 1e9 / pk["bf16_tflops"], 3),
+                            "frac_roofline": round(roof_ms / ms, 3), "cublas_ms": round(ref, 5),
+                            "slowdown_vs_cublas": round(ms / ref, 3)}
+            print(json.dumps(rec), flush=True)
+    for m in M_SWEEP:
+        x = A[:m]
+        y = torch.empty_like(x)
+        ms = timed(lambda: bi.rmsnorm(x, wn, EPS, out=y), True)
+        ref = timed(lambda: torch.nn.functional.rms_norm(x, (K_HIDDEN,), wn, EPS), True)
+        byts = 4.0 * m * K_HIDDEN + 2 * K_HIDDEN
+        print(json.dumps({"sweep": "rmsnorm", "M": m, "K": K_HIDDEN, "ms": round(ms, 5),
+                          "GB/s": round(byts / ms / 1e6, 1), "slowdown_vs_F.rms_norm": round(ms / ref, 3)}), flush=True)
+
+
+# ---------------------------------------------------------------------------
 
 
 def run_reference(args, rank, world):
@@ -500,6 +554,7 @@ def main():
     ap.add_argument("--rows", dest="rows", action="store_true", default=True)
     ap.add_argument("--no-rows", dest="rows", action="store_false")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="the K=4096 M sweep, one JSON line per shape")
     ap.add_argument("--row", choices=["rmsnorm", "decode", "prefill", "lmhead"], default=None,
                     help="measure only this hot-path kernel (for profiling) and print its line")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
@@ -508,7 +563,12 @@ def main():
         args.warmup = 3
     rank, world, local = init_dist()
     try:
-        if args.row is not None:
+        if args.sweep:
+            import invariant_deterministic_04_b200 as bi
+
+            torch.cuda.set_device(local)
+            run_sweep(bi, torch.device("cuda", local), peaks())
+        elif args.row is not None:
             import invariant_deterministic_04_b200 as bi
 
             torch.cuda.set_device(local)

@@ -14,10 +14,12 @@
 //   * one warp reduces one (row, kv-head, split) for the Hq/Hkv query heads that
 //     share the kv-head, page by page in ascending order, with an online softmax
 //     in the base-2 domain (scores pre-multiplied by scale*log2(e));
-//   * inside a page, a token's q.k is an 8-term FMA chain per lane (8 dims)
-//     followed by a fixed xor reduce-scatter tree over the D/8 lanes of the token;
-//     token t of the page is handled by lane group t mod (256/D) and the groups'
-//     partial sums are merged by a fixed xor tree at the end of the split;
+//   * inside a page, a token's q.k is summed per lane over its DPL dims (DPL = 16
+//     or 8, fixed by D and the group size) as two interleaved fp32 FMA chains (even
+//     and odd dims, packed f32x2 FMAs) joined by one add, then by a fixed xor
+//     reduce-scatter tree over the D/DPL lanes of the token; token t of the page
+//     is handled by lane group t mod (32*DPL/D) and the groups' partial sums are
+//     merged by a fixed xor tree at the end of the split;
 //   * splits are folded in ascending order: M = max_s m_s, then
 //     L = sum_s l_s 2^(m_s - M), O = sum_s o_s 2^(m_s - M) (FMA chains from 0),
 //     out = O / L rounded to bf16.
@@ -35,8 +37,6 @@ namespace attn {
 constexpr int PAGE = BI_PAGE_TOKENS;
 constexpr int SPLIT = BI_KV_SPLIT;
 constexpr int PAGES_PER_SPLIT = SPLIT / PAGE;
-constexpr int kWarps = 8;  // warps per CTA in the split kernel, each with its own page ring
-constexpr int NSTAGE = 3;  // pages in flight per warp
 
 // Where a query row reads its keys: decode rows use (row, seq_lens[row]);
 // prefill rows use (q_seq[row], q_pos[row] + 1).
@@ -145,20 +145,36 @@ __device__ __forceinline__ void all_gather(float x, int dl, float (&out)[G]) {
   }
 }
 
-template <int D>
+// Launch shape of the split kernel (a function of D and the group size G only):
+// DPL dims per lane (16 when the registers allow it: fewer lanes per token, a
+// shallower reduction tree), WARPS warps per CTA, each with its own ring of NST pages.
+template <int D, int G>
+struct SplitCfg {
+  static constexpr int DPL = (D == 128 && G <= 4) ? 16 : 8;
+  static constexpr int WARPS = 8, NST = 3;
+};
+
+template <int D, int G>
 constexpr int split_smem_bytes() {
-  return kWarps * NSTAGE * 2 * PAGE * D * 2 + kWarps * NSTAGE * 8;
+  return SplitCfg<D, G>::WARPS * SplitCfg<D, G>::NST * (2 * PAGE * D * 2 + 8);
 }
 
 // One warp per (row, kv-head g, split): writes the split's (m, l) per query head
 // and its unnormalised o[D] per query head into the workspace.
+//
+// Lane layout: the LPT = D/DPL lanes of a token own DPL dims each, in 16-byte
+// vectors v = 0..DPL/8-1 covering dims 8*(dl + v*LPT) .. +7 (interleaved so a
+// quarter-warp's shared-memory reads are contiguous); TPW = 32/LPT tokens are
+// processed per warp step, token t of a page by lane group t mod TPW.
 template <int D, int G>
-__global__ void __launch_bounds__(kWarps * 32, 1)
+__global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
     attn_split_kernel(const uint16_t* __restrict__ q, int Hq, int Hkv, const uint16_t* __restrict__ kc,
                       const uint16_t* __restrict__ vc, int64_t num_pages, const int32_t* __restrict__ pt,
                       Rows R, int nrows, const int32_t* __restrict__ off, float* __restrict__ po,
                       float2* __restrict__ pml, float c) {
-  constexpr int LPT = D / 8;        // lanes per token (8 dims per lane)
+  constexpr int DPL = SplitCfg<D, G>::DPL, WARPS = SplitCfg<D, G>::WARPS, NST = SplitCfg<D, G>::NST;
+  constexpr int NV = DPL / 8;       // 16-byte vectors per lane per token row
+  constexpr int LPT = D / DPL;      // lanes per token
   constexpr int TPW = 32 / LPT;     // tokens per warp step
   constexpr int STEPS = PAGE / TPW;
   constexpr int HEAD_LANES = LPT / G;
@@ -170,11 +186,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tg = lane / LPT, dl = lane % LPT;
   const int hd = dl / HEAD_LANES;
-  const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * NSTAGE * STAGE_BYTES);
-  const uint32_t bars = smem_u32(smem) + (uint32_t)(kWarps * NSTAGE * STAGE_BYTES + warp * NSTAGE * 8);
+  const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * NST * STAGE_BYTES);
+  const uint32_t bars = smem_u32(smem) + (uint32_t)(WARPS * NST * STAGE_BYTES + warp * NST * 8);
 
   if (lane == 0) {
-    for (int s = 0; s < NSTAGE; ++s) mbar_init(bars + 8 * s, 1);
+    for (int s = 0; s < NST; ++s) mbar_init(bars + 8 * s, 1);
     fence_mbar_init();
   }
   __syncwarp();
@@ -183,7 +199,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   const int64_t kv_head_stride = (int64_t)PAGE * D;
   uint32_t seq = 0;  // pages this warp has consumed so far
 
-  for (int item = blockIdx.x * kWarps + warp; item < total; item += gridDim.x * kWarps) {
+  for (int item = blockIdx.x * WARPS + warp; item < total; item += gridDim.x * WARPS) {
     const int f = item / Hkv, g = item - (item / Hkv) * Hkv;
     int lo = 0, hi = nrows;  // off[lo] <= f < off[hi]
     while (hi - lo > 1) {
@@ -199,16 +215,19 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     const int np = (t1 - t0 + PAGE - 1) / PAGE;
     const int32_t* prow = pt + (int64_t)pt_row * R.max_pages + s * PAGES_PER_SPLIT;
 
-    float qf[G][8];
+    float2 qf[G][DPL / 2];  // dims (2e, 2e+1) of the lane's slice in pair e
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-      const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + ((int64_t)r * Hq + g * G + j) * D + dl * 8));
-      unpack8(qv, qf[j]);
-    }
+    for (int j = 0; j < G; ++j)
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + ((int64_t)r * Hq + g * G + j) * D +
+                                                              8 * (dl + v * LPT)));
+        unpack8x2(qv, &qf[j][4 * v]);
+      }
 
     // Lane 0 starts the copy of page j of this split into its ring stage.
     auto issue = [&](int j, uint32_t sq) {
-      const uint32_t st = sq % NSTAGE;
+      const uint32_t st = sq % NST;
       const uint32_t bar = bars + 8 * st;
       const int pg = prow[j];
       const int nvalid = min(PAGE, t1 - t0 - j * PAGE);
@@ -226,39 +245,47 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     };
     if (lane == 0) {
       fence_proxy_async_smem();
-      for (int j = 0; j < NSTAGE && j < np; ++j) issue(j, seq + j);
+      for (int j = 0; j < NST && j < np; ++j) issue(j, seq + j);
     }
 
     float m = -INFINITY, l = 0.f;
-    float o[G][8];
+    float2 o[G][DPL / 2];
 #pragma unroll
     for (int j = 0; j < G; ++j)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[j][e] = 0.f;
+      for (int e = 0; e < DPL / 2; ++e) o[j][e] = make_float2(0.f, 0.f);
 
     bool ok = true;
     for (int j = 0; j < np; ++j, ++seq) {
-      const uint32_t st = seq % NSTAGE;
-      ok = __all_sync(kFullMask, mbar_wait(bars + 8 * st, (seq / NSTAGE) & 1u));
+      const uint32_t st = seq % NST;
+      ok = __all_sync(kFullMask, mbar_wait(bars + 8 * st, (seq / NST) & 1u));
       if (!ok) break;
       const int pg = prow[j];
       const int nvalid = (pg < 0 || pg >= num_pages) ? 0 : min(PAGE, t1 - t0 - j * PAGE);
       const uint32_t kb = ring + st * STAGE_BYTES, vb = kb + PAGE_BYTES;
 
+      // scores of this page: lane holds the score of its token for head hd
       float sc[STEPS];
 #pragma unroll
       for (int u = 0; u < STEPS; ++u) {
         const int t = u * TPW + tg;
-        float kf[8];
-        unpack8(ld_shared_v4(kb + (uint32_t)((t * D + dl * 8) * 2)), kf);
+        // two interleaved FMA chains per head (even / odd dims of the slice), then one add
+        float2 acc[G];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          float2 kf[4];
+          unpack8x2(ld_shared_v4(kb + (uint32_t)((t * D + 8 * (dl + v * LPT)) * 2)), kf);
+#pragma unroll
+          for (int i = 0; i < G; ++i) {
+            float2 a = v == 0 ? __fmul2_rn(qf[i][0], kf[0]) : __ffma2_rn(qf[i][4 * v], kf[0], acc[i]);
+#pragma unroll
+            for (int e = 1; e < 4; ++e) a = __ffma2_rn(qf[i][4 * v + e], kf[e], a);
+            acc[i] = a;
+          }
+        }
         float part[G];
 #pragma unroll
-        for (int i = 0; i < G; ++i) {
-          float a = __fmul_rn(qf[i][0], kf[0]);
-#pragma unroll
-          for (int e = 1; e < 8; ++e) a = __fmaf_rn(qf[i][e], kf[e], a);
-          part[i] = a;
-        }
+        for (int i = 0; i < G; ++i) part[i] = __fadd_rn(acc[i].x, acc[i].y);
         const float dot = reduce_scatter<G, LPT>(part, dl);
         sc[u] = t < nvalid ? __fmul_rn(dot, c) : -INFINITY;
       }
@@ -269,13 +296,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       for (int o2 = LPT; o2 < 32; o2 <<= 1) pm = fmaxf(pm, __shfl_xor_sync(kFullMask, pm, o2));
       const float m_new = fmaxf(m, pm);
       const float alpha = m_new == -INFINITY ? 1.f : exp2f(__fsub_rn(m, m_new));
-      l = __fmul_rn(l, alpha);
-      float al[G];
-      all_gather<G, LPT>(alpha, dl, al);
+      // rescale the running sums; skipped when no head's max moved (x * 1 == x exactly)
+      if (!__all_sync(kFullMask, alpha == 1.f)) {
+        l = __fmul_rn(l, alpha);
+        float al[G];
+        all_gather<G, LPT>(alpha, dl, al);
 #pragma unroll
-      for (int i = 0; i < G; ++i)
+        for (int i = 0; i < G; ++i) {
+          const float2 a2 = make_float2(al[i], al[i]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[i][e] = __fmul_rn(o[i][e], al[i]);
+          for (int e = 0; e < DPL / 2; ++e) o[i][e] = __fmul2_rn(o[i][e], a2);
+        }
+      }
 #pragma unroll
       for (int u = 0; u < STEPS; ++u) {
         const int t = u * TPW + tg;
@@ -284,20 +316,25 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
         l = __fadd_rn(l, p);
         float pa[G];
         all_gather<G, LPT>(p, dl, pa);
-        float vf[8];
-        unpack8(ld_shared_v4(vb + (uint32_t)((t * D + dl * 8) * 2)), vf);
-        if (valid) {
 #pragma unroll
-          for (int i = 0; i < G; ++i)
+        for (int v = 0; v < NV; ++v) {
+          float2 vf[4];
+          unpack8x2(ld_shared_v4(vb + (uint32_t)((t * D + 8 * (dl + v * LPT)) * 2)), vf);
+          if (valid) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o[i][e] = __fmaf_rn(pa[i], vf[e], o[i][e]);
+            for (int i = 0; i < G; ++i) {
+              const float2 p2 = make_float2(pa[i], pa[i]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) o[i][4 * v + e] = __ffma2_rn(p2, vf[e], o[i][4 * v + e]);
+            }
+          }
         }
       }
       m = m_new;
       __syncwarp();
-      if (lane == 0 && j + NSTAGE < np) {
+      if (lane == 0 && j + NST < np) {
         fence_proxy_async_smem();
-        issue(j + NSTAGE, seq + NSTAGE);
+        issue(j + NST, seq + NST);
       }
     }
     if (!ok) return;  // a copy never landed: error recorded, leave the warp
@@ -309,15 +346,21 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
 #pragma unroll
       for (int i = 0; i < G; ++i)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[i][e] = __fadd_rn(o[i][e], __shfl_xor_sync(kFullMask, o[i][e], o2));
+        for (int e = 0; e < DPL / 2; ++e) {
+          const float2 other = make_float2(__shfl_xor_sync(kFullMask, o[i][e].x, o2),
+                                           __shfl_xor_sync(kFullMask, o[i][e].y, o2));
+          o[i][e] = __fadd2_rn(o[i][e], other);
+        }
     }
     if (tg == 0) {
 #pragma unroll
-      for (int i = 0; i < G; ++i) {
-        float4* dst = reinterpret_cast<float4*>(po + ((int64_t)f * Hq + g * G + i) * D + dl * 8);
-        dst[0] = make_float4(o[i][0], o[i][1], o[i][2], o[i][3]);
-        dst[1] = make_float4(o[i][4], o[i][5], o[i][6], o[i][7]);
-      }
+      for (int i = 0; i < G; ++i)
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          float4* dst = reinterpret_cast<float4*>(po + ((int64_t)f * Hq + g * G + i) * D + 8 * (dl + v * LPT));
+          dst[0] = make_float4(o[i][4 * v + 0].x, o[i][4 * v + 0].y, o[i][4 * v + 1].x, o[i][4 * v + 1].y);
+          dst[1] = make_float4(o[i][4 * v + 2].x, o[i][4 * v + 2].y, o[i][4 * v + 3].x, o[i][4 * v + 3].y);
+        }
       if (dl % HEAD_LANES == 0) pml[(int64_t)f * Hq + g * G + hd] = make_float2(m, l);
     }
   }

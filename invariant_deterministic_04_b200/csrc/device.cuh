@@ -3,7 +3,9 @@
 // wrappers, and bounded waits.
 //
 // Every floating-point step on a reduction path is written with an explicit
-// rounding intrinsic (__fmaf_rn, __fadd_rn, __fmul_rn) so that the compiler cannot
+// rounding intrinsic (__fmaf_rn, __fadd_rn, __fmul_rn and their packed f32x2 forms
+// __ffma2_rn, __fadd2_rn, __fmul2_rn, which round each element exactly like the
+// scalar ones) so that the compiler cannot
 // contract or reassociate it differently in different kernels or instantiations:
 // the order of a row's reduction is part of the interface.
 #pragma once
@@ -35,6 +37,14 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
   f[4] = bf16lo(v.z); f[5] = bf16hi(v.z);
   f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+
+// Eight bf16 as four (even, odd) fp32 pairs for the packed f32x2 arithmetic.
+__device__ __forceinline__ void unpack8x2(const uint4& v, float2* f) {
+  f[0] = make_float2(bf16lo(v.x), bf16hi(v.x));
+  f[1] = make_float2(bf16lo(v.y), bf16hi(v.y));
+  f[2] = make_float2(bf16lo(v.z), bf16hi(v.z));
+  f[3] = make_float2(bf16lo(v.w), bf16hi(v.w));
 }
 
 // Round two fp32 values to bf16 (nearest even) and pack them, `lo` in the low half.

@@ -61,21 +61,27 @@ size_t attn_ws_size(int64_t rows, int Hq, int D, int max_pages, AttnWs* layout, 
 }
 
 template <int D, int G>
-cudaError_t launch_split(int grid_per_sm, const uint16_t* q, int Hq, int Hkv, const uint16_t* kc,
+cudaError_t launch_split(const uint16_t* q, int Hq, int Hkv, const uint16_t* kc,
                          const uint16_t* vc, int64_t num_pages, const int32_t* pt, bi::attn::Rows R, int nrows,
                          const AttnWs& ws, float c, cudaStream_t st) {
-  constexpr int smem = bi::attn::split_smem_bytes<D>();
+  constexpr int smem = bi::attn::split_smem_bytes<D, G>();
   static std::once_flag once[64];
   int dev = 0;
   cudaGetDevice(&dev);
   cudaError_t attr = cudaSuccess;
+  static int per_sm[64];
   std::call_once(once[dev & 63], [&] {
     attr = cudaFuncSetAttribute(bi::attn::attn_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 smem);
+    if (attr == cudaSuccess)
+      attr = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[dev & 63], bi::attn::attn_split_kernel<D, G>,
+                                                           bi::attn::SplitCfg<D, G>::WARPS * 32, smem);
   });
   if (attr != cudaSuccess) return attr;
-  const int grid = device_sms() * grid_per_sm;
-  bi::attn::attn_split_kernel<D, G><<<grid, bi::attn::kWarps * 32, smem, st>>>(q, Hq, Hkv, kc, vc, num_pages, pt,
+  // persistent grid: as many CTAs as can be resident (shared memory or registers
+  // limit it); the grid only decides which warp takes which (row, head, split)
+  const int grid = device_sms() * (per_sm[dev & 63] > 0 ? per_sm[dev & 63] : 1);
+  bi::attn::attn_split_kernel<D, G><<<grid, bi::attn::SplitCfg<D, G>::WARPS * 32, smem, st>>>(q, Hq, Hkv, kc, vc, num_pages, pt,
                                                                                 R, nrows, ws.off, ws.po, ws.pml, c);
   return cudaGetLastError();
 }
@@ -84,13 +90,11 @@ template <int D>
 cudaError_t launch_split_g(int G, const uint16_t* q, int Hq, int Hkv, const uint16_t* kc, const uint16_t* vc,
                            int64_t num_pages, const int32_t* pt, bi::attn::Rows R, int nrows, const AttnWs& ws,
                            float c, cudaStream_t st) {
-  // D=128 fills ~192 KiB of shared memory per CTA (one CTA per SM); D=64 fits two.
-  const int per_sm = D == 128 ? 1 : 2;
   switch (G) {
-    case 1: return launch_split<D, 1>(per_sm, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
-    case 2: return launch_split<D, 2>(per_sm, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
-    case 4: return launch_split<D, 4>(per_sm, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
-    default: return launch_split<D, 8>(per_sm, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    case 1: return launch_split<D, 1>(q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    case 2: return launch_split<D, 2>(q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    case 4: return launch_split<D, 4>(q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    default: return launch_split<D, 8>(q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
   }
 }
 

@@ -110,66 +110,89 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int32_t* __restrict
 }
 
 // fp32 logits of flagged rows: out[row, v] = sum_k h[row, k] * W[v, k], one FMA
-// chain in ascending k per logit. Tile: 32 flagged rows x 128 vocabulary rows,
-// k staged 32 at a time through shared memory; each thread owns 4 x 4 outputs.
-constexpr int RB = 32, VB = 128, KB = 32;
+// chain in ascending k per logit (the packed f32x2 FMA below carries two logits of
+// two vocabulary entries, each element rounded exactly like a scalar FMA). Tile:
+// 32 flagged rows x 256 vocabulary rows, k staged 32 at a time through shared
+// memory (the next slab is prefetched into registers while the current one is
+// consumed); each thread owns 4 rows x 8 vocabulary entries.
+constexpr int RB = 32, VB = 256, KB = 32;
 
 __global__ void __launch_bounds__(256) recompute_kernel(const uint16_t* __restrict__ h, int64_t ldh,
                                                         const uint16_t* __restrict__ W, int64_t V, int K, int M,
                                                         const int32_t* __restrict__ list,
                                                         float* __restrict__ out) {
   __shared__ __align__(16) float hs[KB][RB];
-  __shared__ __align__(16) float ws[KB][VB];
+  __shared__ __align__(16) float ws[KB][VB + 4];
   const int count = list[M];
   const int f0 = blockIdx.y * RB;
   if (f0 >= count) return;
   const int64_t v0 = (int64_t)blockIdx.x * VB;
   const int tid = threadIdx.x;
-  const int tx = tid & 31, ty = tid >> 5;  // vocab 4*tx.., rows 4*ty..
-  float acc[4][4];
+  const int tx = tid & 31, ty = tid >> 5;  // vocab 8*tx.., rows 4*ty..
+  float2 acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
 
-  for (int k0 = 0; k0 < K; k0 += KB) {
-    // h tile: 32 rows x 32 k (bf16 -> fp32), transposed to [k][row]
-    for (int e = tid; e < RB * KB; e += 256) {
-      const int rr = e / KB, kk = e % KB;
-      const int f = f0 + rr;
-      float val = 0.f;
-      if (f < count) {
-        const uint16_t b = h[(int64_t)list[f] * ldh + k0 + kk];
-        val = __uint_as_float((uint32_t)b << 16);
-      }
-      hs[kk][rr] = val;
+  // staging of one k-slab: each thread loads 1 h value (32 x 32) and 4 x 8 W values
+  const int hr = tid >> 3, hk = (tid & 7) * 4;  // h: row hr, k hk..hk+3
+  const int hf = f0 + hr;
+  const bool hvalid = hf < count;
+  const uint16_t* hsrc = h + (int64_t)(hvalid ? list[hf] : 0) * ldh;
+  auto load = [&](int k0, float (&hv)[4], uint4 (&wv)[4]) {
+    const uint2 hp = __ldg(reinterpret_cast<const uint2*>(hsrc + k0 + hk));
+    hv[0] = hvalid ? bf16lo(hp.x) : 0.f;
+    hv[1] = hvalid ? bf16hi(hp.x) : 0.f;
+    hv[2] = hvalid ? bf16lo(hp.y) : 0.f;
+    hv[3] = hvalid ? bf16hi(hp.y) : 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int e = tid + r * 256;  // 1024 vectors of 8 bf16: vocab e / 4, k-quarter e % 4
+      const int64_t vv = v0 + (e >> 2);
+      wv[r] = vv < V ? __ldg(reinterpret_cast<const uint4*>(W + vv * K + k0) + (e & 3)) : make_uint4(0, 0, 0, 0);
     }
-    // W tile: 128 vocab x 32 k, transposed to [k][vocab]
-    for (int e = tid; e < VB * (KB / 8); e += 256) {
-      const int vv = e / (KB / 8), kq = e % (KB / 8);
+  };
+  auto store = [&](const float (&hv)[4], const uint4 (&wv)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) hs[hk + e][hr] = hv[e];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int e = tid + r * 256;
       float f[8];
-      if (v0 + vv < V) {
-        unpack8(__ldg(reinterpret_cast<const uint4*>(W + (v0 + vv) * K + k0) + kq), f);
-      } else {
+      unpack8(wv[r], f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) ws[kq * 8 + i][vv] = f[i];
+      for (int i = 0; i < 8; ++i) ws[(e & 3) * 8 + i][e >> 2] = f[i];
     }
-    __syncthreads();
+  };
+  float hv[4];
+  uint4 wv[4];
+  load(0, hv, wv);
+  store(hv, wv);
+  __syncthreads();
+  for (int k0 = 0; k0 < K; k0 += KB) {
+    const bool more = k0 + KB < K;
+    if (more) load(k0 + KB, hv, wv);
 #pragma unroll 8
     for (int kk = 0; kk < KB; ++kk) {
-      const float4 hv = *reinterpret_cast<const float4*>(&hs[kk][ty * 4]);
-      const float4 wv = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
-      const float hr[4] = {hv.x, hv.y, hv.z, hv.w};
-      const float wr[4] = {wv.x, wv.y, wv.z, wv.w};
+      const float4 h4 = *reinterpret_cast<const float4*>(&hs[kk][ty * 4]);
+      const float4 wa = *reinterpret_cast<const float4*>(&ws[kk][tx * 8]);
+      const float4 wb = *reinterpret_cast<const float4*>(&ws[kk][tx * 8 + 4]);
+      const float hr4[4] = {h4.x, h4.y, h4.z, h4.w};
+      const float2 w2[4] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w), make_float2(wb.x, wb.y),
+                            make_float2(wb.z, wb.w)};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i) {
+        const float2 h2 = make_float2(hr4[i], hr4[i]);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(hr[i], wr[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = __ffma2_rn(h2, w2[j], acc[i][j]);
+      }
     }
     __syncthreads();
+    if (more) {
+      store(hv, wv);
+      __syncthreads();
+    }
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -178,8 +201,9 @@ __global__ void __launch_bounds__(256) recompute_kernel(const uint16_t* __restri
     float* dst = out + (int64_t)list[f] * V;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int64_t v = v0 + tx * 4 + j;
-      if (v < V) dst[v] = acc[i][j];
+      const int64_t v = v0 + tx * 8 + 2 * j;
+      if (v < V) dst[v] = acc[i][j].x;
+      if (v + 1 < V) dst[v + 1] = acc[i][j].y;
     }
   }
 }
