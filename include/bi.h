@@ -168,10 +168,13 @@ bi_status bi_attention_decode_static(const bi_bf16* q, const bi_bf16* k_cache, c
  * Each row is computed with exactly the per-row schedule of bi_attention_decode
  * for length q_pos[t] + 1, so a row's bits do not depend on the chunking, on T,
  * or on which other rows are present, and equal the decode result at that length.
- * q: [T, Hq, D] bf16. q_seq, q_pos: [T] int32. page_table: [num_seqs,
- * max_pages_per_seq] int32. out: [T, Hq, D] bf16. T == 0 is a no-op.
+ * A batch may therefore mix prefill chunks and decode tokens (a decode token is a
+ * row at its sequence's newest position).
+ * q: row t at q + t * ldq holds [Hq, D] bf16 (ldq >= Hq*D, ldq % 8 == 0, e.g. the
+ * q part of a fused QKV projection). q_seq, q_pos: [T] int32. page_table:
+ * [num_seqs, max_pages_per_seq] int32. out: [T, Hq, D] bf16. T == 0 is a no-op.
  */
-bi_status bi_attention_prefill(const bi_bf16* q, const int32_t* q_seq, const int32_t* q_pos,
+bi_status bi_attention_prefill(const bi_bf16* q, int64_t ldq, const int32_t* q_seq, const int32_t* q_pos,
                                const bi_bf16* k_cache, const bi_bf16* v_cache, int64_t num_pages,
                                const int32_t* page_table, int num_seqs, int max_pages_per_seq,
                                bi_bf16* out, int T, int Hq, int Hkv, int D, float scale,
@@ -179,14 +182,42 @@ bi_status bi_attention_prefill(const bi_bf16* q, const int32_t* q_seq, const int
 
 /*
  * Glue: write new tokens' K/V into the paged store (the unified layout of the
- * FixedAttention sketch). Token t of k_new/v_new ([T, Hkv, D] bf16) goes to slot
- * q_pos[t] % 16 of page page_table[q_seq[t], q_pos[t] / 16]. Pure copies; T == 0
- * is a no-op. Out-of-range ids set the device error word and skip the token.
+ * FixedAttention sketch). Row t of k_new / v_new starts at t * ld_new and holds
+ * [Hkv, D] bf16 (ld_new >= Hkv*D, ld_new % 8 == 0, e.g. the k / v parts of a fused
+ * QKV projection); it goes to slot q_pos[t] % 16 of page
+ * page_table[q_seq[t], q_pos[t] / 16]. Pure copies; T == 0 is a no-op.
+ * Out-of-range ids set the device error word and skip the token.
  */
-bi_status bi_kv_append(const bi_bf16* k_new, const bi_bf16* v_new, const int32_t* q_seq,
+bi_status bi_kv_append(const bi_bf16* k_new, const bi_bf16* v_new, int64_t ld_new, const int32_t* q_seq,
                        const int32_t* q_pos, bi_bf16* k_cache, bi_bf16* v_cache, int64_t num_pages,
                        const int32_t* page_table, int num_seqs, int max_pages_per_seq, int T,
                        int Hkv, int D, void* stream);
+
+/*
+ * Glue of a Llama-style decoder step. Each output element depends only on its own
+ * row's inputs (copies and elementwise fp32 math), so these are batch-invariant by
+ * construction; they keep a whole decoder step inside this library between the
+ * reductions above. No page describes them; they are the plain Llama operations.
+ *
+ * bi_gather_rows: dst[m, :width] = src[idx[m], :width] (embedding lookup, row
+ *   selection). idx out of [0, nrows_src) sets the device error word and zeroes
+ *   the row. width % 8 == 0.
+ * bi_rope: rotary position embedding, rotate-half form, in place on the H heads of
+ *   D dims in each row t of x (row stride ldx): for i < D/2 with
+ *   (c, s) = cos_sin[2 * (pos[t] * D/2 + i) .. +1] (fp32, [max_pos][D/2][2]),
+ *   x[i] <- x[i] c - x[i+D/2] s,  x[i+D/2] <- x[i+D/2] c + x[i] s, in fp32 as
+ *   fma(a, c, -(b s)) and fma(b, c, a s), rounded to bf16.
+ * bi_swiglu: out[m, j] = bf16(silu(g) * u), g = gate_up[m, j], u = gate_up[m, F+j],
+ *   silu(g) = g / (1 + exp(-g)) in fp32. F % 8 == 0.
+ * bi_add: out = bf16(a + b) elementwise over n (n % 8 == 0); out may alias a or b.
+ */
+bi_status bi_gather_rows(const bi_bf16* src, int64_t ld_src, int64_t nrows_src, const int32_t* idx, int64_t M,
+                         int64_t width, bi_bf16* dst, int64_t ld_dst, void* stream);
+bi_status bi_rope(bi_bf16* x, int64_t ldx, int64_t T, int H, int D, const int32_t* pos, const float* cos_sin,
+                  int max_pos, void* stream);
+bi_status bi_swiglu(const bi_bf16* gate_up, int64_t ld_gu, bi_bf16* out, int64_t ld_out, int64_t M, int64_t F,
+                    void* stream);
+bi_status bi_add(const bi_bf16* a, const bi_bf16* b, bi_bf16* out, int64_t n, void* stream);
 
 /* Workspace bytes for bi_lmhead_argmax with M rows and vocabulary V. */
 size_t bi_lmhead_workspace_size(int64_t M, int64_t V);

@@ -6,8 +6,8 @@ memory and the current stream. There is no CPU or library fallback: if
 libbi.so is missing or fails to load, every call raises ``BIError``.
 
 Operations (see include/bi.h for the exact contracts):
-  rmsnorm, matmul, attention_decode, attention_prefill, kv_append,
-  lmhead_argmax, get_device_error.
+  rmsnorm, matmul, attention_decode, attention_decode_static, attention_prefill,
+  kv_append, lmhead_argmax, gather_rows, rope, swiglu, add, get_device_error.
 """
 from __future__ import annotations
 
@@ -44,9 +44,13 @@ _SIGNATURES = {
     "bi_attention_workspace_size": ([_I64, _I32, _I32, _I32], _SZ),
     "bi_attention_decode": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ, _P], _I32),
     "bi_attention_decode_static": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P], _I32),
-    "bi_attention_prefill": ([_P, _P, _P, _P, _P, _I64, _P, _I32, _I32, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ, _P],
-                             _I32),
-    "bi_kv_append": ([_P, _P, _P, _P, _P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P], _I32),
+    "bi_attention_prefill": ([_P, _I64, _P, _P, _P, _P, _I64, _P, _I32, _I32, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ,
+                              _P], _I32),
+    "bi_kv_append": ([_P, _P, _I64, _P, _P, _P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P], _I32),
+    "bi_gather_rows": ([_P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P], _I32),
+    "bi_rope": ([_P, _I64, _I64, _I32, _I32, _P, _P, _I32, _P], _I32),
+    "bi_swiglu": ([_P, _I64, _P, _I64, _I64, _I64, _P], _I32),
+    "bi_add": ([_P, _P, _P, _I64, _P], _I32),
     "bi_lmhead_workspace_size": ([_I64, _I64], _SZ),
     "bi_lmhead_argmax": ([_P, _I64, _P, _I64, _I64, _I64, _F, _P, _P, _P, _P, _SZ, _P], _I32),
     "bi_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], _I32),
@@ -205,18 +209,30 @@ def attention_decode_static(q, k_cache, v_cache, page_table, seq_lens, scale: fl
     return out
 
 
+def _rows3(t: torch.Tensor, name: str):
+    """[T, H, D] view whose rows may be strided (e.g. a slice of a fused QKV output)."""
+    if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+        raise ValueError(f"{name} must be [T, H, D] with contiguous heads (row stride free)")
+    return t.stride(0)
+
+
 def attention_prefill(q, q_seq, q_pos, k_cache, v_cache, page_table, scale: float | None = None, out=None,
                       workspace=None, stream=None):
-    """Causal prefill; row t of q [T, Hq, D] sees keys 0..q_pos[t] of sequence q_seq[t]."""
+    """Causal prefill; row t of q [T, Hq, D] sees keys 0..q_pos[t] of sequence q_seq[t].
+
+    A decode token is a row at its sequence's newest position, so one call may mix
+    prefill chunks and decode tokens. q's rows may be strided (a fused QKV slice).
+    """
     _req(q, torch.bfloat16, "q", 3)
     _req(q_seq, torch.int32, "q_seq", 1)
     _req(q_pos, torch.int32, "q_pos", 1)
     _req(k_cache, torch.bfloat16, "k_cache", 4)
     _req(v_cache, torch.bfloat16, "v_cache", 4)
     _req(page_table, torch.int32, "page_table", 2)
-    for t, n in ((q, "q"), (q_seq, "q_seq"), (q_pos, "q_pos"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+    for t, n in ((q_seq, "q_seq"), (q_pos, "q_pos"), (k_cache, "k_cache"), (v_cache, "v_cache"),
                  (page_table, "page_table")):
         _contig(t, n)
+    ldq = _rows3(q, "q")
     T, Hq, D = q.shape
     num_pages, Hkv = k_cache.shape[0], k_cache.shape[1]
     if k_cache.shape != v_cache.shape or k_cache.shape[2] != PAGE_TOKENS or k_cache.shape[3] != D:
@@ -225,27 +241,86 @@ def attention_prefill(q, q_seq, q_pos, k_cache, v_cache, page_table, scale: floa
         raise ValueError("q_seq and q_pos need one entry per query row")
     num_seqs, maxp = page_table.shape
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    out = torch.empty_like(q) if out is None else out
+    out = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=q.device) if out is None else out
     ws, nbytes = _workspace(attention_workspace_size(T, Hq, D, maxp), q.device, workspace)
     _check("bi_attention_prefill", lib().bi_attention_prefill(
-        _ptr(q), _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), num_seqs,
-        maxp, _ptr(out), T, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream(stream)))
+        _ptr(q), ldq, _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table),
+        num_seqs, maxp, _ptr(out), T, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream(stream)))
     return out
 
 
 def kv_append(k_new, v_new, q_seq, q_pos, k_cache, v_cache, page_table, stream=None):
-    """Write k_new/v_new [T, Hkv, D] into the paged store at (q_seq[t], q_pos[t])."""
+    """Write k_new/v_new [T, Hkv, D] (rows may be strided) into the paged store at (q_seq[t], q_pos[t])."""
     for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
         _req(t, torch.bfloat16, n)
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
         _contig(t, n)
     for t, n in ((q_seq, "q_seq"), (q_pos, "q_pos"), (page_table, "page_table")):
         _req(t, torch.int32, n)
         _contig(t, n)
+    ld = _rows3(k_new, "k_new")
+    if _rows3(v_new, "v_new") != ld or v_new.shape != k_new.shape:
+        raise ValueError("k_new and v_new must have the same shape and row stride")
     T, Hkv, D = k_new.shape
     num_seqs, maxp = page_table.shape
     _check("bi_kv_append", lib().bi_kv_append(
-        _ptr(k_new), _ptr(v_new), _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
+        _ptr(k_new), _ptr(v_new), ld, _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
         _ptr(page_table), num_seqs, maxp, T, Hkv, D, _stream(stream)))
+
+
+def gather_rows(src, idx, out=None, stream=None):
+    """out[m] = src[idx[m]] (embedding lookup / row selection)."""
+    _req(src, torch.bfloat16, "src", 2)
+    _req(idx, torch.int32, "idx", 1)
+    _contig(idx, "idx")
+    if src.stride(1) != 1:
+        raise ValueError("src rows must be contiguous")
+    M, W = idx.shape[0], src.shape[1]
+    out = torch.empty((M, W), dtype=torch.bfloat16, device=src.device) if out is None else out
+    _check("bi_gather_rows", lib().bi_gather_rows(_ptr(src), src.stride(0), src.shape[0], _ptr(idx), M, W, _ptr(out),
+                                                  out.stride(0), _stream(stream)))
+    return out
+
+
+def rope(x, pos, cos_sin, stream=None):
+    """In-place rotary embedding on x [T, H, D] (rows may be strided); cos_sin fp32 [max_pos, D/2, 2]."""
+    _req(x, torch.bfloat16, "x", 3)
+    _req(pos, torch.int32, "pos", 1)
+    _req(cos_sin, torch.float32, "cos_sin", 3)
+    _contig(pos, "pos")
+    _contig(cos_sin, "cos_sin")
+    ldx = _rows3(x, "x")
+    T, H, D = x.shape
+    if cos_sin.shape[1:] != (D // 2, 2):
+        raise ValueError("cos_sin must be [max_pos, D/2, 2]")
+    _check("bi_rope", lib().bi_rope(_ptr(x), ldx, T, H, D, _ptr(pos), _ptr(cos_sin), cos_sin.shape[0],
+                                    _stream(stream)))
+    return x
+
+
+def swiglu(gate_up, out=None, stream=None):
+    """out = silu(gate_up[:, :F]) * gate_up[:, F:] with F = gate_up.shape[1] // 2."""
+    _req(gate_up, torch.bfloat16, "gate_up", 2)
+    if gate_up.stride(1) != 1:
+        raise ValueError("gate_up rows must be contiguous")
+    M, F2 = gate_up.shape
+    F = F2 // 2
+    out = torch.empty((M, F), dtype=torch.bfloat16, device=gate_up.device) if out is None else out
+    _check("bi_swiglu", lib().bi_swiglu(_ptr(gate_up), gate_up.stride(0), _ptr(out), out.stride(0), M, F,
+                                        _stream(stream)))
+    return out
+
+
+def add(a, b, out=None, stream=None):
+    """out = a + b elementwise (bf16 in, fp32 add, bf16 out); out may be a or b."""
+    for t, n in ((a, "a"), (b, "b")):
+        _req(t, torch.bfloat16, n)
+        _contig(t, n)
+    if a.shape != b.shape:
+        raise ValueError("a and b must have the same shape")
+    out = torch.empty_like(a) if out is None else out
+    _check("bi_add", lib().bi_add(_ptr(a), _ptr(b), _ptr(out), a.numel(), _stream(stream)))
+    return out
 
 
 def lmhead_workspace_size(M: int, V: int) -> int:

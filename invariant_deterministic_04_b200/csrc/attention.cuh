@@ -168,7 +168,7 @@ constexpr int split_smem_bytes() {
 // processed per warp step, token t of a page by lane group t mod TPW.
 template <int D, int G>
 __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
-    attn_split_kernel(const uint16_t* __restrict__ q, int Hq, int Hkv, const uint16_t* __restrict__ kc,
+    attn_split_kernel(const uint16_t* __restrict__ q, int64_t ldq, int Hq, int Hkv, const uint16_t* __restrict__ kc,
                       const uint16_t* __restrict__ vc, int64_t num_pages, const int32_t* __restrict__ pt,
                       Rows R, int nrows, const int32_t* __restrict__ off, float* __restrict__ po,
                       float2* __restrict__ pml, float c) {
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
     for (int j = 0; j < G; ++j)
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + ((int64_t)r * Hq + g * G + j) * D +
+        const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)r * ldq + (int64_t)(g * G + j) * D +
                                                               8 * (dl + v * LPT)));
         unpack8x2(qv, &qf[j][4 * v]);
       }
@@ -404,9 +404,10 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   }
 }
 
-// One warp per (token, kv-head): copy the token's K and V rows into its page slot.
+// One warp per (token, kv-head): copy the token's K and V rows (row t of k_new /
+// v_new starts at t * ld_new) into its page slot.
 __global__ void __launch_bounds__(256) kv_append_kernel(const uint16_t* __restrict__ kn,
-                                                        const uint16_t* __restrict__ vn,
+                                                        const uint16_t* __restrict__ vn, int64_t ld_new,
                                                         const int32_t* __restrict__ q_seq,
                                                         const int32_t* __restrict__ q_pos,
                                                         uint16_t* __restrict__ kc, uint16_t* __restrict__ vc,
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint16_t* __restri
     return;
   }
   const int64_t dst = (((int64_t)pg * Hkv + g) * PAGE + pos % PAGE) * D;
-  const int64_t src = ((int64_t)t * Hkv + g) * D;
+  const int64_t src = (int64_t)t * ld_new + (int64_t)g * D;
   for (int i = lane; i < D / 8; i += 32) {
     reinterpret_cast<uint4*>(kc + dst)[i] = __ldg(reinterpret_cast<const uint4*>(kn + src) + i);
     reinterpret_cast<uint4*>(vc + dst)[i] = __ldg(reinterpret_cast<const uint4*>(vn + src) + i);

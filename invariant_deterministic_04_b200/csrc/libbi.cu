@@ -12,6 +12,7 @@
 #include "gemm.cuh"
 #include "attention.cuh"
 #include "lmhead.cuh"
+#include "glue.cuh"
 
 namespace {
 
@@ -61,7 +62,7 @@ size_t attn_ws_size(int64_t rows, int Hq, int D, int max_pages, AttnWs* layout, 
 }
 
 template <int D, int G>
-cudaError_t launch_split(const uint16_t* q, int Hq, int Hkv, const uint16_t* kc,
+cudaError_t launch_split(const uint16_t* q, int64_t ldq, int Hq, int Hkv, const uint16_t* kc,
                          const uint16_t* vc, int64_t num_pages, const int32_t* pt, bi::attn::Rows R, int nrows,
                          const AttnWs& ws, float c, cudaStream_t st) {
   constexpr int smem = bi::attn::split_smem_bytes<D, G>();
@@ -81,30 +82,31 @@ cudaError_t launch_split(const uint16_t* q, int Hq, int Hkv, const uint16_t* kc,
   // persistent grid: as many CTAs as can be resident (shared memory or registers
   // limit it); the grid only decides which warp takes which (row, head, split)
   const int grid = device_sms() * (per_sm[dev & 63] > 0 ? per_sm[dev & 63] : 1);
-  bi::attn::attn_split_kernel<D, G><<<grid, bi::attn::SplitCfg<D, G>::WARPS * 32, smem, st>>>(q, Hq, Hkv, kc, vc, num_pages, pt,
+  bi::attn::attn_split_kernel<D, G><<<grid, bi::attn::SplitCfg<D, G>::WARPS * 32, smem, st>>>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt,
                                                                                 R, nrows, ws.off, ws.po, ws.pml, c);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_split_g(int G, const uint16_t* q, int Hq, int Hkv, const uint16_t* kc, const uint16_t* vc,
+cudaError_t launch_split_g(int G, const uint16_t* q, int64_t ldq, int Hq, int Hkv, const uint16_t* kc, const uint16_t* vc,
                            int64_t num_pages, const int32_t* pt, bi::attn::Rows R, int nrows, const AttnWs& ws,
                            float c, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_split<D, 1>(q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
-    case 2: return launch_split<D, 2>(q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
-    case 4: return launch_split<D, 4>(q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
-    default: return launch_split<D, 8>(q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    case 1: return launch_split<D, 1>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    case 2: return launch_split<D, 2>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    case 4: return launch_split<D, 4>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
+    default: return launch_split<D, 8>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, ws, c, st);
   }
 }
 
-bi_status attention_common(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int64_t num_pages,
+bi_status attention_common(const uint16_t* q, int64_t ldq, const uint16_t* kc, const uint16_t* vc, int64_t num_pages,
                            const int32_t* pt, int max_pages, bi::attn::Rows R, int nrows, uint16_t* out,
                            int Hq, int Hkv, int D, float scale, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages <= 0 || max_pages <= 0) return BI_ERR_SHAPE;
   const int G = Hq / Hkv;
   if ((D != 64 && D != 128) || (G != 1 && G != 2 && G != 4 && G != 8)) return BI_ERR_UNSUPPORTED;
-  if (!std::isfinite(scale)) return BI_ERR_SHAPE;
+  if (!std::isfinite(scale) || ldq < (int64_t)Hq * D) return BI_ERR_SHAPE;
+  if (ldq % 8) return BI_ERR_ALIGN;
   // index arithmetic of the work list is 32-bit
   if ((int64_t)nrows * max_splits(max_pages) * Hkv >= INT_MAX || (int64_t)nrows * Hq >= INT_MAX / 8)
     return BI_ERR_SHAPE;
@@ -116,8 +118,8 @@ bi_status attention_common(const uint16_t* q, const uint16_t* kc, const uint16_t
   const float c = (float)((double)scale * 1.4426950408889634);  // scale * log2(e)
   bi::attn::split_offsets_kernel<<<1, 1024, 0, st>>>(R, nrows, lay.off);
   if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
-  cudaError_t e = D == 128 ? launch_split_g<128>(G, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st)
-                           : launch_split_g<64>(G, q, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st);
+  cudaError_t e = D == 128 ? launch_split_g<128>(G, q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st)
+                           : launch_split_g<64>(G, q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st);
   if (e != cudaSuccess) return BI_ERR_CUDA;
   const int warps = nrows * Hq;
   const int grid = (warps + 7) / 8;
@@ -195,7 +197,7 @@ const char* bi_status_string(int status) {
   }
 }
 
-int bi_version(void) { return 1; }
+int bi_version(void) { return 2; }
 
 bi_status bi_rmsnorm(const bi_bf16* x, int64_t ldx, const bi_bf16* w, bi_bf16* y, int64_t ldy, int64_t M,
                      int64_t K, float eps, void* stream) {
@@ -236,8 +238,8 @@ bi_status bi_attention_decode(const bi_bf16* q, const bi_bf16* k_cache, const bi
   if (B < 0) return BI_ERR_SHAPE;
   if (!workspace) return B == 0 ? BI_OK : BI_ERR_WORKSPACE;
   bi::attn::Rows R{seq_lens, nullptr, nullptr, B, max_pages_per_seq};
-  return attention_common(q, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, B, out, Hq, Hkv, D,
-                          scale, workspace, workspace_bytes, as_stream(stream));
+  return attention_common(q, (int64_t)Hq * D, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, B, out,
+                          Hq, Hkv, D, scale, workspace, workspace_bytes, as_stream(stream));
 }
 
 bi_status bi_attention_decode_static(const bi_bf16* q, const bi_bf16* k_cache, const bi_bf16* v_cache,
@@ -252,11 +254,11 @@ bi_status bi_attention_decode_static(const bi_bf16* q, const bi_bf16* k_cache, c
   const bi_status s = decode_scratch_address(&scratch);
   if (s != BI_OK) return s;
   bi::attn::Rows R{seq_lens, nullptr, nullptr, B, max_pages_per_seq};
-  return attention_common(q, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, B, out, Hq, Hkv, D,
-                          scale, scratch, BI_STATIC_SCRATCH_BYTES, as_stream(stream));
+  return attention_common(q, (int64_t)Hq * D, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, B, out,
+                          Hq, Hkv, D, scale, scratch, BI_STATIC_SCRATCH_BYTES, as_stream(stream));
 }
 
-bi_status bi_attention_prefill(const bi_bf16* q, const int32_t* q_seq, const int32_t* q_pos,
+bi_status bi_attention_prefill(const bi_bf16* q, int64_t ldq, const int32_t* q_seq, const int32_t* q_pos,
                                const bi_bf16* k_cache, const bi_bf16* v_cache, int64_t num_pages,
                                const int32_t* page_table, int num_seqs, int max_pages_per_seq, bi_bf16* out,
                                int T, int Hq, int Hkv, int D, float scale, void* workspace,
@@ -265,23 +267,25 @@ bi_status bi_attention_prefill(const bi_bf16* q, const int32_t* q_seq, const int
   if (T < 0 || num_seqs <= 0) return BI_ERR_SHAPE;
   if (!workspace) return T == 0 ? BI_OK : BI_ERR_WORKSPACE;
   bi::attn::Rows R{nullptr, q_seq, q_pos, num_seqs, max_pages_per_seq};
-  return attention_common(q, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, T, out, Hq, Hkv, D,
+  return attention_common(q, ldq, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, T, out, Hq, Hkv, D,
                           scale, workspace, workspace_bytes, as_stream(stream));
 }
 
-bi_status bi_kv_append(const bi_bf16* k_new, const bi_bf16* v_new, const int32_t* q_seq, const int32_t* q_pos,
+bi_status bi_kv_append(const bi_bf16* k_new, const bi_bf16* v_new, int64_t ld_new, const int32_t* q_seq, const int32_t* q_pos,
                        bi_bf16* k_cache, bi_bf16* v_cache, int64_t num_pages, const int32_t* page_table,
                        int num_seqs, int max_pages_per_seq, int T, int Hkv, int D, void* stream) {
   if (!k_new || !v_new || !q_seq || !q_pos || !k_cache || !v_cache || !page_table) return BI_ERR_NULL;
   if (T < 0 || num_seqs <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || Hkv <= 0 || D <= 0)
     return BI_ERR_SHAPE;
   if (D % 8 != 0) return BI_ERR_UNSUPPORTED;
-  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache)) return BI_ERR_ALIGN;
+  if (ld_new < (int64_t)Hkv * D) return BI_ERR_SHAPE;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) || ld_new % 8)
+    return BI_ERR_ALIGN;
   if (T == 0) return BI_OK;
   const int64_t warps = (int64_t)T * Hkv;
   if ((warps + 7) / 8 > INT_MAX) return BI_ERR_SHAPE;
   bi::attn::kv_append_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, as_stream(stream)>>>(
-      k_new, v_new, q_seq, q_pos, k_cache, v_cache, num_pages, page_table, num_seqs, max_pages_per_seq, T, Hkv, D);
+      k_new, v_new, ld_new, q_seq, q_pos, k_cache, v_cache, num_pages, page_table, num_seqs, max_pages_per_seq, T, Hkv, D);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
@@ -311,6 +315,54 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
   const dim3 rgrid((unsigned)((V + bi::lmhead::VB - 1) / bi::lmhead::VB), (unsigned)((M + bi::lmhead::RB - 1) / bi::lmhead::RB));
   bi::lmhead::recompute_kernel<<<rgrid, 256, 0, st>>>(h, ldh, W, V, (int)K, (int)M, lay.list, out32);
   bi::lmhead::argmax_kernel<<<(unsigned)M, bi::lmhead::kThreads, 0, st>>>(out32, V, recomputed, tokens);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_gather_rows(const bi_bf16* src, int64_t ld_src, int64_t nrows_src, const int32_t* idx, int64_t M,
+                         int64_t width, bi_bf16* dst, int64_t ld_dst, void* stream) {
+  if (!src || !idx || !dst) return BI_ERR_NULL;
+  if (M < 0 || nrows_src <= 0 || width <= 0 || width % 8 || ld_src < width || ld_dst < width || M > INT_MAX)
+    return BI_ERR_SHAPE;
+  if (!aligned16(src) || !aligned16(dst) || ld_src % 8 || ld_dst % 8) return BI_ERR_ALIGN;
+  if (M == 0) return BI_OK;
+  bi::glue::gather_rows_kernel<<<(unsigned)((M + 7) / 8), 256, 0, as_stream(stream)>>>(src, ld_src, nrows_src, idx,
+                                                                                        (int)M, width, dst, ld_dst);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_rope(bi_bf16* x, int64_t ldx, int64_t T, int H, int D, const int32_t* pos, const float* cos_sin,
+                  int max_pos, void* stream) {
+  if (!x || !pos || !cos_sin) return BI_ERR_NULL;
+  if (T < 0 || H <= 0 || D <= 0 || D % 2 || max_pos <= 0 || ldx < (int64_t)H * D) return BI_ERR_SHAPE;
+  if (T == 0) return BI_OK;
+  const int64_t n = T * H * (D / 2);
+  if ((n + 255) / 256 > INT_MAX) return BI_ERR_SHAPE;
+  bi::glue::rope_kernel<<<(unsigned)((n + 255) / 256), 256, 0, as_stream(stream)>>>(
+      x, ldx, (int)T, H, D, pos, reinterpret_cast<const float2*>(cos_sin), max_pos);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_swiglu(const bi_bf16* gate_up, int64_t ld_gu, bi_bf16* out, int64_t ld_out, int64_t M, int64_t F,
+                    void* stream) {
+  if (!gate_up || !out) return BI_ERR_NULL;
+  if (M < 0 || F <= 0 || F % 8 || ld_gu < 2 * F || ld_out < F) return BI_ERR_SHAPE;
+  if (!aligned16(gate_up) || !aligned16(out) || ld_gu % 8 || ld_out % 8) return BI_ERR_ALIGN;
+  if (M == 0) return BI_OK;
+  const int64_t n = M * (F / 8);
+  if ((n + 255) / 256 > INT_MAX || M > INT_MAX) return BI_ERR_SHAPE;
+  bi::glue::swiglu_kernel<<<(unsigned)((n + 255) / 256), 256, 0, as_stream(stream)>>>(gate_up, ld_gu, out, ld_out,
+                                                                                       (int)M, (int)F);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_add(const bi_bf16* a, const bi_bf16* b, bi_bf16* out, int64_t n, void* stream) {
+  if (!a || !b || !out) return BI_ERR_NULL;
+  if (n < 0 || n % 8) return BI_ERR_SHAPE;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(out)) return BI_ERR_ALIGN;
+  if (n == 0) return BI_OK;
+  const int64_t v = n / 8;
+  if ((v + 255) / 256 > INT_MAX) return BI_ERR_SHAPE;
+  bi::glue::add_kernel<<<(unsigned)((v + 255) / 256), 256, 0, as_stream(stream)>>>(a, b, out, n);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

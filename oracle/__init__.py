@@ -202,3 +202,77 @@ def normwise_rel_err(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
     den = np.abs(r).max(axis=1)
     den[den == 0] = 1.0
     return np.abs(g - r).max(axis=1) / den
+
+
+# ---------------------------------------------------------------------------
+# Decoder-step glue (plain Llama operations, no page describes them): rotary
+# embedding (rotate-half), SwiGLU, and one decoder layer chained in float64.
+
+
+def rope(x: np.ndarray, pos: np.ndarray, theta: float = 10000.0) -> np.ndarray:
+    """Rotary embedding, rotate-half form, in float64.
+
+    x: [T, H, D]; for i < D/2 the pair (x[i], x[i + D/2]) of token t is rotated by
+    the angle pos[t] * theta^(-2i/D).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    T, H, D = x.shape
+    half = D // 2
+    inv = theta ** (-2.0 * np.arange(half) / D)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]  # [T, half]
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    a, b = x[..., :half], x[..., half:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def silu(g: np.ndarray) -> np.ndarray:
+    g = np.asarray(g, dtype=np.float64)
+    return g / (1.0 + np.exp(-g))
+
+
+def swiglu(gate_up: np.ndarray) -> np.ndarray:
+    """silu(gate) * up with gate = first half of the columns, up = second half."""
+    gu = np.asarray(gate_up, dtype=np.float64)
+    F = gu.shape[-1] // 2
+    return silu(gu[..., :F]) * gu[..., F:]
+
+
+def decoder_layer(h, rows_seq, rows_pos, past_k, past_v, w, n_heads, n_kv, eps=1e-6, theta=10000.0):
+    """One pre-norm Llama decoder layer over query rows, in float64.
+
+    h: [T, Hd] hidden rows; row t is token rows_pos[t] of sequence rows_seq[t].
+    past_k/past_v: dict seq -> [L, n_kv, D] keys/values already in the cache for
+    positions 0..L-1 (already rotated). w: dict with wqkv [(n_heads+2 n_kv) D, Hd],
+    wo [Hd, Hd], wgu [2F, Hd], wdown [Hd, F], attn_norm, mlp_norm [Hd].
+    The rows' own keys/values are appended (positions must continue the cache) and
+    each row attends causally over its sequence. Returns the new h [T, Hd].
+    """
+    h = np.asarray(h, dtype=np.float64)
+    T, Hd = h.shape
+    D = Hd // n_heads
+    x = rmsnorm(h, w["attn_norm"], eps)
+    qkv = matmul(x, w["wqkv"])
+    q = qkv[:, : n_heads * D].reshape(T, n_heads, D)
+    k = qkv[:, n_heads * D: (n_heads + n_kv) * D].reshape(T, n_kv, D)
+    v = qkv[:, (n_heads + n_kv) * D:].reshape(T, n_kv, D)
+    q = rope(q, rows_pos, theta)
+    k = rope(k, rows_pos, theta)
+    keys = {s: np.asarray(past_k[s], dtype=np.float64) for s in past_k}
+    vals = {s: np.asarray(past_v[s], dtype=np.float64) for s in past_v}
+    for t in range(T):
+        s, p = int(rows_seq[t]), int(rows_pos[t])
+        kk = keys.setdefault(s, np.zeros((0, n_kv, D)))
+        assert kk.shape[0] == p, "rows must extend their sequence's cache in order"
+        keys[s] = np.concatenate([kk, k[t:t + 1]])
+        vals[s] = np.concatenate([vals.setdefault(s, np.zeros((0, n_kv, D))), v[t:t + 1]])
+    att = np.empty((T, n_heads, D))
+    group = n_heads // n_kv
+    for t in range(T):
+        s, p = int(rows_seq[t]), int(rows_pos[t])
+        for hh in range(n_heads):
+            g = hh // group
+            att[t, hh] = softmax_attend(q[t, hh], keys[s][: p + 1, g], vals[s][: p + 1, g], 1.0 / math.sqrt(D))
+    h = h + matmul(att.reshape(T, Hd), w["wo"])
+    x = rmsnorm(h, w["mlp_norm"], eps)
+    h = h + matmul(swiglu(matmul(x, w["wgu"])), w["wdown"])
+    return h

@@ -208,3 +208,31 @@ def sequence_pages(kv: PagedKV, b: int, L: int):
     k = kv.k_cache[pages].cpu()
     v = kv.v_cache[pages].cpu()
     return k, v, torch.arange(n, dtype=torch.int32).view(1, n)
+
+
+# ---------------------------------------------------------------------------
+# Random-init Llama-style decoder weights and prompts (drawn on the GPU from a
+# seed; N(0, 0.02) for every matrix, norm weights 1, no biases).
+
+
+LLAMA_CFG = dict(layers=16, hidden=2048, heads=32, kv_heads=8, head_dim=64, ffn=8192, vocab=32000, eps=1e-6,
+                 theta=10000.0)
+
+
+def llama_weights(cfg: dict, seed: int, device):
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    H, nh, nkv, D, F, V = (cfg[k] for k in ("hidden", "heads", "kv_heads", "head_dim", "ffn", "vocab"))
+
+    def nrm(shape):
+        return _device_normal_bf16(shape, gen, device).mul_(0.02)
+
+    ones = lambda n: torch.ones(n, dtype=torch.bfloat16, device=device)
+    layers = [dict(wqkv=nrm(((nh + 2 * nkv) * D, H)), wo=nrm((H, nh * D)), wgu=nrm((2 * F, H)), wdown=nrm((H, F)),
+                   attn_norm=ones(H), mlp_norm=ones(H)) for _ in range(cfg["layers"])]
+    return dict(embed=nrm((V, H)), layers=layers, final_norm=ones(H), lm_head=nrm((V, H)))
+
+
+def prompts(n: int, length: int, vocab: int, seed: int) -> np.ndarray:
+    """n prompts of `length` token ids ~ U[0, vocab)."""
+    return torch.randint(0, vocab, (n, length), generator=generator(seed), dtype=torch.int64).numpy()

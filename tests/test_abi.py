@@ -45,7 +45,7 @@ def test_status_strings(L):
     assert L.bi_status_string(0) == b"BI_OK"
     assert L.bi_status_string(4) == b"BI_ERR_WORKSPACE"
     assert L.bi_status_string(99) == b"BI_ERR_UNKNOWN"
-    assert L.bi_version() == 1
+    assert L.bi_version() == 2
 
 
 def test_rmsnorm_validation(L):
@@ -107,19 +107,44 @@ def test_attention_validation(L):
     assert d(*args(B=0, ws=None, wsb=0)) == OK
     p = L.bi_attention_prefill
     wsp = L.bi_attention_workspace_size(10, 32, 64, 8)
-    assert p(P, None, P, P, P, 100, P, 2, 8, P, 10, 32, 8, 64, 0.125, P, wsp, None) == NULL
-    assert p(P, P, P, P, P, 100, P, 0, 8, P, 10, 32, 8, 64, 0.125, P, wsp, None) == SHAPE
-    assert p(P, P, P, P, P, 100, P, 2, 8, P, 10, 32, 8, 64, 0.125, P, wsp - 256, None) == WS
-    assert p(P, P, P, P, P, 100, P, 2, 8, P, 0, 32, 8, 64, 0.125, None, 0, None) == OK
+    assert p(P, 2048, None, P, P, P, 100, P, 2, 8, P, 10, 32, 8, 64, 0.125, P, wsp, None) == NULL
+    assert p(P, 2048, P, P, P, P, 100, P, 0, 8, P, 10, 32, 8, 64, 0.125, P, wsp, None) == SHAPE
+    assert p(P, 2048, P, P, P, P, 100, P, 2, 8, P, 10, 32, 8, 64, 0.125, P, wsp - 256, None) == WS
+    assert p(P, 1024, P, P, P, P, 100, P, 2, 8, P, 10, 32, 8, 64, 0.125, P, wsp, None) == SHAPE   # ldq < Hq*D
+    assert p(P, 3076, P, P, P, P, 100, P, 2, 8, P, 10, 32, 8, 64, 0.125, P, wsp, None) == ALIGN   # ldq % 8
+    assert p(P, 2048, P, P, P, P, 100, P, 2, 8, P, 0, 32, 8, 64, 0.125, None, 0, None) == OK
 
 
 def test_kv_append_validation(L):
     f = L.bi_kv_append
-    assert f(None, P, P, P, P, P, 10, P, 1, 4, 3, 8, 128, None) == NULL
-    assert f(P, P, P, P, P, P, 10, P, 1, 4, -3, 8, 128, None) == SHAPE
-    assert f(P, P, P, P, P, P, 10, P, 1, 4, 3, 8, 100, None) == UNSUP
-    assert f(P + 8, P, P, P, P, P, 10, P, 1, 4, 3, 8, 128, None) == ALIGN
-    assert f(P, P, P, P, P, P, 10, P, 1, 4, 0, 8, 128, None) == OK
+    assert f(None, P, 1024, P, P, P, P, 10, P, 1, 4, 3, 8, 128, None) == NULL
+    assert f(P, P, 1024, P, P, P, P, 10, P, 1, 4, -3, 8, 128, None) == SHAPE
+    assert f(P, P, 1024, P, P, P, P, 10, P, 1, 4, 3, 8, 100, None) == UNSUP
+    assert f(P + 8, P, 1024, P, P, P, P, 10, P, 1, 4, 3, 8, 128, None) == ALIGN
+    assert f(P, P, 512, P, P, P, P, 10, P, 1, 4, 3, 8, 128, None) == SHAPE     # ld_new < Hkv*D
+    assert f(P, P, 1028, P, P, P, P, 10, P, 1, 4, 3, 8, 128, None) == ALIGN    # ld_new % 8
+    assert f(P, P, 1024, P, P, P, P, 10, P, 1, 4, 0, 8, 128, None) == OK
+
+
+def test_glue_validation(L):
+    assert L.bi_gather_rows(None, 2048, 10, P, 4, 2048, P, 2048, None) == NULL
+    assert L.bi_gather_rows(P, 2048, 10, P, 4, 2044, P, 2048, None) == SHAPE    # width % 8
+    assert L.bi_gather_rows(P, 2048, 0, P, 4, 2048, P, 2048, None) == SHAPE
+    assert L.bi_gather_rows(P + 2, 2048, 10, P, 4, 2048, P, 2048, None) == ALIGN
+    assert L.bi_gather_rows(P, 2048, 10, P, 0, 2048, P, 2048, None) == OK
+    assert L.bi_rope(None, 2048, 4, 32, 64, P, P, 384, None) == NULL
+    assert L.bi_rope(P, 2048, 4, 32, 63, P, P, 384, None) == SHAPE              # odd D
+    assert L.bi_rope(P, 1024, 4, 32, 64, P, P, 384, None) == SHAPE              # ldx < H*D
+    assert L.bi_rope(P, 2048, 0, 32, 64, P, P, 384, None) == OK
+    assert L.bi_swiglu(P, 16384, None, 8192, 4, 8192, None) == NULL
+    assert L.bi_swiglu(P, 16000, P, 8192, 4, 8192, None) == SHAPE               # ld_gu < 2F
+    assert L.bi_swiglu(P, 16384, P, 8192, 4, 8190, None) == SHAPE               # F % 8
+    assert L.bi_swiglu(P + 4, 16384, P, 8192, 4, 8192, None) == ALIGN
+    assert L.bi_swiglu(P, 16384, P, 8192, 0, 8192, None) == OK
+    assert L.bi_add(P, None, P, 64, None) == NULL
+    assert L.bi_add(P, P, P, 63, None) == SHAPE
+    assert L.bi_add(P, P + 8, P, 64, None) == ALIGN
+    assert L.bi_add(P, P, P, 0, None) == OK
 
 
 def test_lmhead_validation(L):

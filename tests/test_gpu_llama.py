@@ -1,0 +1,73 @@
+"""The random-init Llama-style decoder (16 layers, hidden 2048, 32/8 heads, SwiGLU
+8192, vocab 32000) on the batch-invariant kernels.
+
+* one decoder layer against the fp64 oracle (same bf16 input rows);
+* greedy streams of 64 prompts x 128 tokens, 256 generated tokens each, under random
+  mixed batching (batch size ~ U[1,64] per step, random subsets and order, random
+  prefill chunks mixed with decode tokens): every repeat must give the same stream
+  for every prompt, and the same stream as the prompt run alone (whole prompt, then
+  one token per step). BI_C5_REPEATS sets the number of mixed repeats
+  (default 2; the 1000-repeat run sets it to 1000). BI_C5_BASELINE_REPEATS > 0 also
+  runs the non-invariant torch path and reports its unique-stream count.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import TOL_BF16, dev, max_rel
+from llama_bi import BaselineLlama, BiLlama, run_repeats
+
+pytestmark = pytest.mark.gpu
+
+
+def test_decoder_layer_matches_oracle():
+    cfg = dict(layers=2, hidden=512, heads=8, kv_heads=2, head_dim=64, ffn=1024, vocab=1000, eps=1e-6, theta=10000.0)
+    w = synth.llama_weights(cfg, seed=11, device=dev())
+    model = BiLlama(cfg, w, n_seqs=2, max_pos=64, device=dev())
+    seqs = [0] * 40 + [1] * 25
+    poss = list(range(40)) + list(range(25))
+    toks = list(synth.prompts(1, 65, 1000, seed=12)[0])
+    h0 = model.hidden(seqs, poss, toks, n_layers=0)
+    h1 = model.hidden(seqs, poss, toks, n_layers=1)
+    lw = {k: synth.to_f64(v.cpu()) for k, v in w["layers"][0].items()}
+    ref = oracle.decoder_layer(synth.to_f64(h0.cpu()), seqs, poss, {}, {}, lw, cfg["heads"], cfg["kv_heads"])
+    assert max_rel(h1, ref) <= TOL_BF16
+
+
+def test_greedy_streams_identical_under_mixed_batching():
+    cfg = synth.LLAMA_CFG
+    repeats = int(os.environ.get("BI_C5_REPEATS", "2"))
+    base_repeats = int(os.environ.get("BI_C5_BASELINE_REPEATS", "0"))
+    w = synth.llama_weights(cfg, seed=0, device=dev())
+    prompts = synth.prompts(64, 128, cfg["vocab"], seed=0)
+    res = run_repeats(BiLlama, cfg, w, prompts, 256, repeats, dev())
+    report = {"repeats": repeats, "max_unique_streams_per_prompt": res["max_unique"],
+              "tokens_per_s": res["tokens_per_s"], "seconds": res["seconds"], "recompute_rate": res["recompute_rate"]}
+    # the same streams with one sequence at a time, whole prompt then token by token
+    solo = BiLlama(cfg, w, 64, 128 + 256, dev())
+    for s in (0, 17, 63):
+        toks = list(prompts[s])
+        out = []
+        t = int(solo.forward([s] * 128, list(range(128)), toks, [127])[0])
+        out.append(t)
+        for i in range(255):
+            t = int(solo.forward([s], [128 + i], [t], [0])[0])
+            out.append(t)
+        assert out == list(res["first"][s]), s
+    if base_repeats:
+        b = run_repeats(BaselineLlama, cfg, w, prompts, 256, base_repeats, dev())
+        report.update(baseline_repeats=base_repeats, baseline_max_unique=b["max_unique"],
+                      baseline_mean_unique=float(b["unique_per_seq"].mean()),
+                      baseline_tokens_per_s=b["tokens_per_s"],
+                      baseline_prompts_diverging=int((b["first"] != res["first"]).any(axis=1).sum()))
+    path = os.environ.get("BI_C5_REPORT")
+    if path:
+        with open(path, "w") as f:
+            json.dump(report, f)
+    print(json.dumps(report))
+    assert res["max_unique"] == 1

@@ -292,3 +292,62 @@ def test_normwise_rel_err():
     got = np.array([[2.0, -4.02, 1.01], [0.0, 1e-3, 0.0]])
     e = oracle.normwise_rel_err(got, ref)
     np.testing.assert_allclose(e, [0.02 / 4.0, 1e-3])
+
+
+# ---------------------------------------------------------------------------
+# Decoder glue: RoPE, SwiGLU, one decoder layer
+
+
+@pytest.mark.parametrize("case", _cases("rope"))
+def test_rope_golden(case):
+    out = oracle.rope(np.array(case["x"]), np.array(case["pos"]), case["theta"])
+    np.testing.assert_allclose(out, np.array(case["expected"]), rtol=0, atol=1e-13)
+
+
+def test_rope_identity_norms_and_composition():
+    x = synth.to_f64(synth.normal_bf16((5, 3, 64), 80))
+    np.testing.assert_array_equal(oracle.rope(x, np.zeros(5)), x)  # position 0: no rotation
+    pos = np.array([1, 7, 100, 383, 5000])
+    y = oracle.rope(x, pos)
+    pair = lambda z: np.hypot(z[..., :32], z[..., 32:])
+    np.testing.assert_allclose(pair(y), pair(x), rtol=1e-13)  # rotations keep each pair's length
+    np.testing.assert_allclose(oracle.rope(oracle.rope(x, pos), pos + 3), oracle.rope(x, 2 * pos + 3), atol=1e-10)
+    # the lowest frequency pair (i = D/2 - 1) turns by pos * theta^(-(D-2)/D)
+    ang = 100 * 10000.0 ** (-62 / 64)
+    z = np.zeros((1, 1, 64))
+    z[0, 0, 31] = 1.0
+    r = oracle.rope(z, np.array([100]))
+    assert abs(r[0, 0, 31] - math.cos(ang)) < 1e-15 and abs(r[0, 0, 63] - math.sin(ang)) < 1e-15
+
+
+@pytest.mark.parametrize("case", _cases("swiglu"))
+def test_swiglu_golden(case):
+    np.testing.assert_allclose(oracle.swiglu(np.array(case["gate_up"])), np.array(case["expected"]), rtol=1e-15)
+
+
+def test_silu_limits():
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    assert abs(oracle.silu(np.array([40.0]))[0] - 40.0) < 1e-15
+    assert abs(oracle.silu(np.array([-40.0]))[0]) < 1e-15
+
+
+def test_decoder_layer_structure():
+    # With wo = wdown = 0 the layer is the identity on h; with one kv head and
+    # identical keys the attention output is the mean of the values.
+    rng = np.random.default_rng(3)
+    Hd, nh, nkv, F = 16, 4, 2, 24
+    D = Hd // nh
+    w = dict(wqkv=rng.normal(0, 0.2, ((nh + 2 * nkv) * D, Hd)), wo=np.zeros((Hd, Hd)),
+             wgu=rng.normal(0, 0.2, (2 * F, Hd)), wdown=np.zeros((Hd, F)), attn_norm=np.ones(Hd),
+             mlp_norm=np.ones(Hd))
+    h = rng.normal(size=(3, Hd))
+    out = oracle.decoder_layer(h, [0, 0, 1], [0, 1, 0], {}, {}, w, nh, nkv)
+    np.testing.assert_array_equal(out, h)
+    # a row that sees only itself: attention returns its own value vector, so with
+    # wo = I the update is exactly v (rotation does not touch v)
+    w2 = dict(w, wo=np.eye(Hd))
+    out2 = oracle.decoder_layer(h[:1], [0], [0], {}, {}, w2, nh, nkv)
+    x = oracle.rmsnorm(h[:1], w["attn_norm"], 1e-6)
+    v = oracle.matmul(x, w["wqkv"])[:, (nh + nkv) * D:].reshape(1, nkv, D)
+    expect = h[:1] + np.repeat(v, nh // nkv, axis=1).reshape(1, Hd)
+    np.testing.assert_allclose(out2, expect, rtol=1e-13, atol=1e-13)
