@@ -111,82 +111,87 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int32_t* __restrict
 
 // fp32 logits of flagged rows: out[row, v] = sum_k h[row, k] * W[v, k], one FMA
 // chain in ascending k per logit (the packed f32x2 FMA below carries two logits of
-// two vocabulary entries, each element rounded exactly like a scalar FMA). Tile:
-// 32 flagged rows x 256 vocabulary rows, k staged 32 at a time through shared
-// memory (the next slab is prefetched into registers while the current one is
-// consumed); each thread owns 4 rows x 8 vocabulary entries.
-constexpr int RB = 32, VB = 256, KB = 32;
+// two vocabulary entries, each element rounded exactly like a scalar FMA).
+// Tile: 64 flagged rows x 256 vocabulary rows per CTA of 8 warps; warp w owns rows
+// 8w .. 8w+7 and lane l the vocabulary entries 4l .. 4l+3 and 128+4l .. 128+4l+3
+// (8 x 8 logits per thread). k is staged KB at a time through shared memory: W
+// transposed to [k][vocab], h as duplicated pairs [k][row] (one 16-byte load gives
+// two rows ready for the packed FMA); a warp's staging stores cover one k-row, so
+// they are free of bank conflicts, and the next slab is prefetched into registers
+// while the current one is consumed.
+constexpr int RB = 64, VB = 256, KB = 16;
 
 __global__ void __launch_bounds__(256) recompute_kernel(const uint16_t* __restrict__ h, int64_t ldh,
                                                         const uint16_t* __restrict__ W, int64_t V, int K, int M,
                                                         const int32_t* __restrict__ list,
                                                         float* __restrict__ out) {
-  __shared__ __align__(16) float hs[KB][RB];
-  __shared__ __align__(16) float ws[KB][VB + 4];
+  __shared__ __align__(16) float2 hs[KB][RB];  // (h, h) per row
+  __shared__ __align__(16) float ws[KB][VB];
   const int count = list[M];
   const int f0 = blockIdx.y * RB;
   if (f0 >= count) return;
   const int64_t v0 = (int64_t)blockIdx.x * VB;
-  const int tid = threadIdx.x;
-  const int tx = tid & 31, ty = tid >> 5;  // vocab 8*tx.., rows 4*ty..
-  float2 acc[4][4];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float2 acc[8][4];  // [row][vocab pair]
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
 
-  // staging of one k-slab: each thread loads 1 h value (32 x 32) and 4 x 8 W values
-  const int hr = tid >> 3, hk = (tid & 7) * 4;  // h: row hr, k hk..hk+3
-  const int hf = f0 + hr;
-  const bool hvalid = hf < count;
-  const uint16_t* hsrc = h + (int64_t)(hvalid ? list[hf] : 0) * ldh;
-  auto load = [&](int k0, float (&hv)[4], uint4 (&wv)[4]) {
-    const uint2 hp = __ldg(reinterpret_cast<const uint2*>(hsrc + k0 + hk));
-    hv[0] = hvalid ? bf16lo(hp.x) : 0.f;
-    hv[1] = hvalid ? bf16hi(hp.x) : 0.f;
-    hv[2] = hvalid ? bf16lo(hp.y) : 0.f;
-    hv[3] = hvalid ? bf16hi(hp.y) : 0.f;
+  // staging: W slab 256 vocab x KB k = 512 vectors of 8 (vocab = e % 256, k-half = e / 256);
+  //          h slab 64 rows x KB k = 128 vectors of 8 (row = e % 64, k-half = e / 64), threads < 128
+  const int hrow = tid & 63, hk = (tid >> 6) & 1;
+  const bool hload = tid < 128 && f0 + hrow < count;
+  const uint16_t* hsrc = h + (int64_t)(hload ? list[f0 + hrow] : 0) * ldh + hk * 8;
+  auto load = [&](int k0, uint4& hv, uint4 (&wv)[2]) {
+    hv = hload ? __ldg(reinterpret_cast<const uint4*>(hsrc + k0)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int e = tid + r * 256;  // 1024 vectors of 8 bf16: vocab e / 4, k-quarter e % 4
-      const int64_t vv = v0 + (e >> 2);
-      wv[r] = vv < V ? __ldg(reinterpret_cast<const uint4*>(W + vv * K + k0) + (e & 3)) : make_uint4(0, 0, 0, 0);
+    for (int r = 0; r < 2; ++r) {
+      const int e = tid + r * 256;
+      const int64_t vv = v0 + (e & 255);
+      wv[r] = vv < V ? __ldg(reinterpret_cast<const uint4*>(W + vv * K + k0 + (e >> 8) * 8))
+                     : make_uint4(0, 0, 0, 0);
     }
   };
-  auto store = [&](const float (&hv)[4], const uint4 (&wv)[4]) {
+  auto store = [&](const uint4& hv, const uint4 (&wv)[2]) {
+    float f[8];
+    if (tid < 128) {
+      unpack8(hv, f);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) hs[hk + e][hr] = hv[e];
+      for (int i = 0; i < 8; ++i) hs[hk * 8 + i][hrow] = make_float2(f[i], f[i]);
+    }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < 2; ++r) {
       const int e = tid + r * 256;
-      float f[8];
       unpack8(wv[r], f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ws[(e & 3) * 8 + i][e >> 2] = f[i];
+      for (int i = 0; i < 8; ++i) ws[(e >> 8) * 8 + i][e & 255] = f[i];
     }
   };
-  float hv[4];
-  uint4 wv[4];
+  uint4 hv, wv[2];
   load(0, hv, wv);
   store(hv, wv);
   __syncthreads();
   for (int k0 = 0; k0 < K; k0 += KB) {
     const bool more = k0 + KB < K;
     if (more) load(k0 + KB, hv, wv);
-#pragma unroll 8
+#pragma unroll
     for (int kk = 0; kk < KB; ++kk) {
-      const float4 h4 = *reinterpret_cast<const float4*>(&hs[kk][ty * 4]);
-      const float4 wa = *reinterpret_cast<const float4*>(&ws[kk][tx * 8]);
-      const float4 wb = *reinterpret_cast<const float4*>(&ws[kk][tx * 8 + 4]);
-      const float hr4[4] = {h4.x, h4.y, h4.z, h4.w};
+      float2 h2[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 t = *reinterpret_cast<const float4*>(&hs[kk][warp * 8 + 2 * i]);
+        h2[2 * i] = make_float2(t.x, t.y);
+        h2[2 * i + 1] = make_float2(t.z, t.w);
+      }
+      const float4 wa = *reinterpret_cast<const float4*>(&ws[kk][lane * 4]);
+      const float4 wb = *reinterpret_cast<const float4*>(&ws[kk][128 + lane * 4]);
       const float2 w2[4] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w), make_float2(wb.x, wb.y),
                             make_float2(wb.z, wb.w)};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 h2 = make_float2(hr4[i], hr4[i]);
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = __ffma2_rn(h2, w2[j], acc[i][j]);
-      }
+        for (int j = 0; j < 4; ++j) acc[i][j] = __ffma2_rn(h2[i], w2[j], acc[i][j]);
     }
     __syncthreads();
     if (more) {
@@ -195,13 +200,13 @@ __global__ void __launch_bounds__(256) recompute_kernel(const uint16_t* __restri
     }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int f = f0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int f = f0 + warp * 8 + i;
     if (f >= count) continue;
     float* dst = out + (int64_t)list[f] * V;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int64_t v = v0 + tx * 8 + 2 * j;
+      const int64_t v = v0 + (j < 2 ? lane * 4 + 2 * j : 128 + lane * 4 + 2 * (j - 2));
       if (v < V) dst[v] = acc[i][j].x;
       if (v + 1 < V) dst[v + 1] = acc[i][j].y;
     }

@@ -211,3 +211,100 @@ def run_repeats(model_cls, cfg, weights, prompts, gen_len, repeats, device, seed
     uniq = np.array([len(d) for d in seen])
     return dict(unique_per_seq=uniq, max_unique=int(uniq.max()), first=first, tokens_per_s=tokens / t_total,
                 seconds=t_total, recompute_rate=(model.recomputed / model.lm_rows) if model.lm_rows else None)
+
+
+class FastBiLlama(BiLlama):
+    """BiLlama with preallocated buffers and direct C-ABI calls (raw pointers, no
+    per-call tensor checks): the same kernels and arguments, less host overhead."""
+
+    def __init__(self, cfg, weights, n_seqs, max_pos, device, threshold=0.5, max_rows=8192, max_want=64):
+        super().__init__(cfg, weights, n_seqs, max_pos, device, threshold)
+        c = cfg
+        H, nh, nkv, D, F, V = (c[k] for k in ("hidden", "heads", "kv_heads", "head_dim", "ffn", "vocab"))
+        self.L = bi.lib()
+        e = lambda *shape: torch.empty(shape, dtype=torch.bfloat16, device=device)
+        self.h, self.x, self.o = e(max_rows, H), e(max_rows, H), e(max_rows, H)
+        self.qkv, self.att = e(max_rows, (nh + 2 * nkv) * D), e(max_rows, nh * D)
+        self.gu, self.a = e(max_rows, 2 * F), e(max_rows, F)
+        self.meta = torch.empty((3, max_rows), dtype=torch.int32, device=device)
+        # ring of pinned staging buffers; a buffer is refilled only after its last copy completed
+        self.meta_host = [torch.empty((3, max_rows), dtype=torch.int32).pin_memory() for _ in range(4)]
+        self.meta_ev = [torch.cuda.Event() for _ in range(4)]
+        self.meta_i = 0
+        self.sel = torch.empty(max_want, dtype=torch.int32, device=device)
+        self.hs, self.hn = e(max_want, H), e(max_want, H)
+        self.tok = torch.empty(max_want, dtype=torch.int32, device=device)
+        self.rec = torch.empty(max_want, dtype=torch.int32, device=device)
+        self.ws_att = torch.empty(bi.attention_workspace_size(max_rows, nh, D, self.store.max_pages),
+                                  dtype=torch.uint8, device=device)
+        self.ws_lm = torch.empty(bi.lmhead_workspace_size(max_want, V), dtype=torch.uint8, device=device)
+        self.max_rows, self.max_want = max_rows, max_want
+
+    def _ok(self, name, status):
+        if status != 0:
+            raise bi.BIError(name, status)
+
+    def hidden(self, seqs, poss, toks, n_layers=None):
+        c, w, st, L = self.cfg, self.w, self.store, self.L
+        H, nh, nkv, D, F = (c[k] for k in ("hidden", "heads", "kv_heads", "head_dim", "ffn"))
+        T = len(toks)
+        assert T <= self.max_rows
+        s = torch.cuda.current_stream().cuda_stream
+        i = self.meta_i = (self.meta_i + 1) % len(self.meta_host)
+        mh = self.meta_host[i]
+        self.meta_ev[i].synchronize()
+        mh[0, :T] = torch.from_numpy(np.asarray(seqs, dtype=np.int32))
+        mh[1, :T] = torch.from_numpy(np.asarray(poss, dtype=np.int32))
+        mh[2, :T] = torch.from_numpy(np.asarray(toks, dtype=np.int32))
+        self.meta[:, :T].copy_(mh[:, :T], non_blocking=True)
+        self.meta_ev[i].record()
+        mp = self.meta.data_ptr()
+        q_seq, q_pos, ids = mp, mp + 4 * self.max_rows, mp + 8 * self.max_rows
+        QKV = (nh + 2 * nkv) * D
+        h, x, o, qkv, att, gu, a = (t.data_ptr() for t in (self.h, self.x, self.o, self.qkv, self.att, self.gu, self.a))
+        E = w["embed"]
+        self._ok("gather", L.bi_gather_rows(E.data_ptr(), H, E.shape[0], ids, T, H, h, H, s))
+        npages, maxp, pt = st.k[0].shape[0], st.max_pages, st.page_table.data_ptr()
+        tab = self.table.data_ptr()
+        scale = 1.0 / math.sqrt(D)
+        ws, wsb = self.ws_att.data_ptr(), self.ws_att.numel()
+        n_seqs = st.page_table.shape[0]
+        for l, lw in enumerate(w["layers"][:n_layers]):
+            kc, vc = st.k[l].data_ptr(), st.v[l].data_ptr()
+            self._ok("rmsnorm", L.bi_rmsnorm(h, H, lw["attn_norm"].data_ptr(), x, H, T, H, c["eps"], s))
+            self._ok("qkv", L.bi_matmul(x, H, lw["wqkv"].data_ptr(), H, qkv, QKV, T, QKV, H, s))
+            self._ok("rope q", L.bi_rope(qkv, QKV, T, nh, D, q_pos, tab, self.table.shape[0], s))
+            self._ok("rope k", L.bi_rope(qkv + 2 * nh * D, QKV, T, nkv, D, q_pos, tab, self.table.shape[0], s))
+            self._ok("append", L.bi_kv_append(qkv + 2 * nh * D, qkv + 2 * (nh + nkv) * D, QKV, q_seq, q_pos, kc, vc,
+                                              npages, pt, n_seqs, maxp, T, nkv, D, s))
+            self._ok("attn", L.bi_attention_prefill(qkv, QKV, q_seq, q_pos, kc, vc, npages, pt, n_seqs, maxp, att, T,
+                                                    nh, nkv, D, scale, ws, wsb, s))
+            self._ok("o", L.bi_matmul(att, nh * D, lw["wo"].data_ptr(), nh * D, o, H, T, H, nh * D, s))
+            self._ok("add", L.bi_add(h, o, h, T * H, s))
+            self._ok("rmsnorm", L.bi_rmsnorm(h, H, lw["mlp_norm"].data_ptr(), x, H, T, H, c["eps"], s))
+            self._ok("gu", L.bi_matmul(x, H, lw["wgu"].data_ptr(), H, gu, 2 * F, T, 2 * F, H, s))
+            self._ok("swiglu", L.bi_swiglu(gu, 2 * F, a, F, T, F, s))
+            self._ok("down", L.bi_matmul(a, F, lw["wdown"].data_ptr(), F, o, H, T, H, F, s))
+            self._ok("add", L.bi_add(h, o, h, T * H, s))
+        return self.h[:T]
+
+    def forward(self, seqs, poss, toks, want):
+        c, w, L = self.cfg, self.w, self.L
+        H, V = c["hidden"], c["vocab"]
+        self.hidden(seqs, poss, toks)
+        n = len(want)
+        if n == 0:
+            return np.zeros(0, dtype=np.int64)
+        s = torch.cuda.current_stream().cuda_stream
+        self.sel[:n].copy_(torch.from_numpy(np.asarray(want, dtype=np.int32)), non_blocking=True)
+        self._ok("select", L.bi_gather_rows(self.h.data_ptr(), H, len(toks), self.sel.data_ptr(), n, H,
+                                            self.hs.data_ptr(), H, s))
+        self._ok("final norm", L.bi_rmsnorm(self.hs.data_ptr(), H, w["final_norm"].data_ptr(), self.hn.data_ptr(), H,
+                                            n, H, c["eps"], s))
+        self._ok("lm head", L.bi_lmhead_argmax(self.hn.data_ptr(), H, w["lm_head"].data_ptr(), n, V, H, self.threshold,
+                                               self.tok.data_ptr(), self.rec.data_ptr(), None,
+                                               self.ws_lm.data_ptr(), self.ws_lm.numel(), s))
+        out = self.tok[:n].cpu().numpy()
+        self.recomputed += int(self.rec[:n].sum())
+        self.lm_rows += n
+        return out

@@ -20,7 +20,7 @@ import torch
 import oracle
 import synth
 from gpu_util import TOL_BF16, dev, max_rel
-from llama_bi import BaselineLlama, BiLlama, run_repeats
+from llama_bi import BaselineLlama, BiLlama, FastBiLlama, run_repeats
 
 pytestmark = pytest.mark.gpu
 
@@ -45,10 +45,11 @@ def test_greedy_streams_identical_under_mixed_batching():
     base_repeats = int(os.environ.get("BI_C5_BASELINE_REPEATS", "0"))
     w = synth.llama_weights(cfg, seed=0, device=dev())
     prompts = synth.prompts(64, 128, cfg["vocab"], seed=0)
-    res = run_repeats(BiLlama, cfg, w, prompts, 256, repeats, dev())
+    res = run_repeats(FastBiLlama, cfg, w, prompts, 256, repeats, dev())
     report = {"repeats": repeats, "max_unique_streams_per_prompt": res["max_unique"],
               "tokens_per_s": res["tokens_per_s"], "seconds": res["seconds"], "recompute_rate": res["recompute_rate"]}
-    # the same streams with one sequence at a time, whole prompt then token by token
+    # the same streams with one sequence at a time, whole prompt then token by token,
+    # through the checked binding (BiLlama) rather than the direct-call path
     solo = BiLlama(cfg, w, 64, 128 + 256, dev())
     for s in (0, 17, 63):
         toks = list(prompts[s])
