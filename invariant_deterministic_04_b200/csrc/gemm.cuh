@@ -32,13 +32,9 @@
 namespace bi {
 namespace gemm {
 
-#ifndef BI_GEMM_TILE_N
-#define BI_GEMM_TILE_N 256
-#endif
-constexpr int BM = 128, BN = BI_GEMM_TILE_N, BK = 64;
-constexpr int STAGES = BN >= 256 ? 4 : 6;  // ~192 KiB of operand ring either way
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KiB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KiB at BN = 256
+constexpr int B_BYTES = BN * BK * 2;  // 32 KiB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;  // two fp32 accumulators
 constexpr int kThreads = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
