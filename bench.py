@@ -38,6 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 import torch.distributed as dist  # noqa: E402
 
@@ -324,6 +325,25 @@ def _row_decode(bi, device, pk):
     gbs = kv_bytes / ms / 1e6
     out["decode_b64_l32k"] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3), "ms": round(ms, 4),
                               "kv_bytes": kv_bytes}
+    # non-invariant comparison: flashinfer's paged decode with its own split-KV heuristic, same store
+    try:
+        import flashinfer
+
+        npages = [(int(L) + 15) // 16 for L in lens.tolist()]
+        indptr = torch.tensor([0] + list(np.cumsum(npages)), dtype=torch.int32, device=device)
+        indices = torch.cat([kv.page_table[b, :n] for b, n in enumerate(npages)]).contiguous()
+        last = torch.tensor([(int(L) - 1) % 16 + 1 for L in lens.tolist()], dtype=torch.int32, device=device)
+        fws = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        wrapper = flashinfer.BatchDecodeWithPagedKVCacheWrapper(fws, kv_layout="HND")
+        wrapper.plan(indptr, indices, last, 32, 8, 128, 16, q_data_type=torch.bfloat16, kv_data_type=torch.bfloat16)
+        fo = wrapper.run(q, (kv.k_cache, kv.v_cache))
+        ms_ref = _events_ms(lambda: wrapper.run(q, (kv.k_cache, kv.v_cache)))
+        err = float(((fo.float() - o.float()).abs().max() / o.float().abs().max()).item())
+        out["decode_b64_l32k"].update({"flashinfer_ms": round(ms_ref, 4), "slowdown_vs_flashinfer": round(ms / ms_ref, 3),
+                                       "flashinfer_GB/s": round(kv_bytes / ms_ref / 1e6, 1),
+                                       "max_rel_diff_vs_flashinfer": round(err, 5)})
+    except Exception as e:  # the comparison path is optional
+        out["decode_b64_l32k"]["flashinfer"] = f"unavailable: {type(e).__name__}: {str(e)[:120]}"
     return out
 
 
@@ -343,6 +363,18 @@ def _row_prefill(bi, device, pk):
     alu_peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
     out["prefill_s4096"] = {"TFLOP/s": round(flops / ms / 1e9, 2), "frac_fp32_alu": round(flops / ms / 1e9 / alu_peak, 3),
                             "ms": round(ms, 3)}
+    # non-invariant comparison: torch SDPA (flash, tensor cores) on the same K/V laid out contiguously
+    try:
+        t = torch.arange(S, device=device)
+        pages = kvp.page_table[0, t // 16].long()
+        kc = kvp.k_cache[pages, :, t % 16, :].permute(1, 0, 2).unsqueeze(0)  # [1, 8, S, D]
+        vc = kvp.v_cache[pages, :, t % 16, :].permute(1, 0, 2).unsqueeze(0)
+        qs4 = qp.permute(1, 0, 2).unsqueeze(0)  # [1, 32, S, D]
+        sdpa = torch.nn.functional.scaled_dot_product_attention
+        ms_ref = _events_ms(lambda: sdpa(qs4, kc, vc, is_causal=True, enable_gqa=True), iters=10, warmup=2)
+        out["prefill_s4096"].update({"sdpa_ms": round(ms_ref, 4), "slowdown_vs_sdpa": round(ms / ms_ref, 2)})
+    except Exception as e:
+        out["prefill_s4096"]["sdpa"] = f"unavailable: {type(e).__name__}: {str(e)[:120]}"
     return out
 
 

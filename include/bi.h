@@ -244,6 +244,16 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
                            void* stream);
 
 /*
+ * Self-test of the device-side failure detection (no page describes it). Launches
+ * one thread that waits on an mbarrier nothing will complete, using the same
+ * bounded wait as every kernel here but a limit of limit_ms milliseconds (1..2000;
+ * the kernels use 2000). When the limit expires the kernel records
+ * BI_ERR_DEVICE_TIMEOUT in the device error word and returns, so the context stays
+ * usable. Returns BI_ERR_SHAPE for a limit outside 1..2000.
+ */
+bi_status bi_selftest_wait_timeout(int limit_ms, void* stream);
+
+/*
  * Reads and clears the device error word of the current device (synchronises the
  * device first). *code receives BI_OK, BI_ERR_DEVICE_TIMEOUT or
  * BI_ERR_DEVICE_INDEX (the first error recorded since the last read). Returns

@@ -54,6 +54,7 @@ _SIGNATURES = {
     "bi_lmhead_workspace_size": ([_I64, _I64], _SZ),
     "bi_lmhead_argmax": ([_P, _I64, _P, _I64, _I64, _I64, _F, _P, _P, _P, _P, _SZ, _P], _I32),
     "bi_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], _I32),
+    "bi_selftest_wait_timeout": ([_I32, _P], _I32),
 }
 
 _lib = None
@@ -350,6 +351,11 @@ def lmhead_argmax(h, w, margin_threshold: float = 0.5, want_logits: bool = False
         _ptr(h), h.stride(0), _ptr(w), M, V, K, margin_threshold, _ptr(tokens), _ptr(recomputed),
         _ptr(logits_fp32), _ptr(ws), nbytes, _stream(stream)))
     return tokens, recomputed, logits_fp32
+
+
+def selftest_wait_timeout(limit_ms: int = 50, stream=None):
+    """Launch a kernel whose bounded wait is made to expire (records BI_ERR_DEVICE_TIMEOUT)."""
+    _check("bi_selftest_wait_timeout", lib().bi_selftest_wait_timeout(limit_ms, _stream(stream)))
 
 
 def get_device_error() -> int:

@@ -111,15 +111,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Waits for the phase with the given parity to complete. Returns false (and
-// records BI_ERR_DEVICE_TIMEOUT) if it does not within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// records BI_ERR_DEVICE_TIMEOUT) if it does not within limit_ns (kWaitLimitNs).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       record_error(BI_ERR_DEVICE_TIMEOUT);
       return false;
     }
@@ -223,5 +223,15 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 }
 
 constexpr unsigned kFullMask = 0xFFFFFFFFu;
+
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// completes; the wait gives up after limit_ns and records BI_ERR_DEVICE_TIMEOUT.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_mbar_init();
+  mbar_wait(b, 0, limit_ns);
+}
 
 }  // namespace bi

@@ -366,6 +366,12 @@ bi_status bi_add(const bi_bf16* a, const bi_bf16* b, bi_bf16* out, int64_t n, vo
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
+bi_status bi_selftest_wait_timeout(int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return BI_ERR_SHAPE;
+  bi::selftest_wait_kernel<<<1, 1, 0, as_stream(stream)>>>((uint64_t)limit_ms * 1000000ull);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
 bi_status bi_get_device_error(int32_t* code) {
   if (!code) return BI_ERR_NULL;
   if (cudaDeviceSynchronize() != cudaSuccess) return BI_ERR_CUDA;

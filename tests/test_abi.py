@@ -170,3 +170,8 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mod, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         mod.lib()
+
+
+def test_selftest_validation(L):
+    assert L.bi_selftest_wait_timeout(0, None) == SHAPE
+    assert L.bi_selftest_wait_timeout(2001, None) == SHAPE

@@ -156,6 +156,17 @@ def test_device_index_errors_are_reported_not_faulted():
     assert bi.get_device_error() == 0
 
 
+def test_bounded_wait_expires_with_status_and_context_stays_usable():
+    # a wait on an mbarrier that nothing completes gives up after 50 ms
+    assert bi.get_device_error() == 0
+    bi.selftest_wait_timeout(50)
+    assert bi.get_device_error() == 7  # BI_ERR_DEVICE_TIMEOUT
+    q, kv = synth.decode_inputs(2, 32, 8, 128, max_len=300, seed=45, lens=[300, 17])
+    out = _decode(q.to(dev()), _to_dev(kv))
+    assert max_rel(out, _oracle_decode(q, kv)) <= TOL_BF16
+    assert bi.get_device_error() == 0
+
+
 # ---------------------------------------------------------------------------
 # Full-size configurations (sampled oracle rows)
 
