@@ -363,6 +363,15 @@ def _row_prefill(bi, device, pk):
     alu_peak = 148 * 128 * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
     out["prefill_s4096"] = {"TFLOP/s": round(flops / ms / 1e9, 2), "frac_fp32_alu": round(flops / ms / 1e9 / alu_peak, 3),
                             "ms": round(ms, 3)}
+    # the tensor-core prefill (same whole/chunked invariance, different fixed arithmetic)
+    try:
+        otc = torch.empty_like(qp)
+        ms_tc = _events_ms(lambda: bi.attention_prefill_tc(qp, 0, 0, kvp.k_cache, kvp.v_cache, kvp.page_table, out=otc),
+                           iters=10, warmup=2)
+        out["prefill_s4096"].update({"tc_ms": round(ms_tc, 4), "tc_TFLOP/s": round(flops / ms_tc / 1e9, 1),
+                                     "tc_frac_bf16_tensor": round(flops / ms_tc / 1e9 / pk["bf16_tflops"], 3)})
+    except Exception as e:
+        out["prefill_s4096"]["tc"] = f"unavailable: {type(e).__name__}: {str(e)[:120]}"
     # non-invariant comparison: torch SDPA (flash, tensor cores) on the same K/V laid out contiguously
     try:
         t = torch.arange(S, device=device)
@@ -373,6 +382,8 @@ def _row_prefill(bi, device, pk):
         sdpa = torch.nn.functional.scaled_dot_product_attention
         ms_ref = _events_ms(lambda: sdpa(qs4, kc, vc, is_causal=True, enable_gqa=True), iters=10, warmup=2)
         out["prefill_s4096"].update({"sdpa_ms": round(ms_ref, 4), "slowdown_vs_sdpa": round(ms / ms_ref, 2)})
+        if "tc_ms" in out["prefill_s4096"]:
+            out["prefill_s4096"]["tc_slowdown_vs_sdpa"] = round(out["prefill_s4096"]["tc_ms"] / ms_ref, 2)
     except Exception as e:
         out["prefill_s4096"]["sdpa"] = f"unavailable: {type(e).__name__}: {str(e)[:120]}"
     return out

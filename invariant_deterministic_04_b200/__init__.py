@@ -46,6 +46,8 @@ _SIGNATURES = {
     "bi_attention_decode_static": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P], _I32),
     "bi_attention_prefill": ([_P, _I64, _P, _P, _P, _P, _I64, _P, _I32, _I32, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ,
                               _P], _I32),
+    "bi_attention_prefill_tc": ([_P, _I64, _I32, _I32, _I32, _P, _P, _I64, _P, _I32, _I32, _P, _I32, _I32, _I32, _F,
+                                 _P], _I32),
     "bi_kv_append": ([_P, _P, _I64, _P, _P, _P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P], _I32),
     "bi_gather_rows": ([_P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P], _I32),
     "bi_rope": ([_P, _I64, _I64, _I32, _I32, _P, _P, _I32, _P], _I32),
@@ -247,6 +249,29 @@ def attention_prefill(q, q_seq, q_pos, k_cache, v_cache, page_table, scale: floa
     _check("bi_attention_prefill", lib().bi_attention_prefill(
         _ptr(q), ldq, _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table),
         num_seqs, maxp, _ptr(out), T, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def attention_prefill_tc(q, seq: int, pos0: int, k_cache, v_cache, page_table, scale: float | None = None, out=None,
+                         stream=None):
+    """Causal prefill of positions pos0 .. pos0+T-1 of one sequence on tensor cores (q [T, Hq, D])."""
+    _req(q, torch.bfloat16, "q", 3)
+    _req(k_cache, torch.bfloat16, "k_cache", 4)
+    _req(v_cache, torch.bfloat16, "v_cache", 4)
+    _req(page_table, torch.int32, "page_table", 2)
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (page_table, "page_table")):
+        _contig(t, n)
+    ldq = _rows3(q, "q")
+    T, Hq, D = q.shape
+    num_pages, Hkv = k_cache.shape[0], k_cache.shape[1]
+    if k_cache.shape != v_cache.shape or k_cache.shape[2] != PAGE_TOKENS or k_cache.shape[3] != D:
+        raise ValueError("k_cache/v_cache must be [num_pages, Hkv, 16, D]")
+    num_seqs, maxp = page_table.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=q.device) if out is None else out
+    _check("bi_attention_prefill_tc", lib().bi_attention_prefill_tc(
+        _ptr(q), ldq, seq, pos0, T, _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), num_seqs, maxp,
+        _ptr(out), Hq, Hkv, D, scale, _stream(stream)))
     return out
 
 

@@ -1,0 +1,391 @@
+// Causal prefill attention on 5th-generation tensor cores, batch- and chunk-invariant.
+//
+// Source: "Defeating Nondeterminism in LLM Inference" technical summary
+// (mobiles-han blog), section 対応策：バッチ不変なカーネル設計, kernel table, row
+// Attention (one layout for cache and chunk; a schedule that does not depend on the
+// chunking), and the French article's "Le prix d'une sortie bit à bit identique"
+// section (a faster attention kernel recovers most of the cost: 55 s -> 42 s).
+//
+// One chunk of one sequence: query rows at positions pos0 .. pos0 + T - 1, keys
+// 0 .. pos from the paged store (the chunk's own K/V already appended).
+// Per-row schedule, a function of the row's position only:
+//   * keys are processed in blocks of 128 at absolute positions 0, 128, 256, ...,
+//     in ascending order, up to the block holding the row's position;
+//   * S = q . k for a block by tcgen05.mma (bf16 x bf16, fp32 accumulation over D in
+//     ascending 16-wide steps), masked to keys <= pos, scaled by scale*log2(e);
+//   * online softmax in fp32 by the thread that owns the row: block max, then
+//     m = max(m, block max), l = l * 2^(m_old - m) + sum_j p_j (keys in order),
+//     O rescaled by 2^(m_old - m) only when m moved (x * 1 == x exactly);
+//   * p rounded to bf16, O += P V by tcgen05.mma (fp32, ascending 16-key steps);
+//   * out = O / l rounded to bf16.
+// The tensor core's result for an output element depends on that element's row and
+// column operands and the fixed K order only, not on the other rows of the tile or
+// the tile shape (checked on this hardware by the matmul tests), and a block with
+// no visible key leaves a row's state unchanged; so a row's bits do not depend on
+// how the sequence was chunked or which other rows shared its tile.
+#pragma once
+
+#include "device.cuh"
+
+namespace bi {
+namespace attn_tc {
+
+constexpr int PAGE = BI_PAGE_TOKENS;
+constexpr int KB = 128;                 // keys per block
+constexpr int PAGES_PER_BLOCK = KB / PAGE;
+constexpr int ROWS = 128;               // query rows per tile
+constexpr int kThreads = 192;           // warp 0 TMA, warp 1 MMA, warps 2..5 softmax (one row per thread)
+
+template <int D>
+struct Cfg {
+  static constexpr int HALVES = D / 64;                       // 64-dim (128-byte) halves
+  static constexpr int Q_BYTES = ROWS * D * 2;                // Q tile
+  static constexpr int KV_HALF = KB * 128;                    // one 64-dim half of a 128-key block
+  static constexpr int K_BYTES = HALVES * KV_HALF;
+  static constexpr int STAGE = 2 * K_BYTES;                   // K and V of one block
+  static constexpr int P_BYTES = ROWS * KB * 2;               // P tile (bf16), two 64-key halves
+  static constexpr int STAGES = 2;
+  static constexpr int SMEM = 1024 + Q_BYTES + STAGES * STAGE + P_BYTES + 256;
+  static constexpr int TMEM_COLS = 256;                       // S: 128 cols, O: D cols
+};
+
+// Instruction descriptors (kind::f16, bf16 inputs, fp32 accumulate, M = 128).
+// S = Q K^T: A = Q K-major, B = K K-major, N = 128 keys.
+constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(KB >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+// O += P V: A = P K-major (keys contiguous), B = V MN-major (dims contiguous), N = D.
+template <int D>
+__host__ __device__ constexpr uint32_t idesc_pv() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// K-major, 128-byte swizzle: 128-byte rows, 8-row atoms 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// MN-major, 128-byte swizzle: 64 MN elements per 128-byte row, K rows 128 bytes
+// apart, 8-K-row groups 1024 bytes apart (SBO), 64-element MN chunks lbo bytes apart.
+__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Tiles: (q-head h, row block rb); heavier row blocks (more key blocks) first.
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ page_row,
+                      int64_t num_pages, int Hq, int Hkv, int pos0, int T, int pages_avail,
+                      uint16_t* __restrict__ out, float c) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t q_s = base;
+  const uint32_t kv_s = base + C::Q_BYTES;           // stage s: K at kv_s + s*STAGE, V at + K_BYTES
+  const uint32_t p_s = kv_s + C::STAGES * C::STAGE;
+  const uint32_t bar0 = p_s + C::P_BYTES;
+  // barriers
+  const uint32_t Q_FULL = bar0, Q_EMPTY = bar0 + 8;
+  auto KV_FULL = [&](int s) { return bar0 + 16 + 16 * s; };
+  auto KV_EMPTY = [&](int s) { return bar0 + 24 + 16 * s; };
+  const uint32_t S_FULL = bar0 + 16 + 16 * C::STAGES, S_EMPTY = S_FULL + 8, P_FULL = S_FULL + 16, O_DONE = S_FULL + 24,
+                 O_FREE = S_FULL + 32;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (bar0 - base) + 16 + 16 * C::STAGES + 48);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rblocks = (T + ROWS - 1) / ROWS;
+  const int tiles = rblocks * Hq;
+  const int G = Hq / Hkv;
+
+  if (threadIdx.x == 0) {
+    mbar_init(Q_FULL, 1);
+    mbar_init(Q_EMPTY, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(KV_FULL(s), 1);
+      mbar_init(KV_EMPTY(s), 1);
+    }
+    mbar_init(S_FULL, 1);
+    mbar_init(S_EMPTY, 128);
+    mbar_init(P_FULL, 128);
+    mbar_init(O_DONE, 1);
+    mbar_init(O_FREE, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    prefetch_tensormap(&tmQ);
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + KB;
+
+  // tile t -> (head, row block): row blocks from the last (heaviest) to the first
+  auto tile_of = [&](int t, int& h, int& rb) {
+    rb = rblocks - 1 - t / Hq;
+    h = t % Hq;
+  };
+  auto nblocks_of = [&](int rb) {
+    const int last_row = min(T, (rb + 1) * ROWS) - 1;
+    return (pos0 + last_row) / KB + 1;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---- TMA producer
+      int s = 0;
+      uint32_t ph = 0, qph = 0;
+      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+        int h, rb;
+        tile_of(t, h, rb);
+        const int g = h / G;
+        if (!mbar_wait(Q_EMPTY, qph ^ 1u)) { *abort_flag = 1; break; }
+        qph ^= 1u;
+        mbar_arrive_expect_tx(Q_FULL, C::Q_BYTES);
+        for (int hh = 0; hh < C::HALVES; ++hh)
+          tma_load_2d(q_s + hh * (ROWS * 128), &tmQ, h * D + hh * 64, rb * ROWS, Q_FULL);
+        const int nb = nblocks_of(rb);
+        bool ok = true;
+        for (int j = 0; j < nb && ok; ++j) {
+          if (!mbar_wait(KV_EMPTY(s), ph ^ 1u)) { ok = false; break; }
+          // pages of this block that exist in the sequence's page-table row
+          int np = pages_avail - j * PAGES_PER_BLOCK;
+          np = np < 0 ? 0 : (np > PAGES_PER_BLOCK ? PAGES_PER_BLOCK : np);
+          int valid_pages = 0;
+          for (int p = 0; p < np; ++p) {
+            const int pg = page_row[j * PAGES_PER_BLOCK + p];
+            if (pg >= 0 && pg < num_pages) ++valid_pages;
+            else record_error(BI_ERR_DEVICE_INDEX);
+          }
+          mbar_arrive_expect_tx(KV_FULL(s), (uint32_t)(valid_pages * PAGE * D * 2 * 2));
+          const uint32_t ks = kv_s + s * C::STAGE, vs = ks + C::K_BYTES;
+          for (int p = 0; p < np; ++p) {
+            const int pg = page_row[j * PAGES_PER_BLOCK + p];
+            if (pg < 0 || pg >= num_pages) continue;
+            const int row = (pg * Hkv + g) * PAGE;  // first row of this page in the [pages*Hkv*16, D] view
+            for (int hh = 0; hh < C::HALVES; ++hh) {
+              tma_load_2d(ks + hh * C::KV_HALF + p * (PAGE * 128), &tmK, hh * 64, row, KV_FULL(s));
+              tma_load_2d(vs + hh * C::KV_HALF + p * (PAGE * 128), &tmV, hh * 64, row, KV_FULL(s));
+            }
+          }
+          if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) { *abort_flag = 1; break; }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---- MMA issuer
+      int s = 0;
+      uint32_t ph = 0, qph = 0, sph = 0, pph = 0, oph = 0;
+      int blocks_done = 0;  // S blocks issued so far (S_EMPTY phase)
+      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+        int h, rb;
+        tile_of(t, h, rb);
+        const int nb = nblocks_of(rb);
+        if (!mbar_wait(Q_FULL, qph)) { *abort_flag = 1; break; }
+        qph ^= 1u;
+        // O of the previous tile must have been read out
+        if (!mbar_wait(O_FREE, oph ^ 1u)) { *abort_flag = 1; break; }
+        oph ^= 1u;
+        bool ok = true;
+        for (int j = 0; j < nb && ok; ++j) {
+          if (!mbar_wait(KV_FULL(s), ph)) { ok = false; break; }
+          if (blocks_done > 0 && !mbar_wait(S_EMPTY, (sph ^ 1u))) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t ks = kv_s + s * C::STAGE, vs = ks + C::K_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk / 4) * (ROWS * 128) + (kk % 4) * 32;
+            const uint32_t koff = (kk / 4) * C::KV_HALF + (kk % 4) * 32;
+            tc_mma_f16(tS, desc_k(q_s + off), desc_k(ks + koff), kIdescS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(S_FULL);
+          if (j == nb - 1) tc_commit(Q_EMPTY);  // Q no longer needed after the last S of the tile
+          ++blocks_done;
+          sph ^= 1u;
+          // wait for P (and any rescale of O) from the softmax warps
+          if (!mbar_wait(P_FULL, pph)) { ok = false; break; }
+          pph ^= 1u;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < KB / 16; ++kk) {
+            const uint32_t poff = (kk / 4) * (ROWS * 128) + (kk % 4) * 32;
+            const uint32_t voff = kk * (16 * 128);  // keys 16kk .. 16kk+15 (128-byte rows)
+            tc_mma_f16(tO, desc_k(p_s + poff), desc_mn(vs + voff, C::KV_HALF), idesc_pv<D>(),
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(O_DONE);
+          tc_commit(KV_EMPTY(s));
+          if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) { *abort_flag = 1; break; }
+      }
+    }
+  } else {  // ---- softmax: warps 2..5, thread = query row (TMEM lane)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // row within the tile
+    uint32_t sph = 0, oph = 0, kvph = 0;
+    int s = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      int h, rb;
+      tile_of(t, h, rb);
+      const int nb = nblocks_of(rb);
+      const int row = rb * ROWS + r;               // row within the chunk
+      const int pos = pos0 + (row < T ? row : T - 1);
+      const int max_pos = pos0 + min(T, (rb + 1) * ROWS) - 1;
+      float m = -INFINITY, l = 0.f;
+      const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+      for (int j = 0; j < nb; ++j) {
+        ok = __all_sync(kFullMask, mbar_wait(S_FULL, sph));
+        if (!ok) break;
+        sph ^= 1u;
+        tc_fence_after();
+        uint32_t sv[KB];
+#pragma unroll
+        for (int cc = 0; cc < KB / 32; ++cc) {
+          uint32_t tmp[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(tS + lane_base + cc * 32, tmp);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sv[cc * 32 + e] = tmp[e];
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(S_EMPTY);
+        // scores and block max (keys in ascending order)
+        const int key0 = j * KB;
+        float bmax = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < KB; ++e) {
+          const float sc = (key0 + e <= pos) ? __fmul_rn(__uint_as_float(sv[e]), c) : -INFINITY;
+          sv[e] = __float_as_uint(sc);
+          bmax = fmaxf(bmax, sc);
+        }
+        const float m_new = fmaxf(m, bmax);
+        const float alpha = (m == -INFINITY) ? 1.f : exp2f(__fsub_rn(m, m_new));
+        float psum = 0.f;
+        // previous P . V must be done before P is overwritten and O rescaled
+        if (j > 0) {
+          ok = __all_sync(kFullMask, mbar_wait(O_DONE, oph));
+          if (!ok) break;
+          oph ^= 1u;
+          tc_fence_after();
+        }
+        // P row, bf16, into the two 64-key swizzled halves; l in key order
+#pragma unroll
+        for (int q8 = 0; q8 < KB / 8; ++q8) {
+          float pv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float sc = __uint_as_float(sv[q8 * 8 + e]);
+            pv[e] = sc == -INFINITY ? 0.f : exp2f(__fsub_rn(sc, m_new));
+            psum = __fadd_rn(psum, pv[e]);
+          }
+          uint4 pk;
+          pk.x = pack_bf16x2(pv[0], pv[1]);
+          pk.y = pack_bf16x2(pv[2], pv[3]);
+          pk.z = pack_bf16x2(pv[4], pv[5]);
+          pk.w = pack_bf16x2(pv[6], pv[7]);
+          const int half = q8 / 8, chunk = q8 % 8;
+          st_shared_v4(p_s + half * (ROWS * 128) + r * 128 + ((chunk ^ (r & 7)) << 4), pk);
+        }
+        l = __fadd_rn(__fmul_rn(l, alpha), psum);
+        if (j > 0 && __any_sync(kFullMask, alpha != 1.f)) {
+          // rescale this warp's rows of O in tensor memory (rows with alpha == 1 are unchanged)
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t ov[32];
+            __syncwarp();
+            tmem_ld_32x32b_x32(tO + lane_base + cc * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__fmul_rn(__uint_as_float(ov[e]), alpha));
+            tmem_st_32x32b_x32(tO + lane_base + cc * 32, ov);
+          }
+          tmem_wait_st();
+        }
+        m = m_new;
+        // V rows of keys past the chunk may be stale (even NaN): zero them before P . V
+        {
+          const int stage = s;
+          const bool wait_ok = mbar_wait(KV_FULL(stage), kvph);  // already complete; acquires the TMA writes
+          (void)wait_ok;
+          const int valid = max_pos + 1 - key0;  // keys of this block that may be read
+          if (valid < KB && r >= valid) {
+            const uint32_t vs = kv_s + stage * C::STAGE + C::K_BYTES;
+            for (int hh = 0; hh < C::HALVES; ++hh)
+              for (int ch = 0; ch < 8; ++ch) st_shared_v4(vs + hh * C::KV_HALF + r * 128 + ch * 16, make_uint4(0, 0, 0, 0));
+          }
+          if (++s == C::STAGES) { s = 0; kvph ^= 1u; }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(P_FULL);
+      }
+      if (!ok) break;
+      // final O / l for this tile
+      ok = __all_sync(kFullMask, mbar_wait(O_DONE, oph));
+      if (!ok) break;
+      oph ^= 1u;
+      tc_fence_after();
+      uint16_t* dst = out + ((int64_t)row * Hq + h) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ov[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tO + lane_base + cc * 32, ov);
+        tmem_wait_ld();
+        if (row < T) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 o;
+            o.x = pack_bf16x2(__fdiv_rn(__uint_as_float(ov[8 * v + 0]), l), __fdiv_rn(__uint_as_float(ov[8 * v + 1]), l));
+            o.y = pack_bf16x2(__fdiv_rn(__uint_as_float(ov[8 * v + 2]), l), __fdiv_rn(__uint_as_float(ov[8 * v + 3]), l));
+            o.z = pack_bf16x2(__fdiv_rn(__uint_as_float(ov[8 * v + 4]), l), __fdiv_rn(__uint_as_float(ov[8 * v + 5]), l));
+            o.w = pack_bf16x2(__fdiv_rn(__uint_as_float(ov[8 * v + 6]), l), __fdiv_rn(__uint_as_float(ov[8 * v + 7]), l));
+            reinterpret_cast<uint4*>(dst + cc * 32)[v] = o;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(O_FREE);
+    }
+    if (!ok) *abort_flag = 1;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace attn_tc
+}  // namespace bi

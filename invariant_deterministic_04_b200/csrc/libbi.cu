@@ -13,6 +13,7 @@
 #include "attention.cuh"
 #include "lmhead.cuh"
 #include "glue.cuh"
+#include "attention_tc.cuh"
 
 namespace {
 
@@ -269,6 +270,56 @@ bi_status bi_attention_prefill(const bi_bf16* q, int64_t ldq, const int32_t* q_s
   bi::attn::Rows R{nullptr, q_seq, q_pos, num_seqs, max_pages_per_seq};
   return attention_common(q, ldq, k_cache, v_cache, num_pages, page_table, max_pages_per_seq, R, T, out, Hq, Hkv, D,
                           scale, workspace, workspace_bytes, as_stream(stream));
+}
+
+bi_status bi_attention_prefill_tc(const bi_bf16* q, int64_t ldq, int seq, int pos0, int T, const bi_bf16* k_cache,
+                                  const bi_bf16* v_cache, int64_t num_pages, const int32_t* page_table, int num_seqs,
+                                  int max_pages_per_seq, bi_bf16* out, int Hq, int Hkv, int D, float scale,
+                                  void* stream) {
+  if (!q || !k_cache || !v_cache || !page_table || !out) return BI_ERR_NULL;
+  if (T < 0 || pos0 < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages <= 0 || num_seqs <= 0 ||
+      max_pages_per_seq <= 0 || seq < 0 || seq >= num_seqs || !std::isfinite(scale))
+    return BI_ERR_SHAPE;
+  if (D != 64 && D != 128) return BI_ERR_UNSUPPORTED;
+  if ((int64_t)pos0 + T > (int64_t)max_pages_per_seq * BI_PAGE_TOKENS || ldq < (int64_t)Hq * D) return BI_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || ldq % 8) return BI_ERR_ALIGN;
+  if (T == 0) return BI_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
+  bi::gemm::DeviceInfo* info = bi::gemm::device_info(dev);
+  if (!info) return BI_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  const int64_t kv_rows = num_pages * Hkv * BI_PAGE_TOKENS;
+  if (!bi::gemm::make_map(&tq, q, T, (int64_t)Hq * D, ldq, bi::attn_tc::ROWS) ||
+      !bi::gemm::make_map(&tk, k_cache, kv_rows, D, D, BI_PAGE_TOKENS) ||
+      !bi::gemm::make_map(&tv, v_cache, kv_rows, D, D, BI_PAGE_TOKENS))
+    return BI_ERR_CUDA;
+  const int tiles = ((T + bi::attn_tc::ROWS - 1) / bi::attn_tc::ROWS) * Hq;
+  const int grid = tiles < info->sms ? tiles : info->sms;
+  const int pages_avail = (pos0 + T + BI_PAGE_TOKENS - 1) / BI_PAGE_TOKENS;
+  const int32_t* prow = page_table + (int64_t)seq * max_pages_per_seq;
+  const float c = (float)((double)scale * 1.4426950408889634);
+  cudaStream_t st = as_stream(stream);
+  static std::once_flag once[2][64];
+  cudaError_t attr = cudaSuccess;
+  if (D == 128) {
+    std::call_once(once[0][dev & 63], [&] {
+      attr = cudaFuncSetAttribute(bi::attn_tc::prefill_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bi::attn_tc::Cfg<128>::SMEM);
+    });
+    if (attr != cudaSuccess) return BI_ERR_CUDA;
+    bi::attn_tc::prefill_tc_kernel<128><<<grid, bi::attn_tc::kThreads, bi::attn_tc::Cfg<128>::SMEM, st>>>(
+        tq, tk, tv, prow, num_pages, Hq, Hkv, pos0, T, pages_avail, out, c);
+  } else {
+    std::call_once(once[1][dev & 63], [&] {
+      attr = cudaFuncSetAttribute(bi::attn_tc::prefill_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bi::attn_tc::Cfg<64>::SMEM);
+    });
+    if (attr != cudaSuccess) return BI_ERR_CUDA;
+    bi::attn_tc::prefill_tc_kernel<64><<<grid, bi::attn_tc::kThreads, bi::attn_tc::Cfg<64>::SMEM, st>>>(
+        tq, tk, tv, prow, num_pages, Hq, Hkv, pos0, T, pages_avail, out, c);
+  }
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
 bi_status bi_kv_append(const bi_bf16* k_new, const bi_bf16* v_new, int64_t ld_new, const int32_t* q_seq, const int32_t* q_pos,

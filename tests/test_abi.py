@@ -175,3 +175,13 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 def test_selftest_validation(L):
     assert L.bi_selftest_wait_timeout(0, None) == SHAPE
     assert L.bi_selftest_wait_timeout(2001, None) == SHAPE
+
+
+def test_prefill_tc_validation(L):
+    f = L.bi_attention_prefill_tc
+    assert f(None, 4096, 0, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == NULL
+    assert f(P, 4096, 1, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == SHAPE    # seq out of range
+    assert f(P, 4096, 0, 4000, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == SHAPE  # past the table
+    assert f(P, 4096, 0, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 96, 0.088, None) == UNSUP
+    assert f(P, 4100, 0, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == ALIGN
+    assert f(P, 4096, 0, 0, 0, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == OK
