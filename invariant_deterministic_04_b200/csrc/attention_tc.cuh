@@ -12,12 +12,14 @@
 //   * keys are processed in blocks of 128 at absolute positions 0, 128, 256, ...,
 //     in ascending order, up to the block holding the row's position;
 //   * S = q . k for a block by tcgen05.mma (bf16 x bf16, fp32 accumulation over D in
-//     ascending 16-wide steps), masked to keys <= pos, scaled by scale*log2(e);
-//   * online softmax in fp32 by the thread that owns the row: block max, then
-//     m = max(m, block max), l = l * 2^(m_old - m) + sum_j p_j (keys in order),
-//     O rescaled by 2^(m_old - m) only when m moved (x * 1 == x exactly);
+//     ascending 16-wide steps), masked to keys <= pos;
+//   * online softmax in fp32 by the thread that owns the row: block max of the
+//     masked q.k times c, m = max(m, block max), p_j = 2^(q.k_j * c - m) (one FMA,
+//     one SFU exp2), l = l * 2^(m_old - m) + the block's p summed as eight partial
+//     sums (key index mod 8, keys in order) joined by a fixed tree; O rescaled by
+//     2^(m_old - m) only when m moved (x * 1 == x exactly);
 //   * p rounded to bf16, O += P V by tcgen05.mma (fp32, ascending 16-key steps);
-//   * out = O / l rounded to bf16.
+//   * out = O * (1 / l) rounded to bf16.
 // The tensor core's result for an output element depends on that element's row and
 // column operands and the fixed K order only, not on the other rows of the tile or
 // the tile shape (checked on this hardware by the matmul tests), and a block with
@@ -80,6 +82,12 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+// 2^x by the SFU (one instruction; 2^-inf = +0, subnormal results flushed to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
@@ -278,18 +286,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(S_EMPTY);
-        // scores and block max (keys in ascending order)
+        // mask keys past the row's position (raw q.k; NaN of stale slots never survives the select)
         const int key0 = j * KB;
-        float bmax = -INFINITY;
+        float bm[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) bm[e] = -INFINITY;
 #pragma unroll
         for (int e = 0; e < KB; ++e) {
-          const float sc = (key0 + e <= pos) ? __fmul_rn(__uint_as_float(sv[e]), c) : -INFINITY;
-          sv[e] = __float_as_uint(sc);
-          bmax = fmaxf(bmax, sc);
+          const float v = (key0 + e <= pos) ? __uint_as_float(sv[e]) : -INFINITY;
+          sv[e] = __float_as_uint(v);
+          bm[e & 7] = fmaxf(bm[e & 7], v);
         }
-        const float m_new = fmaxf(m, bmax);
-        const float alpha = (m == -INFINITY) ? 1.f : exp2f(__fsub_rn(m, m_new));
-        float psum = 0.f;
+        const float bmax = fmaxf(fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3])), fmaxf(fmaxf(bm[4], bm[5]), fmaxf(bm[6], bm[7])));
+        // scores are q.k * c (c = scale * log2 e > 0): the block max of the scores is bmax * c
+        const float m_new = fmaxf(m, __fmul_rn(bmax, c));
+        const float alpha = (m == -INFINITY) ? 1.f : ex2_approx(__fsub_rn(m, m_new));
+        const float neg_m = -m_new;
         // previous P . V must be done before P is overwritten and O rescaled
         if (j > 0) {
           ok = __all_sync(kFullMask, mbar_wait(O_DONE, oph));
@@ -297,15 +309,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           oph ^= 1u;
           tc_fence_after();
         }
-        // P row, bf16, into the two 64-key swizzled halves; l in key order
+        // p = 2^(q.k * c - m) (masked keys give 2^-inf = 0); eight partial sums by key
+        // index mod 8 in key order, joined by a fixed tree; P row as bf16 into the two
+        // 64-key swizzled halves
+        float ps[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ps[e] = 0.f;
 #pragma unroll
         for (int q8 = 0; q8 < KB / 8; ++q8) {
           float pv[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float sc = __uint_as_float(sv[q8 * 8 + e]);
-            pv[e] = sc == -INFINITY ? 0.f : exp2f(__fsub_rn(sc, m_new));
-            psum = __fadd_rn(psum, pv[e]);
+            pv[e] = ex2_approx(__fmaf_rn(__uint_as_float(sv[q8 * 8 + e]), c, neg_m));
+            ps[e] = __fadd_rn(ps[e], pv[e]);
           }
           uint4 pk;
           pk.x = pack_bf16x2(pv[0], pv[1]);
@@ -315,6 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int half = q8 / 8, chunk = q8 % 8;
           st_shared_v4(p_s + half * (ROWS * 128) + r * 128 + ((chunk ^ (r & 7)) << 4), pk);
         }
+        const float psum = __fadd_rn(__fadd_rn(__fadd_rn(ps[0], ps[1]), __fadd_rn(ps[2], ps[3])),
+                                     __fadd_rn(__fadd_rn(ps[4], ps[5]), __fadd_rn(ps[6], ps[7])));
         l = __fadd_rn(__fmul_rn(l, alpha), psum);
         if (j > 0 && __any_sync(kFullMask, alpha != 1.f)) {
           // rescale this warp's rows of O in tensor memory (rows with alpha == 1 are unchanged)
@@ -355,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       oph ^= 1u;
       tc_fence_after();
       uint16_t* dst = out + ((int64_t)row * Hq + h) * D;
+      const float inv_l = __frcp_rn(l);
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t ov[32];
@@ -365,10 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 o;
-            o.x = pack_bf16x2(__fdiv_rn(__uint_as_float(ov[8 * v + 0]), l), __fdiv_rn(__uint_as_float(ov[8 * v + 1]), l));
-            o.y = pack_bf16x2(__fdiv_rn(__uint_as_float(ov[8 * v + 2]), l), __fdiv_rn(__uint_as_float(ov[8 * v + 3]), l));
-            o.z = pack_bf16x2(__fdiv_rn(__uint_as_float(ov[8 * v + 4]), l), __fdiv_rn(__uint_as_float(ov[8 * v + 5]), l));
-            o.w = pack_bf16x2(__fdiv_rn(__uint_as_float(ov[8 * v + 6]), l), __fdiv_rn(__uint_as_float(ov[8 * v + 7]), l));
+            o.x = pack_bf16x2(__fmul_rn(__uint_as_float(ov[8 * v + 0]), inv_l), __fmul_rn(__uint_as_float(ov[8 * v + 1]), inv_l));
+            o.y = pack_bf16x2(__fmul_rn(__uint_as_float(ov[8 * v + 2]), inv_l), __fmul_rn(__uint_as_float(ov[8 * v + 3]), inv_l));
+            o.z = pack_bf16x2(__fmul_rn(__uint_as_float(ov[8 * v + 4]), inv_l), __fmul_rn(__uint_as_float(ov[8 * v + 5]), inv_l));
+            o.w = pack_bf16x2(__fmul_rn(__uint_as_float(ov[8 * v + 6]), inv_l), __fmul_rn(__uint_as_float(ov[8 * v + 7]), inv_l));
             reinterpret_cast<uint4*>(dst + cc * 32)[v] = o;
           }
         }
