@@ -186,13 +186,15 @@ bi_status bi_attention_prefill(const bi_bf16* q, int64_t ldq, const int32_t* q_s
  * (a faster attention kernel brought 55 s back to 42 s). The query rows are
  * positions pos0 .. pos0+T-1 of sequence `seq`; row t of q starts at q + t * ldq
  * and holds [Hq, D] bf16; the chunk's own K/V must already be in the store.
- * out: [T, Hq, D] bf16. Per row: keys in blocks of 128 at absolute positions,
+ * out: [T, Hq, D] bf16. Per row: keys in blocks of 64 at absolute positions,
  * ascending; S = q.k by tcgen05 (fp32), online softmax in fp32 by one thread per
  * row, P rounded to bf16, O += P V by tcgen05; out = O / l. A row's bits depend on
  * its position and the keys only, so whole and chunked prefill give the same bits.
  * They are NOT the bits of bi_attention_prefill / bi_attention_decode (a different,
  * also fixed, arithmetic; the two agree within the bf16 tolerance).
- * D in {64, 128}; Hq % Hkv == 0; pos0 + T <= max_pages_per_seq * 16. No workspace.
+ * D in {64, 128} and Hq / Hkv even (two query heads of one kv-head share each
+ * K/V block), else BI_ERR_UNSUPPORTED; scale > 0; pos0 + T <= max_pages_per_seq * 16.
+ * No workspace.
  */
 bi_status bi_attention_prefill_tc(const bi_bf16* q, int64_t ldq, int seq, int pos0, int T, const bi_bf16* k_cache,
                                   const bi_bf16* v_cache, int64_t num_pages, const int32_t* page_table, int num_seqs,

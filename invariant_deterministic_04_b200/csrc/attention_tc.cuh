@@ -9,15 +9,17 @@
 // One chunk of one sequence: query rows at positions pos0 .. pos0 + T - 1, keys
 // 0 .. pos from the paged store (the chunk's own K/V already appended).
 // Per-row schedule, a function of the row's position only:
-//   * keys are processed in blocks of 128 at absolute positions 0, 128, 256, ...,
-//     in ascending order, up to the block holding the row's position;
+//   * keys are processed in blocks of 64 at absolute positions 0, 64, 128, ..., in
+//     ascending order, up to the block holding the row's position;
 //   * S = q . k for a block by tcgen05.mma (bf16 x bf16, fp32 accumulation over D in
 //     ascending 16-wide steps), masked to keys <= pos;
-//   * online softmax in fp32 by the thread that owns the row: block max of the
-//     masked q.k times c, m = max(m, block max), p_j = 2^(q.k_j * c - m) (one FMA,
-//     one SFU exp2), l = l * 2^(m_old - m) + the block's p summed as eight partial
-//     sums (key index mod 8, keys in order) joined by a fixed tree; O rescaled by
-//     2^(m_old - m) only when m moved (x * 1 == x exactly);
+//   * online softmax in fp32 by the thread that owns the row: b = block max of the
+//     masked q.k times c (c = scale * log2 e); the reference point m becomes b only
+//     when b > m + 8 (lazy rescaling: p stays <= 2^8, exact in fp32, and the final
+//     division by l cancels the choice of m); p_j = 2^(q.k_j * c - m) (one FMA, one
+//     SFU exp2); l = l * 2^(m_old - m) + the block's p summed as eight partial sums
+//     (key index mod 8, keys in order) joined by a fixed tree; O rescaled by
+//     2^(m_old - m) only when m moved (x * 1 == x);
 //   * p rounded to bf16, O += P V by tcgen05.mma (fp32, ascending 16-key steps);
 //   * out = O * (1 / l) rounded to bf16.
 // The tensor core's result for an output element depends on that element's row and
@@ -25,6 +27,11 @@
 // the tile shape (checked on this hardware by the matmul tests), and a block with
 // no visible key leaves a row's state unchanged; so a row's bits do not depend on
 // how the sequence was chunked or which other rows shared its tile.
+//
+// Work: a CTA takes two 128-row Q tiles at once, query heads h and h+1 of one kv-head
+// over the same row block, so every K/V block is fetched once for both. Warp 0 loads
+// (TMA), warp 1 issues the MMAs in a software pipeline (S of one tile while the
+// other tile's softmax runs), warps 2-5 and 6-9 run the two softmaxes.
 #pragma once
 
 #include "device.cuh"
@@ -33,26 +40,27 @@ namespace bi {
 namespace attn_tc {
 
 constexpr int PAGE = BI_PAGE_TOKENS;
-constexpr int KB = 128;                 // keys per block
+constexpr int KB = 64;                  // keys per block
 constexpr int PAGES_PER_BLOCK = KB / PAGE;
 constexpr int ROWS = 128;               // query rows per tile
-constexpr int kThreads = 192;           // warp 0 TMA, warp 1 MMA, warps 2..5 softmax (one row per thread)
+constexpr int kThreads = 320;           // warp 0 TMA, warp 1 MMA, warps 2-5 / 6-9 softmax of tiles A / B
+constexpr float kLazy = 8.f;            // the softmax reference point moves by more than 2^8 or not at all
 
 template <int D>
 struct Cfg {
-  static constexpr int HALVES = D / 64;                       // 64-dim (128-byte) halves
-  static constexpr int Q_BYTES = ROWS * D * 2;                // Q tile
-  static constexpr int KV_HALF = KB * 128;                    // one 64-dim half of a 128-key block
+  static constexpr int HALVES = D / 64;                 // 64-dim (128-byte) halves
+  static constexpr int Q_BYTES = ROWS * D * 2;          // one Q tile
+  static constexpr int KV_HALF = KB * 128;              // one 64-dim half of a 64-key block
   static constexpr int K_BYTES = HALVES * KV_HALF;
-  static constexpr int STAGE = 2 * K_BYTES;                   // K and V of one block
-  static constexpr int P_BYTES = ROWS * KB * 2;               // P tile (bf16), two 64-key halves
-  static constexpr int STAGES = 2;
-  static constexpr int SMEM = 1024 + Q_BYTES + STAGES * STAGE + P_BYTES + 256;
-  static constexpr int TMEM_COLS = 256;                       // S: 128 cols, O: D cols
+  static constexpr int STAGE = 2 * K_BYTES;             // K and V of one block
+  static constexpr int P_BYTES = ROWS * KB * 2;         // one P tile (bf16, 128-byte rows)
+  static constexpr int STAGES = 3;
+  static constexpr int SMEM = 1024 + 2 * Q_BYTES + STAGES * STAGE + 2 * P_BYTES + 256;
+  static constexpr int TMEM_COLS = (2 * KB + 2 * D) <= 256 ? 256 : 512;  // S_A, S_B, O_A, O_B
 };
 
 // Instruction descriptors (kind::f16, bf16 inputs, fp32 accumulate, M = 128).
-// S = Q K^T: A = Q K-major, B = K K-major, N = 128 keys.
+// S = Q K^T: A = Q K-major, B = K K-major, N = 64 keys.
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(KB >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 // O += P V: A = P K-major (keys contiguous), B = V MN-major (dims contiguous), N = D.
 template <int D>
@@ -95,7 +103,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-// Tiles: (q-head h, row block rb); heavier row blocks (more key blocks) first.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -107,23 +114,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t q_s = base;
-  const uint32_t kv_s = base + C::Q_BYTES;           // stage s: K at kv_s + s*STAGE, V at + K_BYTES
-  const uint32_t p_s = kv_s + C::STAGES * C::STAGE;
-  const uint32_t bar0 = p_s + C::P_BYTES;
-  // barriers
+  const uint32_t q_s = base;                            // tile X at q_s + X * Q_BYTES
+  const uint32_t kv_s = base + 2 * C::Q_BYTES;          // stage s: K at kv_s + s*STAGE, V at + K_BYTES
+  const uint32_t p_s = kv_s + C::STAGES * C::STAGE;     // tile X at p_s + X * P_BYTES
+  const uint32_t bar0 = p_s + 2 * C::P_BYTES;
+  // barriers: Q_FULL, Q_EMPTY, KV_FULL[s], KV_EMPTY[s], then per tile X: S_FULL, P_FULL, O_DONE, O_FREE
   const uint32_t Q_FULL = bar0, Q_EMPTY = bar0 + 8;
   auto KV_FULL = [&](int s) { return bar0 + 16 + 16 * s; };
   auto KV_EMPTY = [&](int s) { return bar0 + 24 + 16 * s; };
-  const uint32_t S_FULL = bar0 + 16 + 16 * C::STAGES, S_EMPTY = S_FULL + 8, P_FULL = S_FULL + 16, O_DONE = S_FULL + 24,
-                 O_FREE = S_FULL + 32;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (bar0 - base) + 16 + 16 * C::STAGES + 48);
+  const uint32_t XB = bar0 + 16 + 16 * C::STAGES;
+  auto S_FULL = [&](int x) { return XB + 32 * x; };
+  auto P_FULL = [&](int x) { return XB + 32 * x + 8; };
+  auto O_DONE = [&](int x) { return XB + 32 * x + 16; };
+  auto O_FREE = [&](int x) { return XB + 32 * x + 24; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (XB - base) + 64);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rblocks = (T + ROWS - 1) / ROWS;
-  const int tiles = rblocks * Hq;
   const int G = Hq / Hkv;
+  const int pairs = Hkv * (G / 2);                      // tile pairs per row block
+  const int rblocks = (T + ROWS - 1) / ROWS;
+  const int work = rblocks * pairs;
 
   if (threadIdx.x == 0) {
     mbar_init(Q_FULL, 1);
@@ -132,11 +143,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(KV_FULL(s), 1);
       mbar_init(KV_EMPTY(s), 1);
     }
-    mbar_init(S_FULL, 1);
-    mbar_init(S_EMPTY, 128);
-    mbar_init(P_FULL, 128);
-    mbar_init(O_DONE, 1);
-    mbar_init(O_FREE, 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(S_FULL(x), 1);
+      mbar_init(P_FULL(x), 128);
+      mbar_init(O_DONE(x), 1);
+      mbar_init(O_FREE(x), 128);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -152,12 +164,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + KB;
+  auto tS = [&](int x) { return tmem + (uint32_t)(x * KB); };
+  auto tO = [&](int x) { return tmem + (uint32_t)(2 * KB + x * D); };
 
-  // tile t -> (head, row block): row blocks from the last (heaviest) to the first
-  auto tile_of = [&](int t, int& h, int& rb) {
-    rb = rblocks - 1 - t / Hq;
-    h = t % Hq;
+  // work item w -> (kv-head g, first query head hA = g*G + 2*hp, row block rb);
+  // heavier row blocks (more key blocks) first
+  auto item_of = [&](int w, int& g, int& hA, int& rb) {
+    rb = rblocks - 1 - w / pairs;
+    const int pr = w % pairs;
+    g = pr / (G / 2);
+    hA = g * G + 2 * (pr % (G / 2));
   };
   auto nblocks_of = [&](int rb) {
     const int last_row = min(T, (rb + 1) * ROWS) - 1;
@@ -168,20 +184,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {  // ---- TMA producer
       int s = 0;
       uint32_t ph = 0, qph = 0;
-      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
-        int h, rb;
-        tile_of(t, h, rb);
-        const int g = h / G;
+      for (int w = blockIdx.x; w < work && !*abort_flag; w += gridDim.x) {
+        int g, hA, rb;
+        item_of(w, g, hA, rb);
         if (!mbar_wait(Q_EMPTY, qph ^ 1u)) { *abort_flag = 1; break; }
         qph ^= 1u;
-        mbar_arrive_expect_tx(Q_FULL, C::Q_BYTES);
-        for (int hh = 0; hh < C::HALVES; ++hh)
-          tma_load_2d(q_s + hh * (ROWS * 128), &tmQ, h * D + hh * 64, rb * ROWS, Q_FULL);
+        mbar_arrive_expect_tx(Q_FULL, 2 * C::Q_BYTES);
+        for (int x = 0; x < 2; ++x)
+          for (int hh = 0; hh < C::HALVES; ++hh)
+            tma_load_2d(q_s + x * C::Q_BYTES + hh * (ROWS * 128), &tmQ, (hA + x) * D + hh * 64, rb * ROWS, Q_FULL);
         const int nb = nblocks_of(rb);
         bool ok = true;
-        for (int j = 0; j < nb && ok; ++j) {
+        for (int j = 0; j < nb; ++j) {
           if (!mbar_wait(KV_EMPTY(s), ph ^ 1u)) { ok = false; break; }
-          // pages of this block that exist in the sequence's page-table row
           int np = pages_avail - j * PAGES_PER_BLOCK;
           np = np < 0 ? 0 : (np > PAGES_PER_BLOCK ? PAGES_PER_BLOCK : np);
           int valid_pages = 0;
@@ -207,132 +222,153 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {  // ---- MMA issuer
+    if (lane == 0) {  // ---- MMA issuer (software-pipelined over the two tiles)
       int s = 0;
-      uint32_t ph = 0, qph = 0, sph = 0, pph = 0, oph = 0;
-      int blocks_done = 0;  // S blocks issued so far (S_EMPTY phase)
-      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
-        int h, rb;
-        tile_of(t, h, rb);
-        const int nb = nblocks_of(rb);
-        if (!mbar_wait(Q_FULL, qph)) { *abort_flag = 1; break; }
-        qph ^= 1u;
-        // O of the previous tile must have been read out
-        if (!mbar_wait(O_FREE, oph ^ 1u)) { *abort_flag = 1; break; }
-        oph ^= 1u;
-        bool ok = true;
-        for (int j = 0; j < nb && ok; ++j) {
-          if (!mbar_wait(KV_FULL(s), ph)) { ok = false; break; }
-          if (blocks_done > 0 && !mbar_wait(S_EMPTY, (sph ^ 1u))) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t ks = kv_s + s * C::STAGE, vs = ks + C::K_BYTES;
+      uint32_t ph = 0, qph = 0;
+      uint32_t pph[2] = {0, 0}, oph[2] = {0, 0};
+      bool ok = true;
+      auto issue_s = [&](int x, int st) {
+        const uint32_t ks = kv_s + st * C::STAGE;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * (ROWS * 128) + (kk % 4) * 32;
-            const uint32_t koff = (kk / 4) * C::KV_HALF + (kk % 4) * 32;
-            tc_mma_f16(tS, desc_k(q_s + off), desc_k(ks + koff), kIdescS, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(S_FULL);
-          if (j == nb - 1) tc_commit(Q_EMPTY);  // Q no longer needed after the last S of the tile
-          ++blocks_done;
-          sph ^= 1u;
-          // wait for P (and any rescale of O) from the softmax warps
-          if (!mbar_wait(P_FULL, pph)) { ok = false; break; }
-          pph ^= 1u;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < KB / 16; ++kk) {
-            const uint32_t poff = (kk / 4) * (ROWS * 128) + (kk % 4) * 32;
-            const uint32_t voff = kk * (16 * 128);  // keys 16kk .. 16kk+15 (128-byte rows)
-            tc_mma_f16(tO, desc_k(p_s + poff), desc_mn(vs + voff, C::KV_HALF), idesc_pv<D>(),
-                       (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(O_DONE);
-          tc_commit(KV_EMPTY(s));
-          if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qoff = x * C::Q_BYTES + (kk / 4) * (ROWS * 128) + (kk % 4) * 32;
+          const uint32_t koff = (kk / 4) * C::KV_HALF + (kk % 4) * 32;
+          tc_mma_f16(tS(x), desc_k(q_s + qoff), desc_k(ks + koff), kIdescS, kk > 0 ? 1u : 0u);
         }
-        if (!ok) { *abort_flag = 1; break; }
+        tc_commit(S_FULL(x));
+      };
+      auto issue_pv = [&](int x, int st, int j) {
+        const uint32_t vs = kv_s + st * C::STAGE + C::K_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < KB / 16; ++kk)
+          tc_mma_f16(tO(x), desc_k(p_s + x * C::P_BYTES + kk * 32), desc_mn(vs + kk * (16 * 128), C::KV_HALF),
+                     idesc_pv<D>(), (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(O_DONE(x));
+      };
+      for (int w = blockIdx.x; w < work && ok && !*abort_flag; w += gridDim.x) {
+        int g, hA, rb;
+        item_of(w, g, hA, rb);
+        const int nb = nblocks_of(rb);
+        if (!mbar_wait(Q_FULL, qph)) { ok = false; break; }
+        qph ^= 1u;
+        // prologue: S of block 0 for both tiles
+        if (!mbar_wait(KV_FULL(s), ph)) { ok = false; break; }
+        tc_fence_after();
+        issue_s(0, s);
+        issue_s(1, s);
+        for (int j = 0; j < nb && ok; ++j) {
+          const int sj = s;
+          const int sn = (s + 1 == C::STAGES) ? 0 : s + 1;
+          const uint32_t phn = (s + 1 == C::STAGES) ? (ph ^ 1u) : ph;
+          for (int x = 0; x < 2 && ok; ++x) {
+            if (j == 0) {  // the previous tile's O of this group has been read out
+              if (!mbar_wait(O_FREE(x), oph[x] ^ 1u)) { ok = false; break; }
+              oph[x] ^= 1u;
+            }
+            if (!mbar_wait(P_FULL(x), pph[x])) { ok = false; break; }
+            pph[x] ^= 1u;
+            tc_fence_after();
+            issue_pv(x, sj, j);
+            if (x == 1) tc_commit(KV_EMPTY(sj));  // both tiles are done with block j
+            if (j + 1 < nb) {
+              if (x == 0 && !mbar_wait(KV_FULL(sn), phn)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(x, sn);
+            }
+          }
+          s = sn;
+          ph = phn;
+        }
+        if (!ok) break;
+        tc_commit(Q_EMPTY);  // all S of this tile pair were issued before this point
       }
+      if (!ok) *abort_flag = 1;
     }
-  } else {  // ---- softmax: warps 2..5, thread = query row (TMEM lane)
+  } else {  // ---- softmax: warps 2..5 (tile A) and 6..9 (tile B); thread = query row (TMEM lane)
+    const int x = (warp - 2) / 4;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row within the tile
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     uint32_t sph = 0, oph = 0, kvph = 0;
     int s = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-      int h, rb;
-      tile_of(t, h, rb);
+    for (int w = blockIdx.x; w < work; w += gridDim.x) {
+      int g, hA, rb;
+      item_of(w, g, hA, rb);
+      const int h = hA + x;
       const int nb = nblocks_of(rb);
       const int row = rb * ROWS + r;               // row within the chunk
       const int pos = pos0 + (row < T ? row : T - 1);
       const int max_pos = pos0 + min(T, (rb + 1) * ROWS) - 1;
       float m = -INFINITY, l = 0.f;
-      const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
       for (int j = 0; j < nb; ++j) {
-        ok = __all_sync(kFullMask, mbar_wait(S_FULL, sph));
+        ok = __all_sync(kFullMask, mbar_wait(S_FULL(x), sph));
         if (!ok) break;
         sph ^= 1u;
         tc_fence_after();
-        uint32_t sv[KB];
-#pragma unroll
-        for (int cc = 0; cc < KB / 32; ++cc) {
-          uint32_t tmp[32];
-          __syncwarp();
-          tmem_ld_32x32b_x32(tS + lane_base + cc * 32, tmp);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) sv[cc * 32 + e] = tmp[e];
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(S_EMPTY);
-        // mask keys past the row's position (raw q.k; NaN of stale slots never survives the select)
         const int key0 = j * KB;
+        // every key of the block visible to every row of this warp: no masking needed
+        const bool full = __all_sync(kFullMask, key0 + KB - 1 <= pos);
+        // the block's 64 scores of this row, read from tensor memory once; masked keys
+        // become -inf (NaN of stale slots never survives the select)
+        uint32_t sv[KB];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tS(x) + lane_base, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld_32x32b_x32(tS(x) + lane_base + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+        if (!full) {
+#pragma unroll
+          for (int e = 0; e < KB; ++e)
+            if (key0 + e > pos) sv[e] = __float_as_uint(-INFINITY);
+        }
         float bm[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) bm[e] = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < KB; ++e) {
-          const float v = (key0 + e <= pos) ? __uint_as_float(sv[e]) : -INFINITY;
-          sv[e] = __float_as_uint(v);
-          bm[e & 7] = fmaxf(bm[e & 7], v);
-        }
-        const float bmax = fmaxf(fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3])), fmaxf(fmaxf(bm[4], bm[5]), fmaxf(bm[6], bm[7])));
-        // scores are q.k * c (c = scale * log2 e > 0): the block max of the scores is bmax * c
-        const float m_new = fmaxf(m, __fmul_rn(bmax, c));
-        const float alpha = (m == -INFINITY) ? 1.f : ex2_approx(__fsub_rn(m, m_new));
-        const float neg_m = -m_new;
-        // previous P . V must be done before P is overwritten and O rescaled
+        for (int e = 0; e < KB; ++e) bm[e & 7] = fmaxf(bm[e & 7], __uint_as_float(sv[e]));
+        const float bmax =
+            fmaxf(fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3])), fmaxf(fmaxf(bm[4], bm[5]), fmaxf(bm[6], bm[7])));
+        // the reference point m moves only when the block max exceeds it by more than 2^8;
+        // scores up to 256 * 2^m stay exact in fp32 and the final 1/l cancels the choice
+        const float sb = __fmul_rn(bmax, c);  // scores are q.k * c with c > 0
+        const bool move = sb > __fadd_rn(m, kLazy);
+        const float m_new = move ? sb : m;
+        const float alpha = (move && m != -INFINITY) ? ex2_approx(__fsub_rn(m, m_new)) : 1.f;
+        const float2 neg_m2 = make_float2(-m_new, -m_new);
+        const float2 c2 = make_float2(c, c);
+        // the previous P . V of this tile must be done before P is overwritten and O rescaled
         if (j > 0) {
-          ok = __all_sync(kFullMask, mbar_wait(O_DONE, oph));
+          ok = __all_sync(kFullMask, mbar_wait(O_DONE(x), oph));
           if (!ok) break;
           oph ^= 1u;
           tc_fence_after();
         }
-        // p = 2^(q.k * c - m) (masked keys give 2^-inf = 0); eight partial sums by key
-        // index mod 8 in key order, joined by a fixed tree; P row as bf16 into the two
-        // 64-key swizzled halves
-        float ps[8];
+        // p = 2^(q.k * c - m) (masked keys give 2^-inf = 0), partial sums by key
+        // index mod 8, P row as bf16 into the swizzled 128-byte row
+        float2 ps[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ps[e] = 0.f;
+        for (int e = 0; e < 4; ++e) ps[e] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int q8 = 0; q8 < KB / 8; ++q8) {
-          float pv[8];
+        for (int cc = 0; cc < KB / 32; ++cc) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            pv[e] = ex2_approx(__fmaf_rn(__uint_as_float(sv[q8 * 8 + e]), c, neg_m));
-            ps[e] = __fadd_rn(ps[e], pv[e]);
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 t = __ffma2_rn(make_float2(__uint_as_float(sv[cc * 32 + q8 * 8 + 2 * e]),
+                                                      __uint_as_float(sv[cc * 32 + q8 * 8 + 2 * e + 1])),
+                                          c2, neg_m2);
+              const float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+              ps[e] = __fadd2_rn(ps[e], pv);
+              pk[e] = pack_bf16x2(pv.x, pv.y);
+            }
+            const int chunk = cc * 4 + q8;
+            st_shared_v4(p_s + x * C::P_BYTES + r * 128 + ((chunk ^ (r & 7)) << 4),
+                         make_uint4(pk[0], pk[1], pk[2], pk[3]));
           }
-          uint4 pk;
-          pk.x = pack_bf16x2(pv[0], pv[1]);
-          pk.y = pack_bf16x2(pv[2], pv[3]);
-          pk.z = pack_bf16x2(pv[4], pv[5]);
-          pk.w = pack_bf16x2(pv[6], pv[7]);
-          const int half = q8 / 8, chunk = q8 % 8;
-          st_shared_v4(p_s + half * (ROWS * 128) + r * 128 + ((chunk ^ (r & 7)) << 4), pk);
         }
-        const float psum = __fadd_rn(__fadd_rn(__fadd_rn(ps[0], ps[1]), __fadd_rn(ps[2], ps[3])),
-                                     __fadd_rn(__fadd_rn(ps[4], ps[5]), __fadd_rn(ps[6], ps[7])));
+        const float psum = __fadd_rn(__fadd_rn(__fadd_rn(ps[0].x, ps[0].y), __fadd_rn(ps[1].x, ps[1].y)),
+                                     __fadd_rn(__fadd_rn(ps[2].x, ps[2].y), __fadd_rn(ps[3].x, ps[3].y)));
         l = __fadd_rn(__fmul_rn(l, alpha), psum);
         if (j > 0 && __any_sync(kFullMask, alpha != 1.f)) {
           // rescale this warp's rows of O in tensor memory (rows with alpha == 1 are unchanged)
@@ -340,35 +376,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t ov[32];
             __syncwarp();
-            tmem_ld_32x32b_x32(tO + lane_base + cc * 32, ov);
+            tmem_ld_32x32b_x32(tO(x) + lane_base + cc * 32, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__fmul_rn(__uint_as_float(ov[e]), alpha));
-            tmem_st_32x32b_x32(tO + lane_base + cc * 32, ov);
+            tmem_st_32x32b_x32(tO(x) + lane_base + cc * 32, ov);
           }
           tmem_wait_st();
         }
         m = m_new;
-        // V rows of keys past the chunk may be stale (even NaN): zero them before P . V
-        {
+        // V rows of keys past the chunk may be stale (even NaN): tile A's group zeroes them
+        // before P . V (tile B's P . V is issued after tile A's)
+        if (x == 0) {
           const int stage = s;
-          const bool wait_ok = mbar_wait(KV_FULL(stage), kvph);  // already complete; acquires the TMA writes
-          (void)wait_ok;
-          const int valid = max_pos + 1 - key0;  // keys of this block that may be read
-          if (valid < KB && r >= valid) {
+          (void)mbar_wait(KV_FULL(stage), kvph);  // already complete: acquires the TMA writes
+          const int valid = max_pos + 1 - key0;
+          if (valid < KB && r < KB && r >= valid) {
             const uint32_t vs = kv_s + stage * C::STAGE + C::K_BYTES;
             for (int hh = 0; hh < C::HALVES; ++hh)
               for (int ch = 0; ch < 8; ++ch) st_shared_v4(vs + hh * C::KV_HALF + r * 128 + ch * 16, make_uint4(0, 0, 0, 0));
           }
-          if (++s == C::STAGES) { s = 0; kvph ^= 1u; }
         }
+        if (++s == C::STAGES) { s = 0; kvph ^= 1u; }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(P_FULL);
+        mbar_arrive(P_FULL(x));
       }
       if (!ok) break;
       // final O / l for this tile
-      ok = __all_sync(kFullMask, mbar_wait(O_DONE, oph));
+      ok = __all_sync(kFullMask, mbar_wait(O_DONE(x), oph));
       if (!ok) break;
       oph ^= 1u;
       tc_fence_after();
@@ -378,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t ov[32];
         __syncwarp();
-        tmem_ld_32x32b_x32(tO + lane_base + cc * 32, ov);
+        tmem_ld_32x32b_x32(tO(x) + lane_base + cc * 32, ov);
         tmem_wait_ld();
         if (row < T) {
 #pragma unroll
@@ -393,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(O_FREE);
+      mbar_arrive(O_FREE(x));
     }
     if (!ok) *abort_flag = 1;
   }

@@ -280,7 +280,8 @@ bi_status bi_attention_prefill_tc(const bi_bf16* q, int64_t ldq, int seq, int po
   if (T < 0 || pos0 < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages <= 0 || num_seqs <= 0 ||
       max_pages_per_seq <= 0 || seq < 0 || seq >= num_seqs || !std::isfinite(scale))
     return BI_ERR_SHAPE;
-  if (D != 64 && D != 128) return BI_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128 || (Hq / Hkv) % 2 != 0) return BI_ERR_UNSUPPORTED;
+  if (!(scale > 0.f)) return BI_ERR_SHAPE;
   if ((int64_t)pos0 + T > (int64_t)max_pages_per_seq * BI_PAGE_TOKENS || ldq < (int64_t)Hq * D) return BI_ERR_SHAPE;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || ldq % 8) return BI_ERR_ALIGN;
   if (T == 0) return BI_OK;
@@ -294,8 +295,9 @@ bi_status bi_attention_prefill_tc(const bi_bf16* q, int64_t ldq, int seq, int po
       !bi::gemm::make_map(&tk, k_cache, kv_rows, D, D, BI_PAGE_TOKENS) ||
       !bi::gemm::make_map(&tv, v_cache, kv_rows, D, D, BI_PAGE_TOKENS))
     return BI_ERR_CUDA;
-  const int tiles = ((T + bi::attn_tc::ROWS - 1) / bi::attn_tc::ROWS) * Hq;
-  const int grid = tiles < info->sms ? tiles : info->sms;
+  // one work item = two query heads of one kv-head over one 128-row block
+  const int work = ((T + bi::attn_tc::ROWS - 1) / bi::attn_tc::ROWS) * (Hq / 2);
+  const int grid = work < info->sms ? work : info->sms;
   const int pages_avail = (pos0 + T + BI_PAGE_TOKENS - 1) / BI_PAGE_TOKENS;
   const int32_t* prow = page_table + (int64_t)seq * max_pages_per_seq;
   const float c = (float)((double)scale * 1.4426950408889634);

@@ -183,5 +183,7 @@ def test_prefill_tc_validation(L):
     assert f(P, 4096, 1, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == SHAPE    # seq out of range
     assert f(P, 4096, 0, 4000, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == SHAPE  # past the table
     assert f(P, 4096, 0, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 96, 0.088, None) == UNSUP
+    assert f(P, 1536, 0, 0, 100, P, P, 100, P, 1, 256, P, 12, 4, 128, 0.088, None) == UNSUP  # odd group (3)
+    assert f(P, 4096, 0, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.0, None) == SHAPE     # scale <= 0
     assert f(P, 4100, 0, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == ALIGN
     assert f(P, 4096, 0, 0, 0, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == OK
