@@ -175,6 +175,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     g = pr / (G / 2);
     hA = g * G + 2 * (pr % (G / 2));
   };
+  // the CTA's k-th item: rounds of gridDim.x items in snake order (items are sorted
+  // heaviest first, so alternate rounds hand the lightest to the CTAs that got the heaviest)
+  auto item_at = [&](int k) {
+    return k * (int)gridDim.x + ((k & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+  };
   auto nblocks_of = [&](int rb) {
     const int last_row = min(T, (rb + 1) * ROWS) - 1;
     return (pos0 + last_row) / KB + 1;
@@ -184,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {  // ---- TMA producer
       int s = 0;
       uint32_t ph = 0, qph = 0;
-      for (int w = blockIdx.x; w < work && !*abort_flag; w += gridDim.x) {
+      for (int k = 0, w = item_at(0); w < work && !*abort_flag; w = item_at(++k)) {
         int g, hA, rb;
         item_of(w, g, hA, rb);
         if (!mbar_wait(Q_EMPTY, qph ^ 1u)) { *abort_flag = 1; break; }
@@ -245,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      idesc_pv<D>(), (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(O_DONE(x));
       };
-      for (int w = blockIdx.x; w < work && ok && !*abort_flag; w += gridDim.x) {
+      for (int k = 0, w = item_at(0); w < work && ok && !*abort_flag; w = item_at(++k)) {
         int g, hA, rb;
         item_of(w, g, hA, rb);
         const int nb = nblocks_of(rb);
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t sph = 0, oph = 0, kvph = 0;
     int s = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < work; w += gridDim.x) {
+    for (int k = 0, w = item_at(0); w < work; w = item_at(++k)) {
       int g, hA, rb;
       item_of(w, g, hA, rb);
       const int h = hA + x;
