@@ -18,6 +18,11 @@ the reference. Sources (web pages on batch invariance):
 * "Greedy Decoding Is Not Precision-Invariant" (arXiv 2609.26621), abstract —
   the top-2 logit margin at the LM head decides greedy flips; the LM head is
   recomputed in FP32 only when that margin is below a threshold.
+* same summary, section 他の演算子 (RMSNorm, MatMul, mean/reduction etc.) —
+  log_softmax and mean are replaced by batch-invariant kernels too; Techzine,
+  "Thinking Machines wil AI voorspelbaarder maken" — sampling and training must
+  be bit-identical for on-policy RL; French "température zéro" blog, section "Le
+  mensonge de la température zéro" — sampling made deterministic only in theory.
 
 Readings where the pages are silent (each is pinned by a test):
 * RMSNorm: y = x / sqrt(mean(x^2) + eps) * w, eps inside the root.
@@ -28,6 +33,10 @@ Readings where the pages are silent (each is pinned by a test):
 * LM head: greedy token = argmax of the logits, lowest index on ties; the
   recompute decision compares the top-2 margin of the bf16-rounded logits,
   taken in fp32, against the threshold.
+* Sampling at temperature T > 0 (no page gives a method): the Gumbel-max rule
+  over Philox4x64-10 uniforms keyed by the request's seed and step, so a row's
+  draws never depend on the batch. The sampler and the generator are algorithms,
+  not definitions: the oracle follows their published steps.
 
 Parity pins: every function here is pinned (tests/test_oracle.py).
 """
@@ -187,6 +196,117 @@ def lmhead(h: np.ndarray, w: np.ndarray, threshold: float):
         margin_bf16[m] = float(np.float32(b1) - np.float32(b2))
     return dict(logits=logits, tokens=tokens, margin=margin, margin_bf16=margin_bf16,
                 recompute=margin_bf16 < threshold, tokens_bf16=tokens_bf16)
+
+
+# ---------------------------------------------------------------------------
+# Row reductions and sampling — "Defeating Nondeterminism" summary, section
+# 他の演算子 (RMSNorm, MatMul, mean/reduction etc.): log_softmax and mean are among
+# the operations replaced by batch-invariant kernels, and a mean must be reduced in
+# one fixed order (no split, or a split of fixed size only). Why logprobs and
+# sampled tokens must match bit for bit: Techzine, "Thinking Machines wil AI
+# voorspelbaarder maken" (training and sampling bit-identical, hence truly
+# on-policy RL) and the hakusoku page's discussion of trainer/sampler numerics;
+# the French "température zéro" blog, section "Le mensonge de la température
+# zéro", on sampling made deterministic in theory but not in practice.
+
+
+def log_softmax(x: np.ndarray) -> np.ndarray:
+    """y[m, i] = x[m, i] - log(sum_j exp(x[m, j])), in float64 (max-shifted)."""
+    x = np.asarray(x, dtype=np.float64)
+    mx = x.max(axis=-1, keepdims=True)
+    return x - (mx + np.log(np.exp(x - mx).sum(axis=-1, keepdims=True)))
+
+
+def token_logprob(x: np.ndarray, tokens: np.ndarray) -> np.ndarray:
+    """log_softmax(x)[m, tokens[m]]: the log-probability of each row's token."""
+    ls = log_softmax(x)
+    return ls[np.arange(ls.shape[0]), np.asarray(tokens, dtype=np.int64)]
+
+
+def row_mean(x: np.ndarray) -> np.ndarray:
+    """y[m] = sum_k x[m, k] / K, in float64."""
+    x = np.asarray(x, dtype=np.float64)
+    return x.sum(axis=-1) / x.shape[-1]
+
+
+# Philox4x64-10, the counter-based generator of Salmon, Moraes, Dror and Shaw,
+# "Parallel random numbers: as easy as 1, 2, 3" (SC 2011): ten rounds of two 64x64
+# -> 128-bit multiplications on a 256-bit counter under a 128-bit key, with a Weyl
+# increment of the key between rounds. Written from that definition; its outputs
+# are pinned against numpy's independent implementation.
+_PHILOX_M = (np.uint64(0xD2E7470EE14C6C93), np.uint64(0xCA5A826395121157))
+_PHILOX_W = (np.uint64(0x9E3779B97F4A7C15), np.uint64(0xBB67AE8584CAA73B))
+_LO32 = np.uint64(0xFFFFFFFF)
+
+
+def _mulhilo64(a, b):
+    """(high, low) 64-bit halves of the 128-bit product a * b (uint64 arrays)."""
+    a = np.asarray(a, dtype=np.uint64)
+    b = np.asarray(b, dtype=np.uint64)
+    s32 = np.uint64(32)
+    a0, a1 = a & _LO32, a >> s32
+    b0, b1 = b & _LO32, b >> s32
+    p00, p01, p10, p11 = a0 * b0, a0 * b1, a1 * b0, a1 * b1
+    mid = (p00 >> s32) + (p01 & _LO32) + (p10 & _LO32)
+    hi = p11 + (p01 >> s32) + (p10 >> s32) + (mid >> s32)
+    with np.errstate(over="ignore"):
+        lo = a * b
+    return hi, lo
+
+
+def philox4x64_10(ctr, key):
+    """Philox4x64-10 block: ctr = 4 uint64 words (arrays broadcast), key = 2 words.
+
+    Returns the 4 output words. Round: (x0, x1, x2, x3) -> (hi(M1 x2) ^ x1 ^ k0,
+    lo(M1 x2), hi(M0 x0) ^ x3 ^ k1, lo(M0 x0)); then k += (W0, W1).
+    """
+    x = [np.asarray(c, dtype=np.uint64) for c in ctr]
+    k0, k1 = (np.asarray(k, dtype=np.uint64) for k in key)
+    with np.errstate(over="ignore"):
+        for _ in range(10):
+            hi0, lo0 = _mulhilo64(_PHILOX_M[0], x[0])
+            hi1, lo1 = _mulhilo64(_PHILOX_M[1], x[2])
+            x = [hi1 ^ x[1] ^ k0, lo1, hi0 ^ x[3] ^ k1, lo0]
+            k0 = k0 + _PHILOX_W[0]
+            k1 = k1 + _PHILOX_W[1]
+    return x
+
+
+def sampling_uniforms(seed: int, step: int, V: int) -> np.ndarray:
+    """The uniform u_i in (0, 1) drawn for vocabulary entry i of one row.
+
+    Reading (the pages give no generator): the row's request seed is the key
+    (seed, 0); the counter is (i div 4, step, 0, 0) and u_i comes from output word
+    i mod 4 as (top 23 bits + 1/2) * 2^-23 — exactly representable in fp32, never 0
+    or 1. It depends only on (seed, step, i), never on the batch.
+    """
+    i = np.arange(V, dtype=np.uint64)
+    z = np.zeros(V, dtype=np.uint64)
+    words = philox4x64_10((i >> np.uint64(2), np.full(V, step, dtype=np.uint64), z, z),
+                          (np.uint64(seed), np.uint64(0)))
+    w = np.choose((i & np.uint64(3)).astype(np.int64), words)
+    return ((w >> np.uint64(41)).astype(np.float64) + 0.5) * 2.0 ** -23
+
+
+def gumbel_scores(x: np.ndarray, temperature: float, u: np.ndarray) -> np.ndarray:
+    """x_i / T + g_i with the Gumbel variate g_i = -log(-log(u_i)), in float64."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / temperature - np.log(-np.log(np.asarray(u, dtype=np.float64)))
+
+
+def sample(x: np.ndarray, temperature: float, seeds, steps) -> np.ndarray:
+    """Temperature sampling by the Gumbel-max rule: token = argmax_i (x_i / T + g_i).
+
+    argmax of logits plus independent Gumbel noise is a draw from softmax(x / T)
+    (Gumbel 1954; the "Gumbel-max trick"). One row per request; lowest index wins
+    ties. x: [M, V].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    M, V = x.shape
+    out = np.empty(M, dtype=np.int64)
+    for m in range(M):
+        out[m] = argmax_lowest(gumbel_scores(x[m], temperature, sampling_uniforms(int(seeds[m]), int(steps[m]), V)))
+    return out
 
 
 # ---------------------------------------------------------------------------
