@@ -265,6 +265,58 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
                            void* stream);
 
 /*
+ * Row reductions for log-probabilities and means, and temperature sampling.
+ * Source: "Defeating Nondeterminism" summary, section 他の演算子 (RMSNorm, MatMul,
+ * mean/reduction etc.): log_softmax and mean get batch-invariant kernels too, a
+ * mean reduced in one fixed order. Techzine, "Thinking Machines wil AI
+ * voorspelbaarder maken": sampling and training bit-identical (on-policy RL).
+ * One CTA per row; each row is reduced in one fixed order that depends on the row
+ * length only (256 threads, each folding its 8-element vectors t, t+256, ... in
+ * order; xor-butterfly inside a warp; the 8 warp values left to right), so a row's
+ * result is the same bits whatever M and the other rows are.
+ * Inputs are bf16 [M, N] rows (16-byte aligned, ld % 8 == 0, N % 8 == 0,
+ * 8 <= N <= 2^24); M == 0 is a no-op. Rows of up to 32768 elements are read from
+ * HBM once; longer rows are re-read per pass from L2 in the same order.
+ */
+
+/* y[m, i] = x[m, i] - lse_m with lse_m = max_m + log(sum_i exp(x[m, i] - max_m)),
+ * the sum in fp32 in the order above (exp as 2^(x log2 e - max log2 e), one FMA and
+ * the SFU exp2). y: [M, N] fp32, stride ldy (ldy % 4 == 0, 16-byte aligned). */
+bi_status bi_log_softmax(const bi_bf16* x, int64_t ldx, float* y, int64_t ldy, int64_t M, int64_t N,
+                         void* stream);
+
+/* out[m] = x[m, tokens[m]] - lse_m (the same lse_m as bi_log_softmax): the
+ * log-probability of each row's token. tokens: [M] int32 device; a token outside
+ * 0..N-1 gives NaN and BI_ERR_DEVICE_INDEX in the device error word. out: [M] fp32. */
+bi_status bi_token_logprob(const bi_bf16* x, int64_t ldx, const int32_t* tokens, float* out, int64_t M,
+                           int64_t N, void* stream);
+
+/* y[m] = (sum_k x[m, k]) / K, the sum in fp32 in the order above, one division. y: [M] fp32. */
+bi_status bi_row_mean(const bi_bf16* x, int64_t ldx, float* y, int64_t M, int64_t K, void* stream);
+
+/*
+ * The uniforms the sampler draws: u[m, i] in (0, 1) for vocabulary entry i of row m,
+ * from Philox4x64-10 (Salmon et al., "Parallel random numbers: as easy as 1, 2, 3",
+ * SC 2011) with key (seeds[m], 0) and counter (i / 4, steps[m], 0, 0), output word
+ * i % 4, u = (top 23 bits + 1/2) * 2^-23 (exact in fp32). A row's draws depend on
+ * (seed, step, i) only: the request's seed and its decode step, never the batch.
+ * seeds, steps: [M] uint64 device. u: [M, V] fp32, stride ldu (ldu % 4 == 0).
+ */
+bi_status bi_sampling_uniforms(const uint64_t* seeds, const uint64_t* steps, float* u, int64_t ldu, int64_t M,
+                               int64_t V, void* stream);
+
+/*
+ * Temperature sampling by the Gumbel-max rule: tokens[m] = argmax_i
+ * fma(x[m, i], 1/T, g_i) in fp32 with g_i = -log(-log u[m, i]) (the uniforms of
+ * bi_sampling_uniforms) and 1/T rounded once; lowest index among equal scores. A
+ * draw from softmax(x / T) that depends on (logits, seed, step) only. logits: [M, V]
+ * bf16 (e.g. the bi_matmul LM-head output); temperature: finite, > 0; tokens: [M]
+ * int32 out. A row whose scores are all NaN gives token 0 and BI_ERR_DEVICE_INDEX.
+ */
+bi_status bi_sample(const bi_bf16* logits, int64_t ld, const uint64_t* seeds, const uint64_t* steps,
+                    float temperature, int32_t* tokens, int64_t M, int64_t V, void* stream);
+
+/*
  * Self-test of the device-side failure detection (no page describes it). Launches
  * one thread that waits on an mbarrier nothing will complete, using the same
  * bounded wait as every kernel here but a limit of limit_ms milliseconds (1..2000;

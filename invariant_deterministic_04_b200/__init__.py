@@ -7,7 +7,8 @@ libbi.so is missing or fails to load, every call raises ``BIError``.
 
 Operations (see include/bi.h for the exact contracts):
   rmsnorm, matmul, attention_decode, attention_decode_static, attention_prefill,
-  kv_append, lmhead_argmax, gather_rows, rope, swiglu, add, get_device_error.
+  kv_append, lmhead_argmax, gather_rows, rope, swiglu, add, log_softmax,
+  token_logprob, row_mean, sampling_uniforms, sample, get_device_error.
 """
 from __future__ import annotations
 
@@ -55,6 +56,11 @@ _SIGNATURES = {
     "bi_add": ([_P, _P, _P, _I64, _P], _I32),
     "bi_lmhead_workspace_size": ([_I64, _I64], _SZ),
     "bi_lmhead_argmax": ([_P, _I64, _P, _I64, _I64, _I64, _F, _P, _P, _P, _P, _SZ, _P], _I32),
+    "bi_log_softmax": ([_P, _I64, _P, _I64, _I64, _I64, _P], _I32),
+    "bi_token_logprob": ([_P, _I64, _P, _P, _I64, _I64, _P], _I32),
+    "bi_row_mean": ([_P, _I64, _P, _I64, _I64, _P], _I32),
+    "bi_sampling_uniforms": ([_P, _P, _P, _I64, _I64, _I64, _P], _I32),
+    "bi_sample": ([_P, _I64, _P, _P, _F, _P, _I64, _I64, _P], _I32),
     "bi_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], _I32),
     "bi_selftest_wait_timeout": ([_I32, _P], _I32),
 }
@@ -376,6 +382,70 @@ def lmhead_argmax(h, w, margin_threshold: float = 0.5, want_logits: bool = False
         _ptr(h), h.stride(0), _ptr(w), M, V, K, margin_threshold, _ptr(tokens), _ptr(recomputed),
         _ptr(logits_fp32), _ptr(ws), nbytes, _stream(stream)))
     return tokens, recomputed, logits_fp32
+
+
+def _rows2(x: torch.Tensor, name: str):
+    _req(x, torch.bfloat16, name, 2)
+    if x.stride(1) != 1:
+        raise ValueError(f"{name} rows must be contiguous")
+    return x.shape
+
+
+def _u64(t: torch.Tensor, name: str, M: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype not in (torch.int64, torch.uint64):
+        raise TypeError(f"{name} must be a CUDA int64/uint64 tensor (raw 64-bit words)")
+    if t.shape != (M,):
+        raise ValueError(f"{name} must have shape ({M},)")
+    _contig(t, name)
+
+
+def log_softmax(x, out=None, stream=None):
+    """fp32 log_softmax of each bf16 row, one fixed reduction order per row."""
+    M, N = _rows2(x, "x")
+    y = torch.empty((M, N), dtype=torch.float32, device=x.device) if out is None else out
+    _req(y, torch.float32, "out", 2)
+    _check("bi_log_softmax", lib().bi_log_softmax(_ptr(x), x.stride(0), _ptr(y), y.stride(0), M, N, _stream(stream)))
+    return y
+
+
+def token_logprob(x, tokens, out=None, stream=None):
+    """fp32 log-probability of tokens[m] under log_softmax(x[m])."""
+    M, N = _rows2(x, "x")
+    _req(tokens, torch.int32, "tokens", 1)
+    out = torch.empty(M, dtype=torch.float32, device=x.device) if out is None else out
+    _check("bi_token_logprob", lib().bi_token_logprob(_ptr(x), x.stride(0), _ptr(tokens), _ptr(out), M, N,
+                                                     _stream(stream)))
+    return out
+
+
+def row_mean(x, out=None, stream=None):
+    """fp32 mean of each bf16 row, one fixed reduction order per row."""
+    M, K = _rows2(x, "x")
+    out = torch.empty(M, dtype=torch.float32, device=x.device) if out is None else out
+    _check("bi_row_mean", lib().bi_row_mean(_ptr(x), x.stride(0), _ptr(out), M, K, _stream(stream)))
+    return out
+
+
+def sampling_uniforms(seeds, steps, V: int, out=None, stream=None):
+    """The (0, 1) uniforms the sampler draws for rows (seed, step): fp32 [M, V]."""
+    M = seeds.shape[0]
+    _u64(seeds, "seeds", M)
+    _u64(steps, "steps", M)
+    u = torch.empty((M, V), dtype=torch.float32, device=seeds.device) if out is None else out
+    _check("bi_sampling_uniforms", lib().bi_sampling_uniforms(_ptr(seeds), _ptr(steps), _ptr(u), u.stride(0), M, V,
+                                                             _stream(stream)))
+    return u
+
+
+def sample(logits, seeds, steps, temperature: float, out=None, stream=None):
+    """Gumbel-max temperature sampling: int32 [M] tokens from bf16 logits [M, V]."""
+    M, V = _rows2(logits, "logits")
+    _u64(seeds, "seeds", M)
+    _u64(steps, "steps", M)
+    out = torch.empty(M, dtype=torch.int32, device=logits.device) if out is None else out
+    _check("bi_sample", lib().bi_sample(_ptr(logits), logits.stride(0), _ptr(seeds), _ptr(steps), temperature,
+                                       _ptr(out), M, V, _stream(stream)))
+    return out
 
 
 def selftest_wait_timeout(limit_ms: int = 50, stream=None):

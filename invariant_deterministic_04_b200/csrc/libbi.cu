@@ -14,6 +14,7 @@
 #include "lmhead.cuh"
 #include "glue.cuh"
 #include "attention_tc.cuh"
+#include "reduce.cuh"
 
 namespace {
 
@@ -198,7 +199,7 @@ const char* bi_status_string(int status) {
   }
 }
 
-int bi_version(void) { return 2; }
+int bi_version(void) { return 3; }
 
 bi_status bi_rmsnorm(const bi_bf16* x, int64_t ldx, const bi_bf16* w, bi_bf16* y, int64_t ldy, int64_t M,
                      int64_t K, float eps, void* stream) {
@@ -434,6 +435,70 @@ bi_status bi_get_device_error(int32_t* code) {
   if (cudaMemcpyToSymbol(bi::g_error_word, &zero, sizeof(int)) != cudaSuccess) return BI_ERR_CUDA;
   *code = v;
   return BI_OK;
+}
+
+// ---- row reductions and sampling
+
+namespace {
+
+bi_status rows_check(const void* x, int64_t ldx, int64_t M, int64_t N) {
+  if (M < 0 || M > INT_MAX || N < 8 || N % 8 != 0 || N > (int64_t(1) << 24) || ldx < N) return BI_ERR_SHAPE;
+  if (!aligned16(x) || ldx % 8) return BI_ERR_ALIGN;
+  return BI_OK;
+}
+
+}  // namespace
+
+bi_status bi_log_softmax(const bi_bf16* x, int64_t ldx, float* y, int64_t ldy, int64_t M, int64_t N,
+                         void* stream) {
+  if (!x || !y) return BI_ERR_NULL;
+  if (bi_status e = rows_check(x, ldx, M, N)) return e;
+  if (ldy < N) return BI_ERR_SHAPE;
+  if (!aligned16(y) || ldy % 4) return BI_ERR_ALIGN;
+  if (M == 0) return BI_OK;
+  if (ranges_overlap(x, span_bytes(M, N, ldx, 2), y, span_bytes(M, N, ldy, 4))) return BI_ERR_SHAPE;
+  BI_RED_DISPATCH(bi::red::log_softmax_kernel, N, (unsigned)M, as_stream(stream), x, ldx, y, ldy, (int)N);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_token_logprob(const bi_bf16* x, int64_t ldx, const int32_t* tokens, float* out, int64_t M,
+                           int64_t N, void* stream) {
+  if (!x || !tokens || !out) return BI_ERR_NULL;
+  if (bi_status e = rows_check(x, ldx, M, N)) return e;
+  if (M == 0) return BI_OK;
+  BI_RED_DISPATCH(bi::red::token_logprob_kernel, N, (unsigned)M, as_stream(stream), x, ldx, tokens, out, (int)N);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_row_mean(const bi_bf16* x, int64_t ldx, float* y, int64_t M, int64_t K, void* stream) {
+  if (!x || !y) return BI_ERR_NULL;
+  if (bi_status e = rows_check(x, ldx, M, K)) return e;
+  if (M == 0) return BI_OK;
+  BI_RED_DISPATCH(bi::red::row_mean_kernel, K, (unsigned)M, as_stream(stream), x, ldx, y, (int)K);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_sampling_uniforms(const uint64_t* seeds, const uint64_t* steps, float* u, int64_t ldu, int64_t M,
+                               int64_t V, void* stream) {
+  if (!seeds || !steps || !u) return BI_ERR_NULL;
+  if (M < 0 || M > INT_MAX || V < 8 || V % 8 != 0 || V > (int64_t(1) << 24) || ldu < V) return BI_ERR_SHAPE;
+  if (!aligned16(u) || ldu % 4) return BI_ERR_ALIGN;
+  if (M == 0) return BI_OK;
+  bi::red::uniforms_kernel<<<(unsigned)M, bi::red::kThreads, 0, as_stream(stream)>>>(seeds, steps, u, ldu, (int)V);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status bi_sample(const bi_bf16* logits, int64_t ld, const uint64_t* seeds, const uint64_t* steps,
+                    float temperature, int32_t* tokens, int64_t M, int64_t V, void* stream) {
+  if (!logits || !seeds || !steps || !tokens) return BI_ERR_NULL;
+  if (bi_status e = rows_check(logits, ld, M, V)) return e;
+  if (!std::isfinite(temperature) || !(temperature > 0.f)) return BI_ERR_SHAPE;
+  const float inv_t = 1.0f / temperature;  // IEEE division: 1/T rounded once
+  if (!std::isfinite(inv_t)) return BI_ERR_SHAPE;
+  if (M == 0) return BI_OK;
+  BI_RED_DISPATCH(bi::red::sample_kernel, V, (unsigned)M, as_stream(stream), logits, ld, seeds, steps, inv_t, tokens,
+                  (int)V);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
 }  // extern "C"

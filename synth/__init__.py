@@ -13,7 +13,10 @@ Recipe (all on the CPU, ``torch.Generator`` seeded per call):
     ``[num_pages, Hkv, 16, D]``; each sequence's logical pages map to a seeded
     random permutation of the physical pages; page-table entries past a
     sequence's last page are -1; decode lengths ~ U[1, max_len];
-  * LM head: h ~ N(0, 1), W ~ N(0, 0.02) stored [V, K].
+  * LM head: h ~ N(0, 1), W ~ N(0, 0.02) stored [V, K];
+  * logits for log_softmax / sampling: N(0, 3^2) bf16 rows (the spread of a
+    trained LM head's logits); row means: x ~ N(0.5, 1);
+  * request seeds: uniform 64-bit words; decode steps: small integers.
 """
 from __future__ import annotations
 
@@ -154,6 +157,19 @@ def lmhead_inputs(M: int, V: int, K: int, seed: int = 0):
     h = normal_bf16((M, K), seed)
     w = normal_bf16((V, K), seed + 1, std=0.02)
     return h, w
+
+
+def logits(M: int, V: int, seed: int = 0, std: float = 3.0) -> torch.Tensor:
+    """bf16 [M, V] logit rows ~ N(0, std^2)."""
+    return normal_bf16((M, V), seed, std=std)
+
+
+def request_seeds(M: int, seed: int) -> torch.Tensor:
+    """[M] int64 tensor holding uniform 64-bit words (the bits of uint64 request seeds)."""
+    g = generator(seed)
+    hi = torch.randint(0, 2**32, (M,), generator=g, dtype=torch.int64)
+    lo = torch.randint(0, 2**32, (M,), generator=g, dtype=torch.int64)
+    return (hi << 32) | lo
 
 
 def permutation(n: int, seed: int) -> torch.Tensor:

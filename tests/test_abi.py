@@ -45,7 +45,7 @@ def test_status_strings(L):
     assert L.bi_status_string(0) == b"BI_OK"
     assert L.bi_status_string(4) == b"BI_ERR_WORKSPACE"
     assert L.bi_status_string(99) == b"BI_ERR_UNKNOWN"
-    assert L.bi_version() == 2
+    assert L.bi_version() == 3
 
 
 def test_rmsnorm_validation(L):
@@ -159,6 +159,39 @@ def test_lmhead_validation(L):
     assert f(P, 2048, P, 4, 32000, 2048, 0.5, P, P, None, None, ws, None) == WS
     assert f(P, 2048, P, 4, 32000, 2048, 0.5, P, P, P + 4, P, ws, None) == ALIGN
     assert f(P, 2048, P, 0, 32000, 2048, 0.5, P, P, None, None, 0, None) == OK
+
+
+def test_reduction_and_sampling_validation(L):
+    Y = P + (1 << 30)  # a second, non-overlapping stand-in address
+    ls, tl, mean, uni, smp = (L.bi_log_softmax, L.bi_token_logprob, L.bi_row_mean, L.bi_sampling_uniforms,
+                              L.bi_sample)
+    assert ls(None, 32000, Y, 32000, 4, 32000, None) == NULL
+    assert ls(P, 32000, Y, 32000, 4, 31999, None) == SHAPE          # N % 8
+    assert ls(P, 32000, Y, 32000, 4, 0, None) == SHAPE
+    assert ls(P, 32000, Y, 32000, 4, (1 << 24) + 8, None) == SHAPE  # N > 2^24
+    assert ls(P, 16000, Y, 32000, 4, 32000, None) == SHAPE          # ldx < N
+    assert ls(P, 32000, Y, 16000, 4, 32000, None) == SHAPE          # ldy < N
+    assert ls(P, 32000, P + 8, 32000, 4, 32000, None) == ALIGN      # y not 16-byte aligned
+    assert ls(P, 32000, Y, 32002, 4, 32000, None) == ALIGN          # ldy % 4
+    assert ls(P, 32004, Y, 32000, 4, 32000, None) == ALIGN          # ldx % 8
+    assert ls(P, 32000, P + 64, 32000, 4, 32000, None) == SHAPE     # y overlaps x
+    assert ls(P, 32000, Y, 32000, 0, 32000, None) == OK
+    assert tl(P, 32000, None, Y, 4, 32000, None) == NULL
+    assert tl(P, 32000, P, Y, -1, 32000, None) == SHAPE
+    assert tl(P, 32000, P, Y, 0, 32000, None) == OK
+    assert mean(P, 4096, None, 4, 4096, None) == NULL
+    assert mean(P + 2, 4096, Y, 4, 4096, None) == ALIGN
+    assert mean(P, 4096, Y, 4, 4100, None) == SHAPE                 # ldx < K
+    assert mean(P, 4096, Y, 0, 4096, None) == OK
+    assert uni(None, P, Y, 32000, 4, 32000, None) == NULL
+    assert uni(P, P, Y, 32000, 4, 31996, None) == SHAPE             # V % 8
+    assert uni(P, P, Y + 4, 32000, 4, 32000, None) == ALIGN
+    assert uni(P, P, Y, 32000, 0, 32000, None) == OK
+    assert smp(P, 32000, P, P, 0.8, None, 4, 32000, None) == NULL
+    for t in (0.0, -1.0, float("inf"), float("nan"), 1e-45):        # T <= 0, not finite, 1/T overflows
+        assert smp(P, 32000, P, P, t, Y, 4, 32000, None) == SHAPE, t
+    assert smp(P, 32000, P, P, 0.8, Y, 4, 32004, None) == SHAPE     # ld < V
+    assert smp(P, 32000, P, P, 0.8, Y, 0, 32000, None) == OK
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
