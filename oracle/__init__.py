@@ -276,16 +276,19 @@ def sampling_uniforms(seed: int, step: int, V: int) -> np.ndarray:
     """The uniform u_i in (0, 1) drawn for vocabulary entry i of one row.
 
     Reading (the pages give no generator): the row's request seed is the key
-    (seed, 0); the counter is (i div 4, step, 0, 0) and u_i comes from output word
-    i mod 4 as (top 23 bits + 1/2) * 2^-23 — exactly representable in fp32, never 0
-    or 1. It depends only on (seed, step, i), never on the batch.
+    (seed, 0); the counter is (i div 8, step, 0, 0); one block's four 64-bit words
+    give eight 32-bit halves, entry i taking word (i mod 8) div 2, its low half for
+    even i and its high half for odd i; u_i = (top 23 bits of that half + 1/2) *
+    2^-23 — exactly representable in fp32, never 0 or 1. It depends only on
+    (seed, step, i), never on the batch.
     """
     i = np.arange(V, dtype=np.uint64)
     z = np.zeros(V, dtype=np.uint64)
-    words = philox4x64_10((i >> np.uint64(2), np.full(V, step, dtype=np.uint64), z, z),
+    words = philox4x64_10((i >> np.uint64(3), np.full(V, step, dtype=np.uint64), z, z),
                           (np.uint64(seed), np.uint64(0)))
-    w = np.choose((i & np.uint64(3)).astype(np.int64), words)
-    return ((w >> np.uint64(41)).astype(np.float64) + 0.5) * 2.0 ** -23
+    w = np.choose(((i >> np.uint64(1)) & np.uint64(3)).astype(np.int64), words)
+    half = np.where((i & np.uint64(1)) == 0, w & _LO32, w >> np.uint64(32))
+    return ((half >> np.uint64(9)).astype(np.float64) + 0.5) * 2.0 ** -23
 
 
 def gumbel_scores(x: np.ndarray, temperature: float, u: np.ndarray) -> np.ndarray:

@@ -98,11 +98,13 @@ def test_philox_matches_numpy_bit_generator(counter, key):
 def test_sampling_uniforms_layout_and_range():
     seed, step, V = 0x1234_5678_9ABC_DEF0, 17, 1003
     u = oracle.sampling_uniforms(seed, step, V)
-    # u_i = (top 23 bits of word i mod 4 of block (i div 4, step) + 1/2) * 2^-23
-    for i in (0, 1, 2, 3, 4, 998, 1002):
-        words = oracle.philox4x64_10(_words(i // 4, 1) + [np.uint64(step), np.uint64(0), np.uint64(0)],
+    # u_i = (top 23 bits of 32-bit half i mod 2 (low, high) of word (i mod 8) div 2 of
+    # block (i div 8, step) + 1/2) * 2^-23, by Python integers
+    for i in (0, 1, 2, 3, 7, 8, 9, 998, 1002):
+        words = oracle.philox4x64_10(_words(i // 8, 1) + [np.uint64(step), np.uint64(0), np.uint64(0)],
                                      [np.uint64(seed), np.uint64(0)])
-        assert u[i] == ((int(words[i % 4]) >> 41) + 0.5) / 2**23
+        half = (int(words[(i % 8) // 2]) >> (32 * (i % 2))) & 0xFFFFFFFF
+        assert u[i] == ((half >> 9) + 0.5) / 2**23
     assert np.all((u > 0) & (u < 1))
     assert np.all((u * 2**23 - 0.5) == np.floor(u * 2**23))
     assert np.all(u.astype(np.float32).astype(np.float64) == u)  # exact in fp32
