@@ -281,6 +281,30 @@ def _events_ms(fn, iters=10, warmup=3):
     return s.elapsed_time(e) / iters
 
 
+def _graph_us(fn, n=20, reps=10):
+    """Device microseconds per call of fn, from a CUDA graph of n calls replayed reps times."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(n):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    del g
+    return s.elapsed_time(e) * 1e3 / (n * reps)
+
+
 def other_rows(bi, device, pk, only=None):
     out = {}
     want = (lambda name: only is None or only == name)
@@ -293,6 +317,8 @@ def other_rows(bi, device, pk, only=None):
         out.update(_row_prefill(bi, device, pk))
     if want("lmhead"):
         out.update(_row_lmhead(bi, device, pk))
+    if want("reduce"):
+        out.update(_row_reduce(bi, device, pk))
     return out
 
 
@@ -401,6 +427,50 @@ def _row_lmhead(bi, device, pk):
     ms_ref = _events_ms(lambda: torch.argmax(torch.matmul(h, Wl.t()), dim=1))
     out["lmhead_m64_v32000"] = {"ms": round(ms, 4), "recomputed_rows": int(rec.sum()),
                                 "slowdown_vs_cublas_argmax": round(ms / ms_ref, 3)}
+    return out
+
+
+def _row_reduce(bi, device, pk):
+    out = {}
+    hbm = pk["hbm_gbs"]
+    # log-probabilities of a 4096-token sequence over a 32000 vocabulary (bf16 in,
+    # fp32 out: 786 MB, far above L2), its token log-probabilities, and sampling
+    M, V = 4096, 32000
+    x = synth.logits(M, V, seed=110).to(device)
+    y = torch.empty((M, V), dtype=torch.float32, device=device)
+    tok = torch.randint(0, V, (M,), generator=synth.generator(111), dtype=torch.int32).to(device)
+    lp = torch.empty(M, dtype=torch.float32, device=device)
+    seeds = synth.request_seeds(M, 112).to(device)
+    steps = torch.zeros(M, dtype=torch.int64, device=device)
+    st = torch.empty(M, dtype=torch.int32, device=device)
+    ms = _events_ms(lambda: bi.log_softmax(x, out=y))
+    ms_ref = _events_ms(lambda: torch.log_softmax(x, dim=-1, dtype=torch.float32))
+    gbs = M * V * 6 / ms / 1e6
+    out["log_softmax_m4096_v32000"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+                                       "slowdown_vs_torch": round(ms / ms_ref, 3)}
+    ms = _events_ms(lambda: bi.token_logprob(x, tok, out=lp))
+    gbs = M * V * 2 / ms / 1e6
+    out["token_logprob_m4096_v32000"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3)}
+    ms = _events_ms(lambda: bi.sample(x, seeds, steps, 0.8, out=st))
+    # non-invariant comparison: torch's Gumbel-max with its own generator (batch-dependent draws)
+    ms_ref = _events_ms(lambda: torch.argmax(x.float() / 0.8 - torch.log(-torch.log(torch.rand_like(x, dtype=torch.float32))),
+                                             dim=-1))
+    gbs = M * V * 2 / ms / 1e6
+    out["sample_m4096_v32000"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+                                  "slowdown_vs_torch_gumbel": round(ms / ms_ref, 3)}
+    # a decode-sized batch: 20 launches captured in a CUDA graph, so the host's
+    # per-call cost does not hide the device time
+    xs, s64, t64, o64 = x[:64].contiguous(), seeds[:64].contiguous(), steps[:64].contiguous(), st[:64]
+    out["sample_m64_v32000"] = {"us": round(_graph_us(lambda: bi.sample(xs, s64, t64, 0.8, out=o64)), 2)}
+    out["log_softmax_m64_v32000"] = {"us": round(_graph_us(lambda: bi.log_softmax(xs, out=y[:64])), 2)}
+    # row means of 65536 x 4096 bf16 (512 MiB)
+    xm = synth.normal_bf16((65536, 4096), 113, mean=0.5).to(device)
+    ym = torch.empty(65536, dtype=torch.float32, device=device)
+    ms = _events_ms(lambda: bi.row_mean(xm, out=ym))
+    ms_ref = _events_ms(lambda: torch.mean(xm, dim=-1, dtype=torch.float32))
+    gbs = xm.numel() * 2 / ms / 1e6
+    out["row_mean_m65536_k4096"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 3),
+                                    "slowdown_vs_torch": round(ms / ms_ref, 3)}
     return out
 
 
@@ -598,7 +668,7 @@ def main():
     ap.add_argument("--no-rows", dest="rows", action="store_false")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="the K=4096 M sweep, one JSON line per shape")
-    ap.add_argument("--row", choices=["rmsnorm", "decode", "prefill", "lmhead"], default=None,
+    ap.add_argument("--row", choices=["rmsnorm", "decode", "prefill", "lmhead", "reduce"], default=None,
                     help="measure only this hot-path kernel (for profiling) and print its line")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args()

@@ -297,8 +297,9 @@ bi_status bi_row_mean(const bi_bf16* x, int64_t ldx, float* y, int64_t M, int64_
 /*
  * The uniforms the sampler draws: u[m, i] in (0, 1) for vocabulary entry i of row m,
  * from Philox4x64-10 (Salmon et al., "Parallel random numbers: as easy as 1, 2, 3",
- * SC 2011) with key (seeds[m], 0) and counter (i / 4, steps[m], 0, 0), output word
- * i % 4, u = (top 23 bits + 1/2) * 2^-23 (exact in fp32). A row's draws depend on
+ * SC 2011) with key (seeds[m], 0) and counter (i / 8, steps[m], 0, 0): entry i takes
+ * output word (i % 8) / 2, its low 32 bits for even i and its high 32 bits for odd i,
+ * and u = (top 23 of those 32 bits + 1/2) * 2^-23 (exact in fp32). A row's draws depend on
  * (seed, step, i) only: the request's seed and its decode step, never the batch.
  * seeds, steps: [M] uint64 device. u: [M, V] fp32, stride ldu (ldu % 4 == 0).
  */
@@ -312,6 +313,8 @@ bi_status bi_sampling_uniforms(const uint64_t* seeds, const uint64_t* steps, flo
  * draw from softmax(x / T) that depends on (logits, seed, step) only. logits: [M, V]
  * bf16 (e.g. the bi_matmul LM-head output); temperature: finite, > 0; tokens: [M]
  * int32 out. A row whose scores are all NaN gives token 0 and BI_ERR_DEVICE_INDEX.
+ * Each row runs on a cluster of 8 CTAs, each taking a fixed eighth of the vocabulary
+ * (the argmax is exact, so the split does not change the token).
  */
 bi_status bi_sample(const bi_bf16* logits, int64_t ld, const uint64_t* seeds, const uint64_t* steps,
                     float temperature, int32_t* tokens, int64_t M, int64_t V, void* stream);

@@ -492,12 +492,13 @@ bi_status bi_sample(const bi_bf16* logits, int64_t ld, const uint64_t* seeds, co
                     float temperature, int32_t* tokens, int64_t M, int64_t V, void* stream) {
   if (!logits || !seeds || !steps || !tokens) return BI_ERR_NULL;
   if (bi_status e = rows_check(logits, ld, M, V)) return e;
+  if (M > INT_MAX / bi::red::kSampleParts) return BI_ERR_SHAPE;
   if (!std::isfinite(temperature) || !(temperature > 0.f)) return BI_ERR_SHAPE;
   const float inv_t = 1.0f / temperature;  // IEEE division: 1/T rounded once
   if (!std::isfinite(inv_t)) return BI_ERR_SHAPE;
   if (M == 0) return BI_OK;
-  BI_RED_DISPATCH(bi::red::sample_kernel, V, (unsigned)M, as_stream(stream), logits, ld, seeds, steps, inv_t, tokens,
-                  (int)V);
+  bi::red::sample_kernel<<<(unsigned)(M * bi::red::kSampleParts), bi::red::kThreads, 0, as_stream(stream)>>>(
+      logits, ld, seeds, steps, inv_t, tokens, (int)V);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

@@ -201,19 +201,20 @@ __device__ __forceinline__ U64x4 philox4x64_10(uint64_t c0, uint64_t c1, uint64_
   return U64x4{{c0, c1, c2, c3}};
 }
 
-// u in (0, 1): (top 23 bits of the word + 1/2) * 2^-23, exact in fp32
-__device__ __forceinline__ float word_to_uniform(uint64_t w) {
-  return __fmul_rn(__fadd_rn((float)(uint32_t)(w >> 41), 0.5f), 1.1920928955078125e-07f);
+// u in (0, 1): (top 23 bits of a 32-bit half + 1/2) * 2^-23, exact in fp32
+__device__ __forceinline__ float half_to_uniform(uint32_t h) {
+  return __fmul_rn(__fadd_rn((float)(h >> 9), 0.5f), 1.1920928955078125e-07f);
 }
 
-// The uniforms of vocabulary entries 8 idx .. 8 idx + 7 of a row: two Philox blocks,
-// counters (2 idx, step) and (2 idx + 1, step), key (seed, 0); entry i takes word i mod 4.
+// The uniforms of vocabulary entries 8 idx .. 8 idx + 7 of a row: one Philox block,
+// counter (idx, step), key (seed, 0); entry 8 idx + k takes word k / 2, its low half
+// for even k and its high half for odd k.
 __device__ __forceinline__ void uniforms8(uint64_t seed, uint64_t step, int idx, float (&u)[8]) {
+  const U64x4 r = philox4x64_10((uint64_t)idx, step, 0ull, 0ull, seed, 0ull);
 #pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    const U64x4 r = philox4x64_10((uint64_t)(2 * idx + b), step, 0ull, 0ull, seed, 0ull);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) u[4 * b + k] = word_to_uniform(r.w[k]);
+  for (int k = 0; k < 4; ++k) {
+    u[2 * k] = half_to_uniform((uint32_t)r.w[k]);
+    u[2 * k + 1] = half_to_uniform((uint32_t)(r.w[k] >> 32));
   }
 }
 
@@ -234,32 +235,69 @@ __global__ void __launch_bounds__(kThreads) uniforms_kernel(const uint64_t* __re
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi_) { return v > bv || (v == bv && i < bi_); }
 
 // Temperature sampling by the Gumbel-max rule: token = argmax_i (x_i / T + g_i) with
-// g_i = -log(-log u_i), score = fma(x_i, 1/T, g_i) in fp32 (1/T rounded once).
-template <int NV>
-__global__ void __launch_bounds__(kThreads) sample_kernel(const uint16_t* __restrict__ x, int64_t ldx,
-                                                          const uint64_t* __restrict__ seeds,
-                                                          const uint64_t* __restrict__ steps, float inv_t,
-                                                          int32_t* __restrict__ tokens, int V) {
+// g_i = -log(-log u_i), score = fma(x_i, 1/T, g_i) in fp32 (1/T rounded once). The
+// inner log is the accurate logf (for u near 1, -log u is tiny and its relative
+// error would pass straight into g); the outer one is the SFU log2 times ln 2, whose
+// absolute error (~1e-7) is what g sees.
+// A row is split over a cluster of kSampleParts CTAs, part p taking vectors
+// p * ceil(n/8) .. of the row's n 8-element vectors (a split fixed by V alone); the
+// parts' (score, index) maxima meet in CTA 0 through distributed shared memory. An
+// argmax is exact, so the split does not change the result.
+constexpr int kSampleParts = 8;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t a) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+
+__global__ void __cluster_dims__(kSampleParts, 1, 1) __launch_bounds__(kThreads)
+    sample_kernel(const uint16_t* __restrict__ x, int64_t ldx, const uint64_t* __restrict__ seeds,
+                  const uint64_t* __restrict__ steps, float inv_t, int32_t* __restrict__ tokens, int V) {
   __shared__ float shv[kWarps];
   __shared__ int shi[kWarps];
-  Row<NV> row;
-  row.load(x + (int64_t)blockIdx.x * ldx, V);
-  const uint64_t seed = seeds[blockIdx.x], step = steps[blockIdx.x];
+  __shared__ float part_v;
+  __shared__ int part_i;
+  const int row = blockIdx.x / kSampleParts;
+  const uint32_t part = cluster_rank();
+  const int nvec = V >> 3, per = (nvec + kSampleParts - 1) / kSampleParts;
+  const int v0 = (int)part * per, v1 = min(nvec, v0 + per);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (int64_t)row * ldx);
+  const uint64_t seed = seeds[row], step = steps[row];
   float bv = -INFINITY;
   int bidx = INT_MAX;
-  row.each([&](int idx, const float(&e)[8]) {
-    float u[8];
+  for (int idx = v0 + (int)threadIdx.x; idx < v1; idx += kThreads) {
+    float e[8], u[8];
+    unpack8(__ldcs(xr + idx), e);
     uniforms8(seed, step, idx, u);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float g = -logf(-logf(u[k]));
-      const float s = __fmaf_rn(e[k], inv_t, g);
-      if (better(s, 8 * idx + k, bv, bidx)) {
-        bv = s;
+      const float g = -__logf(-logf(u[k]));
+      const float sc = __fmaf_rn(e[k], inv_t, g);
+      if (better(sc, 8 * idx + k, bv, bidx)) {
+        bv = sc;
         bidx = 8 * idx + k;
       }
     }
-  });
+  }
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) {
     const float ov = __shfl_xor_sync(kFullMask, bv, off);
@@ -282,13 +320,29 @@ __global__ void __launch_bounds__(kThreads) sample_kernel(const uint16_t* __rest
         v = shv[w];
         i = shi[w];
       }
+    part_v = v;
+    part_i = i;
+  }
+  cluster_barrier();  // every part's maximum is in its shared memory
+  if (part == 0 && threadIdx.x == 0) {
+    float v = part_v;
+    int i = part_i;
+    for (uint32_t p = 1; p < kSampleParts; ++p) {
+      const float pv = ld_cluster_f32(map_to_rank(smem_u32(&part_v), p));
+      const int pi = ld_cluster_s32(map_to_rank(smem_u32(&part_i), p));
+      if (better(pv, pi, v, i)) {
+        v = pv;
+        i = pi;
+      }
+    }
     // a row whose scores are all NaN (NaN logits) has no maximum: report index 0 and the error
     if (i == INT_MAX) {
       record_error(BI_ERR_DEVICE_INDEX);
       i = 0;
     }
-    tokens[blockIdx.x] = i;
+    tokens[row] = i;
   }
+  cluster_barrier();  // no part leaves while part 0 may still read its shared memory
 }
 
 // vectors per thread of the register-resident variant for a row of N elements, or 0
