@@ -367,7 +367,8 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
   bi::lmhead::compact_kernel<<<1, 1024, 0, st>>>(recomputed, (int)M, lay.list);
   float* out32 = logits_fp32 ? logits_fp32 : lay.logits32;
   const dim3 rgrid((unsigned)((V + bi::lmhead::VB - 1) / bi::lmhead::VB), (unsigned)((M + bi::lmhead::RB - 1) / bi::lmhead::RB));
-  bi::lmhead::recompute_kernel<<<rgrid, 256, 0, st>>>(h, ldh, W, V, (int)K, (int)M, lay.list, out32);
+  bi::lmhead::recompute_kernel<<<rgrid, bi::lmhead::kRecThreads, 0, st>>>(h, ldh, W, V, (int)K, (int)M, lay.list,
+                                                                         out32);
   bi::lmhead::argmax_kernel<<<(unsigned)M, bi::lmhead::kThreads, 0, st>>>(out32, V, recomputed, tokens);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }

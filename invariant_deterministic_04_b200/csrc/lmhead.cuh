@@ -112,66 +112,68 @@ __global__ void __launch_bounds__(1024) compact_kernel(const int32_t* __restrict
 // fp32 logits of flagged rows: out[row, v] = sum_k h[row, k] * W[v, k], one FMA
 // chain in ascending k per logit (the packed f32x2 FMA below carries two logits of
 // two vocabulary entries, each element rounded exactly like a scalar FMA).
-// Tile: 64 flagged rows x 256 vocabulary rows per CTA of 8 warps; warp w owns rows
-// 8w .. 8w+7 and lane l the vocabulary entries 4l .. 4l+3 and 128+4l .. 128+4l+3
-// (8 x 8 logits per thread). k is staged KB at a time through shared memory: W
-// transposed to [k][vocab], h as duplicated pairs [k][row] (one 16-byte load gives
-// two rows ready for the packed FMA); a warp's staging stores cover one k-row, so
-// they are free of bank conflicts, and the next slab is prefetched into registers
-// while the current one is consumed.
-constexpr int RB = 64, VB = 256, KB = 16;
+// Tile: 64 flagged rows x 128 vocabulary rows per CTA of 4 warps (so that every CTA of
+// a 32000-entry vocabulary is resident at once, three per SM). Warp w owns rows
+// 16w .. 16w+15: lanes 0-15 rows 16w .. 16w+7, lanes 16-31 rows 16w+8 .. 16w+15; lane
+// l owns vocabulary entries 4(l mod 16) .. +3 and 64 + 4(l mod 16) .. +3 (8 x 8
+// logits per thread). k is staged KB at a time through two shared-memory buffers (the
+// next slab is loaded to registers and stored to the other buffer while this one is
+// consumed, one barrier per slab): W transposed to [k][vocab], h as duplicated pairs
+// [k][row] (one 16-byte load gives two rows ready for the packed FMA).
+constexpr int RB = 64, VB = 128, KB = 16, kRecThreads = 128;
 
-__global__ void __launch_bounds__(256) recompute_kernel(const uint16_t* __restrict__ h, int64_t ldh,
-                                                        const uint16_t* __restrict__ W, int64_t V, int K, int M,
-                                                        const int32_t* __restrict__ list,
-                                                        float* __restrict__ out) {
-  __shared__ __align__(16) float2 hs[KB][RB];  // (h, h) per row
-  __shared__ __align__(16) float ws[KB][VB];
+__global__ void __launch_bounds__(kRecThreads, 3) recompute_kernel(const uint16_t* __restrict__ h, int64_t ldh,
+                                                                  const uint16_t* __restrict__ W, int64_t V, int K,
+                                                                  int M, const int32_t* __restrict__ list,
+                                                                  float* __restrict__ out) {
+  __shared__ __align__(16) float2 hs[2][KB][RB];  // (h, h) per row
+  __shared__ __align__(16) float ws[2][KB][VB];
   const int count = list[M];
   const int f0 = blockIdx.y * RB;
   if (f0 >= count) return;
   const int64_t v0 = (int64_t)blockIdx.x * VB;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rbase = warp * 16 + (lane >> 4) * 8;  // first of this thread's 8 rows
+  const int vl = (lane & 15) * 4;                  // first of this thread's vocabulary entries (and vl + 64)
   float2 acc[8][4];  // [row][vocab pair]
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
 
-  // staging: W slab 256 vocab x KB k = 512 vectors of 8 (vocab = e % 256, k-half = e / 256);
-  //          h slab 64 rows x KB k = 128 vectors of 8 (row = e % 64, k-half = e / 64), threads < 128
-  const int hrow = tid & 63, hk = (tid >> 6) & 1;
-  const bool hload = tid < 128 && f0 + hrow < count;
+  // staging of one slab: W 128 vocab x 16 k = 256 vectors of 8 (vocab = e / 2, k-half = e % 2, so a
+  // vocabulary row's 32 bytes are read by adjacent threads); h 64 rows x 16 k = 128 vectors of 8
+  const int hrow = tid >> 1, hk = tid & 1;
+  const bool hload = f0 + hrow < count;
   const uint16_t* hsrc = h + (int64_t)(hload ? list[f0 + hrow] : 0) * ldh + hk * 8;
   auto load = [&](int k0, uint4& hv, uint4 (&wv)[2]) {
     hv = hload ? __ldg(reinterpret_cast<const uint4*>(hsrc + k0)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int e = tid + r * 256;
-      const int64_t vv = v0 + (e & 255);
-      wv[r] = vv < V ? __ldg(reinterpret_cast<const uint4*>(W + vv * K + k0 + (e >> 8) * 8))
+      const int e = tid + r * kRecThreads;
+      const int64_t vv = v0 + (e >> 1);
+      wv[r] = vv < V ? __ldg(reinterpret_cast<const uint4*>(W + vv * K + k0 + (e & 1) * 8))
                      : make_uint4(0, 0, 0, 0);
     }
   };
-  auto store = [&](const uint4& hv, const uint4 (&wv)[2]) {
+  auto store = [&](int buf, const uint4& hv, const uint4 (&wv)[2]) {
     float f[8];
-    if (tid < 128) {
-      unpack8(hv, f);
+    unpack8(hv, f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) hs[hk * 8 + i][hrow] = make_float2(f[i], f[i]);
-    }
+    for (int i = 0; i < 8; ++i) hs[buf][hk * 8 + i][hrow] = make_float2(f[i], f[i]);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int e = tid + r * 256;
+      const int e = tid + r * kRecThreads;
       unpack8(wv[r], f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ws[(e >> 8) * 8 + i][e & 255] = f[i];
+      for (int i = 0; i < 8; ++i) ws[buf][(e & 1) * 8 + i][e >> 1] = f[i];
     }
   };
   uint4 hv, wv[2];
   load(0, hv, wv);
-  store(hv, wv);
+  store(0, hv, wv);
   __syncthreads();
+  int buf = 0;
   for (int k0 = 0; k0 < K; k0 += KB) {
     const bool more = k0 + KB < K;
     if (more) load(k0 + KB, hv, wv);
@@ -180,12 +182,12 @@ __global__ void __launch_bounds__(256) recompute_kernel(const uint16_t* __restri
       float2 h2[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float4 t = *reinterpret_cast<const float4*>(&hs[kk][warp * 8 + 2 * i]);
+        const float4 t = *reinterpret_cast<const float4*>(&hs[buf][kk][rbase + 2 * i]);
         h2[2 * i] = make_float2(t.x, t.y);
         h2[2 * i + 1] = make_float2(t.z, t.w);
       }
-      const float4 wa = *reinterpret_cast<const float4*>(&ws[kk][lane * 4]);
-      const float4 wb = *reinterpret_cast<const float4*>(&ws[kk][128 + lane * 4]);
+      const float4 wa = *reinterpret_cast<const float4*>(&ws[buf][kk][vl]);
+      const float4 wb = *reinterpret_cast<const float4*>(&ws[buf][kk][64 + vl]);
       const float2 w2[4] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w), make_float2(wb.x, wb.y),
                             make_float2(wb.z, wb.w)};
 #pragma unroll
@@ -193,20 +195,19 @@ __global__ void __launch_bounds__(256) recompute_kernel(const uint16_t* __restri
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = __ffma2_rn(h2[i], w2[j], acc[i][j]);
     }
+    // the other buffer was last read in the previous slab, before the barrier that ended it
+    if (more) store(buf ^ 1, hv, wv);
     __syncthreads();
-    if (more) {
-      store(hv, wv);
-      __syncthreads();
-    }
+    buf ^= 1;
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int f = f0 + warp * 8 + i;
+    const int f = f0 + rbase + i;
     if (f >= count) continue;
     float* dst = out + (int64_t)list[f] * V;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int64_t v = v0 + (j < 2 ? lane * 4 + 2 * j : 128 + lane * 4 + 2 * (j - 2));
+      const int64_t v = v0 + (j < 2 ? vl + 2 * j : 64 + vl + 2 * (j - 2));
       if (v < V) dst[v] = acc[i][j].x;
       if (v + 1 < V) dst[v + 1] = acc[i][j].y;
     }
