@@ -33,9 +33,10 @@ def test_prefill_tc_matches_oracle(D, Hq, Hkv):
     assert bi.get_device_error() == 0
 
 
-def test_prefill_tc_whole_equals_chunked_and_agrees_with_cuda_cores():
-    S, Hq, Hkv, D = 1100, 32, 8, 128
-    q, qs, qp, kv = synth.prefill_inputs([S], Hq, Hkv, D, seed=73)
+@pytest.mark.parametrize("D,Hq,Hkv", [(128, 32, 8), (64, 32, 8)])
+def test_prefill_tc_whole_equals_chunked_and_agrees_with_cuda_cores(D, Hq, Hkv):
+    S = 1100
+    q, qs, qp, kv = synth.prefill_inputs([S], Hq, Hkv, D, seed=73 + D)
     kvd = _dev(kv)
     qd = q.to(dev())
     whole = bi.attention_prefill_tc(qd, 0, 0, kvd.k_cache, kvd.v_cache, kvd.page_table)
@@ -49,7 +50,7 @@ def test_prefill_tc_whole_equals_chunked_and_agrees_with_cuda_cores():
     ek = torch.full_like(kvd.k_cache, float("nan"))
     ev = torch.full_like(kvd.v_cache, float("nan"))
     chunked = torch.empty_like(whole)
-    bounds = [0, 77, 128, 333, 512, 1000, 1100]
+    bounds = [0, 77, 128, 333, 512, 513, 1000, 1099, 1100]  # includes 1-row chunks
     for c0, c1 in zip(bounds[:-1], bounds[1:]):
         sl = slice(c0, c1)
         bi.kv_append(k_tok[sl], v_tok[sl], qs[sl].to(dev()), qp[sl].to(dev()), ek, ev, kvd.page_table)
@@ -73,3 +74,26 @@ def test_prefill_tc_full_size_4096_whole_vs_8_chunks():
     ref = oracle.attention_prefill(synth.to_f64(q[rows].cpu()), np.zeros(len(rows), dtype=np.int64), np.array(rows),
                                    synth.to_f64(k), synth.to_f64(v), pt.numpy())
     assert max_rel(whole[rows], ref) <= TOL_BF16
+
+
+def test_prefill_tc_validation_and_device_errors():
+    # odd query-head group: refused on the host; bad page id: recorded on the device, no fault
+    S, D = 200, 128
+    q, qs, qp, kv = synth.prefill_inputs([S], 24, 8, D, seed=75)
+    kvd = _dev(kv)
+    with pytest.raises(bi.BIError, match="UNSUPPORTED"):
+        bi.attention_prefill_tc(q.to(dev()), 0, 0, kvd.k_cache, kvd.v_cache, kvd.page_table)
+    q, qs, qp, kv = synth.prefill_inputs([S], 32, 8, D, seed=76)
+    kvd = _dev(kv)
+    pt = kvd.page_table.clone()
+    pt[0, 3] = kv.k_cache.shape[0] + 5  # outside the store
+    bi.attention_prefill_tc(q.to(dev()), 0, 0, kvd.k_cache, kvd.v_cache, pt)
+    torch.cuda.synchronize()
+    assert bi.get_device_error() == 8
+    # the context stays usable and the next call is correct
+    out = bi.attention_prefill_tc(q.to(dev()), 0, 0, kvd.k_cache, kvd.v_cache, kvd.page_table)
+    rows = [0, 199]
+    ref = oracle.attention_prefill(synth.to_f64(q)[rows], qs.numpy()[rows], qp.numpy()[rows],
+                                   synth.to_f64(kv.k_cache), synth.to_f64(kv.v_cache), kv.page_table.numpy())
+    assert max_rel(out.cpu()[rows], ref) <= TOL_BF16
+    assert bi.get_device_error() == 0
