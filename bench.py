@@ -427,6 +427,19 @@ def _row_lmhead(bi, device, pk):
     ms_ref = _events_ms(lambda: torch.argmax(torch.matmul(h, Wl.t()), dim=1))
     out["lmhead_m64_v32000"] = {"ms": round(ms, 4), "recomputed_rows": int(rec.sum()),
                                 "slowdown_vs_cublas_argmax": round(ms / ms_ref, 3)}
+    # batch 4 with trained-model-like margins (the greedy-decoding abstract's setting):
+    # no row near a tie, then one row near a tie; device time from CUDA-graph replays
+    for ties in (0, 1):
+        h4, W4 = synth.lmhead_planted(4, 32000, 2048, seed=72, ties=ties)
+        h4, W4 = h4.to(device), W4.to(device)
+        t4 = torch.empty(4, dtype=torch.int32, device=device)
+        r4 = torch.empty(4, dtype=torch.int32, device=device)
+        ws4 = torch.empty(bi.lmhead_workspace_size(4, 32000), dtype=torch.uint8, device=device)
+        us = _graph_us(lambda: bi.lmhead_argmax(h4, W4, 0.5, tokens=t4, recomputed=r4, workspace=ws4))
+        us_ref = _graph_us(lambda: torch.argmax(torch.matmul(h4, W4.t()), dim=1))
+        out[f"lmhead_m4_v32000_{ties}tie"] = {"us": round(us, 2), "recomputed_rows": int(r4.sum()),
+                                             "cublas_argmax_us": round(us_ref, 2),
+                                             "overhead_vs_cublas_argmax": round(us / us_ref - 1, 3)}
     return out
 
 

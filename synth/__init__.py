@@ -159,6 +159,26 @@ def lmhead_inputs(M: int, V: int, K: int, seed: int = 0):
     return h, w
 
 
+def lmhead_planted(M: int, V: int, K: int, seed: int, ties: int):
+    """LM-head inputs with a trained-model-like margin structure: W ~ N(0, 0.02) [V, K];
+    row m of h is N(0, 1) plus 40 times the weight row of a seeded target token, so that
+    token's logit stands far above the rest; each of the first `ties` rows is instead
+    20 * (w_a / |w_a|^2 + w_b / |w_b|^2) for two targets a, b (no noise), so logits a and
+    b are both about 20 and nearly tied at the top."""
+    W = normal_bf16((V, K), seed, std=0.02)
+    g = generator(seed + 1)
+    tgt = torch.randint(0, V, (M, 2), generator=g)
+    h = torch.randn((M, K), generator=g, dtype=torch.float32)
+    Wf = W.float()
+    for m in range(M):
+        if m < ties:
+            wa, wb = Wf[tgt[m, 0]], Wf[tgt[m, 1]]
+            h[m] = 20.0 * (wa / wa.dot(wa) + wb / wb.dot(wb))
+        else:
+            h[m] += 40.0 * Wf[tgt[m, 0]]
+    return h.to(torch.bfloat16), W
+
+
 def logits(M: int, V: int, seed: int = 0, std: float = 3.0) -> torch.Tensor:
     """bf16 [M, V] logit rows ~ N(0, std^2)."""
     return normal_bf16((M, V), seed, std=std)
