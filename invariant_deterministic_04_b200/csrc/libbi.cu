@@ -366,9 +366,29 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
                                                                       recomputed);
   bi::lmhead::compact_kernel<<<1, 1024, 0, st>>>(recomputed, (int)M, lay.list);
   float* out32 = logits_fp32 ? logits_fp32 : lay.logits32;
-  const dim3 rgrid((unsigned)((V + bi::lmhead::VB - 1) / bi::lmhead::VB), (unsigned)((M + bi::lmhead::RB - 1) / bi::lmhead::RB));
-  bi::lmhead::recompute_kernel<<<rgrid, bi::lmhead::kRecThreads, 0, st>>>(h, ldh, W, V, (int)K, (int)M, lay.list,
-                                                                         out32);
+  // few flagged rows (with hidden size <= 4096): W streamed once per 8 rows; otherwise
+  // 64-row tiles. Both compute every logit as the same FMA chain, and each returns at
+  // once when the count of flagged rows is not its case.
+  int skip_upto = 0;
+  if (K <= bi::lmhead::kStrMaxK) {
+    static std::once_flag str_once[64];
+    cudaError_t attr = cudaSuccess;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
+    std::call_once(str_once[dev & 63], [&] {
+      attr = cudaFuncSetAttribute(bi::lmhead::recompute_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK));
+    });
+    if (attr != cudaSuccess) return BI_ERR_CUDA;
+    const unsigned sgrid = (unsigned)((V + bi::lmhead::kStrWarps * 32 - 1) / (bi::lmhead::kStrWarps * 32));
+    bi::lmhead::recompute_stream_kernel<<<sgrid, bi::lmhead::kStrThreads, bi::lmhead::stream_smem_bytes((int)K), st>>>(
+        h, ldh, W, V, (int)K, (int)M, lay.list, out32);
+    skip_upto = bi::lmhead::kStrMaxCount;
+  }
+  const dim3 rgrid((unsigned)((V + bi::lmhead::VB - 1) / bi::lmhead::VB),
+                   (unsigned)((M + bi::lmhead::RB - 1) / bi::lmhead::RB));
+  bi::lmhead::recompute_kernel<<<rgrid, bi::lmhead::kRecThreads, 0, st>>>(h, ldh, W, V, (int)K, (int)M, lay.list, out32,
+                                                                         skip_upto);
   bi::lmhead::argmax_kernel<<<(unsigned)M, bi::lmhead::kThreads, 0, st>>>(out32, V, recomputed, tokens);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }

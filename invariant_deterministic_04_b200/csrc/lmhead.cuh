@@ -125,12 +125,12 @@ constexpr int RB = 64, VB = 128, KB = 16, kRecThreads = 128;
 __global__ void __launch_bounds__(kRecThreads, 3) recompute_kernel(const uint16_t* __restrict__ h, int64_t ldh,
                                                                   const uint16_t* __restrict__ W, int64_t V, int K,
                                                                   int M, const int32_t* __restrict__ list,
-                                                                  float* __restrict__ out) {
+                                                                  float* __restrict__ out, int skip_upto) {
   __shared__ __align__(16) float2 hs[2][KB][RB];  // (h, h) per row
   __shared__ __align__(16) float ws[2][KB][VB];
   const int count = list[M];
   const int f0 = blockIdx.y * RB;
-  if (f0 >= count) return;
+  if (f0 >= count || count <= skip_upto) return;  // few flagged rows: the streaming kernel takes them
   const int64_t v0 = (int64_t)blockIdx.x * VB;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rbase = warp * 16 + (lane >> 4) * 8;  // first of this thread's 8 rows
@@ -210,6 +210,96 @@ __global__ void __launch_bounds__(kRecThreads, 3) recompute_kernel(const uint16_
       const int64_t v = v0 + (j < 2 ? vl + 2 * j : 64 + vl + 2 * (j - 2));
       if (v < V) dst[v] = acc[i][j].x;
       if (v + 1 < V) dst[v + 1] = acc[i][j].y;
+    }
+  }
+}
+
+// The same fp32 logits for hidden sizes up to 4096, with W streamed once per 8 flagged
+// rows instead of once per 64-row tile (identical FMA chains, so identical bits). Both
+// kernels are launched; this one takes the call when at most kStrMaxCount rows are flagged
+// (a rare recompute, as with a trained model), the tiled one otherwise.
+// Each warp owns 32 consecutive vocabulary entries (lane = entry) and walks K in tiles of
+// 64: the tile (32 rows x 128 bytes of W) is loaded coalesced (8 lanes per row) one tile
+// ahead into registers, parked in the warp's shared-memory slot (rows padded to 144 bytes,
+// so each lane's 16-byte reads of its own row are conflict-free), and consumed by each lane
+// along its row. The CTA's 8 current flagged rows of h sit in shared memory as fp32,
+// [k][row], read as broadcasts; packed f32x2 FMAs carry two rows each.
+constexpr int kStrRows = 8, kStrWarps = 4, kStrThreads = 128, kStrTK = 64, kStrPad = 72, kStrMaxK = 4096;
+constexpr int kStrMaxCount = 24;
+
+inline int stream_smem_bytes(int K) { return K * kStrRows * 4 + kStrWarps * 32 * kStrPad * 2; }
+
+__global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uint16_t* __restrict__ h, int64_t ldh,
+                                                                      const uint16_t* __restrict__ W, int64_t V,
+                                                                      int K, int M, const int32_t* __restrict__ list,
+                                                                      float* __restrict__ out) {
+  extern __shared__ __align__(16) uint8_t smem_str[];
+  float* hsm = reinterpret_cast<float*>(smem_str);                                     // [K][8]
+  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_str + (size_t)K * kStrRows * 4);  // [warp][32][72]
+  const int count = list[M];
+  if (count == 0 || count > kStrMaxCount) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t vbase = ((int64_t)blockIdx.x * kStrWarps + warp) * 32;
+  const int64_t v = vbase + lane;
+  uint16_t* my = tiles + warp * 32 * kStrPad;
+  const int ntile = K / kStrTK;
+  // tile t: instruction q loads rows 4q .. 4q+3, lane l the 16 bytes (l mod 8) of row 4q + l/8
+  auto load_tile = [&](int t, uint4 (&r)[8]) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int64_t vv = vbase + q * 4 + (lane >> 3);
+      r[q] = vv < V ? __ldg(reinterpret_cast<const uint4*>(W + vv * K + t * kStrTK + (lane & 7) * 8))
+                    : make_uint4(0, 0, 0, 0);
+    }
+  };
+  for (int r0 = 0; r0 < count; r0 += kStrRows) {
+    const int nr = min(kStrRows, count - r0);
+    __syncthreads();  // the previous rows of h are no longer read
+    for (int e = threadIdx.x; e < kStrRows * (K / 8); e += kStrThreads) {
+      const int r = e % kStrRows, kv = e / kStrRows;
+      float f[8];
+      if (r < nr) {
+        unpack8(__ldg(reinterpret_cast<const uint4*>(h + (int64_t)list[r0 + r] * ldh) + kv), f);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hsm[(kv * 8 + i) * kStrRows + r] = f[i];
+    }
+    __syncthreads();
+    float2 acc[kStrRows / 2];
+#pragma unroll
+    for (int j = 0; j < kStrRows / 2; ++j) acc[j] = make_float2(0.f, 0.f);
+    uint4 nxt[8];
+    load_tile(0, nxt);
+    for (int t = 0; t < ntile; ++t) {
+      __syncwarp();  // every lane is done with the previous tile
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<uint4*>(my + (q * 4 + (lane >> 3)) * kStrPad + (lane & 7) * 8) = nxt[q];
+      __syncwarp();
+      if (t + 1 < ntile) load_tile(t + 1, nxt);
+#pragma unroll
+      for (int c = 0; c < kStrTK / 8; ++c) {
+        float w[8];
+        unpack8(*reinterpret_cast<const uint4*>(my + lane * kStrPad + c * 8), w);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float* hk = hsm + (t * kStrTK + c * 8 + i) * kStrRows;
+          const float4 a = *reinterpret_cast<const float4*>(hk);
+          const float4 b = *reinterpret_cast<const float4*>(hk + 4);
+          const float2 ww = make_float2(w[i], w[i]);
+          acc[0] = __ffma2_rn(make_float2(a.x, a.y), ww, acc[0]);
+          acc[1] = __ffma2_rn(make_float2(a.z, a.w), ww, acc[1]);
+          acc[2] = __ffma2_rn(make_float2(b.x, b.y), ww, acc[2]);
+          acc[3] = __ffma2_rn(make_float2(b.z, b.w), ww, acc[3]);
+        }
+      }
+    }
+    if (v < V) {
+      for (int r = 0; r < nr; ++r)
+        out[(int64_t)list[r0 + r] * V + v] = (r & 1) ? acc[r >> 1].y : acc[r >> 1].x;
     }
   }
 }

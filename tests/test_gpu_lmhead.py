@@ -39,7 +39,8 @@ def _check_against_oracle(h, w, tau, tokens, rec, logits):
     return r, rec
 
 
-@pytest.mark.parametrize("M,V,K", [(9, 1000, 256), (1, 32000, 2048), (64, 32000, 2048), (40, 4096, 512)])
+@pytest.mark.parametrize("M,V,K", [(9, 1000, 256), (1, 32000, 2048), (64, 32000, 2048), (40, 4096, 512),
+                                   (6, 2000, 4160)])  # K > 4096: the 64-row tiled recompute
 def test_lmhead_matches_oracle(M, V, K):
     h, w = synth.lmhead_inputs(M, V, K, seed=M + V)
     tok, rec, lg = bi.lmhead_argmax(h.to(dev()), w.to(dev()), TAU, want_logits=True)
