@@ -68,12 +68,16 @@ def peaks():
 
 
 def init_dist():
+    """Process group from the torchrun environment. A rank that fails or never joins ends the
+    others' next collective with an error after BI_PG_TIMEOUT_S seconds (default 300)
+    instead of a hang."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1 and not dist.is_initialized():
         backend = "nccl" if torch.cuda.is_available() else "gloo"
-        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+        timeout = datetime.timedelta(seconds=float(os.environ.get("BI_PG_TIMEOUT_S", "300")))
+        dist.init_process_group(backend=backend, timeout=timeout)
     return rank, world, local
 
 

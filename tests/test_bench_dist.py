@@ -7,6 +7,7 @@ reduction, and that every rank takes the same collective steps.
 """
 import os
 import socket
+import time
 
 import torch.multiprocessing as mp
 
@@ -49,3 +50,31 @@ def test_aggregate_sums_units_and_takes_max_time_over_two_ranks():
 
 def test_single_rank_aggregate_is_identity():
     assert bench.aggregate(123.0, 4.5, 1) == (123.0, 4.5)
+
+
+def _rank_main_failing(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank), BI_PG_TIMEOUT_S="5")
+    r, w, _ = bench.init_dist()
+    if rank == 1:
+        os._exit(0)  # this rank leaves between steps, before the next collective
+    t0 = time.time()
+    try:
+        bench.barrier(w)
+        out[rank] = ("no error", time.time() - t0)
+    except Exception as e:  # the surviving rank learns of it from its collective
+        out[rank] = (type(e).__name__, time.time() - t0)
+
+
+def test_a_rank_that_leaves_ends_the_others_collective_with_an_error():
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_failing, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    kind, seconds = out[0]
+    assert kind != "no error" and seconds < 60, (kind, seconds)
