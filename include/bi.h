@@ -257,7 +257,9 @@ size_t bi_lmhead_workspace_size(int64_t M, int64_t V);
  * recomputed: [M] int32 out (1 if the row took step 3, else 0). logits_fp32:
  * optional [M, V] fp32 out (may be NULL): rows that took step 3 receive their fp32
  * logits, other rows are not written. Requires the bi_matmul rules on K and
- * V % 8 == 0. M == 0 is a no-op.
+ * V % 8 == 0. M == 0 is a no-op. Step 3 reads W once per 8 flagged rows when at most 24
+ * rows are flagged and K <= 4096, and uses 64-row tiles otherwise; the choice is made on
+ * the device from the flagged count, and every logit is the same FMA chain either way.
  */
 bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int64_t M, int64_t V,
                            int64_t K, float margin_threshold, int32_t* tokens, int32_t* recomputed,
