@@ -362,7 +362,7 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
   cudaStream_t st = as_stream(stream);
   bi_status s = bi::gemm::launch(h, ldh, W, K, lay.logits16, V, M, V, K, st);
   if (s != BI_OK) return s;
-  bi::lmhead::top2_kernel<<<(unsigned)M, bi::lmhead::kThreads, 0, st>>>(lay.logits16, V, margin_threshold, tokens,
+  bi::lmhead::top2_kernel<<<(unsigned)(M * bi::lmhead::kParts), bi::lmhead::kThreads, 0, st>>>(lay.logits16, V, margin_threshold, tokens,
                                                                       recomputed);
   bi::lmhead::compact_kernel<<<1, 1024, 0, st>>>(recomputed, (int)M, lay.list);
   float* out32 = logits_fp32 ? logits_fp32 : lay.logits32;
@@ -389,7 +389,8 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
                    (unsigned)((M + bi::lmhead::RB - 1) / bi::lmhead::RB));
   bi::lmhead::recompute_kernel<<<rgrid, bi::lmhead::kRecThreads, 0, st>>>(h, ldh, W, V, (int)K, (int)M, lay.list, out32,
                                                                          skip_upto);
-  bi::lmhead::argmax_kernel<<<(unsigned)M, bi::lmhead::kThreads, 0, st>>>(out32, V, recomputed, tokens);
+  bi::lmhead::argmax_kernel<<<(unsigned)(M * bi::lmhead::kParts), bi::lmhead::kThreads, 0, st>>>(out32, V, recomputed,
+                                                                                                tokens);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

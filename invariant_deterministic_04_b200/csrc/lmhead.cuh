@@ -19,6 +19,8 @@
 // each fp32 logit depends only on its own row, so every row is batch-invariant.
 #pragma once
 
+#include <cstddef>
+
 #include "device.cuh"
 
 namespace bi {
@@ -50,21 +52,10 @@ __device__ __forceinline__ void insert(Top2& t, float v, int i) {
 __device__ __forceinline__ float sanitize(float v) { return v != v ? -INFINITY : v; }
 
 constexpr int kThreads = 256;
+constexpr int kParts = 8;  // CTAs (one cluster) per row for the top-2 and the argmax
 
-__global__ void __launch_bounds__(kThreads) top2_kernel(const uint16_t* __restrict__ logits, int64_t V,
-                                                        float threshold, int32_t* __restrict__ tokens,
-                                                        int32_t* __restrict__ flags) {
-  __shared__ Top2 warp_best[kThreads / 32];
-  const int64_t row = blockIdx.x;
-  const uint4* src = reinterpret_cast<const uint4*>(logits + row * V);
-  Top2 t{-INFINITY, 0x7FFFFFFF, -INFINITY, 0x7FFFFFFF};
-  const int64_t nvec = V / 8;
-  for (int64_t j = threadIdx.x; j < nvec; j += kThreads) {
-    float f[8];
-    unpack8(__ldg(src + j), f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) insert(t, sanitize(f[e]), (int)(j * 8 + e));
-  }
+// Merge of a CTA's per-thread top-2 into thread 0 (warp butterfly, then warps in order).
+__device__ __forceinline__ Top2 block_top2(Top2 t, Top2* warp_best) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) {
     const float a1 = __shfl_xor_sync(kFullMask, t.v1, o), a2 = __shfl_xor_sync(kFullMask, t.v2, o);
@@ -74,16 +65,51 @@ __global__ void __launch_bounds__(kThreads) top2_kernel(const uint16_t* __restri
   }
   if ((threadIdx.x & 31) == 0) warp_best[threadIdx.x >> 5] = t;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    Top2 b = warp_best[0];
+  Top2 b = warp_best[0];
+  if (threadIdx.x == 0)
     for (int w = 1; w < kThreads / 32; ++w) {
       insert(b, warp_best[w].v1, warp_best[w].i1);
       insert(b, warp_best[w].v2, warp_best[w].i2);
     }
-    const float margin = __fsub_rn(b.v1, b.v2);  // +inf when V == 1
-    tokens[row] = b.i1;
+  return b;
+}
+
+// Per row, a cluster of kParts CTAs: part p scans vectors p * ceil(n/8) .. of the row's n
+// 8-element vectors (a split fixed by V); CTA 0 merges the parts' top-2 through
+// distributed shared memory. The top-2 under a strict total order is exact, so the split
+// does not change it.
+__global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads)
+    top2_kernel(const uint16_t* __restrict__ logits, int64_t V, float threshold, int32_t* __restrict__ tokens,
+                int32_t* __restrict__ flags) {
+  __shared__ Top2 warp_best[kThreads / 32];
+  __shared__ Top2 part_best;
+  const int64_t row = blockIdx.x / kParts;
+  const uint32_t part = cluster_rank();
+  const uint4* src = reinterpret_cast<const uint4*>(logits + row * V);
+  const int64_t nvec = V / 8, per = (nvec + kParts - 1) / kParts;
+  const int64_t j0 = (int64_t)part * per, j1 = min(nvec, j0 + per);
+  Top2 t{-INFINITY, 0x7FFFFFFF, -INFINITY, 0x7FFFFFFF};
+  for (int64_t j = j0 + threadIdx.x; j < j1; j += kThreads) {
+    float f[8];
+    unpack8(__ldg(src + j), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) insert(t, sanitize(f[e]), (int)(j * 8 + e));
+  }
+  const Top2 b = block_top2(t, warp_best);
+  if (threadIdx.x == 0) part_best = b;
+  cluster_barrier();  // every part's top-2 is in its shared memory
+  if (part == 0 && threadIdx.x == 0) {
+    Top2 m = part_best;
+    for (uint32_t p = 1; p < kParts; ++p) {
+      const uint32_t base = map_to_rank(smem_u32(&part_best), p);
+      insert(m, ld_cluster_f32(base + offsetof(Top2, v1)), ld_cluster_s32(base + offsetof(Top2, i1)));
+      insert(m, ld_cluster_f32(base + offsetof(Top2, v2)), ld_cluster_s32(base + offsetof(Top2, i2)));
+    }
+    const float margin = __fsub_rn(m.v1, m.v2);  // +inf when V == 1
+    tokens[row] = m.i1;
     flags[row] = (margin < threshold) ? 1 : 0;
   }
+  cluster_barrier();  // no part leaves while CTA 0 may still read its shared memory
 }
 
 // list[0..count) = indices of flagged rows, ascending; list[M] = count.
@@ -304,18 +330,25 @@ __global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uin
   }
 }
 
-// Token of each flagged row = argmax of its fp32 logits (lowest index on ties).
-__global__ void __launch_bounds__(kThreads) argmax_kernel(const float* __restrict__ logits, int64_t V,
-                                                          const int32_t* __restrict__ flags,
-                                                          int32_t* __restrict__ tokens) {
+// Token of each flagged row = argmax of its fp32 logits (lowest index on ties), a cluster
+// of kParts CTAs per row as in top2_kernel (the argmax is exact, so the split does not
+// change it).
+__global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads)
+    argmax_kernel(const float* __restrict__ logits, int64_t V, const int32_t* __restrict__ flags,
+                  int32_t* __restrict__ tokens) {
   __shared__ float wv[kThreads / 32];
   __shared__ int wi[kThreads / 32];
-  const int64_t row = blockIdx.x;
-  if (!flags[row]) return;
+  __shared__ float part_v;
+  __shared__ int part_i;
+  const int64_t row = blockIdx.x / kParts;
+  if (!flags[row]) return;  // the same for every CTA of the cluster
+  const uint32_t part = cluster_rank();
   const float* src = logits + row * V;
+  const int64_t per = (V + kParts - 1) / kParts;
+  const int64_t j0 = (int64_t)part * per, j1 = min(V, j0 + per);
   float best = -INFINITY;
   int bi_ = 0x7FFFFFFF;
-  for (int64_t j = threadIdx.x; j < V; j += kThreads) {
+  for (int64_t j = j0 + threadIdx.x; j < j1; j += kThreads) {
     const float v = sanitize(src[j]);
     if (better(v, (int)j, best, bi_)) {
       best = v;
@@ -344,8 +377,24 @@ __global__ void __launch_bounds__(kThreads) argmax_kernel(const float* __restric
         b = wv[w];
         bi2 = wi[w];
       }
+    part_v = b;
+    part_i = bi2;
+  }
+  cluster_barrier();
+  if (part == 0 && threadIdx.x == 0) {
+    float b = part_v;
+    int bi2 = part_i;
+    for (uint32_t p = 1; p < kParts; ++p) {
+      const float v = ld_cluster_f32(map_to_rank(smem_u32(&part_v), p));
+      const int i = ld_cluster_s32(map_to_rank(smem_u32(&part_i), p));
+      if (better(v, i, b, bi2)) {
+        b = v;
+        bi2 = i;
+      }
+    }
     tokens[row] = bi2;
   }
+  cluster_barrier();
 }
 
 }  // namespace lmhead

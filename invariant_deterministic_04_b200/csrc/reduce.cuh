@@ -245,30 +245,6 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi_) { retu
 // argmax is exact, so the split does not change the result.
 constexpr int kSampleParts = 8;
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_barrier() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float ld_cluster_f32(uint32_t a) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-  return v;
-}
-__device__ __forceinline__ int ld_cluster_s32(uint32_t a) {
-  int v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-  return v;
-}
-
 __global__ void __cluster_dims__(kSampleParts, 1, 1) __launch_bounds__(kThreads)
     sample_kernel(const uint16_t* __restrict__ x, int64_t ldx, const uint64_t* __restrict__ seeds,
                   const uint64_t* __restrict__ steps, float inv_t, int32_t* __restrict__ tokens, int V) {
