@@ -177,6 +177,17 @@ def test_attention_two_keys_closed_form_scale():
     np.testing.assert_allclose(out[0, 0, 3], math.exp(b) / (math.exp(a) + math.exp(b)), rtol=1e-15)
 
 
+def _bruteforce_head(qv, k, v, page_row, L, g):
+    """Pure-Python attention of one query vector over tokens 0..L-1 of kv-head g,
+    each token looked up as (page_row[t // 16], slot t % 16); plain softmax
+    without max subtraction (the scores are small in these cases)."""
+    D = len(qv)
+    rows = [(page_row[t // 16], t % 16) for t in range(L)]
+    w = [math.exp(sum(qv[d] * k[p, g, s, d] for d in range(D)) / math.sqrt(D)) for p, s in rows]
+    z = math.fsum(w)
+    return [math.fsum(w[i] * v[p, g, s, d] for i, (p, s) in enumerate(rows)) / z for d in range(D)]
+
+
 def test_attention_bruteforce_through_page_table():
     lens = [5, 33, 18]
     Hq, Hkv, D = 4, 2, 8
@@ -188,14 +199,37 @@ def test_attention_bruteforce_through_page_table():
     out = oracle.attention_decode(q, k, v, np.array(pt), np.array(lens))
     for b, L in enumerate(lens):
         for h in range(Hq):
-            g = h // (Hq // Hkv)
-            rows = [(pt[b][t // 16], t % 16) for t in range(L)]
-            # plain softmax without max subtraction (scores are small here)
-            w = [math.exp(sum(q[b, h, d] * k[p, g, s, d] for d in range(D)) / math.sqrt(D)) for p, s in rows]
-            z = math.fsum(w)
-            for d in range(D):
-                ref = math.fsum(w[i] * v[p, g, s, d] for i, (p, s) in enumerate(rows)) / z
-                assert abs(out[b, h, d] - ref) <= 1e-13
+            ref = _bruteforce_head(q[b, h], k, v, pt[b], L, h // (Hq // Hkv))
+            np.testing.assert_allclose(out[b, h], ref, rtol=0, atol=1e-13)
+
+
+def test_attention_empty_sequence_gives_zeros():
+    # a sequence of length 0 sees no key: its rows are zero, the others are unaffected
+    lens = [0, 5, 0]
+    kv = _tiny_paged([1, 5, 1], Hkv=1, D=8, seed=18)
+    q = synth.to_f64(synth.normal_bf16((3, 2, 8), 19))
+    k, v, pt = synth.to_f64(kv.k_cache), synth.to_f64(kv.v_cache), kv.page_table.numpy()
+    out = oracle.attention_decode(q, k, v, pt, np.array(lens))
+    assert np.all(out[0] == 0) and np.all(out[2] == 0)
+    for h in range(2):
+        np.testing.assert_allclose(out[1, h], _bruteforce_head(q[1, h], k, v, pt[1].tolist(), 5, 0), rtol=0, atol=1e-13)
+
+
+def test_prefill_rows_of_two_sequences_bruteforce():
+    # rows of two sequences, shuffled together: each row reads its own sequence's
+    # pages, keys 0..p inclusive of its position p
+    lens = [21, 35]
+    Hq, Hkv, D = 4, 2, 8
+    q, q_seq, q_pos, kv = synth.prefill_inputs(lens, Hq, Hkv, D, seed=17)
+    perm = np.random.default_rng(5).permutation(sum(lens))
+    q = synth.to_f64(q)[perm]
+    seq, pos = q_seq.numpy()[perm], q_pos.numpy()[perm]
+    k, v, pt = synth.to_f64(kv.k_cache), synth.to_f64(kv.v_cache), kv.page_table.tolist()
+    out = oracle.attention_prefill(q, seq, pos, k, v, np.array(pt))
+    for r in range(len(perm)):
+        for h in range(Hq):
+            ref = _bruteforce_head(q[r, h], k, v, pt[seq[r]], int(pos[r]) + 1, h // (Hq // Hkv))
+            np.testing.assert_allclose(out[r, h], ref, rtol=0, atol=1e-13)
 
 
 def test_attention_invariant_to_physical_page_placement():
@@ -263,6 +297,24 @@ def test_lmhead_planted_margins():
     assert list(r["tokens"]) == [7, 12]
     assert list(r["recompute"]) == [True, False]
     assert r["margin"][0] == 0.125 and r["margin"][1] == 5.0
+    # a margin exactly at the threshold is not below it: no recompute
+    h3 = np.zeros((1, K))
+    h3[0, 2] = 1.0
+    w[:, 2] = np.clip(w[:, 2], -1, 1)
+    w[3, 2], w[20, 2] = 4.0, 3.5
+    r3 = oracle.lmhead(h3, w, 0.5)
+    assert r3["tokens"][0] == 3 and r3["margin"][0] == 0.5 and not r3["recompute"][0]
+
+
+def test_lmhead_margin_is_taken_on_bf16_rounded_logits():
+    # bf16 values between 256 and 512 are 2 apart, so 256.625 rounds to 256: the
+    # exact margin 0.625 would not ask for a recompute, but the bf16 logits tie
+    # (margin 0 < 0.5), and their argmax is the lower index while the exact
+    # argmax is the higher one
+    vals = [256.0, 256.625, 1.0, -3.0]
+    r = oracle.lmhead(np.array([[1.0]]), np.array(vals).reshape(4, 1), 0.5)
+    assert r["tokens"][0] == 1 and r["margin"][0] == 0.625
+    assert r["tokens_bf16"][0] == 0 and r["margin_bf16"][0] == 0.0 and r["recompute"][0]
 
 
 def test_lmhead_bruteforce_argmax_and_ties():
@@ -351,3 +403,37 @@ def test_decoder_layer_structure():
     v = oracle.matmul(x, w["wqkv"])[:, (nh + nkv) * D:].reshape(1, nkv, D)
     expect = h[:1] + np.repeat(v, nh // nkv, axis=1).reshape(1, Hd)
     np.testing.assert_allclose(out2, expect, rtol=1e-13, atol=1e-13)
+
+
+def test_decoder_layer_attention_closed_form():
+    # One head, D = 2, eps = 0, Wq = Wk = Wv = wo = I, wdown = 0. Rows h0 = e0 at
+    # position 0 and h1 = e1 at position 1 of one sequence; RMSNorm makes x_t =
+    # sqrt(2) h_t. At D = 2 RoPE turns the one pair by pos radians, so
+    # q1 = k1 = sqrt(2) (-sin 1, cos 1) and k0 = sqrt(2) e0. With scale 1/sqrt(2) row 1
+    # scores key 0 at -sqrt(2) sin 1 and key 1 at sqrt(2); row 0 sees only itself.
+    I2 = np.eye(2)
+    w = dict(wqkv=np.vstack([I2, I2, I2]), wo=I2, wgu=np.zeros((2, 2)), wdown=np.zeros((2, 1)),
+             attn_norm=np.ones(2), mlp_norm=np.ones(2))
+    r2 = math.sqrt(2)
+    s0, s1 = -r2 * math.sin(1.0), r2
+    p0 = math.exp(s0) / (math.exp(s0) + math.exp(s1))
+    expect = np.array([[1 + r2, 0.0], [r2 * p0, 1 + r2 * (1 - p0)]])
+    out = oracle.decoder_layer(np.eye(2), [0, 0], [0, 1], {}, {}, w, 1, 1, eps=0.0)
+    np.testing.assert_allclose(out, expect, rtol=0, atol=1e-14)
+    # row 1 alone, position 0 supplied by the cache (key as rotated at position 0,
+    # a value of our choosing): the same weights p0, 1 - p0 mix that value and v1
+    v0 = np.array([0.25, -0.75])
+    out1 = oracle.decoder_layer(np.eye(2)[1:], [0], [1], {0: (r2 * I2[0])[None, None]}, {0: v0[None, None]},
+                                w, 1, 1, eps=0.0)
+    np.testing.assert_allclose(out1[0], I2[1] + p0 * v0 + (1 - p0) * r2 * I2[1], rtol=0, atol=1e-14)
+
+
+def test_decoder_layer_mlp_closed_form():
+    # wo = 0 removes attention. The MLP sees x = rmsnorm(h) * mlp_norm: for h = e0,
+    # eps = 0 and mlp_norm = (1/2, 3), x = (sqrt(2)/2, 0). wgu rows (1, 0), (1, 0)
+    # make gate = up = a = sqrt(2)/2, and wdown = (1, 0)^T puts silu(a) * a on column 0.
+    a = math.sqrt(2) / 2
+    w = dict(wqkv=np.ones((6, 2)), wo=np.zeros((2, 2)), wgu=np.array([[1.0, 0.0], [1.0, 0.0]]),
+             wdown=np.array([[1.0], [0.0]]), attn_norm=np.full(2, 5.0), mlp_norm=np.array([0.5, 3.0]))
+    out = oracle.decoder_layer(np.array([[1.0, 0.0]]), [0], [0], {}, {}, w, 1, 1, eps=0.0)
+    np.testing.assert_allclose(out, [[1 + a * a / (1 + math.exp(-a)), 0.0]], rtol=0, atol=1e-15)

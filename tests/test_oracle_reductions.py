@@ -38,6 +38,14 @@ def test_log_softmax_two_values_closed_form(a, b):
                                     abs=1e-12)
 
 
+def test_log_softmax_rows_far_apart():
+    # each row is shifted by its own maximum: rows 1800 apart still give -log N,
+    # and the token log-probability of any entry is the same
+    x = np.array([[900.0, 900.0, 900.0], [-900.0, -900.0, -900.0]])
+    np.testing.assert_allclose(oracle.log_softmax(x), -math.log(3), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(oracle.token_logprob(x, np.array([2, 0])), -math.log(3), rtol=0, atol=1e-12)
+
+
 def test_log_softmax_matches_library_and_normalises():
     rng = np.random.default_rng(0)
     x = rng.normal(0, 3, size=(5, 1000))
@@ -140,6 +148,21 @@ def test_sample_frequencies_follow_softmax(T):
     # and not the distribution of the other temperature (x * T or a flipped variate would match neither)
     other = np.exp(x * T) / np.exp(x * T).sum() if T != 1.0 else np.exp(-x) / np.exp(-x).sum()
     assert np.any(np.abs(counts - n * other) > 6 * np.sqrt(n * other * (1 - other)))
+
+
+def test_sample_rows_do_not_depend_on_the_batch():
+    # each row's token is a function of its own logits, seed and step: sampling a
+    # batch gives, row by row, what sampling each row alone gives
+    rng = np.random.default_rng(4)
+    x = rng.normal(0, 0.5, size=(8, 64))
+    seeds = np.array([11, 12, 13, 14, 15, 16, 17, 18])
+    steps = np.array([0, 5, 5, 9, 2, 7, 1, 3])
+    batch = oracle.sample(x, 1.0, seeds, steps)
+    alone = [oracle.sample(x[m:m + 1], 1.0, seeds[m:m + 1], steps[m:m + 1])[0] for m in range(8)]
+    assert list(batch) == alone
+    # and the draw moves with the seed and with the step (64 near-uniform choices)
+    assert len({int(oracle.sample(x[:1], 1.0, [s], [0])[0]) for s in range(16)}) > 4
+    assert len({int(oracle.sample(x[:1], 1.0, [11], [t])[0]) for t in range(16)}) > 4
 
 
 def test_gumbel_scores_closed_form():
