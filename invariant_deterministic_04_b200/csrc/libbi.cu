@@ -284,6 +284,8 @@ bi_status bi_attention_prefill_tc(const bi_bf16* q, int64_t ldq, int seq, int po
   if (D != 64 && D != 128 || (Hq / Hkv) % 2 != 0) return BI_ERR_UNSUPPORTED;
   if (!(scale > 0.f)) return BI_ERR_SHAPE;
   if ((int64_t)pos0 + T > (int64_t)max_pages_per_seq * BI_PAGE_TOKENS || ldq < (int64_t)Hq * D) return BI_ERR_SHAPE;
+  // the work list (128-row blocks x head pairs) is indexed in 32-bit
+  if (((int64_t)T + bi::attn_tc::ROWS - 1) / bi::attn_tc::ROWS * (Hq / 2) >= INT_MAX / 2) return BI_ERR_SHAPE;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || ldq % 8) return BI_ERR_ALIGN;
   if (T == 0) return BI_OK;
   int dev = 0;
@@ -409,7 +411,8 @@ bi_status bi_gather_rows(const bi_bf16* src, int64_t ld_src, int64_t nrows_src, 
 bi_status bi_rope(bi_bf16* x, int64_t ldx, int64_t T, int H, int D, const int32_t* pos, const float* cos_sin,
                   int max_pos, void* stream) {
   if (!x || !pos || !cos_sin) return BI_ERR_NULL;
-  if (T < 0 || H <= 0 || D <= 0 || D % 2 || max_pos <= 0 || ldx < (int64_t)H * D) return BI_ERR_SHAPE;
+  if (T < 0 || T > INT_MAX || H <= 0 || D <= 0 || D % 2 || max_pos <= 0 || ldx < (int64_t)H * D)
+    return BI_ERR_SHAPE;
   if (T == 0) return BI_OK;
   const int64_t n = T * H * (D / 2);
   if ((n + 255) / 256 > INT_MAX) return BI_ERR_SHAPE;

@@ -136,6 +136,7 @@ def test_glue_validation(L):
     assert L.bi_rope(P, 2048, 4, 32, 63, P, P, 384, None) == SHAPE              # odd D
     assert L.bi_rope(P, 1024, 4, 32, 64, P, P, 384, None) == SHAPE              # ldx < H*D
     assert L.bi_rope(P, 2048, 0, 32, 64, P, P, 384, None) == OK
+    assert L.bi_rope(P, 2, 2**31, 1, 2, P, P, 384, None) == SHAPE             # T beyond int32
     assert L.bi_swiglu(P, 16384, None, 8192, 4, 8192, None) == NULL
     assert L.bi_swiglu(P, 16000, P, 8192, 4, 8192, None) == SHAPE               # ld_gu < 2F
     assert L.bi_swiglu(P, 16384, P, 8192, 4, 8190, None) == SHAPE               # F % 8
@@ -220,3 +221,5 @@ def test_prefill_tc_validation(L):
     assert f(P, 4096, 0, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.0, None) == SHAPE     # scale <= 0
     assert f(P, 4100, 0, 0, 100, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == ALIGN
     assert f(P, 4096, 0, 0, 0, P, P, 100, P, 1, 256, P, 32, 8, 128, 0.088, None) == OK
+    # 2^23 row blocks x 256 head pairs: the 32-bit work list would overflow
+    assert f(P, 32768, 0, 0, 2**30, P, P, 100, P, 1, 2**26, P, 512, 256, 64, 0.125, None) == SHAPE
