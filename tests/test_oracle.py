@@ -119,6 +119,35 @@ def test_attention_golden(case):
     np.testing.assert_allclose(out, np.array(case["expected"]), rtol=0, atol=1e-15)
 
 
+def test_attention_split_merge_algebra_equals_full_softmax():
+    # Partials (m, l, o) of consecutive key splits, folded left with
+    # m = max(m1, m2), l = l1 e^(m1-m) + l2 e^(m2-m), o = o1 e^(m1-m) + o2 e^(m2-m),
+    # give o / l = the softmax over all keys (an identity, exact up to rounding in fp64).
+    rng = np.random.default_rng(21)
+    D, L, split = 16, 700, 256
+    q = rng.normal(size=D)
+    keys, vals = rng.normal(size=(L, D)), rng.normal(size=(L, D))
+    scale = 1.0 / math.sqrt(D)
+    m, l, o = -math.inf, 0.0, np.zeros(D)
+    for s0 in range(0, L, split):
+        sc = keys[s0:s0 + split] @ q * scale
+        m2 = sc.max()
+        e = np.exp(sc - m2)
+        l2, o2 = e.sum(), e @ vals[s0:s0 + split]
+        mn = max(m, m2)
+        a, b = math.exp(m - mn) if m > -math.inf else 0.0, math.exp(m2 - mn)
+        m, l, o = mn, l * a + l2 * b, o * a + o2 * b
+    np.testing.assert_allclose(oracle.softmax_attend(q, keys, vals, scale), o / l, rtol=0, atol=1e-14)
+
+
+def test_attention_key_order_does_not_matter():
+    rng = np.random.default_rng(22)
+    q, keys, vals = rng.normal(size=8), rng.normal(size=(50, 8)), rng.normal(size=(50, 8))
+    perm = rng.permutation(50)
+    np.testing.assert_allclose(oracle.softmax_attend(q, keys[perm], vals[perm], 0.3),
+                               oracle.softmax_attend(q, keys, vals, 0.3), rtol=0, atol=1e-15)
+
+
 def _tiny_paged(lens, Hkv=2, D=8, seed=0):
     return synth.paged_kv(lens, Hkv, D, seed=seed, poison_tail=False)
 
