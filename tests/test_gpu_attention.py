@@ -57,6 +57,27 @@ def test_decode_closed_forms():
     assert max_rel(out[1], mean) <= TOL_BF16
 
 
+def test_decode_zero_length_sequences_give_zero_rows():
+    # a sequence of length 0 sees no key: its rows are +0 in every bit, and the
+    # other rows keep the bits they have alone. The pages stay allocated (lengths
+    # 1, 40, 1) so only seq_lens says the outer two are empty.
+    q, kv = synth.decode_inputs(3, 32, 8, 128, max_len=64, seed=35, lens=[1, 40, 1])
+    kv = synth.PagedKV(kv.k_cache, kv.v_cache, kv.page_table, torch.tensor([0, 40, 0], dtype=torch.int32),
+                       kv.max_pages)
+    qd, kvd = q.to(dev()), _to_dev(kv)
+    out = _decode(qd, kvd)
+    assert bi.get_device_error() == 0
+    assert bool((out[0].view(torch.int16) == 0).all()) and bool((out[2].view(torch.int16) == 0).all())
+    one = bi.attention_decode(qd[1:2].contiguous(), kvd.k_cache, kvd.v_cache, kvd.page_table[1:2].contiguous(),
+                              kvd.seq_lens[1:2].contiguous())
+    assert same_bits(one[0], out[1])
+    # every sequence empty: no split at all, all rows zero
+    empty = bi.attention_decode(qd, kvd.k_cache, kvd.v_cache, kvd.page_table,
+                                torch.zeros(3, dtype=torch.int32, device=dev()))
+    assert bi.get_device_error() == 0
+    assert bool((empty.view(torch.int16) == 0).all())
+
+
 def test_decode_batch_invariant_and_run_to_run():
     lens = [3000, 1, 257, 4096, 77, 1500, 256, 999]
     q, kv = synth.decode_inputs(len(lens), 32, 8, 128, max_len=4096, seed=32, lens=lens)
