@@ -1,0 +1,260 @@
+"""Power of the GPU parity tests (CPU only): would they see a wrong kernel?
+
+A GPU parity test runs a kernel on fixed seeded inputs and requires its output to
+lie within a tolerance of the oracle's (normwise 1e-2 per row for bf16 outputs). A
+kernel bug slips through when its output stays inside that tolerance on those
+inputs. Here each plausible kernel bug is emulated in fp64 on the CPU: a dropped
+last page, split or 16-byte vector, a split combine without its rescaling, a wrong
+GQA head mapping or scale, an off-by-one causal mask, a wrong page lookup, an
+unwritten ragged tail. The emulation runs on exactly the inputs of the GPU parity
+test it targets, and must fail that test's own assertion on at least one of its
+cases, so the GPU test would fail on such a kernel.
+
+Out of reach by design: changes smaller than the tolerance, e.g. eps placed outside
+the square root of RMSNorm (about 1e-6 here) or fp32 instead of fp64 accumulation.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import TOL_BF16
+from test_oracle_mutants import _mutated
+
+PAGE = 16
+
+
+def _fails_parity(buggy: np.ndarray, ref: np.ndarray) -> bool:
+    """True when `max_rel(got, ref) <= TOL_BF16`, the GPU tests' assertion, is false
+    for got = buggy (NaN counts as a failure, as it does there)."""
+    err = oracle.normwise_rel_err(oracle.round_to_bf16(np.nan_to_num(buggy, nan=np.inf)), ref).max()
+    return not (err <= TOL_BF16)
+
+
+# ---------------------------------------------------------------------------
+# Decode attention: the cases of test_decode_matches_oracle
+
+DECODE_CASES = [(32, 8, 128), (32, 8, 64), (8, 8, 128), (32, 4, 128), (16, 8, 64), (8, 1, 64)]
+DECODE_LENS = [1, 16, 17, 255, 256, 257, 700, 513]
+
+
+def _decode_case(Hq, Hkv, D):
+    q, kv = synth.decode_inputs(len(DECODE_LENS), Hq, Hkv, D, max_len=800, seed=Hq + Hkv + D, lens=DECODE_LENS)
+    return (synth.to_f64(q), synth.to_f64(kv.k_cache), synth.to_f64(kv.v_cache), kv.page_table.numpy(),
+            kv.seq_lens.numpy())
+
+
+def _split_combine(q, k, v, pt, lens, rescale=True):
+    """Decode by fixed 256-token splits folded left; without `rescale` the split
+    partials are added as if they shared one maximum (a missing exp(m_s - M))."""
+    B, Hq, D = q.shape
+    group = Hq // k.shape[1]
+    out = np.zeros_like(q)
+    for b in range(B):
+        L = int(lens[b])
+        keys_all = [oracle.gather_kv(k, pt[b], g, L) for g in range(k.shape[1])]
+        vals_all = [oracle.gather_kv(v, pt[b], g, L) for g in range(k.shape[1])]
+        for h in range(Hq):
+            g = h // group
+            M, Lsum, O = -math.inf, 0.0, np.zeros(D)
+            parts = []
+            for s0 in range(0, L, 256):
+                sc = keys_all[g][s0:s0 + 256] @ q[b, h] / math.sqrt(D)
+                m = sc.max()
+                e = np.exp(sc - m)
+                parts.append((m, e.sum(), e @ vals_all[g][s0:s0 + 256]))
+            if not parts:
+                continue
+            M = max(p[0] for p in parts)
+            for m, l, o in parts:
+                w = math.exp(m - M) if rescale else 1.0
+                Lsum, O = Lsum + w * l, O + w * o
+            out[b, h] = O / Lsum
+    return out
+
+
+def _decode_bugs():
+    def scale_over_d(q, k, v, pt, lens):
+        return oracle.attention_decode(q, k, v, pt, lens, scale=1.0 / q.shape[2])
+
+    def drop_last_token(q, k, v, pt, lens):
+        return oracle.attention_decode(q, k, v, pt, lens - 1)
+
+    def drop_partial_page(q, k, v, pt, lens):
+        return oracle.attention_decode(q, k, v, pt, (lens // PAGE) * PAGE)
+
+    def drop_last_split(q, k, v, pt, lens):
+        return oracle.attention_decode(q, k, v, pt, ((lens - 1) // 256) * 256)
+
+    def combine_without_rescale(q, k, v, pt, lens):
+        return _split_combine(q, k, v, pt, lens, rescale=False)
+
+    def mutant(name, old, new):
+        def run(monkeypatch):
+            monkeypatch.setattr(oracle, name, _mutated(name, old, new))
+        return run
+
+    return {
+        "scale 1/D instead of 1/sqrt(D)": (scale_over_d, None),
+        "last token of each sequence dropped": (drop_last_token, None),
+        "last partial page dropped": (drop_partial_page, None),
+        "last 256-token split dropped": (drop_last_split, None),
+        "split partials combined without exp(m_s - M)": (combine_without_rescale, None),
+        "GQA heads interleaved (h -> kv-head h mod Hkv)":
+            (None, mutant("attention_rows", "h = g * group + j", "h = j * Hkv + g")),
+        "logical page index used as the physical page":
+            (None, mutant("gather_kv", "pages = np.asarray(page_row, dtype=np.int64)[t // PAGE]",
+                          "pages = t // PAGE")),
+        "kv-head 0 read for every query head":
+            (None, mutant("gather_kv", "cache[pages, g, t % PAGE]", "cache[pages, 0, t % PAGE]")),
+    }
+
+
+DECODE_BUGS = _decode_bugs()
+
+
+def test_controls_pass_parity():
+    # the correct results, rounded to bf16, pass every case of each GPU test: a
+    # "caught" above is the bug's doing, not the rounding's
+    for case in DECODE_CASES:
+        q, k, v, pt, lens = _decode_case(*case)
+        ref = oracle.attention_decode(q, k, v, pt, lens)
+        assert not _fails_parity(ref, ref)
+    for M, K in RMS_CASES:
+        x, w = (synth.to_f64(t) for t in synth.rmsnorm_inputs(M, K, seed=M + K))
+        assert not _fails_parity(oracle.rmsnorm(x, w, EPS), oracle.rmsnorm(x, w, EPS))
+    for M, N, K in MM_CASES:
+        a, w = (synth.to_f64(t) for t in synth.matmul_inputs(M, N, K, seed=M * 7 + N + K))
+        assert not _fails_parity(oracle.matmul(a, w), oracle.matmul(a, w))
+
+
+def test_split_combine_emulation_is_exact_when_rescaled():
+    q, k, v, pt, lens = _decode_case(32, 8, 64)
+    ref = oracle.attention_decode(q, k, v, pt, lens)
+    np.testing.assert_allclose(_split_combine(q, k, v, pt, lens), ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("bug", list(DECODE_BUGS))
+def test_decode_parity_sees(bug, monkeypatch):
+    fn, patch = DECODE_BUGS[bug]
+    caught = []
+    for case in DECODE_CASES:
+        q, k, v, pt, lens = _decode_case(*case)
+        ref = oracle.attention_decode(q, k, v, pt, lens)
+        if patch is None:
+            buggy = fn(q, k, v, pt, lens)
+        else:
+            with monkeypatch.context() as mp:
+                patch(mp)
+                with np.errstate(all="ignore"):
+                    buggy = oracle.attention_decode(q, k, v, pt, lens)
+        caught.append(_fails_parity(buggy, ref))
+    assert any(caught), f"{bug}: inside the tolerance in every case"
+
+
+# ---------------------------------------------------------------------------
+# Prefill attention: the cases of test_prefill_matches_oracle
+
+PREFILL_ROWS = [0, 1, 15, 16, 100, 255, 256, 257, 299, 300, 320, 344]
+
+
+def _prefill_case(D):
+    q, qs, qp, kv = synth.prefill_inputs([300, 45], 32, 8, D, seed=40 + D)
+    r = PREFILL_ROWS
+    return (synth.to_f64(q)[r], qs.numpy()[r], qp.numpy()[r], synth.to_f64(kv.k_cache), synth.to_f64(kv.v_cache),
+            kv.page_table.numpy())
+
+
+PREFILL_BUGS = {
+    "causal mask excludes the row's own position": ("np.asarray(q_pos) + 1", "np.asarray(q_pos)"),
+    "causal mask lets in the next position": ("np.asarray(q_pos) + 1", "np.asarray(q_pos) + 2"),
+    "every row reads sequence 0": ("np.asarray(q_seq),", "np.zeros(len(q_seq), dtype=np.int64),"),
+}
+
+
+@pytest.mark.parametrize("bug", list(PREFILL_BUGS))
+def test_prefill_parity_sees(bug, monkeypatch):
+    old, new = PREFILL_BUGS[bug]
+    caught = []
+    for D in (128, 64):
+        q, qs, qp, k, v, pt = _prefill_case(D)
+        ref = oracle.attention_prefill(q, qs, qp, k, v, pt)
+        # a row that would read past its sequence reads the store's next slot, which
+        # the inputs fill with NaN (stale data); index the page table safely
+        with monkeypatch.context() as mp:
+            mp.setattr(oracle, "attention_prefill", _mutated("attention_prefill", old, new))
+            with np.errstate(all="ignore"):
+                buggy = oracle.attention_prefill(q, qs, qp, k, v, np.where(pt < 0, pt.max(), pt))
+        caught.append(_fails_parity(buggy, ref))
+    assert any(caught), f"{bug}: inside the tolerance in every case"
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm: the cases of test_rmsnorm_matches_oracle
+
+RMS_CASES = [(1, 512), (7, 512), (32, 512), (129, 4096), (5, 2048), (3, 8), (4, 136), (2, 16384), (300, 1024)]
+EPS = 1e-6
+
+RMS_BUGS = {
+    "sum of squares misses the row's last 16-byte vector":
+        lambda x, w: x / np.sqrt((x[:, :-8] ** 2).sum(axis=1, keepdims=True) / x.shape[1] + EPS) * w,
+    "sum instead of mean": lambda x, w: x / np.sqrt((x ** 2).sum(axis=1, keepdims=True) + EPS) * w,
+    "weight not applied": lambda x, w: oracle.rmsnorm(x, np.ones_like(w), EPS),
+    "weight read one 16-byte vector late": lambda x, w: oracle.rmsnorm(x, np.roll(w, -8), EPS),
+    "row scaled by the next row's rms": lambda x, w: x / np.sqrt(
+        np.roll((x ** 2).mean(axis=1, keepdims=True), -1, axis=0) + EPS) * w,
+}
+
+
+@pytest.mark.parametrize("bug", list(RMS_BUGS))
+def test_rmsnorm_parity_sees(bug):
+    caught = []
+    for M, K in RMS_CASES:
+        x, w = synth.rmsnorm_inputs(M, K, seed=M + K)
+        x, w = synth.to_f64(x), synth.to_f64(w)
+        caught.append(_fails_parity(RMS_BUGS[bug](x, w), oracle.rmsnorm(x, w, EPS)))
+    assert any(caught), f"{bug}: inside the tolerance in every case"
+
+
+def test_a_dropped_vector_is_seen_only_at_small_k():
+    # the ragged small-K cases carry the check: at K >= 512 one 8-element vector
+    # moves the rms by less than the tolerance
+    bug = RMS_BUGS["sum of squares misses the row's last 16-byte vector"]
+    seen = {}
+    for M, K in RMS_CASES:
+        x, w = synth.rmsnorm_inputs(M, K, seed=M + K)
+        x, w = synth.to_f64(x), synth.to_f64(w)
+        seen[K] = _fails_parity(bug(x, w), oracle.rmsnorm(x, w, EPS))
+    assert seen[8] and seen[136] and not seen[4096]
+
+
+# ---------------------------------------------------------------------------
+# MatMul: the cases of test_matmul_matches_oracle
+
+MM_CASES = [(300, 520, 512), (1, 256, 64), (128, 256, 128), (129, 264, 192), (32, 1024, 512), (5, 8, 64),
+            (257, 4096, 1024)]
+
+MM_BUGS = {
+    "last 64-wide K block dropped": lambda a, w: oracle.matmul(a[:, :-64], w[:, :-64]),
+    "first K block accumulated twice": lambda a, w: oracle.matmul(a, w) + oracle.matmul(a[:, :64], w[:, :64]),
+    "columns past the last full 256-wide tile left at zero":
+        lambda a, w: np.where(np.arange(w.shape[0]) < (w.shape[0] // 256) * 256, oracle.matmul(a, w), 0.0),
+    "rows of a ragged last tile read from the tile's first row":
+        lambda a, w: oracle.matmul(a[np.minimum(np.arange(a.shape[0]), (a.shape[0] - 1) // 128 * 128)], w),
+    "K blocks taken in the wrong 64-column order for W":
+        lambda a, w: oracle.matmul(a, np.roll(w, 64, axis=1)),
+}
+
+
+@pytest.mark.parametrize("bug", list(MM_BUGS))
+def test_matmul_parity_sees(bug):
+    caught = []
+    for M, N, K in MM_CASES:
+        a, w = synth.matmul_inputs(M, N, K, seed=M * 7 + N + K)
+        a, w = synth.to_f64(a), synth.to_f64(w)
+        caught.append(_fails_parity(MM_BUGS[bug](a, w), oracle.matmul(a, w)))
+    assert any(caught), f"{bug}: inside the tolerance in every case"
