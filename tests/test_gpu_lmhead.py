@@ -53,16 +53,27 @@ def test_lmhead_matches_oracle(M, V, K):
 def test_lmhead_planted_margins():
     K, V = 128, 512
     _, w = synth.lmhead_inputs(1, V, K, seed=70)
-    h = torch.zeros((3, K), dtype=torch.bfloat16)
-    h[0, 0] = h[1, 1] = h[2, 2] = 1.0
-    w[:, :3] = w[:, :3].clamp(-1, 1)
+    h = torch.zeros((5, K), dtype=torch.bfloat16)
+    h[0, 0] = h[1, 1] = h[2, 2] = h[3, 3] = 1.0
+    h[4, 4] = h[4, 5] = 1.0
+    w[:, :6] = w[:, :6].clamp(-1, 1)
     w[7, 0], w[30, 0] = 3.0, 2.875      # margin 0.125 -> recompute, token 7
     w[12, 1], w[40, 1] = 8.0, 3.0       # margin 5 -> first pass, token 12
     w[5, 2], w[6, 2] = 2.0, 2.0         # exact tie -> margin 0, lowest index wins
+    w[9, 3], w[20, 3] = 4.0, 3.5        # margin exactly 0.5 is not below 0.5 -> first pass
+    # row 4: logits 256 (token 0) and 256 + 0.625 (token 1). Between 256 and 512 bf16
+    # values are 2 apart, so the first pass sees a tie (margin 0, token 0); the fp32
+    # recompute sees 256.625 and must return token 1.
+    w[0, 4], w[0, 5] = 256.0, 0.0
+    w[1, 4], w[1, 5] = 256.0, 0.625
     tok, rec, lg = bi.lmhead_argmax(h.to(dev()), w.to(dev()), TAU, want_logits=True)
-    assert tok.cpu().tolist() == [7, 12, 5]
-    assert rec.cpu().tolist() == [1, 0, 1]
+    assert tok.cpu().tolist() == [7, 12, 5, 9, 1]
+    assert rec.cpu().tolist() == [1, 0, 1, 0, 1]
     assert float(lg[0, 7]) == 3.0 and float(lg[0, 30]) == 2.875
+    assert float(lg[4, 1]) == 256.625 and float(lg[4, 0]) == 256.0
+    # the first pass alone (bf16 logits) could not tell rows 4's two tokens apart
+    first = bi.matmul(h.to(dev()), w.to(dev()))
+    assert float(first[4, 0]) == float(first[4, 1]) == 256.0
 
 
 def test_lmhead_thresholds_force_or_forbid_recompute():

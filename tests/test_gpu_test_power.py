@@ -258,3 +258,104 @@ def test_matmul_parity_sees(bug):
         a, w = synth.to_f64(a), synth.to_f64(w)
         caught.append(_fails_parity(MM_BUGS[bug](a, w), oracle.matmul(a, w)))
     assert any(caught), f"{bug}: inside the tolerance in every case"
+
+
+# ---------------------------------------------------------------------------
+# LM head: the cases of test_gpu_lmhead.py (oracle comparison, planted margins,
+# thresholds that force or forbid the recompute)
+
+LM_CASES = [(9, 1000, 256), (1, 32000, 2048), (64, 32000, 2048), (40, 4096, 512), (6, 2000, 4160)]
+TAU = 0.5
+
+
+def _first_argmax(v, highest):
+    idx = np.flatnonzero(v == v.max())
+    return int(idx[-1] if highest else idx[0])
+
+
+def _lm_emulate(h, w, tau, bug):
+    """What bi_lmhead_argmax returns (tokens, recomputed, fp32 logits or NaN) for a
+    correct kernel (bug None) or for one with the named bug."""
+    r = oracle.lmhead(h, w, tau)
+    lb = oracle.round_to_bf16(r["logits"])
+    b1 = np.array([oracle.top2(row)[0] for row in lb])
+    b2 = np.array([oracle.top2(row)[2] for row in lb])
+    margin = (b1.astype(np.float32) - b2.astype(np.float32)).astype(np.float64)
+    if bug == "top-2 margin taken from the fp32 accumulators, not the bf16 logits":
+        margin = r["margin"]
+    rec = margin <= tau if bug == "threshold test is <= instead of <" else margin < tau
+    lg32 = r["logits"].astype(np.float32).astype(np.float64)
+    if bug == "recompute done in bf16":
+        lg32 = lb
+    if bug == "recompute drops the last 64-wide K block":
+        lg32 = oracle.matmul(h[:, :-64], w[:, :-64]).astype(np.float32).astype(np.float64)
+    highest = bug == "ties go to the highest index"
+    first = np.array([_first_argmax(row, highest) for row in lb])
+    second = np.array([_first_argmax(row, highest) for row in lg32])
+    if bug == "recomputed rows keep the first-pass token":
+        second = first
+    tokens = np.where(rec, second, first)
+    logits = np.where(rec[:, None], lg32, np.nan)
+    return tokens, rec, logits
+
+
+LM_BUGS = ["threshold test is <= instead of <", "top-2 margin taken from the fp32 accumulators, not the bf16 logits",
+           "recompute done in bf16", "recompute drops the last 64-wide K block", "ties go to the highest index",
+           "recomputed rows keep the first-pass token"]
+
+
+def _planted_inputs():
+    K, V = 128, 512
+    _, w = synth.lmhead_inputs(1, V, K, seed=70)
+    h = np.zeros((5, K))
+    h[0, 0] = h[1, 1] = h[2, 2] = h[3, 3] = 1.0
+    h[4, 4] = h[4, 5] = 1.0
+    w = synth.to_f64(w)
+    w[:, :6] = np.clip(w[:, :6], -1, 1)
+    w[7, 0], w[30, 0] = 3.0, 2.875
+    w[12, 1], w[40, 1] = 8.0, 3.0
+    w[5, 2], w[6, 2] = 2.0, 2.0
+    w[9, 3], w[20, 3] = 4.0, 3.5
+    w[0, 4], w[0, 5] = 256.0, 0.0
+    w[1, 4], w[1, 5] = 256.0, 0.625
+    return h, w
+
+
+def _lm_tests_fail(bug, cases):
+    """True when some assertion of the LM-head GPU tests fails on the emulated output."""
+    import torch
+    from test_gpu_lmhead import _check_against_oracle
+
+    try:
+        for h, w in cases:
+            tok, rec, lg = _lm_emulate(h, w, TAU, bug)
+            ht = torch.from_numpy(h).to(torch.bfloat16)
+            wt = torch.from_numpy(w).to(torch.bfloat16)
+            _check_against_oracle(ht, wt, TAU, torch.from_numpy(tok), torch.from_numpy(rec.astype(np.int32)),
+                                  torch.from_numpy(lg.astype(np.float32)))
+            assert np.isnan(lg[~rec]).all()
+        h, w = _planted_inputs()
+        tok, rec, lg = _lm_emulate(h, w, TAU, bug)
+        assert tok.tolist() == [7, 12, 5, 9, 1] and rec.astype(int).tolist() == [1, 0, 1, 0, 1]
+        assert lg[0, 7] == 3.0 and lg[0, 30] == 2.875 and lg[4, 1] == 256.625 and lg[4, 0] == 256.0
+        h, w = (synth.to_f64(t) for t in synth.lmhead_inputs(16, 4096, 512, seed=71))
+        assert _lm_emulate(h, w, 0.0, bug)[1].sum() == 0
+        tok, rec, lg = _lm_emulate(h, w, math.inf, bug)
+        assert rec.sum() == 16 and (tok == np.argmax(lg, axis=1)).all()
+    except AssertionError:
+        return True
+    return False
+
+
+@pytest.fixture(scope="module")
+def lm_cases():
+    return [tuple(synth.to_f64(t) for t in synth.lmhead_inputs(M, V, K, seed=M + V)) for M, V, K in LM_CASES]
+
+
+def test_lmhead_control_passes(lm_cases):
+    assert not _lm_tests_fail(None, lm_cases)
+
+
+@pytest.mark.parametrize("bug", LM_BUGS)
+def test_lmhead_tests_see(bug, lm_cases):
+    assert _lm_tests_fail(bug, lm_cases), f"{bug}: every LM-head GPU test would pass"
