@@ -61,6 +61,34 @@ def test_prefill_tc_whole_equals_chunked_and_agrees_with_cuda_cores(D, Hq, Hkv):
     assert bi.get_device_error() == 0
 
 
+def test_prefill_tc_large_score_jumps_take_the_rescale_path():
+    # With q, k ~ N(0, 1) no later block's maximum exceeds the running reference
+    # point by the lazy threshold (8 in log2 units), so O is never rescaled after
+    # the first block. Keys at positions >= 130 scaled by 8 raise the block maxima
+    # by about 20 (natural units) and force the rescale in the blocks after the jump
+    # (thousands of times over the 300 rows x 32 heads). Parity with the oracle and
+    # whole vs chunked bits must still hold.
+    S, Hq, Hkv, D = 300, 32, 8, 128
+    q, qs, qp, kv = synth.prefill_inputs([S], Hq, Hkv, D, seed=77)
+    t = torch.arange(S)
+    pages = kv.page_table[0, t // 16].long()
+    big = t >= 130
+    k = kv.k_cache.clone()
+    k[pages[big], :, (t % 16)[big], :] = (k[pages[big], :, (t % 16)[big], :].float() * 8).to(torch.bfloat16)
+    kv = synth.PagedKV(k, kv.v_cache, kv.page_table, kv.seq_lens, kv.max_pages)
+    kvd = _dev(kv)
+    qd = q.to(dev())
+    out = bi.attention_prefill_tc(qd, 0, 0, kvd.k_cache, kvd.v_cache, kvd.page_table)
+    assert torch.isfinite(out.float()).all()
+    ref = oracle.attention_prefill(synth.to_f64(q), qs.numpy(), qp.numpy(), synth.to_f64(kv.k_cache),
+                                   synth.to_f64(kv.v_cache), kv.page_table.numpy())
+    assert max_rel(out.cpu(), ref) <= TOL_BF16
+    for c0, c1 in ((0, 130), (130, 200), (200, 300)):  # the jump at a chunk start and inside one
+        part = bi.attention_prefill_tc(qd[c0:c1].contiguous(), 0, c0, kvd.k_cache, kvd.v_cache, kvd.page_table)
+        assert same_bits(part, out[c0:c1]), c0
+    assert bi.get_device_error() == 0
+
+
 def test_prefill_tc_full_size_4096_whole_vs_8_chunks():
     S, Hq, Hkv, D = 4096, 32, 8, 128
     kv = synth.paged_kv_device([S], Hkv, D, seed=60, max_pages=S // 16, device=dev())
