@@ -19,8 +19,9 @@ from gpu_util import TOL_FP32, dev, max_rel, same_bits
 pytestmark = pytest.mark.gpu
 
 # N: one 8-vector, ragged tails across the 256-thread stride, the 32000 vocabulary,
-# the register-resident maximum and the re-read path above it
-SIZES = [8, 1000, 2056, 32000, 32768, 40000]
+# the register-resident maximum and the re-read path above it; together every
+# register variant (vectors per thread 1, 2, 4, 8, 16) and the re-read one
+SIZES = [8, 1000, 2056, 6000, 12000, 32000, 32768, 40000]
 
 
 def _u64(t):
@@ -52,7 +53,7 @@ def test_log_softmax_and_token_logprob_match_oracle(N):
     assert bi.get_device_error() == 0
 
 
-@pytest.mark.parametrize("K", [8, 2048, 4096, 40000])
+@pytest.mark.parametrize("K", [8, 2048, 4096, 6000, 12000, 40000])
 def test_row_mean_matches_oracle(K):
     M = 7
     x = synth.normal_bf16((M, K), 90 + K % 89, mean=0.5)

@@ -12,8 +12,10 @@ pytestmark = pytest.mark.gpu
 EPS = 1e-6
 
 
+# every register variant of the kernel (16-byte vectors per thread NV = 1, 2, 4, 8, 16),
+# each also with a ragged last round (K = 136, 1032, 3080, 5128, 8200)
 @pytest.mark.parametrize("M,K", [(1, 512), (7, 512), (32, 512), (129, 4096), (5, 2048), (3, 8), (4, 136),
-                                 (2, 16384), (300, 1024)])
+                                 (2, 16384), (300, 1024), (3, 1032), (3, 3080), (3, 5128), (2, 8192), (2, 8200)])
 def test_rmsnorm_matches_oracle(M, K):
     x, w = synth.rmsnorm_inputs(M, K, seed=M + K)
     y = bi.rmsnorm(x.to(dev()), w.to(dev()), EPS)
