@@ -32,7 +32,9 @@ def _oracle_decode(q, kv):
                                    kv.page_table.cpu().numpy(), kv.seq_lens.cpu().numpy())
 
 
-@pytest.mark.parametrize("Hq,Hkv,D", [(32, 8, 128), (32, 8, 64), (8, 8, 128), (32, 4, 128), (16, 8, 64), (8, 1, 64)])
+# every instantiation of the split kernel: D in {64, 128} x group size Hq/Hkv in {1, 2, 4, 8}
+@pytest.mark.parametrize("Hq,Hkv,D", [(32, 8, 128), (32, 8, 64), (8, 8, 128), (32, 4, 128), (16, 8, 64), (8, 1, 64),
+                                      (16, 8, 128), (8, 8, 64)])
 def test_decode_matches_oracle(Hq, Hkv, D):
     lens = [1, 16, 17, 255, 256, 257, 700, 513]
     q, kv = synth.decode_inputs(len(lens), Hq, Hkv, D, max_len=800, seed=Hq + Hkv + D, lens=lens)
