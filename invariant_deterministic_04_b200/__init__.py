@@ -12,6 +12,7 @@ Operations (see include/bi.h for the exact contracts):
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -100,6 +101,30 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+@contextlib.contextmanager
+def _on(device, stream):
+    """Launch context: the tensors' device, and the caller's stream if one was given.
+
+    Under it, temporaries (workspace, outputs) are allocated on the stream the
+    kernels run on, so the caching allocator cannot hand their memory to other
+    work before those kernels are done with it."""
+    with torch.cuda.device(device):
+        if stream is None:
+            yield
+        else:
+            with torch.cuda.stream(stream):
+                yield
+
+
+def _same_device(first: torch.Tensor, *others):
+    """The device of `first`; every other tensor given (None entries skipped) must be on it."""
+    d = first.device
+    for t in others:
+        if t is not None and t.device != d:
+            raise ValueError(f"all tensors must be on {d}; got one on {t.device}")
+    return d
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -118,6 +143,21 @@ def _contig(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _out(t: torch.Tensor, dtype, shape, name: str, strided_rows: bool = False):
+    """Check a caller-supplied output (the C calls write exactly `shape` through its
+    pointer, and a row stride where they take one): dtype, shape, and contiguous
+    storage, or contiguous rows (unit inner stride) when `strided_rows`."""
+    _req(t, dtype, name, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if strided_rows:
+        if t.stride(-1) != 1:
+            raise ValueError(f"{name} rows must be contiguous")
+    else:
+        _contig(t, name)
+    return t
+
+
 # ---------------------------------------------------------------------------
 
 
@@ -129,9 +169,13 @@ def rmsnorm(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, out: torch.Tens
     if x.stride(1) != 1:
         raise ValueError("x rows must be contiguous")
     M, K = x.shape
-    y = torch.empty_like(x, memory_format=torch.contiguous_format) if out is None else out
-    _check("bi_rmsnorm", lib().bi_rmsnorm(_ptr(x), x.stride(0), _ptr(w), _ptr(y), y.stride(0), M, K, eps,
-                                         _stream(stream)))
+    device = _same_device(x, w, out)
+    if out is not None:
+        _out(out, torch.bfloat16, (M, K), "out", strided_rows=True)
+    with _on(device, stream):
+        y = torch.empty_like(x, memory_format=torch.contiguous_format) if out is None else out
+        _check("bi_rmsnorm", lib().bi_rmsnorm(_ptr(x), x.stride(0), _ptr(w), _ptr(y), y.stride(0), M, K, eps,
+                                             _stream()))
     return y
 
 
@@ -145,9 +189,13 @@ def matmul(a: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, st
     N = w.shape[0]
     if w.shape[1] != K:
         raise ValueError(f"inner dimensions differ: {tuple(a.shape)} x {tuple(w.shape)}^T")
-    c = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else out
-    _check("bi_matmul", lib().bi_matmul(_ptr(a), a.stride(0), _ptr(w), w.stride(0), _ptr(c), c.stride(0), M, N, K,
-                                       _stream(stream)))
+    device = _same_device(a, w, out)
+    if out is not None:
+        _out(out, torch.bfloat16, (M, N), "out", strided_rows=True)
+    with _on(device, stream):
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=device) if out is None else out
+        _check("bi_matmul", lib().bi_matmul(_ptr(a), a.stride(0), _ptr(w), w.stride(0), _ptr(c), c.stride(0), M, N,
+                                           K, _stream()))
     return c
 
 
@@ -155,7 +203,16 @@ def attention_workspace_size(rows: int, Hq: int, D: int, max_pages_per_seq: int)
     return int(lib().bi_attention_workspace_size(rows, Hq, D, max_pages_per_seq))
 
 
+def _check_workspace(workspace):
+    """A caller-supplied workspace: any dtype, CUDA, contiguous (its byte size is what counts)."""
+    if workspace is not None:
+        if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
+            raise TypeError("workspace must be a CUDA tensor")
+        _contig(workspace, "workspace")
+
+
 def _workspace(nbytes: int, device, workspace):
+    """(tensor, bytes): the caller's workspace, else a fresh one (call under _on)."""
     if workspace is not None:
         return workspace, workspace.numel() * workspace.element_size()
     return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device), nbytes
@@ -180,11 +237,16 @@ def attention_decode(q, k_cache, v_cache, page_table, seq_lens, scale: float | N
         raise ValueError("page_table and seq_lens need a row per sequence")
     maxp = page_table.shape[1]
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    out = torch.empty_like(q) if out is None else out
-    ws, nbytes = _workspace(attention_workspace_size(B, Hq, D, maxp), q.device, workspace)
-    _check("bi_attention_decode", lib().bi_attention_decode(
-        _ptr(q), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), maxp, _ptr(seq_lens), _ptr(out),
-        B, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream(stream)))
+    device = _same_device(q, k_cache, v_cache, page_table, seq_lens, out, workspace)
+    if out is not None:
+        _out(out, torch.bfloat16, (B, Hq, D), "out")
+    _check_workspace(workspace)
+    with _on(device, stream):
+        out = torch.empty_like(q) if out is None else out
+        ws, nbytes = _workspace(attention_workspace_size(B, Hq, D, maxp), device, workspace)
+        _check("bi_attention_decode", lib().bi_attention_decode(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), maxp, _ptr(seq_lens), _ptr(out),
+            B, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream()))
     return out
 
 
@@ -211,10 +273,14 @@ def attention_decode_static(q, k_cache, v_cache, page_table, seq_lens, scale: fl
     if page_table.shape[0] < B or seq_lens.shape[0] < B:
         raise ValueError("page_table and seq_lens need a row per sequence")
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    out = torch.empty_like(q) if out is None else out
-    _check("bi_attention_decode_static", lib().bi_attention_decode_static(
-        _ptr(q), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), page_table.shape[1], _ptr(seq_lens),
-        _ptr(out), B, Hq, Hkv, D, scale, _stream(stream)))
+    device = _same_device(q, k_cache, v_cache, page_table, seq_lens, out)
+    if out is not None:
+        _out(out, torch.bfloat16, (B, Hq, D), "out")
+    with _on(device, stream):
+        out = torch.empty_like(q) if out is None else out
+        _check("bi_attention_decode_static", lib().bi_attention_decode_static(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), page_table.shape[1], _ptr(seq_lens),
+            _ptr(out), B, Hq, Hkv, D, scale, _stream()))
     return out
 
 
@@ -250,11 +316,16 @@ def attention_prefill(q, q_seq, q_pos, k_cache, v_cache, page_table, scale: floa
         raise ValueError("q_seq and q_pos need one entry per query row")
     num_seqs, maxp = page_table.shape
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    out = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=q.device) if out is None else out
-    ws, nbytes = _workspace(attention_workspace_size(T, Hq, D, maxp), q.device, workspace)
-    _check("bi_attention_prefill", lib().bi_attention_prefill(
-        _ptr(q), ldq, _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table),
-        num_seqs, maxp, _ptr(out), T, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream(stream)))
+    device = _same_device(q, q_seq, q_pos, k_cache, v_cache, page_table, out, workspace)
+    if out is not None:
+        _out(out, torch.bfloat16, (T, Hq, D), "out")
+    _check_workspace(workspace)
+    with _on(device, stream):
+        out = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=device) if out is None else out
+        ws, nbytes = _workspace(attention_workspace_size(T, Hq, D, maxp), device, workspace)
+        _check("bi_attention_prefill", lib().bi_attention_prefill(
+            _ptr(q), ldq, _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table),
+            num_seqs, maxp, _ptr(out), T, Hq, Hkv, D, scale, _ptr(ws), nbytes, _stream()))
     return out
 
 
@@ -274,10 +345,14 @@ def attention_prefill_tc(q, seq: int, pos0: int, k_cache, v_cache, page_table, s
         raise ValueError("k_cache/v_cache must be [num_pages, Hkv, 16, D]")
     num_seqs, maxp = page_table.shape
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    out = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=q.device) if out is None else out
-    _check("bi_attention_prefill_tc", lib().bi_attention_prefill_tc(
-        _ptr(q), ldq, seq, pos0, T, _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), num_seqs, maxp,
-        _ptr(out), Hq, Hkv, D, scale, _stream(stream)))
+    device = _same_device(q, k_cache, v_cache, page_table, out)
+    if out is not None:
+        _out(out, torch.bfloat16, (T, Hq, D), "out")
+    with _on(device, stream):
+        out = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=device) if out is None else out
+        _check("bi_attention_prefill_tc", lib().bi_attention_prefill_tc(
+            _ptr(q), ldq, seq, pos0, T, _ptr(k_cache), _ptr(v_cache), num_pages, _ptr(page_table), num_seqs, maxp,
+            _ptr(out), Hq, Hkv, D, scale, _stream()))
     return out
 
 
@@ -294,10 +369,18 @@ def kv_append(k_new, v_new, q_seq, q_pos, k_cache, v_cache, page_table, stream=N
     if _rows3(v_new, "v_new") != ld or v_new.shape != k_new.shape:
         raise ValueError("k_new and v_new must have the same shape and row stride")
     T, Hkv, D = k_new.shape
+    if q_seq.shape != (T,) or q_pos.shape != (T,):
+        raise ValueError("q_seq and q_pos need one entry per new row")
+    if k_cache.dim() != 4 or k_cache.shape != v_cache.shape or k_cache.shape[1:] != (Hkv, PAGE_TOKENS, D):
+        raise ValueError("k_cache/v_cache must be [num_pages, Hkv, 16, D] matching k_new")
+    if page_table.dim() != 2:
+        raise ValueError("page_table must be [num_seqs, max_pages]")
     num_seqs, maxp = page_table.shape
-    _check("bi_kv_append", lib().bi_kv_append(
-        _ptr(k_new), _ptr(v_new), ld, _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
-        _ptr(page_table), num_seqs, maxp, T, Hkv, D, _stream(stream)))
+    device = _same_device(k_new, v_new, q_seq, q_pos, k_cache, v_cache, page_table)
+    with _on(device, stream):
+        _check("bi_kv_append", lib().bi_kv_append(
+            _ptr(k_new), _ptr(v_new), ld, _ptr(q_seq), _ptr(q_pos), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
+            _ptr(page_table), num_seqs, maxp, T, Hkv, D, _stream()))
 
 
 def gather_rows(src, idx, out=None, stream=None):
@@ -308,9 +391,13 @@ def gather_rows(src, idx, out=None, stream=None):
     if src.stride(1) != 1:
         raise ValueError("src rows must be contiguous")
     M, W = idx.shape[0], src.shape[1]
-    out = torch.empty((M, W), dtype=torch.bfloat16, device=src.device) if out is None else out
-    _check("bi_gather_rows", lib().bi_gather_rows(_ptr(src), src.stride(0), src.shape[0], _ptr(idx), M, W, _ptr(out),
-                                                  out.stride(0), _stream(stream)))
+    device = _same_device(src, idx, out)
+    if out is not None:
+        _out(out, torch.bfloat16, (M, W), "out", strided_rows=True)
+    with _on(device, stream):
+        out = torch.empty((M, W), dtype=torch.bfloat16, device=device) if out is None else out
+        _check("bi_gather_rows", lib().bi_gather_rows(_ptr(src), src.stride(0), src.shape[0], _ptr(idx), M, W,
+                                                      _ptr(out), out.stride(0), _stream()))
     return out
 
 
@@ -325,8 +412,12 @@ def rope(x, pos, cos_sin, stream=None):
     T, H, D = x.shape
     if cos_sin.shape[1:] != (D // 2, 2):
         raise ValueError("cos_sin must be [max_pos, D/2, 2]")
-    _check("bi_rope", lib().bi_rope(_ptr(x), ldx, T, H, D, _ptr(pos), _ptr(cos_sin), cos_sin.shape[0],
-                                    _stream(stream)))
+    if pos.shape != (T,):
+        raise ValueError("pos needs one entry per row of x")
+    device = _same_device(x, pos, cos_sin)
+    with _on(device, stream):
+        _check("bi_rope", lib().bi_rope(_ptr(x), ldx, T, H, D, _ptr(pos), _ptr(cos_sin), cos_sin.shape[0],
+                                        _stream()))
     return x
 
 
@@ -337,9 +428,13 @@ def swiglu(gate_up, out=None, stream=None):
         raise ValueError("gate_up rows must be contiguous")
     M, F2 = gate_up.shape
     F = F2 // 2
-    out = torch.empty((M, F), dtype=torch.bfloat16, device=gate_up.device) if out is None else out
-    _check("bi_swiglu", lib().bi_swiglu(_ptr(gate_up), gate_up.stride(0), _ptr(out), out.stride(0), M, F,
-                                        _stream(stream)))
+    device = _same_device(gate_up, out)
+    if out is not None:
+        _out(out, torch.bfloat16, (M, F), "out", strided_rows=True)
+    with _on(device, stream):
+        out = torch.empty((M, F), dtype=torch.bfloat16, device=device) if out is None else out
+        _check("bi_swiglu", lib().bi_swiglu(_ptr(gate_up), gate_up.stride(0), _ptr(out), out.stride(0), M, F,
+                                            _stream()))
     return out
 
 
@@ -350,8 +445,12 @@ def add(a, b, out=None, stream=None):
         _contig(t, n)
     if a.shape != b.shape:
         raise ValueError("a and b must have the same shape")
-    out = torch.empty_like(a) if out is None else out
-    _check("bi_add", lib().bi_add(_ptr(a), _ptr(b), _ptr(out), a.numel(), _stream(stream)))
+    device = _same_device(a, b, out)
+    if out is not None:
+        _out(out, torch.bfloat16, tuple(a.shape), "out")
+    with _on(device, stream):
+        out = torch.empty_like(a) if out is None else out
+        _check("bi_add", lib().bi_add(_ptr(a), _ptr(b), _ptr(out), a.numel(), _stream()))
     return out
 
 
@@ -372,15 +471,25 @@ def lmhead_argmax(h, w, margin_threshold: float = 0.5, want_logits: bool = False
         raise ValueError("h rows must be contiguous")
     M, K = h.shape
     V = w.shape[0]
-    dev = h.device
-    tokens = torch.empty(M, dtype=torch.int32, device=dev) if tokens is None else tokens
-    recomputed = torch.empty(M, dtype=torch.int32, device=dev) if recomputed is None else recomputed
-    if want_logits and logits_fp32 is None:
-        logits_fp32 = torch.full((M, V), float("nan"), dtype=torch.float32, device=dev)
-    ws, nbytes = _workspace(lmhead_workspace_size(M, V), dev, workspace)
-    _check("bi_lmhead_argmax", lib().bi_lmhead_argmax(
-        _ptr(h), h.stride(0), _ptr(w), M, V, K, margin_threshold, _ptr(tokens), _ptr(recomputed),
-        _ptr(logits_fp32), _ptr(ws), nbytes, _stream(stream)))
+    if w.shape[1] != K:
+        raise ValueError(f"h has {K} columns but w has {w.shape[1]}")
+    dev = _same_device(h, w, tokens, recomputed, logits_fp32, workspace)
+    if tokens is not None:
+        _out(tokens, torch.int32, (M,), "tokens")
+    if recomputed is not None:
+        _out(recomputed, torch.int32, (M,), "recomputed")
+    if logits_fp32 is not None:
+        _out(logits_fp32, torch.float32, (M, V), "logits_fp32")
+    _check_workspace(workspace)
+    with _on(dev, stream):
+        tokens = torch.empty(M, dtype=torch.int32, device=dev) if tokens is None else tokens
+        recomputed = torch.empty(M, dtype=torch.int32, device=dev) if recomputed is None else recomputed
+        if want_logits and logits_fp32 is None:
+            logits_fp32 = torch.full((M, V), float("nan"), dtype=torch.float32, device=dev)
+        ws, nbytes = _workspace(lmhead_workspace_size(M, V), dev, workspace)
+        _check("bi_lmhead_argmax", lib().bi_lmhead_argmax(
+            _ptr(h), h.stride(0), _ptr(w), M, V, K, margin_threshold, _ptr(tokens), _ptr(recomputed),
+            _ptr(logits_fp32), _ptr(ws), nbytes, _stream()))
     return tokens, recomputed, logits_fp32
 
 
@@ -402,27 +511,38 @@ def _u64(t: torch.Tensor, name: str, M: int):
 def log_softmax(x, out=None, stream=None):
     """fp32 log_softmax of each bf16 row, one fixed reduction order per row."""
     M, N = _rows2(x, "x")
-    y = torch.empty((M, N), dtype=torch.float32, device=x.device) if out is None else out
-    _req(y, torch.float32, "out", 2)
-    _check("bi_log_softmax", lib().bi_log_softmax(_ptr(x), x.stride(0), _ptr(y), y.stride(0), M, N, _stream(stream)))
+    device = _same_device(x, out)
+    if out is not None:
+        _out(out, torch.float32, (M, N), "out", strided_rows=True)
+    with _on(device, stream):
+        y = torch.empty((M, N), dtype=torch.float32, device=device) if out is None else out
+        _check("bi_log_softmax", lib().bi_log_softmax(_ptr(x), x.stride(0), _ptr(y), y.stride(0), M, N, _stream()))
     return y
 
 
 def token_logprob(x, tokens, out=None, stream=None):
     """fp32 log-probability of tokens[m] under log_softmax(x[m])."""
     M, N = _rows2(x, "x")
-    _req(tokens, torch.int32, "tokens", 1)
-    out = torch.empty(M, dtype=torch.float32, device=x.device) if out is None else out
-    _check("bi_token_logprob", lib().bi_token_logprob(_ptr(x), x.stride(0), _ptr(tokens), _ptr(out), M, N,
-                                                     _stream(stream)))
+    _out(tokens, torch.int32, (M,), "tokens")
+    device = _same_device(x, tokens, out)
+    if out is not None:
+        _out(out, torch.float32, (M,), "out")
+    with _on(device, stream):
+        out = torch.empty(M, dtype=torch.float32, device=device) if out is None else out
+        _check("bi_token_logprob", lib().bi_token_logprob(_ptr(x), x.stride(0), _ptr(tokens), _ptr(out), M, N,
+                                                         _stream()))
     return out
 
 
 def row_mean(x, out=None, stream=None):
     """fp32 mean of each bf16 row, one fixed reduction order per row."""
     M, K = _rows2(x, "x")
-    out = torch.empty(M, dtype=torch.float32, device=x.device) if out is None else out
-    _check("bi_row_mean", lib().bi_row_mean(_ptr(x), x.stride(0), _ptr(out), M, K, _stream(stream)))
+    device = _same_device(x, out)
+    if out is not None:
+        _out(out, torch.float32, (M,), "out")
+    with _on(device, stream):
+        out = torch.empty(M, dtype=torch.float32, device=device) if out is None else out
+        _check("bi_row_mean", lib().bi_row_mean(_ptr(x), x.stride(0), _ptr(out), M, K, _stream()))
     return out
 
 
@@ -431,9 +551,13 @@ def sampling_uniforms(seeds, steps, V: int, out=None, stream=None):
     M = seeds.shape[0]
     _u64(seeds, "seeds", M)
     _u64(steps, "steps", M)
-    u = torch.empty((M, V), dtype=torch.float32, device=seeds.device) if out is None else out
-    _check("bi_sampling_uniforms", lib().bi_sampling_uniforms(_ptr(seeds), _ptr(steps), _ptr(u), u.stride(0), M, V,
-                                                             _stream(stream)))
+    device = _same_device(seeds, steps, out)
+    if out is not None:
+        _out(out, torch.float32, (M, V), "out", strided_rows=True)
+    with _on(device, stream):
+        u = torch.empty((M, V), dtype=torch.float32, device=device) if out is None else out
+        _check("bi_sampling_uniforms", lib().bi_sampling_uniforms(_ptr(seeds), _ptr(steps), _ptr(u), u.stride(0), M,
+                                                                 V, _stream()))
     return u
 
 
@@ -442,9 +566,13 @@ def sample(logits, seeds, steps, temperature: float, out=None, stream=None):
     M, V = _rows2(logits, "logits")
     _u64(seeds, "seeds", M)
     _u64(steps, "steps", M)
-    out = torch.empty(M, dtype=torch.int32, device=logits.device) if out is None else out
-    _check("bi_sample", lib().bi_sample(_ptr(logits), logits.stride(0), _ptr(seeds), _ptr(steps), temperature,
-                                       _ptr(out), M, V, _stream(stream)))
+    device = _same_device(logits, seeds, steps, out)
+    if out is not None:
+        _out(out, torch.int32, (M,), "out")
+    with _on(device, stream):
+        out = torch.empty(M, dtype=torch.int32, device=device) if out is None else out
+        _check("bi_sample", lib().bi_sample(_ptr(logits), logits.stride(0), _ptr(seeds), _ptr(steps), temperature,
+                                           _ptr(out), M, V, _stream()))
     return out
 
 
