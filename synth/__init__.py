@@ -210,6 +210,17 @@ def _device_normal_bf16(shape, gen, device, chunk_elems=1 << 28):
     return out
 
 
+def normal_bf16_device(shape, seed: int, device, std: float = 1.0, mean: float = 0.0) -> torch.Tensor:
+    """Seeded N(mean, std^2) bf16 draws made on the device (for inputs of several GB,
+    too slow to draw on the host). Same distribution as normal_bf16, other values."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    x = _device_normal_bf16(shape, gen, device)
+    if std != 1.0 or mean != 0.0:
+        x = (x.float() * std + mean).to(torch.bfloat16)
+    return x
+
+
 def paged_kv_device(seq_lens, Hkv: int, D: int, seed: int, max_pages: int, device, spare_pages: int = 1) -> PagedKV:
     lens = [int(v) for v in (seq_lens.tolist() if torch.is_tensor(seq_lens) else seq_lens)]
     B = len(lens)

@@ -131,6 +131,35 @@ def test_sample_frequencies_follow_softmax():
     assert np.all(np.abs(counts - n * p) < 4.5 * sigma), (counts, n * p)
 
 
+def test_reductions_full_size_4096x32000_sampled():
+    # the benchmark's reductions workload: log_softmax, token log-probability and
+    # sampling of 4096 rows of 32000 logits, checked on sampled rows
+    M, V, T = 4096, 32000, 0.8
+    x = synth.normal_bf16_device((M, V), 120, dev(), std=3.0)
+    tok = torch.randint(0, V, (M,), generator=synth.generator(121), dtype=torch.int32)
+    seeds = synth.request_seeds(M, 122)
+    steps = torch.arange(M, dtype=torch.int64) % 13
+    y = bi.log_softmax(x)
+    lp = bi.token_logprob(x, tok.to(dev()))
+    st = bi.sample(x, seeds.to(dev()), steps.to(dev()), T).cpu().numpy()
+    rows = [0, 1, 2047, 4095]
+    xf = synth.to_f64(x[rows])
+    ref = oracle.log_softmax(xf)
+    err = np.abs(y[rows].cpu().double().numpy() - ref).max(axis=1) / np.abs(ref).max(axis=1)
+    assert err.max() <= TOL_FP32, err
+    np.testing.assert_allclose(lp[rows].cpu().double().numpy(), oracle.token_logprob(xf, tok.numpy()[rows]),
+                               rtol=TOL_FP32, atol=0)
+    sd, sp = _u64(seeds), _u64(steps)
+    for i, m in enumerate(rows):
+        sc = oracle.gumbel_scores(xf[i], T, oracle.sampling_uniforms(sd[m], sp[m], V))
+        srt = np.sort(sc)
+        bound = 2e-5 * (1.0 + abs(srt[-1]))
+        assert sc[st[m]] >= srt[-1] - bound, m
+        if srt[-1] - srt[-2] > bound:
+            assert st[m] == oracle.argmax_lowest(sc), m
+    assert bi.get_device_error() == 0
+
+
 def test_bad_token_gives_nan_and_device_index_error():
     x = synth.logits(2, 64, seed=103).to(dev())
     out = bi.token_logprob(x, torch.tensor([3, 64], dtype=torch.int32, device=dev()))

@@ -66,3 +66,17 @@ def test_rmsnorm_strided_rows():
     assert same_bits(y, bi.rmsnorm(x.contiguous(), w[:512].contiguous(), EPS))
     ref = oracle.rmsnorm(synth.to_f64(x.cpu()), synth.to_f64(w[:512].cpu()), EPS)
     assert max_rel(y, ref) <= TOL_BF16
+
+
+def test_rmsnorm_full_size_65536x4096_sampled():
+    # the benchmark's RMSNorm workload (512 MiB in, 512 MiB out): parity on sampled
+    # rows, and each sampled row alone gives the same bits
+    M, K = 65536, 4096
+    x = synth.normal_bf16_device((M, K), 15, dev())
+    w = synth.normal_bf16((K,), 16, std=0.1, mean=1.0).to(dev())
+    y = bi.rmsnorm(x, w, EPS)
+    rows = [0, 1, 4095, 32768, 65535]
+    ref = oracle.rmsnorm(synth.to_f64(x[rows]), synth.to_f64(w), EPS)
+    assert max_rel(y[rows], ref) <= TOL_BF16
+    for r in rows:
+        assert same_bits(bi.rmsnorm(x[r:r + 1].contiguous(), w, EPS)[0], y[r]), r
