@@ -115,6 +115,18 @@ def test_sample_matches_oracle_gumbel_max(T):
             assert tok[m] == top, m
 
 
+def test_sample_low_temperature_is_greedy():
+    # at T = 1e-3 logits 1 apart are 1000 apart after the division, far more than the
+    # Gumbel noise (within [-2.9, 16.7] for 23-bit uniforms): the draw is the argmax
+    M, V = 16, 64
+    g = synth.generator(104)
+    x = torch.stack([torch.randperm(V, generator=g) for _ in range(M)]).to(torch.bfloat16)
+    seeds = synth.request_seeds(M, 105)
+    steps = torch.arange(M, dtype=torch.int64)
+    tok = bi.sample(x.to(dev()), seeds.to(dev()), steps.to(dev()), 1e-3).cpu()
+    assert torch.equal(tok.long(), torch.argmax(x.float(), dim=1))
+
+
 def test_sample_frequencies_follow_softmax():
     # 4000 requests (seeds) sampling the same 8-entry row: the token frequencies
     # follow softmax(x / T)
