@@ -127,6 +127,24 @@ def test_sample_low_temperature_is_greedy():
     assert torch.equal(tok.long(), torch.argmax(x.float(), dim=1))
 
 
+def test_sample_nan_row_reports_and_leaves_other_rows_alone():
+    # a row of NaN logits has no maximum: token 0 and BI_ERR_DEVICE_INDEX; the
+    # other rows draw what they draw alone
+    M, V = 4, 1000
+    x = synth.logits(M, V, seed=106)
+    x[2] = float("nan")
+    seeds = synth.request_seeds(M, 107).to(dev())
+    steps = torch.arange(M, dtype=torch.int64, device=dev())
+    xd = x.to(dev())
+    tok = bi.sample(xd, seeds, steps, 0.9)
+    assert bi.get_device_error() == 8
+    assert int(tok[2]) == 0
+    for m in (0, 1, 3):
+        one = bi.sample(xd[m:m + 1].contiguous(), seeds[m:m + 1].contiguous(), steps[m:m + 1].contiguous(), 0.9)
+        assert int(one[0]) == int(tok[m]), m
+    assert bi.get_device_error() == 0
+
+
 def test_sample_frequencies_follow_softmax():
     # 4000 requests (seeds) sampling the same 8-entry row: the token frequencies
     # follow softmax(x / T)
