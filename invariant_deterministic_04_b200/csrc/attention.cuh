@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
   const int total = off[nrows] * Hkv;
   const int64_t kv_head_stride = (int64_t)PAGE * D;
   uint32_t seq = 0;  // pages this warp has consumed so far
+  uint32_t issued = 0, ph_bits = 0;  // lane 0: ring stages filled and their phase parities
 
   for (int item = blockIdx.x * WARPS + warp; item < total; item += gridDim.x * WARPS) {
     const int f = item / Hkv, g = item - (item / Hkv) * Hkv;
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
       const uint32_t bar = bars + 8 * st;
       const int pg = prow[j];
       const int nvalid = min(PAGE, t1 - t0 - j * PAGE);
+      note_fill(issued, ph_bits, (int)st, (sq / NST) & 1u);
       if (pg < 0 || pg >= num_pages) {
         record_error(BI_ERR_DEVICE_INDEX);
         mbar_arrive_expect_tx(bar, 0);
@@ -337,7 +339,11 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
         issue(j + NST, seq + NST);
       }
     }
-    if (!ok) return;  // a copy never landed: error recorded, leave the warp
+    if (!ok) {  // a copy never landed: error recorded; let this warp's other copies land, then leave
+      if (lane == 0) drain_copies(bars, 8, issued, ph_bits);
+      __syncwarp();
+      return;
+    }
 
     // Merge the token groups of the warp (fixed xor tree).
 #pragma unroll

@@ -164,6 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the producer's filled stages and their phase parities (Q, and the K/V ring)
+  uint32_t q_issued = 0, q_ph_bits = 0, kv_issued = 0, kv_ph_bits = 0;
   auto tS = [&](int x) { return tmem + (uint32_t)(x * KB); };
   auto tO = [&](int x) { return tmem + (uint32_t)(2 * KB + x * D); };
 
@@ -198,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x = 0; x < 2; ++x)
           for (int hh = 0; hh < C::HALVES; ++hh)
             tma_load_2d(q_s + x * C::Q_BYTES + hh * (ROWS * 128), &tmQ, (hA + x) * D + hh * 64, rb * ROWS, Q_FULL);
+        note_fill(q_issued, q_ph_bits, 0, qph ^ 1u);
         const int nb = nblocks_of(rb);
         bool ok = true;
         for (int j = 0; j < nb; ++j) {
@@ -221,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_2d(vs + hh * C::KV_HALF + p * (PAGE * 128), &tmV, hh * 64, row, KV_FULL(s));
             }
           }
+          note_fill(kv_issued, kv_ph_bits, s, ph);
           if (++s == C::STAGES) { s = 0; ph ^= 1u; }
         }
         if (!ok) { *abort_flag = 1; break; }
@@ -440,6 +444,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // after an abort, loads may still be landing in stages nobody waited for
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    drain_copies(Q_FULL, 8, q_issued, q_ph_bits);
+    drain_copies(KV_FULL(0), 16, kv_issued, kv_ph_bits);
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

@@ -126,6 +126,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   }
 }
 
+// After a wait gave up: a thread that issued bulk/TMA copies into this CTA's shared
+// memory gives each of its ring stages still expecting bytes a bounded time
+// (kDrainLimitNs) to complete, so the CTA does not exit while a copy may still be
+// writing its shared memory. Stage s has its barrier at bar0 + stride * s; bit s of
+// `issued` marks a stage this thread has filled, bit s of `ph_bits` the phase parity
+// of that last fill. A stage whose fill already completed returns at once.
+constexpr uint64_t kDrainLimitNs = 20000000ull;  // 20 ms per stage
+__device__ __forceinline__ void drain_copies(uint32_t bar0, uint32_t stride, uint32_t issued, uint32_t ph_bits) {
+#pragma unroll 1
+  for (int s = 0; s < 32; ++s)
+    if (issued & (1u << s)) (void)mbar_wait(bar0 + stride * (uint32_t)s, (ph_bits >> s) & 1u, kDrainLimitNs);
+}
+// Records that stage s was just filled for phase parity ph (bits for drain_copies).
+__device__ __forceinline__ void note_fill(uint32_t& issued, uint32_t& ph_bits, int s, uint32_t ph) {
+  issued |= 1u << s;
+  ph_bits = (ph_bits & ~(1u << s)) | ((ph & 1u) << s);
+}
+
 // ---------------------------------------------------------------------------
 // Bulk copies (TMA engine), global -> shared, completing on an mbarrier
 

@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  uint32_t issued = 0, ph_bits = 0;  // the producer's filled stages and their phase parities
 
   if (warp == 0) {
     if (lane == 0) {  // ---- TMA producer
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(FULL(s), STAGE_BYTES);
           tma_load_2d(a_s + s * A_BYTES, &tmA, kb * BK, m0, FULL(s));
           tma_load_2d(b_s + s * B_BYTES, &tmB, kb * BK, n0, FULL(s));
+          note_fill(issued, ph_bits, s, ph);
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;
@@ -216,6 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef TEMPTY
   tc_fence_before();
   __syncthreads();
+  // after an abort, loads may still be landing in stages nobody waited for
+  if (warp == 0 && lane == 0 && *abort_flag) drain_copies(bar0, 8, issued, ph_bits);
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
