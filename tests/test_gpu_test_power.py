@@ -359,3 +359,114 @@ def test_lmhead_control_passes(lm_cases):
 @pytest.mark.parametrize("bug", LM_BUGS)
 def test_lmhead_tests_see(bug, lm_cases):
     assert _lm_tests_fail(bug, lm_cases), f"{bug}: every LM-head GPU test would pass"
+
+
+# ---------------------------------------------------------------------------
+# Tensor-core prefill: the cases of test_prefill_tc_matches_oracle (one sequence
+# of 300 rows, sampled rows, three head configurations)
+
+TC_CASES = [(128, 32, 8), (64, 32, 8), (128, 16, 8)]
+TC_ROWS = [0, 1, 2, 15, 16, 127, 128, 129, 200, 255, 256, 299]
+
+
+def _tc_case(D, Hq, Hkv):
+    q, qs, qp, kv = synth.prefill_inputs([300], Hq, Hkv, D, seed=70 + D + Hq)
+    r = TC_ROWS
+    return (synth.to_f64(q)[r], qs.numpy()[r], qp.numpy()[r], synth.to_f64(kv.k_cache), synth.to_f64(kv.v_cache),
+            kv.page_table.numpy())
+
+
+def _tc_bug_keys_of_block_skipped(q, qs, qp, k, v, pt, block):
+    """A schedule that drops one whole 64-key block (e.g. an off-by-one block count):
+    keys of that block are removed from every row that would see them. A row whose
+    keys all lie in that block keeps them (the emulation understates the bug there)."""
+    out = np.zeros_like(q)
+    D = q.shape[2]
+    group = q.shape[1] // k.shape[1]
+    for i in range(q.shape[0]):
+        L = int(qp[i]) + 1
+        keep = [t for t in range(L) if t // 64 != block] or list(range(L))
+        for h in range(q.shape[1]):
+            keys = oracle.gather_kv(k, pt[int(qs[i])], h // group, L)[keep]
+            vals = oracle.gather_kv(v, pt[int(qs[i])], h // group, L)[keep]
+            out[i, h] = oracle.softmax_attend(q[i, h], keys, vals, 1.0 / math.sqrt(D))
+    return out
+
+
+TC_BUGS = {
+    "diagonal block's mask excludes the row's own key":
+        lambda q, qs, qp, k, v, pt: oracle.attention_rows(q, k, v, pt, qs, qp, None),
+    "diagonal block's mask lets in the next key":
+        lambda q, qs, qp, k, v, pt: oracle.attention_rows(q, k, v, pt, qs, qp + 2, None),
+    "first 64-key block skipped": lambda *a: _tc_bug_keys_of_block_skipped(*a, block=0),
+    "second 64-key block skipped": lambda *a: _tc_bug_keys_of_block_skipped(*a, block=1),
+    "tile B computed with tile A's query head":
+        lambda q, qs, qp, k, v, pt: oracle.attention_prefill(np.repeat(q[:, 0::2], 2, axis=1), qs, qp, k, v, pt),
+}
+
+
+@pytest.mark.parametrize("bug", list(TC_BUGS))
+def test_prefill_tc_parity_sees(bug):
+    caught = []
+    for case in TC_CASES:
+        q, qs, qp, k, v, pt = _tc_case(*case)
+        ref = oracle.attention_prefill(q, qs, qp, k, v, pt)
+        with np.errstate(all="ignore"):
+            buggy = TC_BUGS[bug](q, qs, qp, k, v, np.where(pt < 0, pt.max(), pt))
+        caught.append(_fails_parity(buggy, ref))
+    assert any(caught), f"{bug}: inside the tolerance in every case"
+
+
+# ---------------------------------------------------------------------------
+# Decoder glue: the cases of test_gpu_glue.py (RoPE at three head shapes; SwiGLU)
+
+ROPE_CASES = [(32, 64), (8, 64), (32, 128)]
+
+
+def _rope_case(H, D):
+    import torch
+    x = synth.to_f64(synth.normal_bf16((37, H, D), 2))
+    pos = torch.randint(0, 384, (37,), generator=synth.generator(3), dtype=torch.int32).numpy()
+    return x, pos
+
+
+def _rope_interleaved(x, pos):
+    T, H, D = x.shape
+    inv = 10000.0 ** (-2.0 * np.arange(D // 2) / D)
+    ang = pos[:, None].astype(np.float64) * inv[None, :]
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    a, b = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2], out[..., 1::2] = a * c - b * s, b * c + a * s
+    return out
+
+
+ROPE_BUGS = {
+    "position off by one": lambda x, pos: oracle.rope(x, pos + 1),
+    "rotation the other way": lambda x, pos: oracle.rope(x, -pos),
+    "interleaved pairs instead of halves": _rope_interleaved,
+    "frequency exponent i/D instead of 2i/D": lambda x, pos: oracle.rope(x, pos, theta=100.0),
+}
+
+
+@pytest.mark.parametrize("bug", list(ROPE_BUGS))
+def test_rope_parity_sees(bug):
+    caught = []
+    for H, D in ROPE_CASES:
+        x, pos = _rope_case(H, D)
+        caught.append(_fails_parity(ROPE_BUGS[bug](x, pos), oracle.rope(x, pos)))
+    assert any(caught), f"{bug}: inside the tolerance in every case"
+
+
+SWIGLU_BUGS = {
+    "gate and up halves swapped": lambda gu: oracle.swiglu(np.concatenate([gu[:, gu.shape[1] // 2:],
+                                                                            gu[:, : gu.shape[1] // 2]], axis=1)),
+    "sigmoid instead of silu": lambda gu: (1 / (1 + np.exp(-gu[:, : gu.shape[1] // 2]))) * gu[:, gu.shape[1] // 2:],
+    "gate times up without the activation": lambda gu: gu[:, : gu.shape[1] // 2] * gu[:, gu.shape[1] // 2:],
+}
+
+
+@pytest.mark.parametrize("bug", list(SWIGLU_BUGS))
+def test_swiglu_parity_sees(bug):
+    gu = synth.to_f64(synth.normal_bf16((33, 2 * 8192), 5))
+    assert _fails_parity(SWIGLU_BUGS[bug](gu), oracle.swiglu(gu)), f"{bug}: inside the tolerance"
