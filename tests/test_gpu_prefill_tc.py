@@ -19,7 +19,7 @@ def _dev(kv):
                          kv.seq_lens.to(dev()), kv.max_pages)
 
 
-@pytest.mark.parametrize("D,Hq,Hkv", [(128, 32, 8), (64, 32, 8), (128, 16, 8)])
+@pytest.mark.parametrize("D,Hq,Hkv", [(128, 32, 8), (64, 32, 8), (128, 16, 8), (128, 32, 4)])  # groups 4, 4, 2, 8
 def test_prefill_tc_matches_oracle(D, Hq, Hkv):
     S = 300
     q, qs, qp, kv = synth.prefill_inputs([S], Hq, Hkv, D, seed=70 + D + Hq)
