@@ -40,6 +40,7 @@ def _check_against_oracle(h, w, tau, tokens, rec, logits):
 
 
 @pytest.mark.parametrize("M,V,K", [(9, 1000, 256), (1, 32000, 2048), (64, 32000, 2048), (40, 4096, 512),
+                                   (5, 1000, 4096),   # the largest K of the W-streaming recompute
                                    (6, 2000, 4160)])  # K > 4096: the 64-row tiled recompute
 def test_lmhead_matches_oracle(M, V, K):
     h, w = synth.lmhead_inputs(M, V, K, seed=M + V)

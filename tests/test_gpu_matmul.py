@@ -18,7 +18,8 @@ M_SWEEP = [1, 2, 3, 4, 7, 8, 13, 16, 32, 33, 64, 127, 128, 255, 256, 257, 512, 1
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 520, 512), (1, 256, 64), (128, 256, 128), (129, 264, 192),
-                                   (32, 1024, 512), (5, 8, 64), (257, 4096, 1024)])
+                                   (32, 1024, 512), (5, 8, 64), (257, 4096, 1024),
+                                   (130, 520, 16384)])  # a long K: 256 blocks accumulated in TMEM
 def test_matmul_matches_oracle(M, N, K):
     a, w = synth.matmul_inputs(M, N, K, seed=M * 7 + N + K)
     c = bi.matmul(a.to(dev()), w.to(dev()))
