@@ -87,6 +87,28 @@ def test_lmhead_thresholds_force_or_forbid_recompute():
     assert (tok.cpu() == torch.argmax(lg.cpu(), dim=1).to(torch.int32)).all()
 
 
+def _fp32_fma_chain(h, w):
+    """fp32 logits computed as the header specifies: one FMA chain per logit in ascending
+    k, acc = fma(h[k], w[k], acc) from 0. A product of two bf16 values is exact in fp64,
+    so float64(acc) + h*w is the exact sum here and one rounding to fp32 is the fused
+    result."""
+    hf, wf = synth.to_f64(h), synth.to_f64(w)
+    acc = np.zeros((hf.shape[0], wf.shape[0]), dtype=np.float32)
+    for k in range(hf.shape[1]):
+        acc = (acc.astype(np.float64) + np.outer(hf[:, k], wf[:, k])).astype(np.float32)
+    return acc
+
+
+def test_lmhead_recompute_is_the_documented_fp32_chain_bit_for_bit():
+    # threshold inf sends every row through the recompute: 3 rows take the W-streaming
+    # kernel, 30 rows the tiled one; both must give exactly the ascending-k fp32 FMA chain
+    for M, V, K in ((3, 1000, 256), (30, 520, 128)):
+        h, w = synth.lmhead_inputs(M, V, K, seed=400 + M)
+        tok, rec, lg = bi.lmhead_argmax(h.to(dev()), w.to(dev()), float("inf"), want_logits=True)
+        assert int(rec.sum()) == M
+        np.testing.assert_array_equal(lg.cpu().numpy(), _fp32_fma_chain(h, w))
+
+
 def test_lmhead_batch_invariant():
     M, V, K = 64, 32000, 2048
     h, w = synth.lmhead_inputs(M, V, K, seed=72)
