@@ -65,6 +65,37 @@ def test_row_mean_matches_oracle(K):
     assert y[3].item() == -1.5
 
 
+def _row_mean_model(x):
+    """bi_row_mean's documented order in fp32 (include/bi.h): thread t of 256 adds the
+    elements of its 8-element vectors t, t+256, ... in order; inside each warp an xor
+    butterfly (offsets 16, 8, 4, 2, 1) whose lane-0 value is kept; the 8 warp values
+    added left to right; one division by K. Every step is an IEEE fp32 operation, so
+    numpy float32 reproduces it exactly."""
+    xf = synth.to_f64(x).astype(np.float32)  # bf16 -> fp32 is exact
+    M, K = xf.shape
+    nvec = K // 8
+    s = np.zeros((M, 256), dtype=np.float32)
+    for t in range(256):
+        for idx in range(t, nvec, 256):
+            for k in range(8):
+                s[:, t] = s[:, t] + xf[:, idx * 8 + k]
+    w = s.reshape(M, 8, 32)
+    lanes = np.arange(32)
+    for off in (16, 8, 4, 2, 1):
+        w = w + w[:, :, lanes ^ off]
+    tot = w[:, 0, 0]
+    for i in range(1, 8):
+        tot = tot + w[:, i, 0]
+    return tot / np.float32(K)
+
+
+@pytest.mark.parametrize("K", [8, 2056, 4096, 40000])
+def test_row_mean_is_the_documented_fp32_order_bit_for_bit(K):
+    x = synth.normal_bf16((5, K), 150 + K % 97, mean=0.5)
+    y = bi.row_mean(x.to(dev())).cpu().numpy()
+    np.testing.assert_array_equal(y, _row_mean_model(x))
+
+
 @pytest.mark.parametrize("op", ["log_softmax", "mean", "sample"])
 def test_rows_are_batch_invariant_and_run_to_run(op):
     M, N = 301, 32000
