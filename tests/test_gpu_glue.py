@@ -46,6 +46,33 @@ def test_rope_matches_oracle_and_is_row_invariant(H, D):
     assert same_bits(view, expect)
 
 
+def _rope_model(x, pos, table):
+    """bi_rope's documented fp32 arithmetic (include/bi.h): with (c, s) from the fp32
+    table, y1 = fma(a, c, -(b s)) and y2 = fma(b, c, a s), each rounded to bf16 (nearest
+    even). b s is one fp32 product; a c is exact in fp64 (8 x 24 significant bits), so
+    one rounding of a c - (b s) to fp32 is the fused result."""
+    xf = synth.to_f64(x)
+    half = x.shape[2] // 2
+    cs = table.cpu().double().numpy()[np.asarray(pos, dtype=np.int64)]  # [T, D/2, 2]
+    c, s = cs[..., 0][:, None, :], cs[..., 1][:, None, :]
+    a, b = xf[..., :half], xf[..., half:]
+    bs = (b * s).astype(np.float32).astype(np.float64)
+    as_ = (a * s).astype(np.float32).astype(np.float64)
+    y = np.concatenate([(a * c - bs).astype(np.float32), (b * c + as_).astype(np.float32)], axis=-1)
+    return torch.from_numpy(y).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("H,D", [(32, 64), (32, 128)])
+def test_rope_is_the_documented_fp32_arithmetic_bit_for_bit(H, D):
+    T = 37
+    x = synth.normal_bf16((T, H, D), 9)
+    pos = torch.randint(0, 384, (T,), generator=synth.generator(10), dtype=torch.int32)
+    table = rope_cos_sin(384, D, 10000.0, dev())
+    xd = x.to(dev()).clone()
+    bi.rope(xd, pos.to(dev()), table)
+    assert same_bits(xd.cpu(), _rope_model(x, pos.numpy(), table))
+
+
 def test_swiglu_and_add_match_oracle():
     gu = synth.normal_bf16((33, 2 * 8192), 5)
     out = bi.swiglu(gu.to(dev()))
@@ -54,6 +81,8 @@ def test_swiglu_and_add_match_oracle():
     a, b = synth.normal_bf16((9, 2048), 6), synth.normal_bf16((9, 2048), 7)
     s = bi.add(a.to(dev()), b.to(dev()))
     assert max_rel(s, synth.to_f64(a) + synth.to_f64(b)) <= TOL_BF16
+    # the documented arithmetic exactly: one fp32 add, rounded to bf16 (nearest even)
+    assert same_bits(s.cpu(), (a.float() + b.float()).to(torch.bfloat16))
     ad = a.to(dev())
     bi.add(ad, b.to(dev()), out=ad)
     assert same_bits(ad, s)
