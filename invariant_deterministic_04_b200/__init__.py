@@ -107,7 +107,10 @@ def _on(device, stream):
 
     Under it, temporaries (workspace, outputs) are allocated on the stream the
     kernels run on, so the caching allocator cannot hand their memory to other
-    work before those kernels are done with it."""
+    work before those kernels are done with it. A stream of another device is
+    refused (its kernels would get this device's pointers)."""
+    if stream is not None and getattr(stream, "device", device) != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     with torch.cuda.device(device):
         if stream is None:
             yield

@@ -195,6 +195,15 @@ def test_tensors_on_two_devices_are_refused(fake):
     assert fake.calls == []
 
 
+def test_a_stream_of_another_device_is_refused(fake):
+    class _OtherStream:
+        device = torch.device("meta")
+
+    with pytest.raises(ValueError, match="stream is on"):
+        bi.matmul(_bf(5, 128), _bf(512, 128), stream=_OtherStream())
+    assert fake.calls == []
+
+
 def test_a_callers_stream_is_current_for_the_call(fake):
     s = object()
     bi.matmul(_bf(5, 128), _bf(512, 128), stream=s)
