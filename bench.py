@@ -656,6 +656,9 @@ def run_ours(args, rank, world, local):
             "algorithmic_bytes_per_launch": 2 * (wl.M * K_HIDDEN + NS[-1] * K_HIDDEN + wl.M * NS[-1]),
             "launch_ms": round(big_ms, 4), "all_matmul_launches_tflops": round(step_gemm_tflops, 1),
             "kernel_share": round(gemm_ms / sum(kernel_ms), 3)}
+    if roof["traffic"] is None:
+        roof["traffic_note"] = ("gemm.cuh differs from the file the committed ncu counters "
+                                "(profiles/gemm_bf16_kernel_traffic.txt) were taken with")
     rms_ms = kernel_ms[0] / args.steps
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
