@@ -73,7 +73,7 @@ int bi_version(void);
 #define BI_PAGE_TOKENS 16   /* tokens per KV page */
 #define BI_KV_SPLIT 256     /* tokens per attention split (fixed size, not a fixed count) */
 #define BI_GEMM_BM 128      /* matmul tile rows (tcgen05 M) */
-#define BI_GEMM_BN 256      /* matmul tile columns (tcgen05 N) */
+#define BI_GEMM_BN_MAX 256  /* widest matmul tile (tcgen05 N); see bi_matmul_tile_n */
 #define BI_GEMM_BK 64       /* matmul K block; K is summed block by block in ascending order */
 
 /*
@@ -94,12 +94,28 @@ bi_status bi_rmsnorm(const bi_bf16* x, int64_t ldx, const bi_bf16* w, bi_bf16* y
  *   C[m, n] = bf16_rne( sum_k A[m, k] * W[n, k] ),  fp32 accumulation in TMEM
  * A: [M, K] bf16 row-major (K contiguous), stride lda. W: [N, K] bf16 row-major
  * (the nn.Linear weight layout), stride ldw. C: [M, N] bf16, stride ldc; must not
- * overlap A or W. Tile 128 x 256, K summed in 64-wide blocks in ascending order by
- * tcgen05.mma; the same for every M. M == 0 or N == 0 is a no-op.
- * Requires K % 64 == 0, K >= 64, N % 8 == 0.
+ * overlap A or W. Each C[m, n] is one chain of tcgen05.mma instructions (128 rows x
+ * tile-width columns x 16 k, bf16 operands, fp32 accumulator in tensor memory)
+ * over k = 0, 16, 32, ... in ascending order, then one bf16 rounding; no split-K.
+ * That chain is the same for every M and every position of the row or column
+ * inside its tile. The tile width (bi_matmul_tile_n) only decides how the columns
+ * are dealt out to CTAs, and it does not enter an element's arithmetic: the GPU
+ * tests check that every row of every M in 1..2048 equals the same row of the
+ * 2048-row product, bit for bit, across the widths the sweep uses.
+ * M == 0 or N == 0 is a no-op. Requires K % 64 == 0, K >= 64, N % 8 == 0.
  */
 bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw, bi_bf16* C,
                     int64_t ldc, int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * Tile width (32, 64, 128 or 256 columns) that bi_matmul uses for an M x N
+ * product on the current device; -1 if the device cannot be queried or M, N < 0.
+ * Narrow tiles spread a small-M product over more SMs (each streams a thin slice
+ * of W); wide tiles reuse each block of A for more columns at large M. The choice
+ * follows the tile counts and the SM count; it changes which CTA computes a
+ * column, never how. Host only, launches nothing.
+ */
+int bi_matmul_tile_n(int64_t M, int64_t N);
 
 /*
  * Workspace bytes for bi_attention_decode (rows = B) or bi_attention_prefill

@@ -6,7 +6,7 @@ memory and the current stream. There is no CPU or library fallback: if
 libbi.so is missing or fails to load, every call raises ``BIError``.
 
 Operations (see include/bi.h for the exact contracts):
-  rmsnorm, matmul, attention_decode, attention_decode_static, attention_prefill,
+  rmsnorm, matmul, matmul_tile_n, attention_decode, attention_decode_static, attention_prefill,
   kv_append, lmhead_argmax, gather_rows, rope, swiglu, add, log_softmax,
   token_logprob, row_mean, sampling_uniforms, sample, get_device_error.
 """
@@ -43,6 +43,7 @@ _SIGNATURES = {
     "bi_version": ([], _I32),
     "bi_rmsnorm": ([_P, _I64, _P, _P, _I64, _I64, _I64, _F, _P], _I32),
     "bi_matmul": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _P], _I32),
+    "bi_matmul_tile_n": ([_I64, _I64], _I32),
     "bi_attention_workspace_size": ([_I64, _I32, _I32, _I32], _SZ),
     "bi_attention_decode": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ, _P], _I32),
     "bi_attention_decode_static": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P], _I32),
@@ -183,7 +184,8 @@ def rmsnorm(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, out: torch.Tens
 
 
 def matmul(a: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, stream=None):
-    """C = A W^T with A [M, K], W [N, K] (nn.Linear layout), bf16 out, fixed tile and K order."""
+    """C = A W^T with A [M, K], W [N, K] (nn.Linear layout), bf16 out; every element is one
+    ascending-k chain of tcgen05 MMAs, the same for every M."""
     _req(a, torch.bfloat16, "a", 2)
     _req(w, torch.bfloat16, "w", 2)
     if a.stride(1) != 1 or w.stride(1) != 1:
@@ -200,6 +202,15 @@ def matmul(a: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, st
         _check("bi_matmul", lib().bi_matmul(_ptr(a), a.stride(0), _ptr(w), w.stride(0), _ptr(c), c.stride(0), M, N,
                                            K, _stream()))
     return c
+
+
+def matmul_tile_n(M: int, N: int) -> int:
+    """Tile width bi_matmul uses for an M x N product on the current device (a
+    scheduling choice; it does not enter the arithmetic of an element)."""
+    w = int(lib().bi_matmul_tile_n(M, N))
+    if w < 0:
+        raise RuntimeError("bi_matmul_tile_n: device query failed")
+    return w
 
 
 def attention_workspace_size(rows: int, Hq: int, D: int, max_pages_per_seq: int) -> int:

@@ -6,21 +6,37 @@
 // split-K, no switch between tensor-core and non-tensor-core paths — and accept a
 // modest loss of speed.
 //
+// What fixes the bits of C[m, n]: the chain of tcgen05.mma.kind::f16 instructions
+// (128 rows x BN columns x 16 k, A and B from shared memory, fp32 accumulator in
+// tensor memory) that adds A[m, k0:k0+16] . W[n, k0:k0+16] for k0 = 0, 16, 32, ...
+// in ascending order, then one round to bf16 (nearest even). Nothing else enters:
+// no split-K, no second accumulator, no reduction across CTAs. The chain is the
+// same for every M, for every position of row m inside its 128-row tile and for
+// every position of column n inside its BN-wide tile; the GPU tests check both
+// (a row alone equals the row at every tile position; every row of the M = 1..2048
+// sweep equals the same row of the 2048-row product).
+//
+// The tile width BN (32, 64, 128 or 256 columns) only decides how the N columns
+// are dealt out to CTAs. A narrow tile gives many CTAs when M is small (each CTA
+// then streams a thin slice of W, so more SMs pull W from HBM at once); a wide tile
+// reads each A block from shared memory for more columns when M is large. The host
+// picks the width from the tile counts (pick_bn); the width is not part of an
+// element's arithmetic, so the choice cannot change a bit (tested over the sweep).
+//
 // Design (sm_100a):
-//   * one output tile = 128 rows x 256 columns, held as fp32 in tensor memory
-//     (TMEM, 256 columns per accumulator, two accumulators per CTA so the
-//     epilogue of one tile overlaps the main loop of the next);
-//   * K is consumed in 64-wide blocks in ascending order; each block is four
-//     tcgen05.mma.kind::f16 instructions of shape 128x256x16, again in ascending
-//     k. Every output element therefore sees the same sequence of tensor-core
-//     accumulations for every M and every position of its row in the tile;
-//   * A and W tiles are brought into shared memory by TMA (128-byte swizzle,
-//     K-major) through a 4-stage mbarrier ring; out-of-range rows of a ragged tile
-//     are zero-filled by TMA and masked in the epilogue, so they cannot touch other rows;
+//   * K is consumed in 64-wide blocks, each four 128xBNx16 MMAs in ascending k;
+//   * A and W tiles come into shared memory by TMA (128-byte swizzle, K-major)
+//     through an mbarrier ring of as many stages as ~200 KB holds (4 at BN = 256,
+//     up to 9 at BN = 32); a ragged tile's out-of-range rows and columns are
+//     zero-filled by TMA and masked in the epilogue, so they cannot touch other rows;
+//   * when M < 128 the A box holds only the first ceil8(M) rows: rows past it are
+//     never loaded, and what the MMAs compute for them lands in output rows >= M,
+//     which are never stored (row m of the product depends on row m of A only);
 //   * warp 0 issues TMA, warp 1 (one thread) issues the MMAs, warps 2-5 drain
-//     TMEM (tcgen05.ld), round to bf16 (nearest even) and store;
-//   * persistent grid of min(#tiles, #SMs) CTAs; tile t goes to CTA t mod grid.
-//     The grid only decides which CTA computes a tile, never how.
+//     TMEM (tcgen05.ld), round to bf16 (nearest even) and store; two TMEM
+//     accumulators let the epilogue of one tile overlap the main loop of the next;
+//   * persistent grid of min(#tiles, #SMs) CTAs; tile t goes to CTA t mod grid,
+//     m-tiles of one W slice on neighbouring CTAs so the slice is read from HBM once;
 //   * every mbarrier wait is bounded; on expiry the kernel records
 //     BI_ERR_DEVICE_TIMEOUT, all roles leave their loops, TMEM is freed.
 #pragma once
@@ -32,20 +48,26 @@
 namespace bi {
 namespace gemm {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KiB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int TMEM_COLS = 2 * BN;  // two fp32 accumulators
-constexpr int kThreads = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int BM = 128, BK = 64;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KiB: room for a full 128-row A block per stage
+constexpr int kThreads = 192;         // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kEpiThreads = 128;
-constexpr int BAR_BYTES = 8 * (2 * STAGES + 4) + 16;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+constexpr int kRingBudget = 198 * 1024;  // shared memory for the stage ring
 
-// Instruction descriptor for kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 =
-// 1), B bf16 (bits 10-12 = 1), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+template <int BN>
+struct Cfg {
+  static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "tcgen05 M=128 tile widths used here");
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = kRingBudget / STAGE_BYTES;  // 4 / 6 / 8 / 9
+  static constexpr int TMEM_COLS = 2 * BN;                   // two fp32 accumulators (power of 2 >= 32)
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4) + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  // Instruction descriptor for kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 =
+  // 1), B bf16 (bits 10-12 = 1), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                    ((uint32_t)(BM >> 4) << 24);
+};
 
 // Shared-memory matrix descriptor for a K-major operand written by TMA with the
 // 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart (stride byte
@@ -56,22 +78,26 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// a_bytes: bytes one A box brings (rows of the A box x 128).
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     uint16_t* __restrict__ C, int64_t ldc, int M, int N, int K) {
+                     uint16_t* __restrict__ C, int64_t ldc, int M, int N, int K, uint32_t a_bytes) {
+  using G = Cfg<BN>;
+  constexpr int STAGES = G::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t a_s = base;
   const uint32_t b_s = base + STAGES * A_BYTES;
-  const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+  const uint32_t bar0 = base + STAGES * G::STAGE_BYTES;
   // barriers: full[0..S), empty[0..S), tfull[0..2), tempty[0..2)
 #define FULL(s) (bar0 + 8u * (s))
 #define EMPTY(s) (bar0 + 8u * (STAGES + (s)))
 #define TFULL(a) (bar0 + 8u * (2 * STAGES + (a)))
 #define TEMPTY(a) (bar0 + 8u * (2 * STAGES + 2 + (a)))
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 4));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * G::STAGE_BYTES + 8 * (2 * STAGES + 4));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -95,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_alloc(smem_u32(tmem_slot), G::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -108,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {  // ---- TMA producer
       int s = 0;
       uint32_t ph = 0;
+      const uint32_t stage_tx = a_bytes + (uint32_t)G::B_BYTES;
       for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
         const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -115,9 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             *abort_flag = 1;
             break;
           }
-          mbar_arrive_expect_tx(FULL(s), STAGE_BYTES);
+          mbar_arrive_expect_tx(FULL(s), stage_tx);
           tma_load_2d(a_s + s * A_BYTES, &tmA, kb * BK, m0, FULL(s));
-          tma_load_2d(b_s + s * B_BYTES, &tmB, kb * BK, n0, FULL(s));
+          tma_load_2d(b_s + s * G::B_BYTES, &tmB, kb * BK, n0, FULL(s));
           note_fill(issued, ph_bits, s, ph);
           if (++s == STAGES) {
             s = 0;
@@ -147,8 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = sw128_desc(a_s + s * A_BYTES + kk * 32);
-            const uint64_t bd = sw128_desc(b_s + s * B_BYTES + kk * 32);
-            tc_mma_f16(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t bd = sw128_desc(b_s + s * G::B_BYTES + kk * 32);
+            tc_mma_f16(d, ad, bd, G::IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit(EMPTY(s));  // frees the stage once these MMAs have read it
           if (++s == STAGES) {
@@ -223,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, G::TMEM_COLS);
   }
 }
 
@@ -262,41 +289,89 @@ inline bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t co
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-struct DeviceInfo {
-  int sms = 0;
-  bool smem_set = false;
-};
-
-inline DeviceInfo* device_info(int dev) {
-  static DeviceInfo infos[64];
+// Number of SMs of a device (cached; 0 if the query fails).
+inline int device_sms(int dev) {
+  static int sms[64];
   static std::mutex mu;
-  if (dev < 0 || dev >= 64) return nullptr;
+  if (dev < 0 || dev >= 64) return 0;
   std::lock_guard<std::mutex> lock(mu);
-  DeviceInfo* d = &infos[dev];
-  if (d->sms == 0) {
-    if (cudaDeviceGetAttribute(&d->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
-  }
-  if (!d->smem_set) {
-    if (cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-        cudaSuccess)
-      return nullptr;
-    d->smem_set = true;
-  }
-  return d;
+  if (sms[dev] == 0 && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms[dev] = 0;
+  return sms[dev];
 }
 
+// Raises the dynamic shared-memory limit of kernel `fn` once per device and keeps
+// the result, so that a failure is reported on every later call too.
+template <typename F>
+inline cudaError_t set_smem_once(F fn, int bytes, std::once_flag* once, cudaError_t* result, int dev) {
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] { result[dev] = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes); });
+  return result[dev];
+}
+
+template <int BN>
+inline cudaError_t prepare(int dev) {
+  static std::once_flag once[64];
+  static cudaError_t result[64];
+  return set_smem_once(gemm_bf16_kernel<BN>, Cfg<BN>::SMEM_BYTES, once, result, dev);
+}
+
+// Rows of A one stage loads: a whole 128-row block, or only ceil8(M) rows when the
+// product has fewer than 128 rows.
+inline uint32_t a_box_rows(int64_t M) { return M >= BM ? (uint32_t)BM : (uint32_t)((M + 7) / 8 * 8); }
+
+// Tile width for an M x N product on `sms` SMs. Cost of one tile per 64-wide K
+// block, in shared-memory cycles (128 bytes per cycle): the A box written by TMA,
+// A read by the four MMAs, the W block written and read, i.e. rows + 128 + 2 BN.
+// Tiles run in waves of `sms`; the width with the fewest cycles in total wins, ties
+// to the wider tile (fewer re-reads of A from L2). A scheduling choice only.
+inline int pick_bn(int64_t M, int64_t N, int sms) {
+  if (sms <= 0) sms = 1;
+  const int64_t mt = (M + BM - 1) / BM;
+  const int64_t rows = a_box_rows(M);
+  int best = 256;
+  int64_t best_cost = INT64_MAX;
+  for (int bn : {256, 128, 64, 32}) {
+    const int64_t tiles = mt * ((N + bn - 1) / bn);
+    const int64_t waves = (tiles + sms - 1) / sms;
+    const int64_t cost = waves * (rows + 128 + 2 * bn);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+template <int BN>
+inline bi_status launch_bn(const uint16_t* A, int64_t lda, const uint16_t* W, int64_t ldw, uint16_t* C,
+                           int64_t ldc, int64_t M, int64_t N, int64_t K, int dev, int sms, cudaStream_t st) {
+  if (prepare<BN>(dev) != cudaSuccess) return BI_ERR_CUDA;
+  const uint32_t arows = a_box_rows(M);
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, lda, arows) || !make_map(&tb, W, N, K, ldw, BN)) return BI_ERR_CUDA;
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  gemm_bf16_kernel<BN><<<grid, kThreads, Cfg<BN>::SMEM_BYTES, st>>>(ta, tb, C, ldc, (int)M, (int)N, (int)K,
+                                                                     arows * (uint32_t)(BK * 2));
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
+// bn: tile width (0 = pick_bn's choice for this device).
 inline bi_status launch(const uint16_t* A, int64_t lda, const uint16_t* W, int64_t ldw, uint16_t* C,
-                        int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st) {
+                        int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st, int bn = 0) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
-  DeviceInfo* info = device_info(dev);
-  if (!info) return BI_ERR_CUDA;
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K, lda, BM) || !make_map(&tb, W, N, K, ldw, BN)) return BI_ERR_CUDA;
-  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  const int grid = (int)(tiles < info->sms ? tiles : info->sms);
-  gemm_bf16_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(ta, tb, C, ldc, (int)M, (int)N, (int)K);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  const int sms = device_sms(dev);
+  if (sms <= 0) return BI_ERR_CUDA;
+  if (bn == 0) bn = pick_bn(M, N, sms);
+  switch (bn) {
+    case 32: return launch_bn<32>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
+    case 64: return launch_bn<64>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
+    case 128: return launch_bn<128>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
+    case 256: return launch_bn<256>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
+    default: return BI_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace gemm

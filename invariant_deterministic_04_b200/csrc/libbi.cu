@@ -68,24 +68,30 @@ cudaError_t launch_split(const uint16_t* q, int64_t ldq, int Hq, int Hkv, const 
                          const uint16_t* vc, int64_t num_pages, const int32_t* pt, bi::attn::Rows R, int nrows,
                          const AttnWs& ws, float c, cudaStream_t st) {
   constexpr int smem = bi::attn::split_smem_bytes<D, G>();
-  static std::once_flag once[64];
+  constexpr int threads = bi::attn::SplitCfg<D, G>::WARPS * 32;
   int dev = 0;
-  cudaGetDevice(&dev);
-  cudaError_t attr = cudaSuccess;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  // the shared-memory limit and the occupancy query run once per device; their
+  // result is kept, so a failure is returned on every later call as well
+  static std::once_flag once[64];
+  static cudaError_t result[64];
   static int per_sm[64];
-  std::call_once(once[dev & 63], [&] {
-    attr = cudaFuncSetAttribute(bi::attn::attn_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                smem);
-    if (attr == cudaSuccess)
-      attr = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[dev & 63], bi::attn::attn_split_kernel<D, G>,
-                                                           bi::attn::SplitCfg<D, G>::WARPS * 32, smem);
+  std::call_once(once[dev], [&] {
+    cudaError_t e = cudaFuncSetAttribute(bi::attn::attn_split_kernel<D, G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[dev], bi::attn::attn_split_kernel<D, G>, threads,
+                                                        smem);
+    if (e == cudaSuccess && per_sm[dev] <= 0) e = cudaErrorInvalidConfiguration;
+    result[dev] = e;
   });
-  if (attr != cudaSuccess) return attr;
+  if (result[dev] != cudaSuccess) return result[dev];
   // persistent grid: as many CTAs as can be resident (shared memory or registers
   // limit it); the grid only decides which warp takes which (row, head, split)
-  const int grid = device_sms() * (per_sm[dev & 63] > 0 ? per_sm[dev & 63] : 1);
-  bi::attn::attn_split_kernel<D, G><<<grid, bi::attn::SplitCfg<D, G>::WARPS * 32, smem, st>>>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt,
-                                                                                R, nrows, ws.off, ws.po, ws.pml, c);
+  const int grid = device_sms() * per_sm[dev];
+  bi::attn::attn_split_kernel<D, G><<<grid, threads, smem, st>>>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows,
+                                                                 ws.off, ws.po, ws.pml, c);
   return cudaGetLastError();
 }
 
@@ -101,9 +107,10 @@ cudaError_t launch_split_g(int G, const uint16_t* q, int64_t ldq, int Hq, int Hk
   }
 }
 
-bi_status attention_common(const uint16_t* q, int64_t ldq, const uint16_t* kc, const uint16_t* vc, int64_t num_pages,
-                           const int32_t* pt, int max_pages, bi::attn::Rows R, int nrows, uint16_t* out,
-                           int Hq, int Hkv, int D, float scale, void* ws, size_t ws_bytes, cudaStream_t st) {
+// Host checks of an attention request that need no workspace: head counts, head
+// size, scale, strides, the 32-bit range of the work list, pointer alignment.
+bi_status attention_check(const uint16_t* q, int64_t ldq, const uint16_t* kc, const uint16_t* vc, int64_t num_pages,
+                          int max_pages, int nrows, const uint16_t* out, int Hq, int Hkv, int D, float scale) {
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || num_pages <= 0 || max_pages <= 0) return BI_ERR_SHAPE;
   const int G = Hq / Hkv;
   if ((D != 64 && D != 128) || (G != 1 && G != 2 && G != 4 && G != 8)) return BI_ERR_UNSUPPORTED;
@@ -112,7 +119,16 @@ bi_status attention_common(const uint16_t* q, int64_t ldq, const uint16_t* kc, c
   // index arithmetic of the work list is 32-bit
   if ((int64_t)nrows * max_splits(max_pages) * Hkv >= INT_MAX || (int64_t)nrows * Hq >= INT_MAX / 8)
     return BI_ERR_SHAPE;
-  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(out) || !aligned16(ws)) return BI_ERR_ALIGN;
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(out)) return BI_ERR_ALIGN;
+  return BI_OK;
+}
+
+bi_status attention_common(const uint16_t* q, int64_t ldq, const uint16_t* kc, const uint16_t* vc, int64_t num_pages,
+                           const int32_t* pt, int max_pages, bi::attn::Rows R, int nrows, uint16_t* out,
+                           int Hq, int Hkv, int D, float scale, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (bi_status e = attention_check(q, ldq, kc, vc, num_pages, max_pages, nrows, out, Hq, Hkv, D, scale)) return e;
+  if (!aligned16(ws)) return BI_ERR_ALIGN;
+  const int G = Hq / Hkv;
   AttnWs lay{};
   const size_t need = attn_ws_size(nrows, Hq, D, max_pages, &lay, ws);
   if (ws_bytes < need) return BI_ERR_WORKSPACE;
@@ -199,7 +215,7 @@ const char* bi_status_string(int status) {
   }
 }
 
-int bi_version(void) { return 3; }
+int bi_version(void) { return 4; }
 
 bi_status bi_rmsnorm(const bi_bf16* x, int64_t ldx, const bi_bf16* w, bi_bf16* y, int64_t ldy, int64_t M,
                      int64_t K, float eps, void* stream) {
@@ -228,6 +244,14 @@ bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw
   return bi::gemm::launch(A, lda, W, ldw, C, ldc, M, N, K, as_stream(stream));
 }
 
+int bi_matmul_tile_n(int64_t M, int64_t N) {
+  if (M < 0 || N < 0) return -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  const int sms = bi::gemm::device_sms(dev);
+  return sms > 0 ? bi::gemm::pick_bn(M, N, sms) : -1;
+}
+
 size_t bi_attention_workspace_size(int64_t rows, int Hq, int D, int max_pages_per_seq) {
   return attn_ws_size(rows, Hq, D, max_pages_per_seq, nullptr, nullptr);
 }
@@ -251,6 +275,11 @@ bi_status bi_attention_decode_static(const bi_bf16* q, const bi_bf16* k_cache, c
   if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out) return BI_ERR_NULL;
   if (B < 0) return BI_ERR_SHAPE;
   if (B == 0) return BI_OK;
+  // every check that needs no scratch runs before the size check and before the
+  // first use of the device (the symbol lookup)
+  if (bi_status e = attention_check(q, (int64_t)Hq * D, k_cache, v_cache, num_pages, max_pages_per_seq, B, out, Hq,
+                                    Hkv, D, scale))
+    return e;
   if (attn_ws_size(B, Hq, D, max_pages_per_seq, nullptr, nullptr) > BI_STATIC_SCRATCH_BYTES) return BI_ERR_WORKSPACE;
   void* scratch = nullptr;
   const bi_status s = decode_scratch_address(&scratch);
@@ -290,8 +319,8 @@ bi_status bi_attention_prefill_tc(const bi_bf16* q, int64_t ldq, int seq, int po
   if (T == 0) return BI_OK;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
-  bi::gemm::DeviceInfo* info = bi::gemm::device_info(dev);
-  if (!info) return BI_ERR_CUDA;
+  const int sms = bi::gemm::device_sms(dev);
+  if (sms <= 0) return BI_ERR_CUDA;
   CUtensorMap tq, tk, tv;
   const int64_t kv_rows = num_pages * Hkv * BI_PAGE_TOKENS;
   if (!bi::gemm::make_map(&tq, q, T, (int64_t)Hq * D, ldq, bi::attn_tc::ROWS) ||
@@ -300,27 +329,23 @@ bi_status bi_attention_prefill_tc(const bi_bf16* q, int64_t ldq, int seq, int po
     return BI_ERR_CUDA;
   // one work item = two query heads of one kv-head over one 128-row block
   const int work = ((T + bi::attn_tc::ROWS - 1) / bi::attn_tc::ROWS) * (Hq / 2);
-  const int grid = work < info->sms ? work : info->sms;
+  const int grid = work < sms ? work : sms;
   const int pages_avail = (pos0 + T + BI_PAGE_TOKENS - 1) / BI_PAGE_TOKENS;
   const int32_t* prow = page_table + (int64_t)seq * max_pages_per_seq;
   const float c = (float)((double)scale * 1.4426950408889634);
   cudaStream_t st = as_stream(stream);
   static std::once_flag once[2][64];
-  cudaError_t attr = cudaSuccess;
+  static cudaError_t attr[2][64];
   if (D == 128) {
-    std::call_once(once[0][dev & 63], [&] {
-      attr = cudaFuncSetAttribute(bi::attn_tc::prefill_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  bi::attn_tc::Cfg<128>::SMEM);
-    });
-    if (attr != cudaSuccess) return BI_ERR_CUDA;
+    if (bi::gemm::set_smem_once(bi::attn_tc::prefill_tc_kernel<128>, bi::attn_tc::Cfg<128>::SMEM, once[0], attr[0],
+                                dev) != cudaSuccess)
+      return BI_ERR_CUDA;
     bi::attn_tc::prefill_tc_kernel<128><<<grid, bi::attn_tc::kThreads, bi::attn_tc::Cfg<128>::SMEM, st>>>(
         tq, tk, tv, prow, num_pages, Hq, Hkv, pos0, T, pages_avail, out, c);
   } else {
-    std::call_once(once[1][dev & 63], [&] {
-      attr = cudaFuncSetAttribute(bi::attn_tc::prefill_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  bi::attn_tc::Cfg<64>::SMEM);
-    });
-    if (attr != cudaSuccess) return BI_ERR_CUDA;
+    if (bi::gemm::set_smem_once(bi::attn_tc::prefill_tc_kernel<64>, bi::attn_tc::Cfg<64>::SMEM, once[1], attr[1],
+                                dev) != cudaSuccess)
+      return BI_ERR_CUDA;
     bi::attn_tc::prefill_tc_kernel<64><<<grid, bi::attn_tc::kThreads, bi::attn_tc::Cfg<64>::SMEM, st>>>(
         tq, tk, tv, prow, num_pages, Hq, Hkv, pos0, T, pages_avail, out, c);
   }
@@ -374,14 +399,12 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
   int skip_upto = 0;
   if (K <= bi::lmhead::kStrMaxK) {
     static std::once_flag str_once[64];
-    cudaError_t attr = cudaSuccess;
+    static cudaError_t str_attr[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
-    std::call_once(str_once[dev & 63], [&] {
-      attr = cudaFuncSetAttribute(bi::lmhead::recompute_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK));
-    });
-    if (attr != cudaSuccess) return BI_ERR_CUDA;
+    if (bi::gemm::set_smem_once(bi::lmhead::recompute_stream_kernel, bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK),
+                                str_once, str_attr, dev) != cudaSuccess)
+      return BI_ERR_CUDA;
     const unsigned sgrid = (unsigned)((V + bi::lmhead::kStrWarps * 32 - 1) / (bi::lmhead::kStrWarps * 32));
     bi::lmhead::recompute_stream_kernel<<<sgrid, bi::lmhead::kStrThreads, bi::lmhead::stream_smem_bytes((int)K), st>>>(
         h, ldh, W, V, (int)K, (int)M, lay.list, out32);

@@ -45,7 +45,7 @@ def test_status_strings(L):
     assert L.bi_status_string(0) == b"BI_OK"
     assert L.bi_status_string(4) == b"BI_ERR_WORKSPACE"
     assert L.bi_status_string(99) == b"BI_ERR_UNKNOWN"
-    assert L.bi_version() == 3
+    assert L.bi_version() == 4
 
 
 def test_rmsnorm_validation(L):

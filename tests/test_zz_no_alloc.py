@@ -33,6 +33,22 @@ def test_static_decode_host_validation():
     need = L.bi_attention_workspace_size(256, 32, 128, 2048)
     assert need > bi.STATIC_SCRATCH_BYTES
     assert f(P, P, P, 100, P, 2048, P, P, 256, 32, 8, 128, 0.088, None) == 4        # BI_ERR_WORKSPACE
+    # shape errors are reported as such even when the size query would pass
+    assert f(P, P, P, 100, P, 64, P, P, 4, 0, 8, 128, 0.088, None) == 2              # Hq = 0: BI_ERR_SHAPE
+    assert f(P, P, P, 100, P, 64, P, P, 4, 32, 8, 96, 0.088, None) == 5              # D = 96: BI_ERR_UNSUPPORTED
+    # the smallest batch whose scratch no longer fits is refused; the one below it fits exactly
+    B = max_batch_in_scratch(L, 16)
+    assert L.bi_attention_workspace_size(B, 32, 128, 16) <= bi.STATIC_SCRATCH_BYTES
+    assert L.bi_attention_workspace_size(B + 1, 32, 128, 16) > bi.STATIC_SCRATCH_BYTES
+    assert f(P, P, P, 100, P, 16, P, P, B + 1, 32, 8, 128, 0.088, None) == 4
+
+
+def max_batch_in_scratch(L, max_pages):
+    """Largest batch whose decode scratch (Hq 32, D 128) fits the fixed array."""
+    B = 1
+    while L.bi_attention_workspace_size(B + 1, 32, 128, max_pages) <= bi.STATIC_SCRATCH_BYTES:
+        B += 1
+    return B
 
 
 @pytest.mark.gpu
@@ -54,4 +70,28 @@ def test_static_decode_matches_workspace_decode_on_two_calls_in_a_row():
     for got, ref in results:
         assert max_rel(got, synth.to_f64(ref.cpu())) <= TOL_BF16
         assert same_bits(got, ref)
+    assert bi.get_device_error() == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("max_pages,long_lens", [(16, []), (2048, [32768, 20000])])
+def test_static_decode_with_scratch_filled_to_its_end(max_pages, long_lens):
+    # The largest batch that fits: the split partials of the last rows lie at the
+    # end of the fixed array (with one page per sequence the scratch is filled to
+    # its last byte). Two call shapes: thousands of one-split rows, and a few rows
+    # with up to 128 splits next to short ones.
+    L = bi.lib()
+    B = max_batch_in_scratch(L, max_pages)
+    assert L.bi_attention_workspace_size(B, 32, 128, max_pages) > bi.STATIC_SCRATCH_BYTES - (2 << 20)
+    g = synth.generator(92 + max_pages)
+    short = torch.randint(1, 257, (B - len(long_lens),), generator=g).tolist()
+    lens = long_lens + short
+    q, kv = synth.decode_inputs(B, 32, 8, 128, max_len=max_pages * 16, seed=93, lens=lens)
+    assert kv.max_pages == max_pages
+    qd = q.to(dev())
+    kc, vc, ptd, sl = kv.k_cache.to(dev()), kv.v_cache.to(dev()), kv.page_table.to(dev()), kv.seq_lens.to(dev())
+    got = bi.attention_decode_static(qd, kc, vc, ptd, sl)
+    ref = bi.attention_decode(qd, kc, vc, ptd, sl)
+    torch.cuda.synchronize()
+    assert same_bits(got, ref)
     assert bi.get_device_error() == 0
