@@ -15,7 +15,11 @@ torch.matmul + F.rms_norm) on the same box, an end-to-end figure through the
 public API with host buffers, the clocks seen during the timed region, the fp64
 CPU oracle timed on a bounded sample, and (``--rows``, default on) one
 measurement of every other hot-path kernel: RMSNorm bandwidth, decode attention
-bandwidth, causal prefill throughput and the LM head.
+bandwidth, causal prefill throughput and the LM head; and (``--sweeps``, default
+on) the configuration sweeps: bi_matmul over M = 1..2048 at K = 4096 for N = 4096,
+6144 and 14336 (W warm and W cold), RMSNorm over the same M at hidden 4096, and
+decode attention over B = 1..256 with lengths ~ U[1, 32768], each entry with its
+fraction of the applicable peak.
 
 ``--impl reference`` times the fp64 CPU oracle on the same workload and metric
 (bounded samples per step) and prints the reference line.
@@ -501,60 +505,145 @@ def _row_reduce(bi, device, pk):
 
 
 # ---------------------------------------------------------------------------
-# the K=4096 sweep (one JSON line per (M, N)): bi_matmul vs cuBLAS, W warm and W cold
+# the configuration sweeps: bi_matmul over M (K=4096, three N, W warm and W cold),
+# RMSNorm over M at hidden 4096, decode attention over the batch size
 
 
 M_SWEEP = [1, 2, 3, 4, 7, 8, 13, 16, 32, 33, 64, 127, 128, 255, 256, 257, 512, 1023, 1024, 2047, 2048]
+B_SWEEP = [1, 2, 4, 8, 16, 32, 64, 128, 256]
 
 
-def run_sweep(bi, device, pk, iters=20):
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)  # > L2 (126 MB)
+class L2Flush:
+    """Evicts L2 (126 MB) by reading a 512 MiB buffer. A read leaves L2 full of clean
+    lines, so the next kernel pays for its own misses only; a flush by writing would
+    leave dirty lines whose write-back lands inside the next, timed kernel (measured:
+    up to 8 us of a 30 us launch)."""
+
+    def __init__(self, device):
+        self.buf = torch.ones(512 << 20, dtype=torch.uint8, device=device).view(torch.int64)
+        self.sink = torch.empty(1, dtype=torch.int64, device=device)
+
+    def __call__(self):
+        self.sink.copy_(self.buf.sum().view(1))
+
+
+def _launch_ms(fn, flush, iters, cold):
+    """Median device time of one launch of fn (CUDA events on the current stream);
+    when `cold`, an L2 flush precedes every launch. A spin of about 100 us on the
+    device precedes the start event, so that the host's work of issuing the call
+    (argument checks, tensor maps) happens while the device is busy and is not
+    counted in a kernel of a few microseconds."""
+    ts = []
+    for i in range(iters + 3):
+        if cold:
+            flush()
+        torch.cuda._sleep(200000)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(s.elapsed_time(e))
+    return statistics.median(ts)
+
+
+def sweep_matmul(bi, device, pk, flush, iters=7, ms_list=M_SWEEP):
+    """One entry per (M, N): TFLOP/s W warm (in L2) and W cold (L2 flushed), the
+    fraction of the bf16 burst peak (each launch is timed alone) and of the roofline
+    max(FLOPs / peak, bytes / HBM), and cuBLAS (torch.matmul) on the same operands."""
     A = synth.normal_bf16((2048, K_HIDDEN), 100).to(device)
-    wn = synth.normal_bf16((K_HIDDEN,), 110, std=0.1, mean=1.0).to(device)
-
-    def timed(fn, cold):
-        ts = []
-        for i in range(iters + 3):
-            if cold:
-                flush.zero_()
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s.record()
-            fn()
-            e.record()
-            torch.cuda.synchronize()
-            if i >= 3:
-                ts.append(s.elapsed_time(e))
-        return statistics.median(ts)
-
+    out = []
     for j, n in enumerate(NS):
         W = synth.normal_bf16((n, K_HIDDEN), 120 + j, std=0.02).to(device)
         C = torch.empty((2048, n), dtype=torch.bfloat16, device=device)
-        for m in M_SWEEP:
+        for m in ms_list:
             a, c = A[:m], C[:m]
             flops = 2.0 * m * n * K_HIDDEN
             byts = 2.0 * (m * K_HIDDEN + n * K_HIDDEN + m * n)
-            rec = {"sweep": "matmul", "M": m, "N": n, "K": K_HIDDEN}
-            for cold in (False, True):
-                ms = timed(lambda: bi.matmul(a, W, out=c), cold)
-                ref = timed(lambda: torch.matmul(a, W.t(), out=c), cold)
-                roof_ms = max(flops / pk["bf16_tflops"] / 1e9, byts / pk["hbm_gbs"] / 1e6)
-                key = "cold" if cold else "warm"
-                rec[key] = {"ms": round(ms, 5), "TFLOP/s": round(flops / ms / 1e9, 1),
-                            "frac_tensor_peak": round(flops / ms / 1e9 / pk["bf16_tflops"], 3),
-                            "frac_roofline": round(roof_ms / ms, 3), "cublas_ms": round(ref, 5),
-                            "slowdown_vs_cublas": round(ms / ref, 3)}
-            print(json.dumps(rec), flush=True)
-    for m in M_SWEEP:
-        x = A[:m]
-        y = torch.empty_like(x)
-        ms = timed(lambda: bi.rmsnorm(x, wn, EPS, out=y), True)
-        ref = timed(lambda: torch.nn.functional.rms_norm(x, (K_HIDDEN,), wn, EPS), True)
-        byts = 4.0 * m * K_HIDDEN + 2 * K_HIDDEN
-        print(json.dumps({"sweep": "rmsnorm", "M": m, "K": K_HIDDEN, "ms": round(ms, 5),
-                          "GB/s": round(byts / ms / 1e6, 1), "slowdown_vs_F.rms_norm": round(ms / ref, 3)}), flush=True)
+            roof_ms = max(flops / pk["bf16_tflops"] / 1e9, byts / pk["hbm_gbs"] / 1e6)
+            warm = _launch_ms(lambda: bi.matmul(a, W, out=c), flush, iters, False)
+            cold = _launch_ms(lambda: bi.matmul(a, W, out=c), flush, iters, True)
+            ref = _launch_ms(lambda: torch.matmul(a, W.t(), out=c), flush, iters, True)
+            out.append({"M": m, "N": n, "tile_n": bi.matmul_tile_n(m, n),
+                        "warm_tflops": round(flops / warm / 1e9, 1),
+                        "warm_frac_peak": round(flops / warm / 1e9 / pk["bf16_tflops"], 3),
+                        "cold_us": round(cold * 1e3, 2), "cold_tflops": round(flops / cold / 1e9, 1),
+                        "cold_frac_peak": round(flops / cold / 1e9 / pk["bf16_tflops"], 3),
+                        "cold_frac_roofline": round(roof_ms / cold, 3),
+                        "cold_frac_hbm": round(byts / cold / 1e6 / pk["hbm_gbs"], 3),
+                        "cublas_cold_us": round(ref * 1e3, 2), "slowdown_vs_cublas": round(cold / ref, 3)})
+        del W, C
+    return out
+
+
+def sweep_rmsnorm(bi, device, pk, flush, iters=7, ms_list=M_SWEEP):
+    """RMSNorm at hidden 4096 over M, L2 flushed before each launch: GB/s of x in + y
+    out + w, fraction of the HBM copy peak, and F.rms_norm on the same rows."""
+    x = synth.normal_bf16((2048, K_HIDDEN), 100).to(device)
+    wn = synth.normal_bf16((K_HIDDEN,), 110, std=0.1, mean=1.0).to(device)
+    y = torch.empty_like(x)
+    out = []
+    for m in ms_list:
+        xm, ym = x[:m], y[:m]
+        t = _launch_ms(lambda: bi.rmsnorm(xm, wn, EPS, out=ym), flush, iters, True)
+        ref = _launch_ms(lambda: torch.nn.functional.rms_norm(xm, (K_HIDDEN,), wn, EPS), flush, iters, True)
+        gbs = (4.0 * m * K_HIDDEN + 2 * K_HIDDEN) / t / 1e6
+        out.append({"M": m, "us": round(t * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3),
+                    "slowdown_vs_F.rms_norm": round(t / ref, 3)})
+    return out
+
+
+def sweep_decode(bi, device, pk, flush, iters=5, bs=B_SWEEP):
+    """Decode attention (32 q-heads / 8 kv-heads, D 128, 16-token pages) over the batch
+    size: the first B sequences of one store of 256 with lengths ~ U[1, 32768]
+    (17 GB of K/V). KV bytes read per launch / time, against the HBM copy peak;
+    L2 flushed before each launch."""
+    Bmax, Lmax = max(bs), 32768
+    lens = synth.decode_lengths(Bmax, Lmax, seed=50)
+    kv = synth.paged_kv_device(lens, 8, 128, seed=51, max_pages=Lmax // 16, device=device)
+    q = synth.normal_bf16((Bmax, 32, 128), 52).to(device)
+    o = torch.empty_like(q)
+    ws = torch.empty(bi.attention_workspace_size(Bmax, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
+    out = []
+    for B in bs:
+        qb, ob = q[:B], o[:B]
+        pt, sl = kv.page_table[:B], kv.seq_lens[:B]
+        t = _launch_ms(lambda: bi.attention_decode(qb, kv.k_cache, kv.v_cache, pt, sl, out=ob, workspace=ws),
+                       flush, iters, True)
+        kv_bytes = 4096.0 * int(lens[:B].sum())
+        gbs = kv_bytes / t / 1e6
+        out.append({"B": B, "kv_tokens": int(lens[:B].sum()), "us": round(t * 1e3, 2), "GB/s": round(gbs, 1),
+                    "frac_hbm": round(gbs / pk["hbm_gbs"], 3)})
+    del kv, ws
+    return out
+
+
+def run_sweeps(bi, device, pk):
+    flush = L2Flush(device)
+    res = {"matmul_k4096": sweep_matmul(bi, device, pk, flush),
+           "rmsnorm_k4096": sweep_rmsnorm(bi, device, pk, flush),
+           "decode_h32_8_d128_l32k": sweep_decode(bi, device, pk, flush)}
+    del flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_sweep(bi, device, pk):
+    """--sweep: the sweeps alone, one JSON line per entry."""
+    for name, entries in run_sweeps(bi, device, pk).items():
+        for e in entries:
+            print(json.dumps({"sweep": name, **e}), flush=True)
 
 
 # ---------------------------------------------------------------------------
+
+
+def ours_config(M, world):
+    """The workload description both arms print (the same dict, so the two lines compare)."""
+    return {"workload": WORKLOAD, "M": M, "K": K_HIDDEN, "N": list(NS), "step": "bi_rmsnorm + 3 x bi_matmul",
+            "parallelism": f"replicas x{world}",
+            "l2": "working set > L2 (201 MB of weights per step; two activation buffers rotate)"}
 
 
 def run_reference(args, rank, world):
@@ -576,7 +665,7 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": 2048, "K": K_HIDDEN, "N": list(NS), "rows_per_step": per},
+            "config": ours_config(2048, world),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -648,11 +737,17 @@ def run_ours(args, rank, world, local):
     achieved = big_flops / (big_ms / 1e3) / 1e12
     gemm_ms = sum(kernel_ms[1:])
     step_gemm_tflops = 2.0 * wl.M * K_HIDDEN * sum(NS) * args.steps / (gemm_ms / 1e3) / 1e12
+    # The denominator follows the length of the timed region: the burst peak (cuBLAS
+    # timed alone, clocks at their maximum) for a region under two seconds, the
+    # sustained one (seconds of back-to-back GEMMs under the power cap) otherwise.
+    sustained = ms_total > 2000.0
+    peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
     roof = {"bound": "tensor", "kernel": "gemm_bf16_kernel (tcgen05), M=2048 N=14336 K=4096 launch",
-            "achieved": round(achieved, 1), "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-            "frac": round(achieved / pk["bf16_tflops_sustained"], 3),
-            "peak_kind": f"bf16 sustained ({pk['source']}); the step runs back to back for the whole timed region",
-            "frac_of_burst": round(achieved / pk["bf16_tflops"], 3), "traffic": traffic_from_profile(),
+            "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 3),
+            "peak_kind": (f"bf16 {'sustained' if sustained else 'burst'} ({pk['source']}); timed region "
+                          f"{ms_total / 1e3:.3f} s"),
+            "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 3), "traffic": traffic_from_profile(),
             "algorithmic_bytes_per_launch": 2 * (wl.M * K_HIDDEN + NS[-1] * K_HIDDEN + wl.M * NS[-1]),
             "launch_ms": round(big_ms, 4), "all_matmul_launches_tflops": round(step_gemm_tflops, 1),
             "kernel_share": round(gemm_ms / sum(kernel_ms), 3)}
@@ -664,9 +759,7 @@ def run_ours(args, rank, world, local):
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "M": wl.M, "K": K_HIDDEN, "N": list(NS), "step": "bi_rmsnorm + 3 x bi_matmul",
-                   "parallelism": f"replicas x{world}",
-                   "l2": "working set > L2 (201 MB of weights per step; two activation buffers rotate)"},
+        "config": ours_config(wl.M, world),
         "roofline": roof,
         "rmsnorm_in_step": {"GB/s": round(wl.rms_bytes / rms_ms / 1e6, 1), "ms": round(rms_ms, 4),
                             "note": "16 MiB in + 16 MiB out per launch"},
@@ -679,10 +772,13 @@ def run_ours(args, rank, world, local):
     }
     if world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
-    if world == 1 and args.rows:
+    if world == 1 and (args.rows or args.sweeps):
         del wl
         torch.cuda.empty_cache()
+    if world == 1 and args.rows:
         line["rows"] = other_rows(bi, device, pk)
+    if world == 1 and args.sweeps:
+        line["sweeps"] = run_sweeps(bi, device, pk)
     print(json.dumps(line), flush=True)
 
 
@@ -696,7 +792,10 @@ def main():
     ap.add_argument("--rows", dest="rows", action="store_true", default=True)
     ap.add_argument("--no-rows", dest="rows", action="store_false")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--sweep", action="store_true", help="the K=4096 M sweep, one JSON line per shape")
+    ap.add_argument("--sweeps", dest="sweeps", action="store_true", default=True,
+                    help="add the matmul / RMSNorm / decode sweeps to the line (default on)")
+    ap.add_argument("--no-sweeps", dest="sweeps", action="store_false")
+    ap.add_argument("--sweep", action="store_true", help="only the sweeps, one JSON line per entry")
     ap.add_argument("--row", choices=["rmsnorm", "decode", "prefill", "lmhead", "reduce"], default=None,
                     help="measure only this hot-path kernel (for profiling) and print its line")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
