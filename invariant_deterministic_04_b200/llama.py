@@ -1,5 +1,6 @@
 """Random-init Llama-style decoder on the batch-invariant kernels, with a mixed-batch
-greedy scheduler (test harness for the 1000-repeat determinism check).
+greedy scheduler: the model of the 1000-repeat determinism check and of the
+config-5 benchmark row.
 
 Every operation of a step runs in libbi through the binding: row gather (embedding),
 RMSNorm, the tcgen05 matmul, RoPE, KV append into the paged store, causal attention

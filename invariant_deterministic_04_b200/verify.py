@@ -1,4 +1,4 @@
-"""Selective determinism by verify and rollback, on the config-5 random Llama (test harness).
+"""Selective determinism by verify and rollback, on the config-5 random Llama.
 
 Source: French "température zéro" blog, section "Vous n'avez pas à le payer partout":
 LLM-42 keeps a fast nondeterministic path and enforces determinism with a light
@@ -31,7 +31,7 @@ import time
 import numpy as np
 import torch
 
-from llama_bi import PAGE, BaselineLlama, FastBiLlama
+from .llama import PAGE, BaselineLlama, FastBiLlama
 
 
 class FastPathLlama(BaselineLlama):

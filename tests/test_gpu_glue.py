@@ -8,7 +8,7 @@ import invariant_deterministic_04_b200 as bi
 import oracle
 import synth
 from gpu_util import TOL_BF16, dev, max_rel, same_bits
-from llama_bi import rope_cos_sin
+from invariant_deterministic_04_b200.llama import rope_cos_sin
 
 pytestmark = pytest.mark.gpu
 

@@ -20,7 +20,7 @@ import torch
 import oracle
 import synth
 from gpu_util import TOL_BF16, dev, max_rel
-from llama_bi import BaselineLlama, BiLlama, FastBiLlama, run_repeats
+from invariant_deterministic_04_b200.llama import BaselineLlama, BiLlama, FastBiLlama, run_repeats
 
 pytestmark = pytest.mark.gpu
 

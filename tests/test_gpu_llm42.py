@@ -16,8 +16,8 @@ import pytest
 
 import synth
 from gpu_util import dev
-from llama_bi import FastBiLlama, run_schedule
-from llm42 import FastPathLlama, generate, timed_generate
+from invariant_deterministic_04_b200.llama import FastBiLlama, run_schedule
+from invariant_deterministic_04_b200.verify import FastPathLlama, generate, timed_generate
 
 pytestmark = pytest.mark.gpu
 
