@@ -225,9 +225,14 @@ bi_status bi_rmsnorm(const bi_bf16* x, int64_t ldx, const bi_bf16* w, bi_bf16* y
   if (K > 16384) return BI_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(w) || !aligned16(y) || ldx % 8 || ldy % 8) return BI_ERR_ALIGN;
   if (M == 0) return BI_OK;
-  if (x != y && ranges_overlap(x, span_bytes(M, K, ldx, 2), y, span_bytes(M, K, ldy, 2))) return BI_ERR_SHAPE;
-  return bi::rms::launch(x, ldx, w, y, ldy, M, (int)K, eps, as_stream(stream)) == cudaSuccess ? BI_OK
-                                                                                              : BI_ERR_CUDA;
+  // in place only row for row: an alias with another row stride would let one row's
+  // output overwrite another row's input before it is read
+  if (x == y ? ldx != ldy : ranges_overlap(x, span_bytes(M, K, ldx, 2), y, span_bytes(M, K, ldy, 2)))
+    return BI_ERR_SHAPE;
+  const int sms = device_sms();
+  if (sms <= 0) return BI_ERR_CUDA;
+  return bi::rms::launch(x, ldx, w, y, ldy, M, (int)K, eps, sms, as_stream(stream)) == cudaSuccess ? BI_OK
+                                                                                                   : BI_ERR_CUDA;
 }
 
 bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw, bi_bf16* C, int64_t ldc,

@@ -61,6 +61,8 @@ def test_rmsnorm_validation(L):
     assert f(P, 512, P, P, 512, 0, 512, 1e-6, None) == OK           # empty: no-op
     # partially overlapping input and output rows are rejected (exact aliasing is allowed)
     assert f(P, 512, P + 0x100000, P + 16, 512, 4, 512, 1e-6, None) == SHAPE
+    # in place needs the same row stride on both sides
+    assert f(P, 512, P + 0x100000, P, 1024, 4, 512, 1e-6, None) == SHAPE
 
 
 def test_matmul_validation(L):

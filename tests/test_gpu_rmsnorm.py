@@ -80,3 +80,21 @@ def test_rmsnorm_full_size_65536x4096_sampled():
     assert max_rel(y[rows], ref) <= TOL_BF16
     for r in rows:
         assert same_bits(bi.rmsnorm(x[r:r + 1].contiguous(), w, EPS)[0], y[r]), r
+
+
+# Batches larger than the persistent grid (8, 4 or 2 CTAs per SM by register
+# variant), so every CTA takes several rows and prefetches the next one while it
+# writes the current one: every row equals the same row computed alone (grid of one
+# CTA) and in a reversed batch, and sampled rows match the oracle.
+@pytest.mark.parametrize("M,K", [(2500, 512), (2500, 2048), (2600, 4096), (1300, 8192), (700, 16384), (2501, 1032)])
+def test_rmsnorm_rows_beyond_the_persistent_grid(M, K):
+    x, w = synth.rmsnorm_inputs(M, K, seed=17 + K)
+    x, w = x.to(dev()), w.to(dev())
+    full = bi.rmsnorm(x, w, EPS)
+    rev = torch.arange(M - 1, -1, -1, device=dev())
+    assert same_bits(bi.rmsnorm(x[rev].contiguous(), w, EPS), full[rev])
+    for r in (0, 1, M // 3, M - 2, M - 1):
+        assert same_bits(bi.rmsnorm(x[r:r + 1].contiguous(), w, EPS)[0], full[r]), r
+    rows = [0, 7, M // 2, M - 1]
+    ref = oracle.rmsnorm(synth.to_f64(x[rows].cpu()), synth.to_f64(w.cpu()), EPS)
+    assert max_rel(full[rows], ref) <= TOL_BF16
