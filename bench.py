@@ -513,118 +513,143 @@ M_SWEEP = [1, 2, 3, 4, 7, 8, 13, 16, 32, 33, 64, 127, 128, 255, 256, 257, 512, 1
 B_SWEEP = [1, 2, 4, 8, 16, 32, 64, 128, 256]
 
 
-class L2Flush:
-    """Evicts L2 (126 MB) by reading a 512 MiB buffer. A read leaves L2 full of clean
-    lines, so the next kernel pays for its own misses only; a flush by writing would
-    leave dirty lines whose write-back lands inside the next, timed kernel (measured:
-    up to 8 us of a 30 us launch)."""
-
-    def __init__(self, device):
-        self.buf = torch.ones(512 << 20, dtype=torch.uint8, device=device).view(torch.int64)
-        self.sink = torch.empty(1, dtype=torch.int64, device=device)
-
-    def __call__(self):
-        self.sink.copy_(self.buf.sum().view(1))
-
-
-def _launch_ms(fn, flush, iters, cold):
-    """Median device time of one launch of fn (CUDA events on the current stream);
-    when `cold`, an L2 flush precedes every launch. A spin of about 100 us on the
-    device precedes the start event, so that the host's work of issuing the call
-    (argument checks, tensor maps) happens while the device is busy and is not
-    counted in a kernel of a few microseconds."""
-    ts = []
-    for i in range(iters + 3):
-        if cold:
-            flush()
-        torch.cuda._sleep(200000)
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        fn()
-        e.record()
-        torch.cuda.synchronize()
-        if i >= 3:
-            ts.append(s.elapsed_time(e))
-    return statistics.median(ts)
+def _graph_per_call_us(calls, reps=5):
+    """Device microseconds per call: the calls (closures issuing one launch each) are
+    captured back to back in one CUDA graph, replayed `reps` times between two CUDA
+    events, and the time is divided by the number of calls. Graph replay keeps the
+    device busy from one launch to the next, so neither the host's issue cost nor the
+    overhead of an event pair is counted. Callers rotate through inputs whose total
+    size exceeds L2 (126 MB) to time them cold, or repeat one input to time it warm."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for fn in calls[:2]:
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for fn in calls:
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    del g
+    return s.elapsed_time(e) * 1e3 / (len(calls) * reps)
 
 
-def sweep_matmul(bi, device, pk, flush, iters=7, ms_list=M_SWEEP):
-    """One entry per (M, N): TFLOP/s W warm (in L2) and W cold (L2 flushed), the
-    fraction of the bf16 burst peak (each launch is timed alone) and of the roofline
-    max(FLOPs / peak, bytes / HBM), and cuBLAS (torch.matmul) on the same operands."""
+def _copies(nbytes_one, floor=384 << 20, cap=64):
+    """Number of rotating copies whose total exceeds `floor` bytes (three times L2)."""
+    return int(max(2, min(cap, -(-floor // max(1, nbytes_one)))))
+
+
+# tcgen05 dependent-accumulation latency: one 128 x N x 16 MMA into the accumulator
+# the previous one wrote costs about 195 SM cycles, whatever N (measured on this
+# B200 with the chain probe; see DESIGN). Every output tile is one such chain of
+# K/16 MMAs, so no tile of the invariant matmul finishes in less than K/16 x 195
+# cycles.
+MMA_CHAIN_CYCLES = 195.0
+
+
+def sweep_matmul(bi, device, pk, clocks_mhz, ms_list=M_SWEEP, calls=12):
+    """One entry per (M, N): bi_matmul and cuBLAS (torch.matmul), each as CUDA-graph
+    replays of back-to-back launches. W warm: one W repeated (it stays in L2). W cold:
+    launches rotate through copies of W larger than L2 together (A, the activations,
+    stays resident, as between the layers of a model). Fractions: of the bf16 burst
+    peak; of the roofline max(FLOPs / peak, bytes / HBM); of the chain bound
+    max(roofline time, K/16 x 195 cycles at the sampled SM clock)."""
     A = synth.normal_bf16((2048, K_HIDDEN), 100).to(device)
     out = []
+    chain_ms = (K_HIDDEN / 16) * MMA_CHAIN_CYCLES / (clocks_mhz * 1e3)
     for j, n in enumerate(NS):
         W = synth.normal_bf16((n, K_HIDDEN), 120 + j, std=0.02).to(device)
+        R = _copies(W.numel() * 2)
+        Ws = [W] + [W.clone() for _ in range(R - 1)]
         C = torch.empty((2048, n), dtype=torch.bfloat16, device=device)
         for m in ms_list:
             a, c = A[:m], C[:m]
             flops = 2.0 * m * n * K_HIDDEN
             byts = 2.0 * (m * K_HIDDEN + n * K_HIDDEN + m * n)
             roof_ms = max(flops / pk["bf16_tflops"] / 1e9, byts / pk["hbm_gbs"] / 1e6)
-            warm = _launch_ms(lambda: bi.matmul(a, W, out=c), flush, iters, False)
-            cold = _launch_ms(lambda: bi.matmul(a, W, out=c), flush, iters, True)
-            ref = _launch_ms(lambda: torch.matmul(a, W.t(), out=c), flush, iters, True)
+            warm = _graph_per_call_us([lambda: bi.matmul(a, W, out=c)] * calls) / 1e3
+            cold = _graph_per_call_us([lambda w=Ws[i % R]: bi.matmul(a, w, out=c) for i in range(max(calls, R))]) / 1e3
+            ref = _graph_per_call_us([lambda w=Ws[i % R]: torch.matmul(a, w.t(), out=c)
+                                      for i in range(max(calls, R))]) / 1e3
             out.append({"M": m, "N": n, "tile_n": bi.matmul_tile_n(m, n),
-                        "warm_tflops": round(flops / warm / 1e9, 1),
+                        "warm_us": round(warm * 1e3, 2), "warm_tflops": round(flops / warm / 1e9, 1),
                         "warm_frac_peak": round(flops / warm / 1e9 / pk["bf16_tflops"], 3),
                         "cold_us": round(cold * 1e3, 2), "cold_tflops": round(flops / cold / 1e9, 1),
                         "cold_frac_peak": round(flops / cold / 1e9 / pk["bf16_tflops"], 3),
                         "cold_frac_roofline": round(roof_ms / cold, 3),
                         "cold_frac_hbm": round(byts / cold / 1e6 / pk["hbm_gbs"], 3),
+                        "cold_frac_chain_bound": round(max(roof_ms, chain_ms) / cold, 3),
                         "cublas_cold_us": round(ref * 1e3, 2), "slowdown_vs_cublas": round(cold / ref, 3)})
-        del W, C
+        del W, Ws, C
     return out
 
 
-def sweep_rmsnorm(bi, device, pk, flush, iters=7, ms_list=M_SWEEP):
-    """RMSNorm at hidden 4096 over M, L2 flushed before each launch: GB/s of x in + y
-    out + w, fraction of the HBM copy peak, and F.rms_norm on the same rows."""
-    x = synth.normal_bf16((2048, K_HIDDEN), 100).to(device)
+def sweep_rmsnorm(bi, device, pk, ms_list=M_SWEEP):
+    """RMSNorm at hidden 4096 over M, CUDA-graph replays of back-to-back launches
+    rotating through (x, y) pairs larger than L2 together (up to 64 pairs; below
+    M = 64 the rows stay in L2 whatever the rotation): GB/s of x in + y out + w,
+    fraction of the HBM copy peak, and F.rms_norm on the same rows."""
     wn = synth.normal_bf16((K_HIDDEN,), 110, std=0.1, mean=1.0).to(device)
-    y = torch.empty_like(x)
     out = []
     for m in ms_list:
-        xm, ym = x[:m], y[:m]
-        t = _launch_ms(lambda: bi.rmsnorm(xm, wn, EPS, out=ym), flush, iters, True)
-        ref = _launch_ms(lambda: torch.nn.functional.rms_norm(xm, (K_HIDDEN,), wn, EPS), flush, iters, True)
-        gbs = (4.0 * m * K_HIDDEN + 2 * K_HIDDEN) / t / 1e6
-        out.append({"M": m, "us": round(t * 1e3, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3),
-                    "slowdown_vs_F.rms_norm": round(t / ref, 3)})
+        R = _copies(2 * 2 * m * K_HIDDEN)
+        xs = [synth.normal_bf16_device((m, K_HIDDEN), 130 + i, device) for i in range(R)]
+        ys = [torch.empty_like(x) for x in xs]
+        t = _graph_per_call_us([lambda i=i: bi.rmsnorm(xs[i], wn, EPS, out=ys[i]) for i in range(R)] * max(1, 16 // R))
+        ref = _graph_per_call_us([lambda i=i: torch.nn.functional.rms_norm(xs[i], (K_HIDDEN,), wn, EPS)
+                                  for i in range(R)] * max(1, 16 // R))
+        gbs = (4.0 * m * K_HIDDEN + 2 * K_HIDDEN) / t / 1e3
+        out.append({"M": m, "us": round(t, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3),
+                    "slowdown_vs_F.rms_norm": round(t / ref, 3), "rotating_buffers": R})
+        del xs, ys
     return out
 
 
-def sweep_decode(bi, device, pk, flush, iters=5, bs=B_SWEEP):
+def sweep_decode(bi, device, pk, bs=B_SWEEP):
     """Decode attention (32 q-heads / 8 kv-heads, D 128, 16-token pages) over the batch
-    size: the first B sequences of one store of 256 with lengths ~ U[1, 32768]
-    (17 GB of K/V). KV bytes read per launch / time, against the HBM copy peak;
-    L2 flushed before each launch."""
+    size, from one store of 256 sequences with lengths ~ U[1, 32768] (17 GB of K/V).
+    Each B is timed as CUDA-graph replays of back-to-back launches over disjoint
+    batches of B sequences (sequences rB .. rB + B - 1 for r = 0 .. 256/B - 1, at most
+    16 batches), so consecutive launches read different K/V: KV bytes of all
+    launches / their time, against the HBM copy peak."""
     Bmax, Lmax = max(bs), 32768
     lens = synth.decode_lengths(Bmax, Lmax, seed=50)
     kv = synth.paged_kv_device(lens, 8, 128, seed=51, max_pages=Lmax // 16, device=device)
     q = synth.normal_bf16((Bmax, 32, 128), 52).to(device)
     o = torch.empty_like(q)
-    ws = torch.empty(bi.attention_workspace_size(Bmax, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
     out = []
     for B in bs:
-        qb, ob = q[:B], o[:B]
-        pt, sl = kv.page_table[:B], kv.seq_lens[:B]
-        t = _launch_ms(lambda: bi.attention_decode(qb, kv.k_cache, kv.v_cache, pt, sl, out=ob, workspace=ws),
-                       flush, iters, True)
-        kv_bytes = 4096.0 * int(lens[:B].sum())
-        gbs = kv_bytes / t / 1e6
-        out.append({"B": B, "kv_tokens": int(lens[:B].sum()), "us": round(t * 1e3, 2), "GB/s": round(gbs, 1),
-                    "frac_hbm": round(gbs / pk["hbm_gbs"], 3)})
-    del kv, ws
+        R = max(1, min(16, Bmax // B))
+        ws = torch.empty(bi.attention_workspace_size(B, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
+        calls = []
+        for r in range(R):
+            sl = slice(r * B, (r + 1) * B)
+            calls.append(lambda sl=sl: bi.attention_decode(q[sl], kv.k_cache, kv.v_cache, kv.page_table[sl],
+                                                           kv.seq_lens[sl], out=o[sl], workspace=ws))
+        reps = max(1, 16 // R)
+        t = _graph_per_call_us(calls * reps if R < 16 else calls)
+        tokens = int(lens[: R * B].sum())
+        kv_bytes = 4096.0 * tokens / R
+        gbs = kv_bytes / t / 1e3
+        out.append({"B": B, "batches": R, "kv_tokens_per_launch": round(tokens / R), "us": round(t, 2),
+                    "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3)})
+        del ws
+    del kv
     return out
 
 
-def run_sweeps(bi, device, pk):
-    flush = L2Flush(device)
-    res = {"matmul_k4096": sweep_matmul(bi, device, pk, flush),
-           "rmsnorm_k4096": sweep_rmsnorm(bi, device, pk, flush),
-           "decode_h32_8_d128_l32k": sweep_decode(bi, device, pk, flush)}
-    del flush
+def run_sweeps(bi, device, pk, clocks_mhz=None):
+    res = {"matmul_k4096": sweep_matmul(bi, device, pk, clocks_mhz or pk["sm_max_mhz"]),
+           "rmsnorm_k4096": sweep_rmsnorm(bi, device, pk),
+           "decode_h32_8_d128_l32k": sweep_decode(bi, device, pk)}
     torch.cuda.empty_cache()
     return res
 
@@ -778,7 +803,7 @@ def run_ours(args, rank, world, local):
     if world == 1 and args.rows:
         line["rows"] = other_rows(bi, device, pk)
     if world == 1 and args.sweeps:
-        line["sweeps"] = run_sweeps(bi, device, pk)
+        line["sweeps"] = run_sweeps(bi, device, pk, (clocks or {}).get("sm_mhz"))
     print(json.dumps(line), flush=True)
 
 

@@ -33,6 +33,21 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(s) <= t for s in SOURCES + [HEADER])
 
 
+PROBE_SRC = os.path.join(PKG, "probes", "mma_chain.cu")
+PROBE_BIN = os.path.join(ROOT, "_build", "mma_chain")
+
+
+def build_probe() -> str:
+    """Compile the tcgen05 chain-latency probe (a standalone diagnostic program) into
+    _build/; returns its path."""
+    os.makedirs(os.path.dirname(PROBE_BIN), exist_ok=True)
+    cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-o", PROBE_BIN, PROBE_SRC]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
+    return PROBE_BIN
+
+
 def build_library(force: bool = False, verbose: bool = False) -> str:
     """Compile csrc/libbi.cu into libbi.so next to this file; returns its path."""
     if not force and up_to_date():
