@@ -273,9 +273,11 @@ size_t bi_lmhead_workspace_size(int64_t M, int64_t V);
  * recomputed: [M] int32 out (1 if the row took step 3, else 0). logits_fp32:
  * optional [M, V] fp32 out (may be NULL): rows that took step 3 receive their fp32
  * logits, other rows are not written. Requires the bi_matmul rules on K and
- * V % 8 == 0. M == 0 is a no-op. Step 3 reads W once per 8 flagged rows when at most 24
- * rows are flagged and K <= 4096, and uses 64-row tiles otherwise; the choice is made on
- * the device from the flagged count, and every logit is the same FMA chain either way.
+ * V % 8 == 0. M == 0 is a no-op.
+ * How step 3 is laid out (never the arithmetic of a logit): with K <= 4096 it reads W
+ * once for a single flagged row, once per group of 8 rows for 2..24 flagged rows, and
+ * uses 64-row tiles beyond that; the choice is made on the device from the flagged
+ * count. Every fp32 logit is the same FMA chain on every path (tested bit for bit).
  */
 bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int64_t M, int64_t V,
                            int64_t K, float margin_threshold, int32_t* tokens, int32_t* recomputed,

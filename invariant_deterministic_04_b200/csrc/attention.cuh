@@ -151,7 +151,11 @@ __device__ __forceinline__ void all_gather(float x, int dl, float (&out)[G]) {
 template <int D, int G>
 struct SplitCfg {
   static constexpr int DPL = (D == 128 && G <= 4) ? 16 : 8;
-  static constexpr int WARPS = 8, NST = 3;
+  // 12 warps with 2-page rings where 16 dims per lane apply (measured on a B200 at
+  // D = 128, group 4: 5-8 % more HBM bandwidth than 8 warps with 3-page rings at
+  // B >= 4, same bits), 8 warps with 3-page rings otherwise
+  static constexpr int WARPS = DPL == 16 ? 12 : 8;
+  static constexpr int NST = DPL == 16 ? 2 : 3;
 };
 
 template <int D, int G>

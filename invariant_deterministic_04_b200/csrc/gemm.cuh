@@ -78,6 +78,93 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// Barrier layout shared by the kernels built on this main loop: full[0..S),
+// empty[0..S), tfull[0..2), tempty[0..2), 8 bytes each from bar0.
+struct Bars {
+  uint32_t bar0;
+  int stages;
+  __device__ __forceinline__ uint32_t full(int s) const { return bar0 + 8u * (uint32_t)s; }
+  __device__ __forceinline__ uint32_t empty(int s) const { return bar0 + 8u * (uint32_t)(stages + s); }
+  __device__ __forceinline__ uint32_t tfull(int a) const { return bar0 + 8u * (uint32_t)(2 * stages + a); }
+  __device__ __forceinline__ uint32_t tempty(int a) const { return bar0 + 8u * (uint32_t)(2 * stages + 2 + a); }
+};
+
+// TMA producer (one thread): for every tile t = blockIdx.x, +gridDim.x, ... (m-tile
+// t mod mt, n-tile t / mt) and every 64-wide K block in ascending order, waits for a
+// free stage and loads the A block (a_bytes of rows) and the W block into it.
+// `issued` / `ph_bits` record the stages filled and their parities (drain_copies).
+template <int BN, int STAGES>
+__device__ __forceinline__ void tma_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, uint32_t a_s, uint32_t b_s,
+                                             const Bars& bars, int tiles, int mt, int nkb, uint32_t a_bytes,
+                                             volatile int* abort_flag, uint32_t& issued, uint32_t& ph_bits) {
+  int s = 0;
+  uint32_t ph = 0;
+  const uint32_t stage_tx = a_bytes + (uint32_t)Cfg<BN>::B_BYTES;
+  for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+    const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!mbar_wait(bars.empty(s), ph ^ 1u)) {
+        *abort_flag = 1;
+        break;
+      }
+      mbar_arrive_expect_tx(bars.full(s), stage_tx);
+      tma_load_2d(a_s + s * A_BYTES, tmA, kb * BK, m0, bars.full(s));
+      tma_load_2d(b_s + s * Cfg<BN>::B_BYTES, tmB, kb * BK, n0, bars.full(s));
+      note_fill(issued, ph_bits, s, ph);
+      if (++s == STAGES) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+  }
+}
+
+// MMA issuer (one thread): per tile, waits for a free accumulator (two, BN columns
+// apart in TMEM), then per K block for its stage, and issues the four 128xBNx16
+// MMAs in ascending k; the first MMA of a tile overwrites the accumulator. Each
+// stage is released by tcgen05.commit once its MMAs have read it, each accumulator
+// once its last MMA completes.
+template <int BN, int STAGES>
+__device__ __forceinline__ void mma_issuer(uint32_t a_s, uint32_t b_s, const Bars& bars, uint32_t tmem, int tiles,
+                                           int nkb, volatile int* abort_flag) {
+  int s = 0, acc = 0;
+  uint32_t ph = 0, aph = 0;
+  for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+    if (!mbar_wait(bars.tempty(acc), aph ^ 1u)) {
+      *abort_flag = 1;
+      break;
+    }
+    tc_fence_after();
+    const uint32_t d = tmem + (uint32_t)(acc * BN);
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!mbar_wait(bars.full(s), ph)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk) {
+        const uint64_t ad = sw128_desc(a_s + s * A_BYTES + kk * 32);
+        const uint64_t bd = sw128_desc(b_s + s * Cfg<BN>::B_BYTES + kk * 32);
+        tc_mma_f16(d, ad, bd, Cfg<BN>::IDESC, (kb | kk) != 0 ? 1u : 0u);
+      }
+      tc_commit(bars.empty(s));  // frees the stage once these MMAs have read it
+      if (++s == STAGES) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      break;
+    }
+    tc_commit(bars.tfull(acc));  // accumulator complete
+    acc ^= 1;
+    if (acc == 0) aph ^= 1u;
+  }
+}
+
 // a_bytes: bytes one A box brings (rows of the A box x 128).
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -91,12 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t a_s = base;
   const uint32_t b_s = base + STAGES * A_BYTES;
-  const uint32_t bar0 = base + STAGES * G::STAGE_BYTES;
-  // barriers: full[0..S), empty[0..S), tfull[0..2), tempty[0..2)
-#define FULL(s) (bar0 + 8u * (s))
-#define EMPTY(s) (bar0 + 8u * (STAGES + (s)))
-#define TFULL(a) (bar0 + 8u * (2 * STAGES + (a)))
-#define TEMPTY(a) (bar0 + 8u * (2 * STAGES + 2 + (a)))
+  const Bars bars{base + STAGES * G::STAGE_BYTES, STAGES};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * G::STAGE_BYTES + 8 * (2 * STAGES + 4));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -107,12 +189,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(FULL(s), 1);
-      mbar_init(EMPTY(s), 1);
+      mbar_init(bars.full(s), 1);
+      mbar_init(bars.empty(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(TFULL(a), 1);
-      mbar_init(TEMPTY(a), kEpiThreads);
+      mbar_init(bars.tfull(a), 1);
+      mbar_init(bars.tempty(a), kEpiThreads);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -131,74 +213,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t issued = 0, ph_bits = 0;  // the producer's filled stages and their phase parities
 
   if (warp == 0) {
-    if (lane == 0) {  // ---- TMA producer
-      int s = 0;
-      uint32_t ph = 0;
-      const uint32_t stage_tx = a_bytes + (uint32_t)G::B_BYTES;
-      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
-        const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(EMPTY(s), ph ^ 1u)) {
-            *abort_flag = 1;
-            break;
-          }
-          mbar_arrive_expect_tx(FULL(s), stage_tx);
-          tma_load_2d(a_s + s * A_BYTES, &tmA, kb * BK, m0, FULL(s));
-          tma_load_2d(b_s + s * G::B_BYTES, &tmB, kb * BK, n0, FULL(s));
-          note_fill(issued, ph_bits, s, ph);
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1u;
-          }
-        }
-      }
-    }
+    if (lane == 0)
+      tma_producer<BN, STAGES>(&tmA, &tmB, a_s, b_s, bars, tiles, mt, nkb, a_bytes, abort_flag, issued, ph_bits);
   } else if (warp == 1) {
-    if (lane == 0) {  // ---- MMA issuer (single thread)
-      int s = 0, acc = 0;
-      uint32_t ph = 0, aph = 0;
-      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
-        if (!mbar_wait(TEMPTY(acc), aph ^ 1u)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(acc * BN);
-        bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(FULL(s), ph)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = sw128_desc(a_s + s * A_BYTES + kk * 32);
-            const uint64_t bd = sw128_desc(b_s + s * G::B_BYTES + kk * 32);
-            tc_mma_f16(d, ad, bd, G::IDESC, (kb | kk) != 0 ? 1u : 0u);
-          }
-          tc_commit(EMPTY(s));  // frees the stage once these MMAs have read it
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1u;
-          }
-        }
-        if (!ok) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_commit(TFULL(acc));  // accumulator complete
-        acc ^= 1;
-        if (acc == 0) aph ^= 1u;
-      }
-    }
+    if (lane == 0) mma_issuer<BN, STAGES>(a_s, b_s, bars, tmem, tiles, nkb, abort_flag);
   } else {  // ---- epilogue: warps 2..5; warp w may read TMEM lanes 32*(w%4) .. +31
     const int quarter = warp & 3;
     int acc = 0;
     uint32_t aph = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
-      const bool ok = __all_sync(kFullMask, mbar_wait(TFULL(acc), aph));
+      const bool ok = __all_sync(kFullMask, mbar_wait(bars.tfull(acc), aph));
       if (!ok || *abort_flag) {
         *abort_flag = 1;
         break;
@@ -234,19 +259,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(TEMPTY(acc));
+      mbar_arrive(bars.tempty(acc));
       acc ^= 1;
       if (acc == 0) aph ^= 1u;
     }
   }
-#undef FULL
-#undef EMPTY
-#undef TFULL
-#undef TEMPTY
   tc_fence_before();
   __syncthreads();
   // after an abort, loads may still be landing in stages nobody waited for
-  if (warp == 0 && lane == 0 && *abort_flag) drain_copies(bar0, 8, issued, ph_bits);
+  if (warp == 0 && lane == 0 && *abort_flag) drain_copies(bars.bar0, 8, issued, ph_bits);
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

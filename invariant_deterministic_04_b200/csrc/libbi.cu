@@ -148,23 +148,30 @@ bi_status attention_common(const uint16_t* q, int64_t ldq, const uint16_t* kc, c
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
-// ---- LM head workspace: bf16 logits [M, V], fp32 logits [M, V], flagged list [M + 1]
+// ---- LM head workspace: bf16 logits [M, V], fp32 logits [M, V], flagged list [M + 1],
+// argmax partials of the streaming recompute [24][its CTAs], its completion ticket
 struct LmWs {
   uint16_t* logits16;
   float* logits32;
   int32_t* list;
+  bi::lmhead::ArgBest* arg_part;
+  unsigned int* ticket;
 };
 
 size_t lm_ws_size(int64_t M, int64_t V, LmWs* lay, void* base) {
   if (M < 0 || V <= 0) return 0;
+  const int64_t sctas = (V + bi::lmhead::kStrWarps * 32 - 1) / (bi::lmhead::kStrWarps * 32);
   const size_t a = align256((size_t)M * V * 2), b = align256((size_t)M * V * 4), c = align256((size_t)(M + 1) * 4);
+  const size_t d = align256((size_t)bi::lmhead::kStrMaxCount * sctas * sizeof(bi::lmhead::ArgBest)), e = 256;
   if (lay && base) {
     uint8_t* p = static_cast<uint8_t*>(base);
     lay->logits16 = reinterpret_cast<uint16_t*>(p);
     lay->logits32 = reinterpret_cast<float*>(p + a);
     lay->list = reinterpret_cast<int32_t*>(p + a + b);
+    lay->arg_part = reinterpret_cast<bi::lmhead::ArgBest*>(p + a + b + c);
+    lay->ticket = reinterpret_cast<unsigned int*>(p + a + b + c + d);
   }
-  return a + b + c;
+  return a + b + c + d + e;
 }
 
 }  // namespace
@@ -392,33 +399,42 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
   LmWs lay{};
   if (workspace_bytes < lm_ws_size(M, V, &lay, workspace)) return BI_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
   bi_status s = bi::gemm::launch(h, ldh, W, K, lay.logits16, V, M, V, K, st);
   if (s != BI_OK) return s;
-  bi::lmhead::top2_kernel<<<(unsigned)(M * bi::lmhead::kParts), bi::lmhead::kThreads, 0, st>>>(lay.logits16, V, margin_threshold, tokens,
-                                                                      recomputed);
-  bi::lmhead::compact_kernel<<<1, 1024, 0, st>>>(recomputed, (int)M, lay.list);
+  // small batches (M <= 24, hidden size <= 4096): the streaming recompute lists the
+  // flagged rows and takes their tokens itself; W is streamed once for a single flagged
+  // row, once per group of 8 otherwise. Larger batches: the flagged list, then 64-row
+  // tiles and a separate argmax. Every fp32 logit is the same FMA chain on each path;
+  // each kernel returns at once when the flagged count (known on the device) is not
+  // its case.
+  const bool small = M <= bi::lmhead::kStrMaxCount && K <= bi::lmhead::kStrMaxK;
+  bi::lmhead::top2_kernel<<<(unsigned)(M * bi::lmhead::kParts), bi::lmhead::kThreads, 0, st>>>(
+      lay.logits16, V, margin_threshold, tokens, recomputed, small ? lay.ticket : nullptr);
   float* out32 = logits_fp32 ? logits_fp32 : lay.logits32;
-  // few flagged rows (with hidden size <= 4096): W streamed once per 8 rows; otherwise
-  // 64-row tiles. Both compute every logit as the same FMA chain, and each returns at
-  // once when the count of flagged rows is not its case.
-  int skip_upto = 0;
-  if (K <= bi::lmhead::kStrMaxK) {
-    static std::once_flag str_once[64];
-    static cudaError_t str_attr[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
-    if (bi::gemm::set_smem_once(bi::lmhead::recompute_stream_kernel, bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK),
-                                str_once, str_attr, dev) != cudaSuccess)
+  if (small) {
+    static std::once_flag once1[64], once8[64];
+    static cudaError_t attr1[64], attr8[64];
+    if (bi::gemm::set_smem_once(bi::lmhead::recompute_stream_kernel<1>,
+                                bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK, 1), once1, attr1, dev) != cudaSuccess ||
+        bi::gemm::set_smem_once(bi::lmhead::recompute_stream_kernel<8>,
+                                bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK, 8), once8, attr8, dev) != cudaSuccess)
       return BI_ERR_CUDA;
     const unsigned sgrid = (unsigned)((V + bi::lmhead::kStrWarps * 32 - 1) / (bi::lmhead::kStrWarps * 32));
-    bi::lmhead::recompute_stream_kernel<<<sgrid, bi::lmhead::kStrThreads, bi::lmhead::stream_smem_bytes((int)K), st>>>(
-        h, ldh, W, V, (int)K, (int)M, lay.list, out32);
-    skip_upto = bi::lmhead::kStrMaxCount;
+    bi::lmhead::recompute_stream_kernel<1><<<sgrid, bi::lmhead::kStrThreads, bi::lmhead::stream_smem_bytes((int)K, 1), st>>>(
+        h, ldh, W, V, (int)K, (int)M, recomputed, out32, lay.arg_part, tokens, lay.ticket);
+    if (M > 1)
+      bi::lmhead::recompute_stream_kernel<8><<<sgrid, bi::lmhead::kStrThreads, bi::lmhead::stream_smem_bytes((int)K, 8),
+                                               st>>>(h, ldh, W, V, (int)K, (int)M, recomputed, out32, lay.arg_part,
+                                                     tokens, lay.ticket);
+    return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
   }
+  bi::lmhead::compact_kernel<<<1, 1024, 0, st>>>(recomputed, (int)M, lay.list);
   const dim3 rgrid((unsigned)((V + bi::lmhead::VB - 1) / bi::lmhead::VB),
                    (unsigned)((M + bi::lmhead::RB - 1) / bi::lmhead::RB));
   bi::lmhead::recompute_kernel<<<rgrid, bi::lmhead::kRecThreads, 0, st>>>(h, ldh, W, V, (int)K, (int)M, lay.list, out32,
-                                                                         skip_upto);
+                                                                         0);
   bi::lmhead::argmax_kernel<<<(unsigned)(M * bi::lmhead::kParts), bi::lmhead::kThreads, 0, st>>>(out32, V, recomputed,
                                                                                                 tokens);
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;

@@ -12,8 +12,9 @@
 //      never wins), margin = top1 - top2 in fp32, flag = margin < threshold;
 //      token = top-1 index.
 //   3. compact_kernel: ascending list of flagged rows.
-//   4. recompute_kernel: fp32 logits of the flagged rows from bf16 operands
-//      widened to fp32, each logit one FMA chain over k = 0..K-1 (CUDA cores).
+//   4. recompute_kernel, or recompute_stream_kernel<1 | 8> for few flagged rows: fp32
+//      logits of the flagged rows from bf16 operands widened to fp32, each logit one
+//      FMA chain over k = 0..K-1 (CUDA cores).
 //   5. argmax_kernel: token of each flagged row = argmax of its fp32 logits.
 // The top-2 and argmax merges are order-independent (a strict total order), and
 // each fp32 logit depends only on its own row, so every row is batch-invariant.
@@ -31,6 +32,11 @@ struct Top2 {
   int i1;
   float v2;
   int i2;
+};
+
+struct ArgBest {
+  float v;
+  int i;
 };
 
 __device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
@@ -80,11 +86,12 @@ __device__ __forceinline__ Top2 block_top2(Top2 t, Top2* warp_best) {
 // does not change it.
 __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads)
     top2_kernel(const uint16_t* __restrict__ logits, int64_t V, float threshold, int32_t* __restrict__ tokens,
-                int32_t* __restrict__ flags) {
+                int32_t* __restrict__ flags, unsigned int* __restrict__ ticket) {
   __shared__ Top2 warp_best[kThreads / 32];
   __shared__ Top2 part_best;
   const int64_t row = blockIdx.x / kParts;
   const uint32_t part = cluster_rank();
+  if (blockIdx.x == 0 && threadIdx.x == 0 && ticket) *ticket = 0;  // for recompute_stream_kernel
   const uint4* src = reinterpret_cast<const uint4*>(logits + row * V);
   const int64_t nvec = V / 8, per = (nvec + kParts - 1) / kParts;
   const int64_t j0 = (int64_t)part * per, j1 = min(nvec, j0 + per);
@@ -240,31 +247,47 @@ __global__ void __launch_bounds__(kRecThreads, 3) recompute_kernel(const uint16_
   }
 }
 
-// The same fp32 logits for hidden sizes up to 4096, with W streamed once per 8 flagged
-// rows instead of once per 64-row tile (identical FMA chains, so identical bits). Both
-// kernels are launched; this one takes the call when at most kStrMaxCount rows are flagged
-// (a rare recompute, as with a trained model), the tiled one otherwise.
+// The same fp32 logits for batches of at most kStrMaxCount rows and hidden sizes up to
+// 4096, with W streamed once per NR flagged rows instead of once per 64-row tile
+// (identical FMA chains, so identical bits), and the flagged rows' tokens taken in the
+// same kernel. Both are launched; the on-device count of flagged rows picks the one
+// that works: recompute_stream_kernel<1> when exactly one row is flagged (the common
+// case of a trained model's rare near-tie), <8> for two or more.
 // Each warp owns 32 consecutive vocabulary entries (lane = entry) and walks K in tiles of
-// 64: the tile (32 rows x 128 bytes of W) is loaded coalesced (8 lanes per row) one tile
+// 64: the tile (32 rows x 128 bytes of W) is loaded coalesced (8 lanes per row) two tiles
 // ahead into registers, parked in the warp's shared-memory slot (rows padded to 144 bytes,
 // so each lane's 16-byte reads of its own row are conflict-free), and consumed by each lane
-// along its row. The CTA's 8 current flagged rows of h sit in shared memory as fp32,
+// along its row. The CTA's NR current flagged rows of h sit in shared memory as fp32,
 // [k][row], read as broadcasts; packed f32x2 FMAs carry two rows each.
-constexpr int kStrRows = 8, kStrWarps = 4, kStrThreads = 128, kStrTK = 64, kStrPad = 72, kStrMaxK = 4096;
+constexpr int kStrWarps = 4, kStrThreads = 128, kStrTK = 64, kStrPad = 72, kStrMaxK = 4096;
 constexpr int kStrMaxCount = 24;
 
-inline int stream_smem_bytes(int K) { return K * kStrRows * 4 + kStrWarps * 32 * kStrPad * 2; }
+inline int stream_smem_bytes(int K, int NR) { return K * NR * 4 + kStrWarps * 32 * kStrPad * 2; }
 
+template <int NR>
 __global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uint16_t* __restrict__ h, int64_t ldh,
                                                                       const uint16_t* __restrict__ W, int64_t V,
-                                                                      int K, int M, const int32_t* __restrict__ list,
-                                                                      float* __restrict__ out) {
+                                                                      int K, int M, const int32_t* __restrict__ flags,
+                                                                      float* __restrict__ out,
+                                                                      ArgBest* __restrict__ arg_part,
+                                                                      int32_t* __restrict__ tokens,
+                                                                      unsigned int* __restrict__ ticket) {
   extern __shared__ __align__(16) uint8_t smem_str[];
-  float* hsm = reinterpret_cast<float*>(smem_str);                                     // [K][8]
-  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_str + (size_t)K * kStrRows * 4);  // [warp][32][72]
-  const int count = list[M];
-  if (count == 0 || count > kStrMaxCount) return;
+  float* hsm = reinterpret_cast<float*>(smem_str);                               // [K][NR]
+  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_str + (size_t)K * NR * 4);  // [warp][32][72]
+  __shared__ int list[kStrMaxCount + 1];  // flagged rows, ascending (M <= kStrMaxCount)
+  __shared__ ArgBest warp_arg[kStrWarps][NR];
+  __shared__ int last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {  // the flagged rows in order: one ballot over M <= 24 rows
+    const bool f = lane < M && flags[lane] != 0;
+    const unsigned mask = __ballot_sync(kFullMask, f);
+    if (f) list[__popc(mask & ((1u << lane) - 1u))] = lane;
+    if (lane == 0) list[kStrMaxCount] = __popc(mask);
+  }
+  __syncthreads();
+  const int count = list[kStrMaxCount];
+  if (NR == 1 ? count != 1 : count < 2) return;
   const int64_t vbase = ((int64_t)blockIdx.x * kStrWarps + warp) * 32;
   const int64_t v = vbase + lane;
   uint16_t* my = tiles + warp * 32 * kStrPad;
@@ -278,11 +301,11 @@ __global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uin
                     : make_uint4(0, 0, 0, 0);
     }
   };
-  for (int r0 = 0; r0 < count; r0 += kStrRows) {
-    const int nr = min(kStrRows, count - r0);
-    __syncthreads();  // the previous rows of h are no longer read
-    for (int e = threadIdx.x; e < kStrRows * (K / 8); e += kStrThreads) {
-      const int r = e % kStrRows, kv = e / kStrRows;
+  for (int r0 = 0; r0 < count; r0 += NR) {
+    const int nr = min(NR, count - r0);
+    __syncthreads();  // the previous rows of h and the previous partials are no longer read
+    for (int e = threadIdx.x; e < NR * (K / 8); e += kStrThreads) {
+      const int r = e % NR, kv = e / NR;
       float f[8];
       if (r < nr) {
         unpack8(__ldg(reinterpret_cast<const uint4*>(h + (int64_t)list[r0 + r] * ldh) + kv), f);
@@ -291,41 +314,108 @@ __global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uin
         for (int i = 0; i < 8; ++i) f[i] = 0.f;
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) hsm[(kv * 8 + i) * kStrRows + r] = f[i];
+      for (int i = 0; i < 8; ++i) hsm[(kv * 8 + i) * NR + r] = f[i];
     }
     __syncthreads();
-    float2 acc[kStrRows / 2];
+    float acc[NR];
 #pragma unroll
-    for (int j = 0; j < kStrRows / 2; ++j) acc[j] = make_float2(0.f, 0.f);
-    uint4 nxt[8];
-    load_tile(0, nxt);
-    for (int t = 0; t < ntile; ++t) {
+    for (int j = 0; j < NR; ++j) acc[j] = 0.f;
+    // two tiles in flight in registers ahead of the one being consumed
+    uint4 b0[8], b1[8];
+    load_tile(0, b0);
+    if (ntile > 1) load_tile(1, b1);
+    auto step = [&](int t, uint4 (&buf)[8]) {
       __syncwarp();  // every lane is done with the previous tile
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<uint4*>(my + (q * 4 + (lane >> 3)) * kStrPad + (lane & 7) * 8) = nxt[q];
+        *reinterpret_cast<uint4*>(my + (q * 4 + (lane >> 3)) * kStrPad + (lane & 7) * 8) = buf[q];
       __syncwarp();
-      if (t + 1 < ntile) load_tile(t + 1, nxt);
+      if (t + 2 < ntile) load_tile(t + 2, buf);
 #pragma unroll
       for (int c = 0; c < kStrTK / 8; ++c) {
         float w[8];
         unpack8(*reinterpret_cast<const uint4*>(my + lane * kStrPad + c * 8), w);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float* hk = hsm + (t * kStrTK + c * 8 + i) * kStrRows;
-          const float4 a = *reinterpret_cast<const float4*>(hk);
-          const float4 b = *reinterpret_cast<const float4*>(hk + 4);
-          const float2 ww = make_float2(w[i], w[i]);
-          acc[0] = __ffma2_rn(make_float2(a.x, a.y), ww, acc[0]);
-          acc[1] = __ffma2_rn(make_float2(a.z, a.w), ww, acc[1]);
-          acc[2] = __ffma2_rn(make_float2(b.x, b.y), ww, acc[2]);
-          acc[3] = __ffma2_rn(make_float2(b.z, b.w), ww, acc[3]);
+          const float* hk = hsm + (t * kStrTK + c * 8 + i) * NR;
+          if constexpr (NR == 1) {
+            acc[0] = __fmaf_rn(hk[0], w[i], acc[0]);
+          } else {
+            // packed pairs of rows; each element rounds exactly like a scalar FMA
+#pragma unroll
+            for (int j = 0; j < NR; j += 4) {
+              const float4 a = *reinterpret_cast<const float4*>(hk + j);
+              const float2 ww = make_float2(w[i], w[i]);
+              const float2 p0 = __ffma2_rn(make_float2(a.x, a.y), ww, make_float2(acc[j], acc[j + 1]));
+              const float2 p1 = __ffma2_rn(make_float2(a.z, a.w), ww, make_float2(acc[j + 2], acc[j + 3]));
+              acc[j] = p0.x;
+              acc[j + 1] = p0.y;
+              acc[j + 2] = p1.x;
+              acc[j + 3] = p1.y;
+            }
+          }
         }
       }
+    };
+    for (int t = 0; t < ntile; t += 2) {
+      step(t, b0);
+      if (t + 1 < ntile) step(t + 1, b1);
     }
-    if (v < V) {
-      for (int r = 0; r < nr; ++r)
-        out[(int64_t)list[r0 + r] * V + v] = (r & 1) ? acc[r >> 1].y : acc[r >> 1].x;
+    // fp32 logits out, and this CTA's argmax of each row over its 128 entries (lowest
+    // index on ties, NaN never wins): lanes by an xor tree, then the warps in order
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      if (r < nr && v < V) out[(int64_t)list[r0 + r] * V + v] = acc[r];
+      ArgBest b{v < V ? sanitize(acc[r]) : -INFINITY, v < V ? (int)v : 0x7FFFFFFF};
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        const float ov = __shfl_xor_sync(kFullMask, b.v, o);
+        const int oi = __shfl_xor_sync(kFullMask, b.i, o);
+        if (better(ov, oi, b.v, b.i)) b = ArgBest{ov, oi};
+      }
+      if (lane == 0) warp_arg[warp][r] = b;
+    }
+    __syncthreads();
+    if (threadIdx.x < nr) {
+      ArgBest b = warp_arg[0][threadIdx.x];
+      for (int w2 = 1; w2 < kStrWarps; ++w2)
+        if (better(warp_arg[w2][threadIdx.x].v, warp_arg[w2][threadIdx.x].i, b.v, b.i)) b = warp_arg[w2][threadIdx.x];
+      arg_part[(int64_t)(r0 + threadIdx.x) * gridDim.x + blockIdx.x] = b;
+    }
+  }
+  // the CTA that finishes last (an integer ticket zeroed by top2_kernel; it orders no
+  // value) merges the CTAs' partials in CTA order and writes the tokens
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  // per flagged row: thread t takes partials t, t + 128, ... (read from L2, where the
+  // other CTAs' writes are), then an xor tree over the lanes and the warps in order
+  for (int f = 0; f < count; ++f) {
+    const ArgBest* p = arg_part + (int64_t)f * gridDim.x;
+    ArgBest b{-INFINITY, 0x7FFFFFFF};
+    for (unsigned c = threadIdx.x; c < gridDim.x; c += kStrThreads) {
+      const float cv = __ldcg(&p[c].v);
+      const int ci = __ldcg(&p[c].i);
+      if (better(cv, ci, b.v, b.i)) b = ArgBest{cv, ci};
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const float ov = __shfl_xor_sync(kFullMask, b.v, o);
+      const int oi = __shfl_xor_sync(kFullMask, b.i, o);
+      if (better(ov, oi, b.v, b.i)) b = ArgBest{ov, oi};
+    }
+    __syncthreads();  // warp_arg of the previous row is read
+    if (lane == 0) warp_arg[warp][0] = b;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w2 = 1; w2 < kStrWarps; ++w2)
+        if (better(warp_arg[w2][0].v, warp_arg[w2][0].i, b.v, b.i)) b = warp_arg[w2][0];
+      tokens[list[f]] = b.i;
     }
   }
 }

@@ -40,6 +40,9 @@ def _check_against_oracle(h, w, tau, tokens, rec, logits):
 
 
 @pytest.mark.parametrize("M,V,K", [(9, 1000, 256), (1, 32000, 2048), (64, 32000, 2048), (40, 4096, 512),
+                                   (4, 32000, 2048), (3, 16384, 512),
+                                   (2, 1000, 4096),   # the streaming recompute's largest K
+                                   (4, 1000, 4160),   # K > 4096: the tiled recompute
                                    (5, 1000, 4096),   # the largest K of the W-streaming recompute
                                    (6, 2000, 4160)])  # K > 4096: the 64-row tiled recompute
 def test_lmhead_matches_oracle(M, V, K):
@@ -99,14 +102,19 @@ def _fp32_fma_chain(h, w):
     return acc
 
 
-def test_lmhead_recompute_is_the_documented_fp32_chain_bit_for_bit():
-    # threshold inf sends every row through the recompute: 3 rows take the W-streaming
-    # kernel, 30 rows the tiled one; both must give exactly the ascending-k fp32 FMA chain
-    for M, V, K in ((3, 1000, 256), (30, 520, 128)):
-        h, w = synth.lmhead_inputs(M, V, K, seed=400 + M)
-        tok, rec, lg = bi.lmhead_argmax(h.to(dev()), w.to(dev()), float("inf"), want_logits=True)
-        assert int(rec.sum()) == M
-        np.testing.assert_array_equal(lg.cpu().numpy(), _fp32_fma_chain(h, w))
+@pytest.mark.parametrize("M,V,K", [(1, 1000, 256),     # W-streaming recompute of a single row
+                                   (2, 520, 128),      # the 8-row streaming kernel, two rows used
+                                   (3, 1000, 256),
+                                   (4, 4096, 1024),
+                                   (10, 1000, 256),    # a group of eight rows, then a group of two
+                                   (30, 520, 128)])    # the 64-row tiled recompute
+def test_lmhead_recompute_is_the_documented_fp32_chain_bit_for_bit(M, V, K):
+    # threshold inf flags every row; each path that produces fp32 logits must give
+    # exactly the ascending-k fp32 FMA chain
+    h, w = synth.lmhead_inputs(M, V, K, seed=400 + M)
+    tok, rec, lg = bi.lmhead_argmax(h.to(dev()), w.to(dev()), float("inf"), want_logits=True)
+    assert int(rec.sum()) == M
+    np.testing.assert_array_equal(lg.cpu().numpy(), _fp32_fma_chain(h, w))
 
 
 def test_lmhead_batch_invariant():
@@ -119,7 +127,9 @@ def test_lmhead_batch_invariant():
         assert int(t1[0]) == int(tok[r]) and int(r1[0]) == int(rec[r])
         if int(r1[0]):
             assert same_bits(l1[0], lg[r])
-    for m in (1, 2, 7, 33):
+    # small batches put their flagged rows through the streaming recompute (one row, or
+    # groups of 8), the 64-row batch through the tiled one: the same bits
+    for m in (1, 2, 4, 5, 7, 33):
         t2, r2, l2 = bi.lmhead_argmax(hd[:m].contiguous(), wd, TAU, want_logits=True)
         assert torch.equal(t2, tok[:m]) and torch.equal(r2, rec[:m])
         mask = r2.bool()
