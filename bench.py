@@ -15,7 +15,9 @@ torch.matmul + F.rms_norm) on the same box, an end-to-end figure through the
 public API with host buffers, the clocks seen during the timed region, the fp64
 CPU oracle timed on a bounded sample, and (``--rows``, default on) one
 measurement of every other hot-path kernel: RMSNorm bandwidth, decode attention
-bandwidth, causal prefill throughput and the LM head; and (``--sweeps``, default
+bandwidth, causal prefill throughput, the LM head, the row reductions, and the
+random-Llama decoder under mixed batching (streams per prompt, tokens/s,
+recompute rate, against stock torch ops); and (``--sweeps``, default
 on) the configuration sweeps: bi_matmul over M = 1..2048 at K = 4096 for N = 4096,
 6144 and 14336 (W warm and W cold), RMSNorm over the same M at hidden 4096, and
 decode attention over B = 1..256 with lengths ~ U[1, 32768], each entry with its
@@ -336,7 +338,39 @@ def other_rows(bi, device, pk, only=None):
         out.update(_row_lmhead(bi, device, pk))
     if want("reduce"):
         out.update(_row_reduce(bi, device, pk))
+    if want("config5"):
+        out.update(_row_config5(bi, device, pk))
     return out
+
+
+def _row_config5(bi, device, pk, repeats=3, base_repeats=2):
+    """The random-init Llama decoder (16 layers, hidden 2048, 32/8 heads, SwiGLU 8192,
+    vocab 32000, weights ~ N(0, 0.02), seed 0): 64 prompts of 128 tokens, 256 greedy
+    tokens each, under random mixed batching (batch ~ U[1, 64] per step, random
+    subsets and order, prefill chunks mixed with decode tokens; schedule seed r for
+    repeat r). Reported: the most distinct 256-token streams any prompt produced over
+    the repeats (1 = bit-identical), wall-clock tokens/s, the share of LM-head rows
+    that took the FP32 recompute, and the same for stock torch ops (cuBLAS,
+    F.rms_norm, padded attention, matmul + argmax) on the same weights."""
+    from invariant_deterministic_04_b200.llama import BaselineLlama, FastBiLlama, run_repeats, run_schedule
+
+    cfg = synth.LLAMA_CFG
+    w = synth.llama_weights(cfg, seed=0, device=device)
+    prompts = synth.prompts(64, 128, cfg["vocab"], seed=0)
+    run_schedule(FastBiLlama(cfg, w, 64, 128 + 8, device), prompts, 8, seed=10_000)  # warm-up
+    inv = run_repeats(FastBiLlama, cfg, w, prompts, 256, repeats, device)
+    base = run_repeats(BaselineLlama, cfg, w, prompts, 256, base_repeats, device)
+    diverging = int((base["first"] != inv["first"]).any(axis=1).sum())
+    row = {"repeats": repeats, "max_unique_streams_per_prompt": inv["max_unique"],
+           "tokens_per_s": round(inv["tokens_per_s"], 1), "recompute_rate": round(inv["recompute_rate"], 4),
+           "baseline_repeats": base_repeats, "baseline_max_unique_streams_per_prompt": base["max_unique"],
+           "baseline_mean_unique_streams_per_prompt": round(float(base["unique_per_seq"].mean()), 2),
+           "baseline_prompts_diverging_from_invariant": diverging,
+           "baseline_tokens_per_s": round(base["tokens_per_s"], 1),
+           "speed_vs_baseline": round(inv["tokens_per_s"] / base["tokens_per_s"], 3)}
+    del w
+    torch.cuda.empty_cache()
+    return {"config5_llama_64x128_gen256": row}
 
 
 def _row_rmsnorm(bi, device, pk):
@@ -547,12 +581,11 @@ def _copies(nbytes_one, floor=384 << 20, cap=64):
     return int(max(2, min(cap, -(-floor // max(1, nbytes_one)))))
 
 
-# tcgen05 dependent-accumulation latency: one 128 x N x 16 MMA into the accumulator
-# the previous one wrote costs about 195 SM cycles, whatever N (measured on this
-# B200 with the chain probe; see DESIGN). Every output tile is one such chain of
-# K/16 MMAs, so no tile of the invariant matmul finishes in less than K/16 x 195
-# cycles.
-MMA_CHAIN_CYCLES = 195.0
+# tcgen05 dependent-accumulation step: one 128 x N x 16 MMA into the accumulator the
+# previous one wrote costs about 83 SM cycles for N <= 128 and 130 for N = 256
+# (measured on this B200 with probes/mma_chain.cu). Every output tile is one such
+# chain of K/16 MMAs, so no tile finishes in less than K/16 steps.
+MMA_CHAIN_CYCLES = {32: 83.0, 64: 83.0, 128: 83.0, 256: 130.0}
 
 
 def sweep_matmul(bi, device, pk, clocks_mhz, ms_list=M_SWEEP, calls=12):
@@ -561,10 +594,9 @@ def sweep_matmul(bi, device, pk, clocks_mhz, ms_list=M_SWEEP, calls=12):
     launches rotate through copies of W larger than L2 together (A, the activations,
     stays resident, as between the layers of a model). Fractions: of the bf16 burst
     peak; of the roofline max(FLOPs / peak, bytes / HBM); of the chain bound
-    max(roofline time, K/16 x 195 cycles at the sampled SM clock)."""
+    max(roofline time, K/16 chain steps at the sampled SM clock)."""
     A = synth.normal_bf16((2048, K_HIDDEN), 100).to(device)
     out = []
-    chain_ms = (K_HIDDEN / 16) * MMA_CHAIN_CYCLES / (clocks_mhz * 1e3)
     for j, n in enumerate(NS):
         W = synth.normal_bf16((n, K_HIDDEN), 120 + j, std=0.02).to(device)
         R = _copies(W.numel() * 2)
@@ -575,11 +607,13 @@ def sweep_matmul(bi, device, pk, clocks_mhz, ms_list=M_SWEEP, calls=12):
             flops = 2.0 * m * n * K_HIDDEN
             byts = 2.0 * (m * K_HIDDEN + n * K_HIDDEN + m * n)
             roof_ms = max(flops / pk["bf16_tflops"] / 1e9, byts / pk["hbm_gbs"] / 1e6)
+            tile_n = bi.matmul_tile_n(m, n)
+            chain_ms = (K_HIDDEN / 16) * MMA_CHAIN_CYCLES[tile_n] / (clocks_mhz * 1e3)
             warm = _graph_per_call_us([lambda: bi.matmul(a, W, out=c)] * calls) / 1e3
             cold = _graph_per_call_us([lambda w=Ws[i % R]: bi.matmul(a, w, out=c) for i in range(max(calls, R))]) / 1e3
             ref = _graph_per_call_us([lambda w=Ws[i % R]: torch.matmul(a, w.t(), out=c)
                                       for i in range(max(calls, R))]) / 1e3
-            out.append({"M": m, "N": n, "tile_n": bi.matmul_tile_n(m, n),
+            out.append({"M": m, "N": n, "tile_n": tile_n,
                         "warm_us": round(warm * 1e3, 2), "warm_tflops": round(flops / warm / 1e9, 1),
                         "warm_frac_peak": round(flops / warm / 1e9 / pk["bf16_tflops"], 3),
                         "cold_us": round(cold * 1e3, 2), "cold_tflops": round(flops / cold / 1e9, 1),
@@ -821,7 +855,7 @@ def main():
                     help="add the matmul / RMSNorm / decode sweeps to the line (default on)")
     ap.add_argument("--no-sweeps", dest="sweeps", action="store_false")
     ap.add_argument("--sweep", action="store_true", help="only the sweeps, one JSON line per entry")
-    ap.add_argument("--row", choices=["rmsnorm", "decode", "prefill", "lmhead", "reduce"], default=None,
+    ap.add_argument("--row", choices=["rmsnorm", "decode", "prefill", "lmhead", "reduce", "config5"], default=None,
                     help="measure only this hot-path kernel (for profiling) and print its line")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args()

@@ -22,16 +22,26 @@ __device__ __forceinline__ uint64_t sw128(uint32_t saddr) {
 // smem: A 16 KiB (128 rows x 128 B), B 32 KiB (256 rows x 128 B), barrier.
 // unrolled = 0: one MMA per loop trip, descriptors advanced in the loop;
 // unrolled = 1: as the matmul kernel issues them, four MMAs (k = 0, 16, 32, 48 of a
-// 64-wide block) with precomputed descriptors per trip.
+// 64-wide block) with precomputed descriptors per trip;
+// unrolled = 2: the matmul's whole per-block sequence with the data already present:
+// a wait on a stage barrier that is already complete, the fence, the four MMAs, and
+// a tcgen05.commit of the stage to a barrier nobody waits on;
+// unrolled = 3: the same without the commit; 4: without the wait and the fence;
+// 5: the fence and the four MMAs only.
 __global__ void __launch_bounds__(128, 1) lat_kernel(int m_instr, int n_instr, int chains, int iters, int unrolled,
                                                       long long* out) {
   extern __shared__ __align__(1024) uint8_t sm[];
   const uint32_t base = (smem_u32(sm) + 1023u) & ~1023u;
   uint8_t* g = sm + (base - smem_u32(sm));
   __shared__ uint32_t tslot;
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bar, bar_full, bar_empty;
   for (int i = threadIdx.x; i < (16384 + 32768) / 16; i += 128) reinterpret_cast<uint4*>(g)[i] = make_uint4(0, 0, 0, 0);
-  if (threadIdx.x == 0) { mbar_init(smem_u32(&bar), 1); fence_mbar_init(); }
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    mbar_init(smem_u32(&bar_full), 1);   // never arrived on: its previous phase counts as complete
+    mbar_init(smem_u32(&bar_empty), 1);
+    fence_mbar_init();
+  }
   fence_proxy_async_smem();
   if (threadIdx.x < 32) { tmem_alloc(smem_u32(&tslot), 512); tmem_relinquish(); }
   tc_fence_before(); __syncthreads(); tc_fence_after();
@@ -48,6 +58,20 @@ __global__ void __launch_bounds__(128, 1) lat_kernel(int m_instr, int n_instr, i
       t0 = clock64();
       for (int i = 0; i < iters; ++i)
         for (int c = 0; c < chains; ++c) tc_mma_f16(tmem + c * n_instr, ad + ((i & 3) * 2), bd + ((i & 3) * 2), idesc, 1u);
+      t1 = clock64();
+    } else if (unrolled >= 2) {
+      uint64_t a4[4], b4[4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) { a4[kk] = sw128(base + kk * 32); b4[kk] = sw128(base + 16384 + kk * 32); }
+      t0 = clock64();
+      for (int i = 0; i < iters; i += 4)
+        for (int c = 0; c < chains; ++c) {
+          if (unrolled == 2 || unrolled == 3) mbar_wait(smem_u32(&bar_full), 1u);
+          if (unrolled != 4) tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) tc_mma_f16(tmem + c * n_instr, a4[kk], b4[kk], idesc, 1u);
+          if (unrolled == 2 || unrolled == 4) tc_commit(smem_u32(&bar_empty));
+        }
       t1 = clock64();
     } else {
       uint64_t a4[4], b4[4];
@@ -75,7 +99,7 @@ int main() {
   cudaFuncSetAttribute(lat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 50 * 1024);
   const int iters = 256;
   int ns[] = {32, 64, 128, 256};
-  for (int unrolled = 0; unrolled < 2; ++unrolled)
+  for (int unrolled = 0; unrolled < 6; ++unrolled)
     for (int m : {128, 64})
       for (int n : ns)
         for (int chains = 1; chains <= 8; chains *= 2) {
