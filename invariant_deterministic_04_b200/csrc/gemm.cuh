@@ -49,24 +49,31 @@ namespace bi {
 namespace gemm {
 
 constexpr int BM = 128, BK = 64;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KiB: room for a full 128-row A block per stage
+constexpr int A_BYTES = BM * BK * 2;  // 16 KiB: a full 128-row A block
 constexpr int kThreads = 192;         // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kEpiThreads = 128;
-constexpr int kRingBudget = 198 * 1024;  // shared memory for the stage ring
+constexpr int kSmemBytes = 227 * 1024;   // dynamic shared memory of every launch
+constexpr int kBarBytes = 8 * (2 * 32 + 4) + 16;  // barriers for up to 32 stages, TMEM slot, flag
+constexpr int kMaxStages = 32;
 
 template <int BN>
 struct Cfg {
   static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "tcgen05 M=128 tile widths used here");
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = kRingBudget / STAGE_BYTES;  // 4 / 6 / 8 / 9
-  static constexpr int TMEM_COLS = 2 * BN;                   // two fp32 accumulators (power of 2 >= 32)
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4) + 16;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;  // two fp32 accumulators (power of 2 >= 32)
   // Instruction descriptor for kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 =
   // 1), B bf16 (bits 10-12 = 1), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                     ((uint32_t)(BM >> 4) << 24);
+};
+
+// Stage ring of one launch (host-computed, a function of M and the tile width only):
+// a K block is an A slot (the rows of the A box, 128 bytes each) followed by a W slot
+// (BN rows); a stage holds kps consecutive K blocks; `stages` stages from the start of
+// the (1024-aligned) dynamic shared memory, then `pad` bytes so that the MMA's 128-row
+// read of the last A slot stays inside the allocation, then the barriers.
+struct Layout {
+  uint32_t a_slot, b_slot, kblk, kps, stages, stage_bytes, bar_offset;
 };
 
 // Shared-memory matrix descriptor for a K-major operand written by TMA with the
@@ -90,28 +97,48 @@ struct Bars {
 };
 
 // TMA producer (one thread): for every tile t = blockIdx.x, +gridDim.x, ... (m-tile
-// t mod mt, n-tile t / mt) and every 64-wide K block in ascending order, waits for a
-// free stage and loads the A block (a_bytes of rows) and the W block into it.
+// t mod mt, n-tile t / mt) and every group of up to kps 64-wide K blocks in ascending
+// order, waits for a free stage and loads each K block's A rows and W rows into it.
 // `issued` / `ph_bits` record the stages filled and their parities (drain_copies).
-template <int BN, int STAGES>
-__device__ __forceinline__ void tma_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, uint32_t a_s, uint32_t b_s,
-                                             const Bars& bars, int tiles, int mt, int nkb, uint32_t a_bytes,
+// Byte strides of the stage ring: compile-time with full 128-row A slots (one K block
+// per stage), from the host's Layout with compact A slots (the A box's rows).
+template <int BN, int KPS, bool COMPACT>
+struct Strides {
+  uint32_t a_slot, kblk, stage;
+  __device__ __forceinline__ explicit Strides(const Layout& L)
+      : a_slot(COMPACT ? L.a_slot : (uint32_t)A_BYTES),
+        kblk(COMPACT ? L.kblk : (uint32_t)(A_BYTES + Cfg<BN>::B_BYTES)),
+        stage(COMPACT ? L.stage_bytes : (uint32_t)(A_BYTES + Cfg<BN>::B_BYTES)) {}
+};
+
+template <int BN, int KPS, bool COMPACT>
+__device__ __forceinline__ void tma_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, uint32_t base,
+                                             const Layout& L, const Bars& bars, int tiles, int mt, int nkb,
                                              volatile int* abort_flag, uint32_t& issued, uint32_t& ph_bits) {
+  const Strides<BN, KPS, COMPACT> S(L);
+  const int stages = (int)L.stages;
+  const uint32_t a_bytes = L.a_slot;  // bytes one A box brings (its rows x 128)
   int s = 0;
   uint32_t ph = 0;
-  const uint32_t stage_tx = a_bytes + (uint32_t)Cfg<BN>::B_BYTES;
   for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
     const int m0 = (t % mt) * BM, n0 = (t / mt) * BN;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb0 = 0; kb0 < nkb; kb0 += KPS) {
+      const int nk = min(KPS, nkb - kb0);
       if (!mbar_wait(bars.empty(s), ph ^ 1u)) {
         *abort_flag = 1;
         break;
       }
-      mbar_arrive_expect_tx(bars.full(s), stage_tx);
-      tma_load_2d(a_s + s * A_BYTES, tmA, kb * BK, m0, bars.full(s));
-      tma_load_2d(b_s + s * Cfg<BN>::B_BYTES, tmB, kb * BK, n0, bars.full(s));
+      mbar_arrive_expect_tx(bars.full(s), (uint32_t)nk * (a_bytes + (uint32_t)Cfg<BN>::B_BYTES));
+      const uint32_t st = base + (uint32_t)s * S.stage;
+#pragma unroll
+      for (int j = 0; j < KPS; ++j) {
+        if (j < nk) {
+          tma_load_2d(st + j * S.kblk, tmA, (kb0 + j) * BK, m0, bars.full(s));
+          tma_load_2d(st + j * S.kblk + S.a_slot, tmB, (kb0 + j) * BK, n0, bars.full(s));
+        }
+      }
       note_fill(issued, ph_bits, s, ph);
-      if (++s == STAGES) {
+      if (++s == stages) {
         s = 0;
         ph ^= 1u;
       }
@@ -120,13 +147,16 @@ __device__ __forceinline__ void tma_producer(const CUtensorMap* tmA, const CUten
 }
 
 // MMA issuer (one thread): per tile, waits for a free accumulator (two, BN columns
-// apart in TMEM), then per K block for its stage, and issues the four 128xBNx16
-// MMAs in ascending k; the first MMA of a tile overwrites the accumulator. Each
-// stage is released by tcgen05.commit once its MMAs have read it, each accumulator
-// once its last MMA completes.
-template <int BN, int STAGES>
-__device__ __forceinline__ void mma_issuer(uint32_t a_s, uint32_t b_s, const Bars& bars, uint32_t tmem, int tiles,
+// apart in TMEM), then per stage for its data, and issues for each of its K blocks the
+// four 128xBNx16 MMAs in ascending k; the first MMA of a tile overwrites the
+// accumulator. A stage is released by one tcgen05.commit once all its MMAs have read
+// it, an accumulator once its last MMA completes. The MMAs of an element are the same
+// sequence whatever kps is: kps only sets how many of them share one wait and commit.
+template <int BN, int KPS, bool COMPACT>
+__device__ __forceinline__ void mma_issuer(uint32_t base, const Layout& L, const Bars& bars, uint32_t tmem, int tiles,
                                            int nkb, volatile int* abort_flag) {
+  const Strides<BN, KPS, COMPACT> S(L);
+  const int stages = (int)L.stages;
   int s = 0, acc = 0;
   uint32_t ph = 0, aph = 0;
   for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
@@ -137,20 +167,26 @@ __device__ __forceinline__ void mma_issuer(uint32_t a_s, uint32_t b_s, const Bar
     tc_fence_after();
     const uint32_t d = tmem + (uint32_t)(acc * BN);
     bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb0 = 0; kb0 < nkb; kb0 += KPS) {
+      const int nk = min(KPS, nkb - kb0);
       if (!mbar_wait(bars.full(s), ph)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      const uint32_t st = base + (uint32_t)s * S.stage;
 #pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk) {
-        const uint64_t ad = sw128_desc(a_s + s * A_BYTES + kk * 32);
-        const uint64_t bd = sw128_desc(b_s + s * Cfg<BN>::B_BYTES + kk * 32);
-        tc_mma_f16(d, ad, bd, Cfg<BN>::IDESC, (kb | kk) != 0 ? 1u : 0u);
+      for (int j = 0; j < KPS; ++j) {
+        if (j < nk) {
+          const uint32_t a = st + j * S.kblk, b = a + S.a_slot;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16(d, sw128_desc(a + kk * 32), sw128_desc(b + kk * 32), Cfg<BN>::IDESC,
+                       ((kb0 + j) | kk) != 0 ? 1u : 0u);
+        }
       }
       tc_commit(bars.empty(s));  // frees the stage once these MMAs have read it
-      if (++s == STAGES) {
+      if (++s == stages) {
         s = 0;
         ph ^= 1u;
       }
@@ -165,21 +201,17 @@ __device__ __forceinline__ void mma_issuer(uint32_t a_s, uint32_t b_s, const Bar
   }
 }
 
-// a_bytes: bytes one A box brings (rows of the A box x 128).
-template <int BN>
+template <int BN, int KPS, bool COMPACT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     uint16_t* __restrict__ C, int64_t ldc, int M, int N, int K, uint32_t a_bytes) {
+                     uint16_t* __restrict__ C, int64_t ldc, int M, int N, int K, const Layout L) {
   using G = Cfg<BN>;
-  constexpr int STAGES = G::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t a_s = base;
-  const uint32_t b_s = base + STAGES * A_BYTES;
-  const Bars bars{base + STAGES * G::STAGE_BYTES, STAGES};
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * G::STAGE_BYTES + 8 * (2 * STAGES + 4));
+  const Bars bars{base + L.bar_offset, (int)L.stages};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.bar_offset + 8 * (2 * L.stages + 4));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkb = K / BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < (int)L.stages; ++s) {
       mbar_init(bars.full(s), 1);
       mbar_init(bars.empty(s), 1);
     }
@@ -214,9 +246,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0)
-      tma_producer<BN, STAGES>(&tmA, &tmB, a_s, b_s, bars, tiles, mt, nkb, a_bytes, abort_flag, issued, ph_bits);
+      tma_producer<BN, KPS, COMPACT>(&tmA, &tmB, base, L, bars, tiles, mt, nkb, abort_flag, issued, ph_bits);
   } else if (warp == 1) {
-    if (lane == 0) mma_issuer<BN, STAGES>(a_s, b_s, bars, tmem, tiles, nkb, abort_flag);
+    if (lane == 0) mma_issuer<BN, KPS, COMPACT>(base, L, bars, tmem, tiles, nkb, abort_flag);
   } else {  // ---- epilogue: warps 2..5; warp w may read TMEM lanes 32*(w%4) .. +31
     const int quarter = warp & 3;
     int acc = 0;
@@ -330,11 +362,11 @@ inline cudaError_t set_smem_once(F fn, int bytes, std::once_flag* once, cudaErro
   return result[dev];
 }
 
-template <int BN>
+template <int BN, int KPS, bool COMPACT>
 inline cudaError_t prepare(int dev) {
   static std::once_flag once[64];
   static cudaError_t result[64];
-  return set_smem_once(gemm_bf16_kernel<BN>, Cfg<BN>::SMEM_BYTES, once, result, dev);
+  return set_smem_once(gemm_bf16_kernel<BN, KPS, COMPACT>, kSmemBytes, once, result, dev);
 }
 
 // Rows of A one stage loads: a whole 128-row block, or only ceil8(M) rows when the
@@ -364,18 +396,62 @@ inline int pick_bn(int64_t M, int64_t N, int sms) {
   return best;
 }
 
+// The stage ring for an M-row product with tile width bn. From 65 rows of A on: one K
+// block per stage, full 128-row A slots, as many stages as 198 KB hold (4 at BN = 256,
+// 6, 8 and 9 at 128, 64 and 32). Up to 64 rows: the A slot holds only the rows of the
+// A box, and the most K blocks per stage (4, else 2) that still leave three stages
+// share one wait and one commit (16 or 8 MMAs instead of 4), so more W is in flight.
+constexpr uint32_t kRingBudget = 198 * 1024;
+inline Layout make_layout(int64_t M, int bn) {
+  Layout L{};
+  const uint32_t arows = a_box_rows(M);
+  L.b_slot = (uint32_t)bn * BK * 2;
+  if (arows > 64) {
+    L.a_slot = arows * BK * 2;  // the A box's bytes; its slot is a full 16 KiB
+    L.kblk = (uint32_t)A_BYTES + L.b_slot;
+    L.kps = 1;
+    L.stage_bytes = L.kblk;
+    L.stages = kRingBudget / L.stage_bytes;
+    L.bar_offset = L.stages * L.stage_bytes;
+    return L;
+  }
+  L.a_slot = arows * BK * 2;
+  L.kblk = L.a_slot + L.b_slot;
+  const uint32_t pad = (uint32_t)A_BYTES - L.a_slot;  // the MMA reads 128 rows from every A slot
+  const uint32_t ring = (uint32_t)kSmemBytes - 1024 - kBarBytes - pad;
+  for (uint32_t kps : {4u, 2u, 1u}) {
+    L.kps = kps;
+    L.stage_bytes = kps * L.kblk;
+    L.stages = ring / L.stage_bytes;
+    if (L.stages >= 3) break;
+  }
+  if (L.stages > (uint32_t)kMaxStages) L.stages = kMaxStages;
+  L.bar_offset = (L.stages * L.stage_bytes + pad + 7u) & ~7u;
+  return L;
+}
+
+template <int BN, int KPS, bool COMPACT>
+inline bi_status launch_kps(const uint16_t* A, int64_t lda, const uint16_t* W, int64_t ldw, uint16_t* C, int64_t ldc,
+                            int64_t M, int64_t N, int64_t K, const Layout& L, int dev, int sms, cudaStream_t st) {
+  if (prepare<BN, KPS, COMPACT>(dev) != cudaSuccess) return BI_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, lda, a_box_rows(M)) || !make_map(&tb, W, N, K, ldw, BN)) return BI_ERR_CUDA;
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  const int smem = (int)(1024 + L.bar_offset + kBarBytes);
+  gemm_bf16_kernel<BN, KPS, COMPACT><<<grid, kThreads, smem, st>>>(ta, tb, C, ldc, (int)M, (int)N, (int)K, L);
+  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
 template <int BN>
 inline bi_status launch_bn(const uint16_t* A, int64_t lda, const uint16_t* W, int64_t ldw, uint16_t* C,
                            int64_t ldc, int64_t M, int64_t N, int64_t K, int dev, int sms, cudaStream_t st) {
-  if (prepare<BN>(dev) != cudaSuccess) return BI_ERR_CUDA;
-  const uint32_t arows = a_box_rows(M);
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K, lda, arows) || !make_map(&tb, W, N, K, ldw, BN)) return BI_ERR_CUDA;
-  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  const int grid = (int)(tiles < sms ? tiles : sms);
-  gemm_bf16_kernel<BN><<<grid, kThreads, Cfg<BN>::SMEM_BYTES, st>>>(ta, tb, C, ldc, (int)M, (int)N, (int)K,
-                                                                     arows * (uint32_t)(BK * 2));
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  const Layout L = make_layout(M, BN);
+  if (L.stages < 2) return BI_ERR_UNSUPPORTED;
+  if (a_box_rows(M) > 64) return launch_kps<BN, 1, false>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
+  if (L.kps == 4) return launch_kps<BN, 4, true>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
+  if (L.kps == 2) return launch_kps<BN, 2, true>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
+  return launch_kps<BN, 1, true>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
 }
 
 // bn: tile width (0 = pick_bn's choice for this device).
