@@ -100,15 +100,15 @@ struct Bars {
 // t mod mt, n-tile t / mt) and every group of up to kps 64-wide K blocks in ascending
 // order, waits for a free stage and loads each K block's A rows and W rows into it.
 // `issued` / `ph_bits` record the stages filled and their parities (drain_copies).
-// Byte strides of the stage ring: compile-time with full 128-row A slots (one K block
-// per stage), from the host's Layout with compact A slots (the A box's rows).
+// Byte strides of the stage ring: compile-time with full 128-row A slots, from the
+// host's Layout with compact A slots (the A box's rows).
 template <int BN, int KPS, bool COMPACT>
 struct Strides {
   uint32_t a_slot, kblk, stage;
   __device__ __forceinline__ explicit Strides(const Layout& L)
       : a_slot(COMPACT ? L.a_slot : (uint32_t)A_BYTES),
         kblk(COMPACT ? L.kblk : (uint32_t)(A_BYTES + Cfg<BN>::B_BYTES)),
-        stage(COMPACT ? L.stage_bytes : (uint32_t)(A_BYTES + Cfg<BN>::B_BYTES)) {}
+        stage(COMPACT ? L.stage_bytes : (uint32_t)(KPS * (A_BYTES + Cfg<BN>::B_BYTES))) {}
 };
 
 template <int BN, int KPS, bool COMPACT>
@@ -396,11 +396,12 @@ inline int pick_bn(int64_t M, int64_t N, int sms) {
   return best;
 }
 
-// The stage ring for an M-row product with tile width bn. From 65 rows of A on: one K
-// block per stage, full 128-row A slots, as many stages as 198 KB hold (4 at BN = 256,
-// 6, 8 and 9 at 128, 64 and 32). Up to 64 rows: the A slot holds only the rows of the
-// A box, and the most K blocks per stage (4, else 2) that still leave three stages
-// share one wait and one commit (16 or 8 MMAs instead of 4), so more W is in flight.
+// The stage ring for an M-row product with tile width bn. From 65 rows of A on: full
+// 128-row A slots in 198 KB, two K blocks per stage where that leaves three stages
+// (tile widths up to 128), else one (width 256: four stages). Up to 64 rows: the A
+// slot holds only the rows of the A box, and the most K blocks per stage (4, else 2)
+// that still leave three stages. Grouping K blocks lets 8 or 16 MMAs share one wait
+// and one commit instead of 4; compact A slots leave room for more W in flight.
 constexpr uint32_t kRingBudget = 198 * 1024;
 inline Layout make_layout(int64_t M, int bn) {
   Layout L{};
@@ -409,8 +410,8 @@ inline Layout make_layout(int64_t M, int bn) {
   if (arows > 64) {
     L.a_slot = arows * BK * 2;  // the A box's bytes; its slot is a full 16 KiB
     L.kblk = (uint32_t)A_BYTES + L.b_slot;
-    L.kps = 1;
-    L.stage_bytes = L.kblk;
+    L.kps = kRingBudget / (2 * L.kblk) >= 3 ? 2 : 1;
+    L.stage_bytes = L.kps * L.kblk;
     L.stages = kRingBudget / L.stage_bytes;
     L.bar_offset = L.stages * L.stage_bytes;
     return L;
@@ -448,7 +449,9 @@ inline bi_status launch_bn(const uint16_t* A, int64_t lda, const uint16_t* W, in
                            int64_t ldc, int64_t M, int64_t N, int64_t K, int dev, int sms, cudaStream_t st) {
   const Layout L = make_layout(M, BN);
   if (L.stages < 2) return BI_ERR_UNSUPPORTED;
-  if (a_box_rows(M) > 64) return launch_kps<BN, 1, false>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
+  if (a_box_rows(M) > 64)
+    return L.kps == 2 ? launch_kps<BN, 2, false>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st)
+                      : launch_kps<BN, 1, false>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
   if (L.kps == 4) return launch_kps<BN, 4, true>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
   if (L.kps == 2) return launch_kps<BN, 2, true>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
   return launch_kps<BN, 1, true>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
