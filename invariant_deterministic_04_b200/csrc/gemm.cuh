@@ -26,12 +26,16 @@
 // Design (sm_100a):
 //   * K is consumed in 64-wide blocks, each four 128xBNx16 MMAs in ascending k;
 //   * A and W tiles come into shared memory by TMA (128-byte swizzle, K-major)
-//     through an mbarrier ring of as many stages as ~200 KB holds (4 at BN = 256,
-//     up to 9 at BN = 32); a ragged tile's out-of-range rows and columns are
-//     zero-filled by TMA and masked in the epilogue, so they cannot touch other rows;
-//   * when M < 128 the A box holds only the first ceil8(M) rows: rows past it are
-//     never loaded, and what the MMAs compute for them lands in output rows >= M,
-//     which are never stored (row m of the product depends on row m of A only);
+//     through an mbarrier ring (make_layout); a stage holds 1, 2 or 4 K blocks, so
+//     that 4, 8 or 16 MMAs share one stage wait and one tcgen05.commit (the probe in
+//     probes/mma_chain.cu measures that pair at about one MMA chain step); a ragged
+//     tile's out-of-range rows and columns are zero-filled by TMA and masked in the
+//     epilogue, so they cannot touch other rows;
+//   * when M < 128 the A box holds only the first ceil8(M) rows; up to 64 rows the
+//     A slot in shared memory holds only those rows too (more stages fit). Rows past
+//     the box are never loaded: the MMAs read whatever lies there, and the result of
+//     those rows lands in output rows >= M, which are never stored (row m of the
+//     product depends on row m of A only);
 //   * warp 0 issues TMA, warp 1 (one thread) issues the MMAs, warps 2-5 drain
 //     TMEM (tcgen05.ld), round to bf16 (nearest even) and store; two TMEM
 //     accumulators let the epilogue of one tile overlap the main loop of the next;
@@ -96,10 +100,6 @@ struct Bars {
   __device__ __forceinline__ uint32_t tempty(int a) const { return bar0 + 8u * (uint32_t)(2 * stages + 2 + a); }
 };
 
-// TMA producer (one thread): for every tile t = blockIdx.x, +gridDim.x, ... (m-tile
-// t mod mt, n-tile t / mt) and every group of up to kps 64-wide K blocks in ascending
-// order, waits for a free stage and loads each K block's A rows and W rows into it.
-// `issued` / `ph_bits` record the stages filled and their parities (drain_copies).
 // Byte strides of the stage ring: compile-time with full 128-row A slots, from the
 // host's Layout with compact A slots (the A box's rows).
 template <int BN, int KPS, bool COMPACT>
@@ -111,6 +111,10 @@ struct Strides {
         stage(COMPACT ? L.stage_bytes : (uint32_t)(KPS * (A_BYTES + Cfg<BN>::B_BYTES))) {}
 };
 
+// TMA producer (one thread): for every tile t = blockIdx.x, +gridDim.x, ... (m-tile
+// t mod mt, n-tile t / mt) and every group of up to KPS 64-wide K blocks in ascending
+// order, waits for a free stage and loads each K block's A rows and W rows into it.
+// `issued` / `ph_bits` record the stages filled and their parities (drain_copies).
 template <int BN, int KPS, bool COMPACT>
 __device__ __forceinline__ void tma_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, uint32_t base,
                                              const Layout& L, const Bars& bars, int tiles, int mt, int nkb,
