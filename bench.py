@@ -698,6 +698,48 @@ def run_sweep(bi, device, pk):
 # ---------------------------------------------------------------------------
 
 
+PROFILE_CASES = ("decode_b16", "rmsnorm", "lmhead_m4", "matmul_small")
+
+
+def profile_case(bi, device, name):
+    """A few plain launches of one kernel case, for an ncu capture (nothing timed):
+    decode_b16 = decode attention over the first 16 sequences of the decode sweep's
+    store (lengths ~ U[1, 32768], 1.1 GB of K/V); rmsnorm = RMSNorm at 65536 x 4096
+    then 2048 x 4096; lmhead_m4 = the LM head at 4 rows, V = 32000, K = 2048, with no
+    near-tie and with one (then the cuBLAS matmul + argmax of the same shapes);
+    matmul_small = bi_matmul at M = 1 and 128, K = N = 4096."""
+    if name == "decode_b16":
+        lens = synth.decode_lengths(16, 32768, seed=50)
+        kv = synth.paged_kv_device(lens, 8, 128, seed=51, max_pages=2048, device=device)
+        q = synth.normal_bf16((16, 32, 128), 52).to(device)
+        o = torch.empty_like(q)
+        ws = torch.empty(bi.attention_workspace_size(16, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
+        for _ in range(3):
+            bi.attention_decode(q, kv.k_cache, kv.v_cache, kv.page_table, kv.seq_lens, out=o, workspace=ws)
+    elif name == "rmsnorm":
+        for M in (65536, 2048):
+            x = synth.normal_bf16_device((M, K_HIDDEN), 15, device)
+            w = synth.normal_bf16((K_HIDDEN,), 16, std=0.1, mean=1.0).to(device)
+            y = torch.empty_like(x)
+            for _ in range(3):
+                bi.rmsnorm(x, w, EPS, out=y)
+    elif name == "lmhead_m4":
+        for ties in (0, 1):
+            h, W = synth.lmhead_planted(4, 32000, 2048, seed=72, ties=ties)
+            h, W = h.to(device), W.to(device)
+            for _ in range(2):
+                bi.lmhead_argmax(h, W, 0.5)
+            torch.argmax(torch.matmul(h, W.t()), dim=1)
+    elif name == "matmul_small":
+        A = synth.normal_bf16((128, K_HIDDEN), 100).to(device)
+        W = synth.normal_bf16((4096, K_HIDDEN), 120, std=0.02).to(device)
+        for m in (1, 128):
+            for _ in range(2):
+                bi.matmul(A[:m], W)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "done": True}))
+
+
 def ours_config(M, world):
     """The workload description both arms print (the same dict, so the two lines compare)."""
     return {"workload": WORKLOAD, "M": M, "K": K_HIDDEN, "N": list(NS), "step": "bi_rmsnorm + 3 x bi_matmul",
@@ -858,12 +900,19 @@ def main():
     ap.add_argument("--row", choices=["rmsnorm", "decode", "prefill", "lmhead", "reduce", "config5"], default=None,
                     help="measure only this hot-path kernel (for profiling) and print its line")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--profile", choices=PROFILE_CASES, default=None,
+                    help="run a few plain launches of one kernel case (for an ncu capture) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     rank, world, local = init_dist()
     try:
-        if args.sweep:
+        if args.profile is not None:
+            import invariant_deterministic_04_b200 as bi
+
+            torch.cuda.set_device(local)
+            profile_case(bi, torch.device("cuda", local), args.profile)
+        elif args.sweep:
             import invariant_deterministic_04_b200 as bi
 
             torch.cuda.set_device(local)
