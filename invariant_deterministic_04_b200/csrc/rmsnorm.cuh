@@ -17,7 +17,8 @@
 // Scheduling (no effect on any row's arithmetic): CTA b takes rows b, b + grid,
 // b + 2 grid, ...; while it reduces and writes one row, the loads of its next row
 // are already in flight, so reads and writes of different rows overlap in HBM
-// instead of the whole batch reading first and writing after.
+// instead of the whole batch reading first and writing after. Batches of more than
+// four waves of resident CTAs get one CTA per row instead.
 #pragma once
 
 #include "device.cuh"
@@ -105,8 +106,11 @@ constexpr int ctas_per_sm() {
 template <int NV>
 inline cudaError_t launch_nv(const uint16_t* x, int64_t ldx, const uint16_t* w, uint16_t* y, int64_t ldy, int64_t M,
                              int K, float eps, int sms, cudaStream_t st) {
+  // up to 4 waves of resident CTAs: the persistent grid (each CTA overlaps its next
+  // row's loads with the current row's stores); beyond that one CTA per row, which
+  // the hardware schedules as CTAs retire (measured faster at M = 65536)
   const int64_t cap = (int64_t)sms * ctas_per_sm<NV>();
-  const unsigned grid = (unsigned)(M < cap ? M : cap);
+  const unsigned grid = (unsigned)(M <= 4 * cap ? (M < cap ? M : cap) : M);
   rmsnorm_kernel<NV><<<grid, kThreads, 0, st>>>(x, ldx, w, y, ldy, M, K, eps);
   return cudaGetLastError();
 }
