@@ -376,41 +376,87 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
   }
 }
 
-// One warp per (row, query head): fold the row's splits in ascending order.
-template <int D>
+// Fold a row's splits in ascending order: one warp per (row, query head, group of
+// 32 * DPL output dims), DPL dims per lane. The maximum of the splits' running maxima
+// is taken lane-parallel (a maximum is exact in any order); lane j computes the weight
+// of split j of each group of 32 and the weights are broadcast, so that every output
+// dim and the normaliser are each one FMA chain in split order whatever DPL is. The
+// partial outputs of 32 / DPL splits are loaded before any of them is folded. DPL only
+// sets how many warps share a row: 1 when the batch gives few (row, head) pairs, D / 32
+// when it gives enough warps to fill the GPU.
+template <int D, int DPL>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ po,
                                                            const float2* __restrict__ pml,
                                                            const int32_t* __restrict__ off, int nrows,
                                                            int Hq, uint16_t* __restrict__ out) {
-  constexpr int DPL = D / 32;  // dims per lane
+  static_assert(DPL == 1 || DPL == 2 || DPL == 4, "dims per lane");
+  static_assert(D % (32 * DPL) == 0, "a warp covers whole groups of dims");
+  constexpr int NG = D / (32 * DPL);  // warps per (row, query head)
+  constexpr int U = 32 / DPL;         // splits whose partial outputs are loaded together
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (w >= nrows * Hq) return;
-  const int r = w / Hq, h = w - (w / Hq) * Hq;
+  if (w >= nrows * Hq * NG) return;
+  const int rh = w / NG, g = w - (w / NG) * NG;
+  const int r = rh / Hq, h = rh - (rh / Hq) * Hq;
   const int f0 = off[r], n = off[r + 1] - off[r];
+  const int d0 = (g * 32 + lane) * DPL;
+  const float2* ml_row = pml + (int64_t)f0 * Hq + h;             // split s at s * Hq
+  const float* po_row = po + ((int64_t)f0 * Hq + h) * D + d0;    // split s at s * Hq * D
+  const int64_t po_step = (int64_t)Hq * D;
+  float M = -INFINITY;
+  for (int s0 = 0; s0 < n; s0 += 32)
+    if (s0 + lane < n) M = fmaxf(M, ml_row[(int64_t)(s0 + lane) * Hq].x);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float O[DPL];
 #pragma unroll
   for (int d = 0; d < DPL; ++d) O[d] = 0.f;
   float L = 0.f;
-  float M = -INFINITY;
-  for (int s = 0; s < n; ++s) M = fmaxf(M, pml[(int64_t)(f0 + s) * Hq + h].x);
   if (M != -INFINITY) {
-    for (int s = 0; s < n; ++s) {
-      const int64_t idx = (int64_t)(f0 + s) * Hq + h;
-      const float2 ml = pml[idx];
-      const float wgt = exp2f(__fsub_rn(ml.x, M));
-      L = __fmaf_rn(ml.y, wgt, L);
-      const float* src = po + idx * D + lane * DPL;
+    for (int s0 = 0; s0 < n; s0 += 32) {
+      const int cnt = min(32, n - s0);
+      const float2 ml = lane < cnt ? ml_row[(int64_t)(s0 + lane) * Hq] : make_float2(-INFINITY, 0.f);
+      const float wl = lane < cnt ? exp2f(__fsub_rn(ml.x, M)) : 0.f;
 #pragma unroll
-      for (int d = 0; d < DPL; ++d) O[d] = __fmaf_rn(src[d], wgt, O[d]);
+      for (int u0 = 0; u0 < 32; u0 += U) {
+        if (u0 >= cnt) break;  // the same for every lane
+        float v[U][DPL];
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+          const float* src = po_row + (int64_t)(u0 + j < cnt ? s0 + u0 + j : s0) * po_step;
+          if constexpr (DPL == 4) {
+            const float4 q = *reinterpret_cast<const float4*>(src);
+            v[j][0] = q.x; v[j][1] = q.y; v[j][2] = q.z; v[j][3] = q.w;
+          } else if constexpr (DPL == 2) {
+            const float2 q = *reinterpret_cast<const float2*>(src);
+            v[j][0] = q.x; v[j][1] = q.y;
+          } else {
+            v[j][0] = *src;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+          const float wk = __shfl_sync(0xffffffffu, wl, u0 + j);
+          const float lk = __shfl_sync(0xffffffffu, ml.y, u0 + j);
+          if (u0 + j < cnt) {
+            L = __fmaf_rn(lk, wk, L);
+#pragma unroll
+            for (int d = 0; d < DPL; ++d) O[d] = __fmaf_rn(v[j][d], wk, O[d]);
+          }
+        }
+      }
     }
   }
-  uint16_t* dst = out + ((int64_t)r * Hq + h) * D + lane * DPL;
+  float y[DPL];
 #pragma unroll
-  for (int d = 0; d < DPL; d += 2) {
-    const float a = L > 0.f ? __fdiv_rn(O[d], L) : 0.f;
-    const float b = L > 0.f ? __fdiv_rn(O[d + 1], L) : 0.f;
-    *reinterpret_cast<uint32_t*>(dst + d) = pack_bf16x2(a, b);
+  for (int d = 0; d < DPL; ++d) y[d] = L > 0.f ? __fdiv_rn(O[d], L) : 0.f;
+  uint16_t* dst = out + (int64_t)rh * D + d0;
+  if constexpr (DPL == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+  } else if constexpr (DPL == 2) {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(y[0], y[1]);
+  } else {
+    *dst = to_bf16_bits(y[0]);
   }
 }
 

@@ -139,12 +139,24 @@ bi_status attention_common(const uint16_t* q, int64_t ldq, const uint16_t* kc, c
   cudaError_t e = D == 128 ? launch_split_g<128>(G, q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st)
                            : launch_split_g<64>(G, q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st);
   if (e != cudaSuccess) return BI_ERR_CUDA;
-  const int warps = nrows * Hq;
+  // one dim per lane while that still leaves at most 32 warps per SM; beyond that
+  // D / 32 dims per lane (fewer, wider loads). The fold is the same either way.
+  const int sms = device_sms();
+  if (sms <= 0) return BI_ERR_CUDA;
+  const bool narrow = (int64_t)nrows * Hq * (D / 32) <= (int64_t)sms * 32;
+  const int warps = narrow ? nrows * Hq * (D / 32) : nrows * Hq;
   const int grid = (warps + 7) / 8;
-  if (D == 128)
-    bi::attn::attn_combine_kernel<128><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
-  else
-    bi::attn::attn_combine_kernel<64><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+  if (D == 128) {
+    if (narrow)
+      bi::attn::attn_combine_kernel<128, 1><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+    else
+      bi::attn::attn_combine_kernel<128, 4><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+  } else {
+    if (narrow)
+      bi::attn::attn_combine_kernel<64, 1><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+    else
+      bi::attn::attn_combine_kernel<64, 2><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+  }
   return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 

@@ -99,6 +99,23 @@ def test_decode_batch_invariant_and_run_to_run():
     assert same_bits(outp, full[perm])
 
 
+@pytest.mark.parametrize("D", [128, 64])
+def test_decode_combine_width_does_not_change_bits(D):
+    """96 sequences x 32 heads fold their splits with D / 32 (or D / 64) dims per
+    lane; 3 sequences with one dim per lane over D / 32 warps. Same bits, and the
+    oracle agrees with both."""
+    q, kv = synth.decode_inputs(96, 32, 8, D, max_len=1300, seed=70 + D)
+    qd, kvd = q.to(dev()), _to_dev(kv)
+    full = _decode(qd, kvd)
+    sub = [0, 41, 95]
+    s = torch.tensor(sub, device=dev())
+    few = bi.attention_decode(qd[s].contiguous(), kvd.k_cache, kvd.v_cache, kvd.page_table[s].contiguous(),
+                              kvd.seq_lens[s].contiguous())
+    assert same_bits(few, full[s])
+    kv_sub = synth.PagedKV(kv.k_cache, kv.v_cache, kv.page_table[sub], kv.seq_lens[sub], kv.max_pages)
+    assert max_rel(few, _oracle_decode(q[sub], kv_sub)) <= TOL_BF16
+
+
 def test_decode_invariant_to_physical_page_placement():
     lens = [1000, 333]
     q, kv = synth.decode_inputs(2, 32, 8, 64, max_len=1024, seed=34, lens=lens)
