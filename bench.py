@@ -698,13 +698,14 @@ def run_sweep(bi, device, pk):
 # ---------------------------------------------------------------------------
 
 
-PROFILE_CASES = ("decode_b16", "rmsnorm", "lmhead_m4", "matmul_small")
+PROFILE_CASES = ("decode_b16", "decode_b1", "rmsnorm", "lmhead_m4", "matmul_small")
 
 
 def profile_case(bi, device, name):
     """A few plain launches of one kernel case, for an ncu capture (nothing timed):
     decode_b16 = decode attention over the first 16 sequences of the decode sweep's
-    store (lengths ~ U[1, 32768], 1.1 GB of K/V); rmsnorm = RMSNorm at 65536 x 4096
+    store (lengths ~ U[1, 32768], 1.1 GB of K/V); decode_b1 = decode attention over
+    one sequence of 16384 tokens (64 splits, 67 MB of K/V); rmsnorm = RMSNorm at 65536 x 4096
     then 2048 x 4096; lmhead_m4 = the LM head at 4 rows, V = 32000, K = 2048, with no
     near-tie and with one (then the cuBLAS matmul + argmax of the same shapes);
     matmul_small = bi_matmul at M = 1 and 128, K = N = 4096."""
@@ -714,6 +715,13 @@ def profile_case(bi, device, name):
         q = synth.normal_bf16((16, 32, 128), 52).to(device)
         o = torch.empty_like(q)
         ws = torch.empty(bi.attention_workspace_size(16, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
+        for _ in range(3):
+            bi.attention_decode(q, kv.k_cache, kv.v_cache, kv.page_table, kv.seq_lens, out=o, workspace=ws)
+    elif name == "decode_b1":
+        kv = synth.paged_kv_device([16384], 8, 128, seed=51, max_pages=2048, device=device)
+        q = synth.normal_bf16((1, 32, 128), 52).to(device)
+        o = torch.empty_like(q)
+        ws = torch.empty(bi.attention_workspace_size(1, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
         for _ in range(3):
             bi.attention_decode(q, kv.k_cache, kv.v_cache, kv.page_table, kv.seq_lens, out=o, workspace=ws)
     elif name == "rmsnorm":

@@ -204,7 +204,9 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
   uint32_t seq = 0;  // pages this warp has consumed so far
   uint32_t issued = 0, ph_bits = 0;  // lane 0: ring stages filled and their phase parities
 
-  for (int item = blockIdx.x * WARPS + warp; item < total; item += gridDim.x * WARPS) {
+  // items are dealt across CTAs first (item = warp * gridDim.x + CTA), so that a
+  // launch with fewer items than warp slots spreads them over every SM
+  for (int item = warp * gridDim.x + blockIdx.x; item < total; item += gridDim.x * WARPS) {
     const int f = item / Hkv, g = item - (item / Hkv) * Hkv;
     int lo = 0, hi = nrows;  // off[lo] <= f < off[hi]
     while (hi - lo > 1) {
