@@ -698,14 +698,15 @@ def run_sweep(bi, device, pk):
 # ---------------------------------------------------------------------------
 
 
-PROFILE_CASES = ("decode_b16", "decode_b1", "rmsnorm", "lmhead_m4", "matmul_small")
+PROFILE_CASES = ("decode_b16", "decode_b1", "prefill_s4096", "rmsnorm", "lmhead_m4", "matmul_small")
 
 
 def profile_case(bi, device, name):
     """A few plain launches of one kernel case, for an ncu capture (nothing timed):
     decode_b16 = decode attention over the first 16 sequences of the decode sweep's
     store (lengths ~ U[1, 32768], 1.1 GB of K/V); decode_b1 = decode attention over
-    one sequence of 16384 tokens (64 splits, 67 MB of K/V); rmsnorm = RMSNorm at 65536 x 4096
+    one sequence of 16384 tokens (64 splits, 67 MB of K/V); prefill_s4096 = causal
+    prefill of one 4096-token sequence on the CUDA cores; rmsnorm = RMSNorm at 65536 x 4096
     then 2048 x 4096; lmhead_m4 = the LM head at 4 rows, V = 32000, K = 2048, with no
     near-tie and with one (then the cuBLAS matmul + argmax of the same shapes);
     matmul_small = bi_matmul at M = 1 and 128, K = N = 4096."""
@@ -724,6 +725,16 @@ def profile_case(bi, device, name):
         ws = torch.empty(bi.attention_workspace_size(1, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
         for _ in range(3):
             bi.attention_decode(q, kv.k_cache, kv.v_cache, kv.page_table, kv.seq_lens, out=o, workspace=ws)
+    elif name == "prefill_s4096":
+        S = 4096
+        kv = synth.paged_kv_device([S], 8, 128, seed=60, max_pages=S // 16, device=device)
+        q = synth.normal_bf16((S, 32, 128), 61).to(device)
+        qs = torch.zeros(S, dtype=torch.int32, device=device)
+        qpos = torch.arange(S, dtype=torch.int32, device=device)
+        o = torch.empty_like(q)
+        ws = torch.empty(bi.attention_workspace_size(S, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
+        for _ in range(2):
+            bi.attention_prefill(q, qs, qpos, kv.k_cache, kv.v_cache, kv.page_table, out=o, workspace=ws)
     elif name == "rmsnorm":
         for M in (65536, 2048):
             x = synth.normal_bf16_device((M, K_HIDDEN), 15, device)

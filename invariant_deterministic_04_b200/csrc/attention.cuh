@@ -163,33 +163,169 @@ constexpr int split_smem_bytes() {
   return SplitCfg<D, G>::WARPS * SplitCfg<D, G>::NST * (2 * PAGE * D * 2 + 8);
 }
 
-// One warp per (row, kv-head g, split): writes the split's (m, l) per query head
-// and its unnormalised o[D] per query head into the workspace.
+// Per-warp state of one (row, kv-head, split) reduction and the three steps that
+// both the decode kernel and the prefill window kernel run on it, so that a row's
+// arithmetic is the same code whichever kernel reduces it.
 //
 // Lane layout: the LPT = D/DPL lanes of a token own DPL dims each, in 16-byte
 // vectors v = 0..DPL/8-1 covering dims 8*(dl + v*LPT) .. +7 (interleaved so a
 // quarter-warp's shared-memory reads are contiguous); TPW = 32/LPT tokens are
 // processed per warp step, token t of a page by lane group t mod TPW.
 template <int D, int G>
+struct SplitLanes {
+  static constexpr int DPL = SplitCfg<D, G>::DPL;
+  static constexpr int NV = DPL / 8;   // 16-byte vectors per lane per token row
+  static constexpr int LPT = D / DPL;  // lanes per token
+  static constexpr int TPW = 32 / LPT; // tokens per warp step
+  static constexpr int STEPS = PAGE / TPW;
+  static constexpr int HEAD_LANES = LPT / G;
+  static constexpr int PAGE_BYTES = PAGE * D * 2;
+  static constexpr int STAGE_BYTES = 2 * PAGE_BYTES;
+};
+
+// The lane's slice of the G query heads that share kv-head g, row r.
+template <int D, int G>
+__device__ __forceinline__ void load_q(const uint16_t* __restrict__ q, int64_t ldq, int r, int g, int dl,
+                                       float2 (&qf)[G][SplitCfg<D, G>::DPL / 2]) {
+  using T = SplitLanes<D, G>;
+#pragma unroll
+  for (int j = 0; j < G; ++j)
+#pragma unroll
+    for (int v = 0; v < T::NV; ++v) {
+      const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)r * ldq + (int64_t)(g * G + j) * D +
+                                                            8 * (dl + v * T::LPT)));
+      unpack8x2(qv, &qf[j][4 * v]);
+    }
+}
+
+// Folds one page (K at kb, V at vb in shared memory, its first nvalid tokens
+// visible) into the running (m, l, o) of the lane's head: scores, the base-2
+// online-softmax rescale, then p * V.
+template <int D, int G>
+__device__ __forceinline__ void fold_page(const float2 (&qf)[G][SplitCfg<D, G>::DPL / 2], uint32_t kb, uint32_t vb,
+                                          int nvalid, float c, int tg, int dl, float& m, float& l,
+                                          float2 (&o)[G][SplitCfg<D, G>::DPL / 2]) {
+  using T = SplitLanes<D, G>;
+  constexpr int NV = T::NV, LPT = T::LPT, TPW = T::TPW, STEPS = T::STEPS, DPL = T::DPL;
+  // scores of this page: lane holds the score of its token for head hd
+  float sc[STEPS];
+#pragma unroll
+  for (int u = 0; u < STEPS; ++u) {
+    const int t = u * TPW + tg;
+    // two interleaved FMA chains per head (even / odd dims of the slice), then one add
+    float2 acc[G];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      float2 kf[4];
+      unpack8x2(ld_shared_v4(kb + (uint32_t)((t * D + 8 * (dl + v * LPT)) * 2)), kf);
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        float2 a = v == 0 ? __fmul2_rn(qf[i][0], kf[0]) : __ffma2_rn(qf[i][4 * v], kf[0], acc[i]);
+#pragma unroll
+        for (int e = 1; e < 4; ++e) a = __ffma2_rn(qf[i][4 * v + e], kf[e], a);
+        acc[i] = a;
+      }
+    }
+    float part[G];
+#pragma unroll
+    for (int i = 0; i < G; ++i) part[i] = __fadd_rn(acc[i].x, acc[i].y);
+    const float dot = reduce_scatter<G, LPT>(part, dl);
+    sc[u] = t < nvalid ? __fmul_rn(dot, c) : -INFINITY;
+  }
+  float pm = sc[0];
+#pragma unroll
+  for (int u = 1; u < STEPS; ++u) pm = fmaxf(pm, sc[u]);
+#pragma unroll
+  for (int o2 = LPT; o2 < 32; o2 <<= 1) pm = fmaxf(pm, __shfl_xor_sync(kFullMask, pm, o2));
+  const float m_new = fmaxf(m, pm);
+  const float alpha = m_new == -INFINITY ? 1.f : exp2f(__fsub_rn(m, m_new));
+  // rescale the running sums; skipped when no head's max moved (x * 1 == x exactly)
+  if (!__all_sync(kFullMask, alpha == 1.f)) {
+    l = __fmul_rn(l, alpha);
+    float al[G];
+    all_gather<G, LPT>(alpha, dl, al);
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      const float2 a2 = make_float2(al[i], al[i]);
+#pragma unroll
+      for (int e = 0; e < DPL / 2; ++e) o[i][e] = __fmul2_rn(o[i][e], a2);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < STEPS; ++u) {
+    const int t = u * TPW + tg;
+    const bool valid = t < nvalid;
+    const float p = valid ? exp2f(__fsub_rn(sc[u], m_new)) : 0.f;
+    l = __fadd_rn(l, p);
+    float pa[G];
+    all_gather<G, LPT>(p, dl, pa);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      float2 vf[4];
+      unpack8x2(ld_shared_v4(vb + (uint32_t)((t * D + 8 * (dl + v * LPT)) * 2)), vf);
+      if (valid) {
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          const float2 p2 = make_float2(pa[i], pa[i]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[i][4 * v + e] = __ffma2_rn(p2, vf[e], o[i][4 * v + e]);
+        }
+      }
+    }
+  }
+  m = m_new;
+}
+
+// Merges the warp's token groups (fixed xor tree) and writes split slot f's
+// unnormalised o[D] and (m, l) for the G query heads of kv-head g.
+template <int D, int G>
+__device__ __forceinline__ void store_split(float m, float l, float2 (&o)[G][SplitCfg<D, G>::DPL / 2], int tg, int dl,
+                                            int f, int Hq, int g, float* __restrict__ po,
+                                            float2* __restrict__ pml) {
+  using T = SplitLanes<D, G>;
+  constexpr int NV = T::NV, LPT = T::LPT, DPL = T::DPL, HEAD_LANES = T::HEAD_LANES;
+#pragma unroll
+  for (int o2 = LPT; o2 < 32; o2 <<= 1) {
+    l = __fadd_rn(l, __shfl_xor_sync(kFullMask, l, o2));
+#pragma unroll
+    for (int i = 0; i < G; ++i)
+#pragma unroll
+      for (int e = 0; e < DPL / 2; ++e) {
+        const float2 other = make_float2(__shfl_xor_sync(kFullMask, o[i][e].x, o2),
+                                         __shfl_xor_sync(kFullMask, o[i][e].y, o2));
+        o[i][e] = __fadd2_rn(o[i][e], other);
+      }
+  }
+  if (tg == 0) {
+#pragma unroll
+    for (int i = 0; i < G; ++i)
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        float4* dst = reinterpret_cast<float4*>(po + ((int64_t)f * Hq + g * G + i) * D + 8 * (dl + v * LPT));
+        dst[0] = make_float4(o[i][4 * v + 0].x, o[i][4 * v + 0].y, o[i][4 * v + 1].x, o[i][4 * v + 1].y);
+        dst[1] = make_float4(o[i][4 * v + 2].x, o[i][4 * v + 2].y, o[i][4 * v + 3].x, o[i][4 * v + 3].y);
+      }
+    if (dl % HEAD_LANES == 0) pml[(int64_t)f * Hq + g * G + dl / HEAD_LANES] = make_float2(m, l);
+  }
+}
+
+// One warp per (row, kv-head g, split): writes the split's (m, l) per query head
+// and its unnormalised o[D] per query head into the workspace. Each warp streams
+// its split's pages through its own ring of NST stages.
+template <int D, int G>
 __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
     attn_split_kernel(const uint16_t* __restrict__ q, int64_t ldq, int Hq, int Hkv, const uint16_t* __restrict__ kc,
                       const uint16_t* __restrict__ vc, int64_t num_pages, const int32_t* __restrict__ pt,
                       Rows R, int nrows, const int32_t* __restrict__ off, float* __restrict__ po,
                       float2* __restrict__ pml, float c) {
-  constexpr int DPL = SplitCfg<D, G>::DPL, WARPS = SplitCfg<D, G>::WARPS, NST = SplitCfg<D, G>::NST;
-  constexpr int NV = DPL / 8;       // 16-byte vectors per lane per token row
-  constexpr int LPT = D / DPL;      // lanes per token
-  constexpr int TPW = 32 / LPT;     // tokens per warp step
-  constexpr int STEPS = PAGE / TPW;
-  constexpr int HEAD_LANES = LPT / G;
-  constexpr int PAGE_BYTES = PAGE * D * 2;
-  constexpr int STAGE_BYTES = 2 * PAGE_BYTES;
+  using T = SplitLanes<D, G>;
+  constexpr int DPL = T::DPL, LPT = T::LPT, PAGE_BYTES = T::PAGE_BYTES, STAGE_BYTES = T::STAGE_BYTES;
+  constexpr int WARPS = SplitCfg<D, G>::WARPS, NST = SplitCfg<D, G>::NST;
   static_assert(G >= 1 && G <= LPT, "group size");
 
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tg = lane / LPT, dl = lane % LPT;
-  const int hd = dl / HEAD_LANES;
   const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * NST * STAGE_BYTES);
   const uint32_t bars = smem_u32(smem) + (uint32_t)(WARPS * NST * STAGE_BYTES + warp * NST * 8);
 
@@ -223,14 +359,7 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
     const int32_t* prow = pt + (int64_t)pt_row * R.max_pages + s * PAGES_PER_SPLIT;
 
     float2 qf[G][DPL / 2];  // dims (2e, 2e+1) of the lane's slice in pair e
-#pragma unroll
-    for (int j = 0; j < G; ++j)
-#pragma unroll
-      for (int v = 0; v < NV; ++v) {
-        const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)r * ldq + (int64_t)(g * G + j) * D +
-                                                              8 * (dl + v * LPT)));
-        unpack8x2(qv, &qf[j][4 * v]);
-      }
+    load_q<D, G>(q, ldq, r, g, dl, qf);
 
     // Lane 0 starts the copy of page j of this split into its ring stage.
     auto issue = [&](int j, uint32_t sq) {
@@ -270,75 +399,8 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
       if (!ok) break;
       const int pg = prow[j];
       const int nvalid = (pg < 0 || pg >= num_pages) ? 0 : min(PAGE, t1 - t0 - j * PAGE);
-      const uint32_t kb = ring + st * STAGE_BYTES, vb = kb + PAGE_BYTES;
-
-      // scores of this page: lane holds the score of its token for head hd
-      float sc[STEPS];
-#pragma unroll
-      for (int u = 0; u < STEPS; ++u) {
-        const int t = u * TPW + tg;
-        // two interleaved FMA chains per head (even / odd dims of the slice), then one add
-        float2 acc[G];
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          float2 kf[4];
-          unpack8x2(ld_shared_v4(kb + (uint32_t)((t * D + 8 * (dl + v * LPT)) * 2)), kf);
-#pragma unroll
-          for (int i = 0; i < G; ++i) {
-            float2 a = v == 0 ? __fmul2_rn(qf[i][0], kf[0]) : __ffma2_rn(qf[i][4 * v], kf[0], acc[i]);
-#pragma unroll
-            for (int e = 1; e < 4; ++e) a = __ffma2_rn(qf[i][4 * v + e], kf[e], a);
-            acc[i] = a;
-          }
-        }
-        float part[G];
-#pragma unroll
-        for (int i = 0; i < G; ++i) part[i] = __fadd_rn(acc[i].x, acc[i].y);
-        const float dot = reduce_scatter<G, LPT>(part, dl);
-        sc[u] = t < nvalid ? __fmul_rn(dot, c) : -INFINITY;
-      }
-      float pm = sc[0];
-#pragma unroll
-      for (int u = 1; u < STEPS; ++u) pm = fmaxf(pm, sc[u]);
-#pragma unroll
-      for (int o2 = LPT; o2 < 32; o2 <<= 1) pm = fmaxf(pm, __shfl_xor_sync(kFullMask, pm, o2));
-      const float m_new = fmaxf(m, pm);
-      const float alpha = m_new == -INFINITY ? 1.f : exp2f(__fsub_rn(m, m_new));
-      // rescale the running sums; skipped when no head's max moved (x * 1 == x exactly)
-      if (!__all_sync(kFullMask, alpha == 1.f)) {
-        l = __fmul_rn(l, alpha);
-        float al[G];
-        all_gather<G, LPT>(alpha, dl, al);
-#pragma unroll
-        for (int i = 0; i < G; ++i) {
-          const float2 a2 = make_float2(al[i], al[i]);
-#pragma unroll
-          for (int e = 0; e < DPL / 2; ++e) o[i][e] = __fmul2_rn(o[i][e], a2);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < STEPS; ++u) {
-        const int t = u * TPW + tg;
-        const bool valid = t < nvalid;
-        const float p = valid ? exp2f(__fsub_rn(sc[u], m_new)) : 0.f;
-        l = __fadd_rn(l, p);
-        float pa[G];
-        all_gather<G, LPT>(p, dl, pa);
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          float2 vf[4];
-          unpack8x2(ld_shared_v4(vb + (uint32_t)((t * D + 8 * (dl + v * LPT)) * 2)), vf);
-          if (valid) {
-#pragma unroll
-            for (int i = 0; i < G; ++i) {
-              const float2 p2 = make_float2(pa[i], pa[i]);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) o[i][4 * v + e] = __ffma2_rn(p2, vf[e], o[i][4 * v + e]);
-            }
-          }
-        }
-      }
-      m = m_new;
+      const uint32_t kb = ring + st * STAGE_BYTES;
+      fold_page<D, G>(qf, kb, kb + PAGE_BYTES, nvalid, c, tg, dl, m, l, o);
       __syncwarp();
       if (lane == 0 && j + NST < np) {
         fence_proxy_async_smem();
@@ -350,31 +412,7 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
       __syncwarp();
       return;
     }
-
-    // Merge the token groups of the warp (fixed xor tree).
-#pragma unroll
-    for (int o2 = LPT; o2 < 32; o2 <<= 1) {
-      l = __fadd_rn(l, __shfl_xor_sync(kFullMask, l, o2));
-#pragma unroll
-      for (int i = 0; i < G; ++i)
-#pragma unroll
-        for (int e = 0; e < DPL / 2; ++e) {
-          const float2 other = make_float2(__shfl_xor_sync(kFullMask, o[i][e].x, o2),
-                                           __shfl_xor_sync(kFullMask, o[i][e].y, o2));
-          o[i][e] = __fadd2_rn(o[i][e], other);
-        }
-    }
-    if (tg == 0) {
-#pragma unroll
-      for (int i = 0; i < G; ++i)
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          float4* dst = reinterpret_cast<float4*>(po + ((int64_t)f * Hq + g * G + i) * D + 8 * (dl + v * LPT));
-          dst[0] = make_float4(o[i][4 * v + 0].x, o[i][4 * v + 0].y, o[i][4 * v + 1].x, o[i][4 * v + 1].y);
-          dst[1] = make_float4(o[i][4 * v + 2].x, o[i][4 * v + 2].y, o[i][4 * v + 3].x, o[i][4 * v + 3].y);
-        }
-      if (dl % HEAD_LANES == 0) pml[(int64_t)f * Hq + g * G + hd] = make_float2(m, l);
-    }
+    store_split<D, G>(m, l, o, tg, dl, f, Hq, g, po, pml);
   }
 }
 

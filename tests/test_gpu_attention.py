@@ -155,6 +155,29 @@ def test_prefill_row_equals_decode_row():
         assert same_bits(dec[0], pre[p]), p
 
 
+@pytest.mark.parametrize("Hq,Hkv,D", [(32, 8, 128), (32, 4, 64), (8, 1, 128)])
+def test_prefill_rows_in_any_order_and_mix(Hq, Hkv, D):
+    """Rows of three sequences in sequence order, then in a seeded shuffle (the
+    prefill kernel's windows of consecutive rows then mix sequences, so rows that
+    share a page-table row are scattered): every row keeps its bits, and equals the
+    decode of that row."""
+    lens = [300, 37, 530]
+    q, qs, qp, kv = synth.prefill_inputs(lens, Hq, Hkv, D, seed=80 + D)
+    kvd = _to_dev(kv)
+    qd, qsd, qpd = q.to(dev()), qs.to(dev()), qp.to(dev())
+    ordered = _prefill(qd, qsd, qpd, kvd)
+    perm = synth.permutation(q.shape[0], 81).to(dev())
+    shuffled = _prefill(qd[perm].contiguous(), qsd[perm].contiguous(), qpd[perm].contiguous(), kvd)
+    assert same_bits(shuffled, ordered[perm])
+    for row in (0, 299, 300, 336, 337, 600, 866):
+        b, p = int(qs[row]), int(qp[row])
+        n = torch.tensor([p + 1], dtype=torch.int32, device=dev())
+        dec = bi.attention_decode(qd[row:row + 1].contiguous(), kvd.k_cache, kvd.v_cache,
+                                  kvd.page_table[b:b + 1].contiguous(), n)
+        assert same_bits(dec[0], ordered[row]), row
+    assert bi.get_device_error() == 0
+
+
 def test_prefill_whole_equals_chunked_with_appends():
     # Whole: every token's K/V written, then one prefill call over all rows.
     # Chunked: the store starts empty (NaN); for each chunk its K/V are appended,
