@@ -698,7 +698,7 @@ def run_sweep(bi, device, pk):
 # ---------------------------------------------------------------------------
 
 
-PROFILE_CASES = ("decode_b16", "decode_b1", "prefill_s4096", "rmsnorm", "lmhead_m4", "matmul_small")
+PROFILE_CASES = ("decode_b16", "decode_b1", "prefill_s4096", "rmsnorm", "lmhead_m4", "lmhead_m64", "matmul_small")
 
 
 def profile_case(bi, device, name):
@@ -709,6 +709,8 @@ def profile_case(bi, device, name):
     prefill of one 4096-token sequence on the CUDA cores; rmsnorm = RMSNorm at 65536 x 4096
     then 2048 x 4096; lmhead_m4 = the LM head at 4 rows, V = 32000, K = 2048, with no
     near-tie and with one (then the cuBLAS matmul + argmax of the same shapes);
+    lmhead_m64 = the LM head at 64 rows, V = 32000, K = 2048, random N(0, 0.02) weights
+    (53 rows flagged);
     matmul_small = bi_matmul at M = 1 and 128, K = N = 4096."""
     if name == "decode_b16":
         lens = synth.decode_lengths(16, 32768, seed=50)
@@ -735,6 +737,14 @@ def profile_case(bi, device, name):
         ws = torch.empty(bi.attention_workspace_size(S, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
         for _ in range(2):
             bi.attention_prefill(q, qs, qpos, kv.k_cache, kv.v_cache, kv.page_table, out=o, workspace=ws)
+    elif name == "lmhead_m64":
+        h = synth.normal_bf16((64, 2048), 70).to(device)
+        Wl = synth.normal_bf16((32000, 2048), 71, std=0.02).to(device)
+        tok = torch.empty(64, dtype=torch.int32, device=device)
+        rec = torch.empty(64, dtype=torch.int32, device=device)
+        wsl = torch.empty(bi.lmhead_workspace_size(64, 32000), dtype=torch.uint8, device=device)
+        for _ in range(3):
+            bi.lmhead_argmax(h, Wl, 0.5, tokens=tok, recomputed=rec, workspace=wsl)
     elif name == "rmsnorm":
         for M in (65536, 2048):
             x = synth.normal_bf16_device((M, K_HIDDEN), 15, device)
