@@ -163,9 +163,12 @@ constexpr int split_smem_bytes() {
   return SplitCfg<D, G>::WARPS * SplitCfg<D, G>::NST * (2 * PAGE * D * 2 + 8);
 }
 
-// Per-warp state of one (row, kv-head, split) reduction and the three steps that
-// both the decode kernel and the prefill window kernel run on it, so that a row's
-// arithmetic is the same code whichever kernel reduces it.
+// The steps that reduce one (row, kv-head, split) for GW of the kv-head's G query
+// heads on one warp: load the heads' query slices, fold pages, store the partials.
+// The lane layout (SplitLanes) depends on D and G only, never on GW, and a head's
+// q.k is summed by the same lanes in the same xor pairing whether its warp carries
+// 1, 2, 4 or G heads (reduce_scatter pairs the same lanes at every level; a lane
+// only drops the heads it does not keep), so a head's bits do not depend on GW.
 //
 // Lane layout: the LPT = D/DPL lanes of a token own DPL dims each, in 16-byte
 // vectors v = 0..DPL/8-1 covering dims 8*(dl + v*LPT) .. +7 (interleaved so a
@@ -178,21 +181,20 @@ struct SplitLanes {
   static constexpr int LPT = D / DPL;  // lanes per token
   static constexpr int TPW = 32 / LPT; // tokens per warp step
   static constexpr int STEPS = PAGE / TPW;
-  static constexpr int HEAD_LANES = LPT / G;
   static constexpr int PAGE_BYTES = PAGE * D * 2;
   static constexpr int STAGE_BYTES = 2 * PAGE_BYTES;
 };
 
-// The lane's slice of the G query heads that share kv-head g, row r.
-template <int D, int G>
-__device__ __forceinline__ void load_q(const uint16_t* __restrict__ q, int64_t ldq, int r, int g, int dl,
-                                       float2 (&qf)[G][SplitCfg<D, G>::DPL / 2]) {
+// The lane's slice of query heads h0 .. h0+GW-1 of row r.
+template <int D, int G, int GW>
+__device__ __forceinline__ void load_q(const uint16_t* __restrict__ q, int64_t ldq, int r, int h0, int dl,
+                                       float2 (&qf)[GW][SplitCfg<D, G>::DPL / 2]) {
   using T = SplitLanes<D, G>;
 #pragma unroll
-  for (int j = 0; j < G; ++j)
+  for (int j = 0; j < GW; ++j)
 #pragma unroll
     for (int v = 0; v < T::NV; ++v) {
-      const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)r * ldq + (int64_t)(g * G + j) * D +
+      const uint4 qv = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)r * ldq + (int64_t)(h0 + j) * D +
                                                             8 * (dl + v * T::LPT)));
       unpack8x2(qv, &qf[j][4 * v]);
     }
@@ -201,35 +203,35 @@ __device__ __forceinline__ void load_q(const uint16_t* __restrict__ q, int64_t l
 // Folds one page (K at kb, V at vb in shared memory, its first nvalid tokens
 // visible) into the running (m, l, o) of the lane's head: scores, the base-2
 // online-softmax rescale, then p * V.
-template <int D, int G>
-__device__ __forceinline__ void fold_page(const float2 (&qf)[G][SplitCfg<D, G>::DPL / 2], uint32_t kb, uint32_t vb,
+template <int D, int G, int GW>
+__device__ __forceinline__ void fold_page(const float2 (&qf)[GW][SplitCfg<D, G>::DPL / 2], uint32_t kb, uint32_t vb,
                                           int nvalid, float c, int tg, int dl, float& m, float& l,
-                                          float2 (&o)[G][SplitCfg<D, G>::DPL / 2]) {
+                                          float2 (&o)[GW][SplitCfg<D, G>::DPL / 2]) {
   using T = SplitLanes<D, G>;
   constexpr int NV = T::NV, LPT = T::LPT, TPW = T::TPW, STEPS = T::STEPS, DPL = T::DPL;
-  // scores of this page: lane holds the score of its token for head hd
+  // scores of this page: lane holds the score of its token for its head
   float sc[STEPS];
 #pragma unroll
   for (int u = 0; u < STEPS; ++u) {
     const int t = u * TPW + tg;
     // two interleaved FMA chains per head (even / odd dims of the slice), then one add
-    float2 acc[G];
+    float2 acc[GW];
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
       float2 kf[4];
       unpack8x2(ld_shared_v4(kb + (uint32_t)((t * D + 8 * (dl + v * LPT)) * 2)), kf);
 #pragma unroll
-      for (int i = 0; i < G; ++i) {
+      for (int i = 0; i < GW; ++i) {
         float2 a = v == 0 ? __fmul2_rn(qf[i][0], kf[0]) : __ffma2_rn(qf[i][4 * v], kf[0], acc[i]);
 #pragma unroll
         for (int e = 1; e < 4; ++e) a = __ffma2_rn(qf[i][4 * v + e], kf[e], a);
         acc[i] = a;
       }
     }
-    float part[G];
+    float part[GW];
 #pragma unroll
-    for (int i = 0; i < G; ++i) part[i] = __fadd_rn(acc[i].x, acc[i].y);
-    const float dot = reduce_scatter<G, LPT>(part, dl);
+    for (int i = 0; i < GW; ++i) part[i] = __fadd_rn(acc[i].x, acc[i].y);
+    const float dot = reduce_scatter<GW, LPT>(part, dl);
     sc[u] = t < nvalid ? __fmul_rn(dot, c) : -INFINITY;
   }
   float pm = sc[0];
@@ -242,10 +244,10 @@ __device__ __forceinline__ void fold_page(const float2 (&qf)[G][SplitCfg<D, G>::
   // rescale the running sums; skipped when no head's max moved (x * 1 == x exactly)
   if (!__all_sync(kFullMask, alpha == 1.f)) {
     l = __fmul_rn(l, alpha);
-    float al[G];
-    all_gather<G, LPT>(alpha, dl, al);
+    float al[GW];
+    all_gather<GW, LPT>(alpha, dl, al);
 #pragma unroll
-    for (int i = 0; i < G; ++i) {
+    for (int i = 0; i < GW; ++i) {
       const float2 a2 = make_float2(al[i], al[i]);
 #pragma unroll
       for (int e = 0; e < DPL / 2; ++e) o[i][e] = __fmul2_rn(o[i][e], a2);
@@ -257,15 +259,15 @@ __device__ __forceinline__ void fold_page(const float2 (&qf)[G][SplitCfg<D, G>::
     const bool valid = t < nvalid;
     const float p = valid ? exp2f(__fsub_rn(sc[u], m_new)) : 0.f;
     l = __fadd_rn(l, p);
-    float pa[G];
-    all_gather<G, LPT>(p, dl, pa);
+    float pa[GW];
+    all_gather<GW, LPT>(p, dl, pa);
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
       float2 vf[4];
       unpack8x2(ld_shared_v4(vb + (uint32_t)((t * D + 8 * (dl + v * LPT)) * 2)), vf);
       if (valid) {
 #pragma unroll
-        for (int i = 0; i < G; ++i) {
+        for (int i = 0; i < GW; ++i) {
           const float2 p2 = make_float2(pa[i], pa[i]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) o[i][4 * v + e] = __ffma2_rn(p2, vf[e], o[i][4 * v + e]);
@@ -277,18 +279,18 @@ __device__ __forceinline__ void fold_page(const float2 (&qf)[G][SplitCfg<D, G>::
 }
 
 // Merges the warp's token groups (fixed xor tree) and writes split slot f's
-// unnormalised o[D] and (m, l) for the G query heads of kv-head g.
-template <int D, int G>
-__device__ __forceinline__ void store_split(float m, float l, float2 (&o)[G][SplitCfg<D, G>::DPL / 2], int tg, int dl,
-                                            int f, int Hq, int g, float* __restrict__ po,
+// unnormalised o[D] and (m, l) for query heads h0 .. h0+GW-1.
+template <int D, int G, int GW>
+__device__ __forceinline__ void store_split(float m, float l, float2 (&o)[GW][SplitCfg<D, G>::DPL / 2], int tg,
+                                            int dl, int f, int Hq, int h0, float* __restrict__ po,
                                             float2* __restrict__ pml) {
   using T = SplitLanes<D, G>;
-  constexpr int NV = T::NV, LPT = T::LPT, DPL = T::DPL, HEAD_LANES = T::HEAD_LANES;
+  constexpr int NV = T::NV, LPT = T::LPT, DPL = T::DPL, HEAD_LANES = LPT / GW;
 #pragma unroll
   for (int o2 = LPT; o2 < 32; o2 <<= 1) {
     l = __fadd_rn(l, __shfl_xor_sync(kFullMask, l, o2));
 #pragma unroll
-    for (int i = 0; i < G; ++i)
+    for (int i = 0; i < GW; ++i)
 #pragma unroll
       for (int e = 0; e < DPL / 2; ++e) {
         const float2 other = make_float2(__shfl_xor_sync(kFullMask, o[i][e].x, o2),
@@ -298,52 +300,44 @@ __device__ __forceinline__ void store_split(float m, float l, float2 (&o)[G][Spl
   }
   if (tg == 0) {
 #pragma unroll
-    for (int i = 0; i < G; ++i)
+    for (int i = 0; i < GW; ++i)
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        float4* dst = reinterpret_cast<float4*>(po + ((int64_t)f * Hq + g * G + i) * D + 8 * (dl + v * LPT));
+        float4* dst = reinterpret_cast<float4*>(po + ((int64_t)f * Hq + h0 + i) * D + 8 * (dl + v * LPT));
         dst[0] = make_float4(o[i][4 * v + 0].x, o[i][4 * v + 0].y, o[i][4 * v + 1].x, o[i][4 * v + 1].y);
         dst[1] = make_float4(o[i][4 * v + 2].x, o[i][4 * v + 2].y, o[i][4 * v + 3].x, o[i][4 * v + 3].y);
       }
-    if (dl % HEAD_LANES == 0) pml[(int64_t)f * Hq + g * G + dl / HEAD_LANES] = make_float2(m, l);
+    if (dl % HEAD_LANES == 0) pml[(int64_t)f * Hq + h0 + dl / HEAD_LANES] = make_float2(m, l);
   }
 }
 
-// One warp per (row, kv-head g, split): writes the split's (m, l) per query head
-// and its unnormalised o[D] per query head into the workspace. Each warp streams
-// its split's pages through its own ring of NST stages.
-template <int D, int G>
-__global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
-    attn_split_kernel(const uint16_t* __restrict__ q, int64_t ldq, int Hq, int Hkv, const uint16_t* __restrict__ kc,
-                      const uint16_t* __restrict__ vc, int64_t num_pages, const int32_t* __restrict__ pt,
-                      Rows R, int nrows, const int32_t* __restrict__ off, float* __restrict__ po,
-                      float2* __restrict__ pml, float c) {
+// Per-warp ring state of the split kernel: pages consumed so far (the ring position)
+// and, for lane 0, the stages it filled and their phase parities (for drain_copies).
+struct RingState {
+  uint32_t seq, issued, ph_bits;
+};
+
+// The split kernel's work loop for GW query heads per warp: items are (split slot f,
+// kv-head g, head part hp) with heads g*G + hp*GW .. +GW-1, dealt across CTAs first
+// (item = warp * gridDim.x + CTA) so that a launch with fewer items than warp slots
+// spreads them over every SM. Returns false if a copy never landed.
+template <int D, int G, int GW>
+__device__ __forceinline__ bool split_items(const uint16_t* __restrict__ q, int64_t ldq, int Hq, int Hkv,
+                                            const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc,
+                                            int64_t num_pages, const int32_t* __restrict__ pt, const Rows& R,
+                                            int nrows, const int32_t* __restrict__ off, float* __restrict__ po,
+                                            float2* __restrict__ pml, float c, int total, uint32_t ring,
+                                            uint32_t bars, RingState& rs) {
   using T = SplitLanes<D, G>;
   constexpr int DPL = T::DPL, LPT = T::LPT, PAGE_BYTES = T::PAGE_BYTES, STAGE_BYTES = T::STAGE_BYTES;
-  constexpr int WARPS = SplitCfg<D, G>::WARPS, NST = SplitCfg<D, G>::NST;
-  static_assert(G >= 1 && G <= LPT, "group size");
-
-  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int WARPS = SplitCfg<D, G>::WARPS, NST = SplitCfg<D, G>::NST, HP = G / GW;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tg = lane / LPT, dl = lane % LPT;
-  const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * NST * STAGE_BYTES);
-  const uint32_t bars = smem_u32(smem) + (uint32_t)(WARPS * NST * STAGE_BYTES + warp * NST * 8);
-
-  if (lane == 0) {
-    for (int s = 0; s < NST; ++s) mbar_init(bars + 8 * s, 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
-
-  const int total = off[nrows] * Hkv;
   const int64_t kv_head_stride = (int64_t)PAGE * D;
-  uint32_t seq = 0;  // pages this warp has consumed so far
-  uint32_t issued = 0, ph_bits = 0;  // lane 0: ring stages filled and their phase parities
-
-  // items are dealt across CTAs first (item = warp * gridDim.x + CTA), so that a
-  // launch with fewer items than warp slots spreads them over every SM
-  for (int item = warp * gridDim.x + blockIdx.x; item < total; item += gridDim.x * WARPS) {
-    const int f = item / Hkv, g = item - (item / Hkv) * Hkv;
+  for (int item = warp * gridDim.x + blockIdx.x; item < total * HP; item += gridDim.x * WARPS) {
+    const int fg = item / HP, hp = item - (item / HP) * HP;
+    const int f = fg / Hkv, g = fg - (fg / Hkv) * Hkv;
+    const int h0 = g * G + hp * GW;
     int lo = 0, hi = nrows;  // off[lo] <= f < off[hi]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -358,8 +352,8 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
     const int np = (t1 - t0 + PAGE - 1) / PAGE;
     const int32_t* prow = pt + (int64_t)pt_row * R.max_pages + s * PAGES_PER_SPLIT;
 
-    float2 qf[G][DPL / 2];  // dims (2e, 2e+1) of the lane's slice in pair e
-    load_q<D, G>(q, ldq, r, g, dl, qf);
+    float2 qf[GW][DPL / 2];  // dims (2e, 2e+1) of the lane's slice in pair e
+    load_q<D, G, GW>(q, ldq, r, h0, dl, qf);
 
     // Lane 0 starts the copy of page j of this split into its ring stage.
     auto issue = [&](int j, uint32_t sq) {
@@ -367,7 +361,7 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
       const uint32_t bar = bars + 8 * st;
       const int pg = prow[j];
       const int nvalid = min(PAGE, t1 - t0 - j * PAGE);
-      note_fill(issued, ph_bits, (int)st, (sq / NST) & 1u);
+      note_fill(rs.issued, rs.ph_bits, (int)st, (sq / NST) & 1u);
       if (pg < 0 || pg >= num_pages) {
         record_error(BI_ERR_DEVICE_INDEX);
         mbar_arrive_expect_tx(bar, 0);
@@ -382,37 +376,78 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
     };
     if (lane == 0) {
       fence_proxy_async_smem();
-      for (int j = 0; j < NST && j < np; ++j) issue(j, seq + j);
+      for (int j = 0; j < NST && j < np; ++j) issue(j, rs.seq + j);
     }
 
     float m = -INFINITY, l = 0.f;
-    float2 o[G][DPL / 2];
+    float2 o[GW][DPL / 2];
 #pragma unroll
-    for (int j = 0; j < G; ++j)
+    for (int j = 0; j < GW; ++j)
 #pragma unroll
       for (int e = 0; e < DPL / 2; ++e) o[j][e] = make_float2(0.f, 0.f);
 
-    bool ok = true;
-    for (int j = 0; j < np; ++j, ++seq) {
-      const uint32_t st = seq % NST;
-      ok = __all_sync(kFullMask, mbar_wait(bars + 8 * st, (seq / NST) & 1u));
-      if (!ok) break;
+    for (int j = 0; j < np; ++j, ++rs.seq) {
+      const uint32_t st = rs.seq % NST;
+      if (!__all_sync(kFullMask, mbar_wait(bars + 8 * st, (rs.seq / NST) & 1u))) return false;
       const int pg = prow[j];
       const int nvalid = (pg < 0 || pg >= num_pages) ? 0 : min(PAGE, t1 - t0 - j * PAGE);
       const uint32_t kb = ring + st * STAGE_BYTES;
-      fold_page<D, G>(qf, kb, kb + PAGE_BYTES, nvalid, c, tg, dl, m, l, o);
+      fold_page<D, G, GW>(qf, kb, kb + PAGE_BYTES, nvalid, c, tg, dl, m, l, o);
       __syncwarp();
       if (lane == 0 && j + NST < np) {
         fence_proxy_async_smem();
-        issue(j + NST, seq + NST);
+        issue(j + NST, rs.seq + NST);
       }
     }
-    if (!ok) {  // a copy never landed: error recorded; let this warp's other copies land, then leave
-      if (lane == 0) drain_copies(bars, 8, issued, ph_bits);
-      __syncwarp();
-      return;
-    }
-    store_split<D, G>(m, l, o, tg, dl, f, Hq, g, po, pml);
+    store_split<D, G, GW>(m, l, o, tg, dl, f, Hq, h0, po, pml);
+  }
+  return true;
+}
+
+// One warp per (row, kv-head g, split) -- or per (row, kv-head, split, half or quarter
+// of the G query heads) when the batch's items would fill at most half (a quarter) of
+// the warp slots: writes the split's (m, l) and unnormalised o[D] per query head into
+// the workspace. Each warp streams its split's pages through its own ring of NST
+// stages. How the heads are spread over warps is a launch shape: every head's
+// arithmetic is the same (see split_items).
+template <int D, int G>
+__global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
+    attn_split_kernel(const uint16_t* __restrict__ q, int64_t ldq, int Hq, int Hkv, const uint16_t* __restrict__ kc,
+                      const uint16_t* __restrict__ vc, int64_t num_pages, const int32_t* __restrict__ pt,
+                      Rows R, int nrows, const int32_t* __restrict__ off, float* __restrict__ po,
+                      float2* __restrict__ pml, float c) {
+  using T = SplitLanes<D, G>;
+  constexpr int LPT = T::LPT, STAGE_BYTES = T::STAGE_BYTES;
+  constexpr int WARPS = SplitCfg<D, G>::WARPS, NST = SplitCfg<D, G>::NST;
+  static_assert(G >= 1 && G <= LPT, "group size");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ring = smem_u32(smem) + (uint32_t)(warp * NST * STAGE_BYTES);
+  const uint32_t bars = smem_u32(smem) + (uint32_t)(WARPS * NST * STAGE_BYTES + warp * NST * 8);
+
+  if (lane == 0) {
+    for (int s = 0; s < NST; ++s) mbar_init(bars + 8 * s, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  const int total = off[nrows] * Hkv;  // (split slot, kv-head) items
+  const int64_t slots = (int64_t)gridDim.x * WARPS;
+  RingState rs{0u, 0u, 0u};
+  bool ok;
+  if (G >= 4 && (int64_t)total * 4 <= slots)
+    ok = split_items<D, G, (G >= 4 ? G / 4 : G)>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, off, po, pml, c,
+                                                 total, ring, bars, rs);
+  else if (G >= 2 && (int64_t)total * 2 <= slots)
+    ok = split_items<D, G, (G >= 2 ? G / 2 : G)>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, off, po, pml, c,
+                                                 total, ring, bars, rs);
+  else
+    ok = split_items<D, G, G>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, off, po, pml, c, total, ring, bars,
+                              rs);
+  if (!ok) {  // a copy never landed: error recorded; let this warp's other copies land, then leave
+    if (lane == 0) drain_copies(bars, 8, rs.issued, rs.ph_bits);
+    __syncwarp();
   }
 }
 

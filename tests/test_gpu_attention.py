@@ -99,6 +99,25 @@ def test_decode_batch_invariant_and_run_to_run():
     assert same_bits(outp, full[perm])
 
 
+def test_decode_heads_per_warp_do_not_change_bits():
+    """Decode reduces a (row, kv-head, split) with all 4 query heads of the kv-head on
+    one warp when the batch's items fill the GPU, with 2 or 1 per warp when they fill
+    at most a half or a quarter of it (on a 148-SM B200: 8 rows of 4096 tokens take
+    4 per warp, 5 of them 2, 3 of them 1). Every head's bits are the same."""
+    lens = [4096] * 8
+    q, kv = synth.decode_inputs(8, 32, 8, 128, max_len=4096, seed=90, lens=lens)
+    qd, kvd = q.to(dev()), _to_dev(kv)
+    full = _decode(qd, kvd)
+    for sub in ([0, 2, 4, 6, 7], [1, 3, 5], [6]):
+        s = torch.tensor(sub, device=dev())
+        part = bi.attention_decode(qd[s].contiguous(), kvd.k_cache, kvd.v_cache, kvd.page_table[s].contiguous(),
+                                   kvd.seq_lens[s].contiguous())
+        assert same_bits(part, full[s]), sub
+    kv_sub = synth.PagedKV(kv.k_cache, kv.v_cache, kv.page_table[[6]], kv.seq_lens[[6]], kv.max_pages)
+    assert max_rel(full[6:7], _oracle_decode(q[6:7], kv_sub)) <= TOL_BF16
+    assert bi.get_device_error() == 0
+
+
 @pytest.mark.parametrize("D", [128, 64])
 def test_decode_combine_width_does_not_change_bits(D):
     """96 sequences x 32 heads fold their splits with D / 32 (or D / 64) dims per
