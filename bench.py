@@ -892,7 +892,10 @@ def run_ours(args, rank, world, local):
         "config": ours_config(wl.M, world),
         "roofline": roof,
         "rmsnorm_in_step": {"GB/s": round(wl.rms_bytes / rms_ms / 1e6, 1), "ms": round(rms_ms, 4),
-                            "note": "16 MiB in + 16 MiB out per launch"},
+                            "note": ("16 MiB in + 16 MiB out per launch, one event pair per launch inside the "
+                                     "step: it includes the event gaps and the write-back of the previous step's "
+                                     "matmul outputs (up to 96 MiB of dirty lines) that its reads evict from L2; "
+                                     "the launch on its own is sweeps.rmsnorm_k4096 at M = 2048")},
         "slowdown_vs_noninvariant": round((ms_total / args.steps) / (ref_ms / args.steps), 3),
         "noninvariant_ms_per_step": round(ref_ms / args.steps, 4),
         "e2e": {"value": round(e2e_units / (e2e_max / 1e3) / 1e12, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
