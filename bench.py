@@ -582,10 +582,10 @@ def _copies(nbytes_one, floor=384 << 20, cap=64):
 
 
 # tcgen05 dependent-accumulation step: one 128 x N x 16 MMA into the accumulator the
-# previous one wrote costs about 83 SM cycles for N <= 128 and 130 for N = 256
-# (measured on this B200 with probes/mma_chain.cu). Every output tile is one such
-# chain of K/16 MMAs, so no tile finishes in less than K/16 steps.
-MMA_CHAIN_CYCLES = {32: 83.0, 64: 83.0, 128: 83.0, 256: 130.0}
+# previous one wrote costs about 83 SM cycles for N <= 128, 98 for N = 192 and 130
+# for N = 256 (measured on this B200 with probes/mma_chain.cu). Every output tile is
+# one such chain of K/16 MMAs, so no tile finishes in less than K/16 steps.
+MMA_CHAIN_CYCLES = {32: 83.0, 64: 83.0, 128: 83.0, 192: 97.6, 256: 130.0}
 
 
 def sweep_matmul(bi, device, pk, clocks_mhz, ms_list=M_SWEEP, calls=12):

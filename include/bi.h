@@ -108,7 +108,7 @@ bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw
                     int64_t ldc, int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
- * Tile width (32, 64, 128 or 256 columns) that bi_matmul uses for an M x N
+ * Tile width (32, 64, 128, 192 or 256 columns) that bi_matmul uses for an M x N
  * product on the current device; -1 if the device cannot be queried or M, N < 0.
  * Narrow tiles spread a small-M product over more SMs (each streams a thin slice
  * of W); wide tiles reuse each block of A for more columns at large M. The choice

@@ -16,12 +16,13 @@
 // (a row alone equals the row at every tile position; every row of the M = 1..2048
 // sweep equals the same row of the 2048-row product).
 //
-// The tile width BN (32, 64, 128 or 256 columns) only decides how the N columns
-// are dealt out to CTAs. A narrow tile gives many CTAs when M is small (each CTA
-// then streams a thin slice of W, so more SMs pull W from HBM at once); a wide tile
-// reads each A block from shared memory for more columns when M is large. The host
-// picks the width from the tile counts (pick_bn); the width is not part of an
-// element's arithmetic, so the choice cannot change a bit (tested over the sweep).
+// The tile width BN (32, 64, 128, 192 or 256 columns) only decides how the N columns
+// are dealt out to CTAs. A narrow tile gives many CTAs when M is small (each CTA then
+// streams a thin slice of W, so more SMs pull W from HBM at once); a wide tile reads
+// each A block from shared memory for more columns when M is large; 192 evens out the
+// waves where 256 leaves SMs idle (N = 6144 at M = 512..1024: 8 % faster on a B200).
+// The host picks the width from the tile counts (pick_bn); the width is not part of
+// an element's arithmetic, so the choice cannot change a bit (tested over the sweep).
 //
 // Design (sm_100a):
 //   * K is consumed in 64-wide blocks, each four 128xBNx16 MMAs in ascending k;
@@ -60,11 +61,14 @@ constexpr int kSmemBytes = 227 * 1024;   // dynamic shared memory of every launc
 constexpr int kBarBytes = 8 * (2 * 32 + 4) + 16;  // barriers for up to 32 stages, TMEM slot, flag
 constexpr int kMaxStages = 32;
 
+// Tensor-memory columns allocated for two BN-wide fp32 accumulators: a power of two.
+constexpr int tmem_cols_for(int bn) { return 2 * bn <= 32 ? 32 : 2 * bn <= 64 ? 64 : 2 * bn <= 128 ? 128 : 2 * bn <= 256 ? 256 : 512; }
+
 template <int BN>
 struct Cfg {
-  static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "tcgen05 M=128 tile widths used here");
-  static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int TMEM_COLS = 2 * BN;  // two fp32 accumulators (power of 2 >= 32)
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tcgen05 M=128 tile widths used here");
+  static constexpr int B_BYTES = BN * BK * 2;   // BN rows of 128 bytes: whole 8-row swizzle atoms
+  static constexpr int TMEM_COLS = tmem_cols_for(BN);  // two fp32 accumulators at columns 0 and BN
   // Instruction descriptor for kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 =
   // 1), B bf16 (bits 10-12 = 1), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -388,7 +392,7 @@ inline int pick_bn(int64_t M, int64_t N, int sms) {
   const int64_t rows = a_box_rows(M);
   int best = 256;
   int64_t best_cost = INT64_MAX;
-  for (int bn : {256, 128, 64, 32}) {
+  for (int bn : {256, 192, 128, 64, 32}) {
     const int64_t tiles = mt * ((N + bn - 1) / bn);
     const int64_t waves = (tiles + sms - 1) / sms;
     const int64_t cost = waves * (rows + 128 + 2 * bn);
@@ -473,6 +477,7 @@ inline bi_status launch(const uint16_t* A, int64_t lda, const uint16_t* W, int64
     case 32: return launch_bn<32>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
     case 64: return launch_bn<64>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
     case 128: return launch_bn<128>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
+    case 192: return launch_bn<192>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
     case 256: return launch_bn<256>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
     default: return BI_ERR_UNSUPPORTED;
   }

@@ -1,7 +1,7 @@
 // Chain probe: cycles per tcgen05.mma.kind::f16 (128 x N x 16, bf16 operands in
 // shared memory, fp32 accumulator in tensor memory) when every MMA accumulates into
 // the tile the previous one wrote (one chain), and when 2, 4 or 8 independent
-// accumulators are interleaved, for N = 32, 64, 128, 256. One CTA on one SM; the
+// accumulators are interleaved, for N = 32, 64, 128, 192, 224, 256. One CTA on one SM; the
 // operands are zeros (their values do not change the timing); clock64() around the
 // issue loop and around the completion (tcgen05.commit -> mbarrier).
 //
@@ -98,7 +98,7 @@ int main() {
   long long* d; cudaMalloc(&d, 16);
   cudaFuncSetAttribute(lat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 50 * 1024);
   const int iters = 256;
-  int ns[] = {32, 64, 128, 256};
+  int ns[] = {32, 64, 128, 192, 224, 256};
   for (int unrolled = 0; unrolled < 6; ++unrolled)
     for (int m : {128, 64})
       for (int n : ns)

@@ -69,6 +69,8 @@ def test_matmul_batch_invariant_over_m_sweep(N):
     full = bi.matmul(a, w)
     for m in M_SWEEP:
         assert same_bits(bi.matmul(a[:m].contiguous(), w), full[:m]), m
+    # the sweep crosses tile widths (on a 148-SM B200: 32/64/128/256, and 192 at N = 6144)
+    assert len({bi.matmul_tile_n(m, N) for m in M_SWEEP + [2048]}) >= 2
     # rows in a permuted batch and a batch taken from the middle
     perm = synth.permutation(2048, 25).to(dev())
     assert same_bits(bi.matmul(a[perm].contiguous(), w), full[perm])
