@@ -77,6 +77,8 @@ __device__ __forceinline__ int num_splits(const Rows& R, int r) {
 __global__ void __launch_bounds__(1024) split_offsets_kernel(Rows R, int nrows, int32_t* off) {
   __shared__ int32_t sums[1024];
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const int per = (nrows + 1023) / 1024;
   const int r0 = tid * per;
   const int r1 = min(r0 + per, nrows);
@@ -431,6 +433,8 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
     fence_mbar_init();
   }
   __syncwarp();
+  pdl_wait();  // the offsets (and the caller's q and K/V) are complete from here on
+  pdl_trigger();
 
   const int total = off[nrows] * Hkv;  // (split slot, kv-head) items
   const int64_t slots = (int64_t)gridDim.x * WARPS;
@@ -470,6 +474,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   constexpr int U = 32 / DPL;         // splits whose partial outputs are loaded together
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_wait();  // the split partials are complete from here on
+  pdl_trigger();
   if (w >= nrows * Hq * NG) return;
   const int rh = w / NG, g = w - (w / NG) * NG;
   const int r = rh / Hq, h = rh - (rh / Hq) * Hq;
@@ -544,6 +550,8 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint16_t* __restri
                                                         uint16_t* __restrict__ kc, uint16_t* __restrict__ vc,
                                                         int64_t num_pages, const int32_t* __restrict__ pt,
                                                         int num_seqs, int max_pages, int T, int Hkv, int D) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= (int64_t)T * Hkv) return;

@@ -27,6 +27,32 @@ __device__ int g_error_word = 0;
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_error_word, 0, code); }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched with launch_pdl may start while
+// the previous kernel on the stream is still running; it calls pdl_wait() before its
+// first access to global memory that the previous kernel may write or read, and
+// pdl_wait() returns once that kernel has completed and its writes are visible (at
+// once when there is no such kernel). pdl_trigger() lets the next kernel's CTAs be
+// scheduled before this one ends; they still wait in their own pdl_wait().
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// ---------------------------------------------------------------------------
 // bf16 <-> fp32
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -42,6 +42,9 @@
 //     accumulators let the epilogue of one tile overlap the main loop of the next;
 //   * persistent grid of min(#tiles, #SMs) CTAs; tile t goes to CTA t mod grid,
 //     m-tiles of one W slice on neighbouring CTAs so the slice is read from HBM once;
+//   * launched as a programmatic dependent of the previous kernel on the stream: the
+//     barrier set-up, TMEM allocation and tensor-map prefetch overlap that kernel's
+//     tail, and the TMA thread waits for it (pdl_wait) before the first load;
 //   * every mbarrier wait is bounded; on expiry the kernel records
 //     BI_ERR_DEVICE_TIMEOUT, all roles leave their loops, TMEM is freed.
 #pragma once
@@ -252,9 +255,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   uint32_t issued = 0, ph_bits = 0;  // the producer's filled stages and their phase parities
 
+  if (threadIdx.x == 0) pdl_trigger();
   if (warp == 0) {
-    if (lane == 0)
+    // the previous kernel on the stream (which may write A or W, or read C) must be
+    // done before the first load; the MMA and epilogue warps only follow the loads
+    if (lane == 0) {
+      pdl_wait();
       tma_producer<BN, KPS, COMPACT>(&tmA, &tmB, base, L, bars, tiles, mt, nkb, abort_flag, issued, ph_bits);
+    }
   } else if (warp == 1) {
     if (lane == 0) mma_issuer<BN, KPS, COMPACT>(base, L, bars, tmem, tiles, nkb, abort_flag);
   } else {  // ---- epilogue: warps 2..5; warp w may read TMEM lanes 32*(w%4) .. +31
@@ -448,8 +456,10 @@ inline bi_status launch_kps(const uint16_t* A, int64_t lda, const uint16_t* W, i
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
   const int smem = (int)(1024 + L.bar_offset + kBarBytes);
-  gemm_bf16_kernel<BN, KPS, COMPACT><<<grid, kThreads, smem, st>>>(ta, tb, C, ldc, (int)M, (int)N, (int)K, L);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  return launch_pdl(gemm_bf16_kernel<BN, KPS, COMPACT>, dim3(grid), dim3(kThreads), (size_t)smem, st, ta, tb, C, ldc,
+                    (int)M, (int)N, (int)K, L) == cudaSuccess
+             ? BI_OK
+             : BI_ERR_CUDA;
 }
 
 template <int BN>

@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
                                                           int64_t nrows_src, const int32_t* __restrict__ idx,
                                                           int M, int64_t width, uint16_t* __restrict__ dst,
                                                           int64_t ld_dst) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   const int64_t m = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (m >= M) return;
@@ -41,6 +43,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 __global__ void __launch_bounds__(256) rope_kernel(uint16_t* __restrict__ x, int64_t ldx, int T, int H, int D,
                                                    const int32_t* __restrict__ pos, const float2* __restrict__ table,
                                                    int max_pos) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   const int half = D / 2;
   const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (e >= (int64_t)T * H * half) return;
@@ -67,6 +71,8 @@ __global__ void __launch_bounds__(256) rope_kernel(uint16_t* __restrict__ x, int
 // silu(g) = g / (1 + exp(-g)) in fp32 (expf, then an IEEE division).
 __global__ void __launch_bounds__(256) swiglu_kernel(const uint16_t* __restrict__ gu, int64_t ld_gu,
                                                      uint16_t* __restrict__ out, int64_t ld_out, int M, int F) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;  // one thread per 8 outputs
   const int64_t per_row = F / 8;
   if (e >= (int64_t)M * per_row) return;
@@ -92,6 +98,8 @@ __global__ void __launch_bounds__(256) swiglu_kernel(const uint16_t* __restrict_
 // out = bf16(a + b) elementwise (fp32 add of the two bf16 values), n % 8 == 0.
 // out may alias a or b (each thread reads its 8 elements before writing them).
 __global__ void __launch_bounds__(256) add_kernel(const uint16_t* a, const uint16_t* b, uint16_t* out, int64_t n) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   const int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (e >= n / 8) return;
   float x[8], y[8];

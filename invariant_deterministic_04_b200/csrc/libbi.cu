@@ -90,9 +90,8 @@ cudaError_t launch_split(const uint16_t* q, int64_t ldq, int Hq, int Hkv, const 
   // persistent grid: as many CTAs as can be resident (shared memory or registers
   // limit it); the grid only decides which warp takes which (row, head, split)
   const int grid = device_sms() * per_sm[dev];
-  bi::attn::attn_split_kernel<D, G><<<grid, threads, smem, st>>>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows,
-                                                                 ws.off, ws.po, ws.pml, c);
-  return cudaGetLastError();
+  return bi::launch_pdl(bi::attn::attn_split_kernel<D, G>, dim3(grid), dim3(threads), (size_t)smem, st, q, ldq, Hq, Hkv,
+                    kc, vc, num_pages, pt, R, nrows, (const int32_t*)ws.off, ws.po, ws.pml, c);
 }
 
 template <int D>
@@ -134,8 +133,8 @@ bi_status attention_common(const uint16_t* q, int64_t ldq, const uint16_t* kc, c
   if (ws_bytes < need) return BI_ERR_WORKSPACE;
   if (nrows == 0) return BI_OK;
   const float c = (float)((double)scale * 1.4426950408889634);  // scale * log2(e)
-  bi::attn::split_offsets_kernel<<<1, 1024, 0, st>>>(R, nrows, lay.off);
-  if (cudaGetLastError() != cudaSuccess) return BI_ERR_CUDA;
+  if (bi::launch_pdl(bi::attn::split_offsets_kernel, dim3(1), dim3(1024), 0, st, R, nrows, lay.off) != cudaSuccess)
+    return BI_ERR_CUDA;
   cudaError_t e = D == 128 ? launch_split_g<128>(G, q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st)
                            : launch_split_g<64>(G, q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, lay, c, st);
   if (e != cudaSuccess) return BI_ERR_CUDA;
@@ -148,16 +147,20 @@ bi_status attention_common(const uint16_t* q, int64_t ldq, const uint16_t* kc, c
   const int grid = (warps + 7) / 8;
   if (D == 128) {
     if (narrow)
-      bi::attn::attn_combine_kernel<128, 1><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+      e = bi::launch_pdl(bi::attn::attn_combine_kernel<128, 1>, dim3(grid), dim3(256), 0, st, (const float*)lay.po,
+                     (const float2*)lay.pml, (const int32_t*)lay.off, nrows, Hq, out);
     else
-      bi::attn::attn_combine_kernel<128, 4><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+      e = bi::launch_pdl(bi::attn::attn_combine_kernel<128, 4>, dim3(grid), dim3(256), 0, st, (const float*)lay.po,
+                     (const float2*)lay.pml, (const int32_t*)lay.off, nrows, Hq, out);
   } else {
     if (narrow)
-      bi::attn::attn_combine_kernel<64, 1><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+      e = bi::launch_pdl(bi::attn::attn_combine_kernel<64, 1>, dim3(grid), dim3(256), 0, st, (const float*)lay.po,
+                     (const float2*)lay.pml, (const int32_t*)lay.off, nrows, Hq, out);
     else
-      bi::attn::attn_combine_kernel<64, 2><<<grid, 256, 0, st>>>(lay.po, lay.pml, lay.off, nrows, Hq, out);
+      e = bi::launch_pdl(bi::attn::attn_combine_kernel<64, 2>, dim3(grid), dim3(256), 0, st, (const float*)lay.po,
+                     (const float2*)lay.pml, (const int32_t*)lay.off, nrows, Hq, out);
   }
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
 // ---- LM head workspace: bf16 logits [M, V], fp32 logits [M, V], flagged list [M + 1],
@@ -389,9 +392,11 @@ bi_status bi_kv_append(const bi_bf16* k_new, const bi_bf16* v_new, int64_t ld_ne
   if (T == 0) return BI_OK;
   const int64_t warps = (int64_t)T * Hkv;
   if ((warps + 7) / 8 > INT_MAX) return BI_ERR_SHAPE;
-  bi::attn::kv_append_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, as_stream(stream)>>>(
-      k_new, v_new, ld_new, q_seq, q_pos, k_cache, v_cache, num_pages, page_table, num_seqs, max_pages_per_seq, T, Hkv, D);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  return bi::launch_pdl(bi::attn::kv_append_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, as_stream(stream),
+                        k_new, v_new, ld_new, q_seq, q_pos, k_cache, v_cache, num_pages, page_table, num_seqs,
+                        max_pages_per_seq, T, Hkv, D) == cudaSuccess
+             ? BI_OK
+             : BI_ERR_CUDA;
 }
 
 size_t bi_lmhead_workspace_size(int64_t M, int64_t V) { return lm_ws_size(M, V, nullptr, nullptr); }
@@ -422,8 +427,10 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
   // each kernel returns at once when the flagged count (known on the device) is not
   // its case.
   const bool small = M <= bi::lmhead::kStrMaxCount && K <= bi::lmhead::kStrMaxK;
-  bi::lmhead::top2_kernel<<<(unsigned)(M * bi::lmhead::kParts), bi::lmhead::kThreads, 0, st>>>(
-      lay.logits16, V, margin_threshold, tokens, recomputed, small ? lay.ticket : nullptr);
+  if (bi::launch_pdl(bi::lmhead::top2_kernel, dim3((unsigned)(M * bi::lmhead::kParts)), dim3(bi::lmhead::kThreads), 0,
+                     st, (const uint16_t*)lay.logits16, V, margin_threshold, tokens, recomputed,
+                     small ? lay.ticket : (unsigned int*)nullptr) != cudaSuccess)
+    return BI_ERR_CUDA;
   float* out32 = logits_fp32 ? logits_fp32 : lay.logits32;
   if (small) {
     static std::once_flag once1[64], once8[64];
@@ -434,22 +441,26 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
                                 bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK, 8), once8, attr8, dev) != cudaSuccess)
       return BI_ERR_CUDA;
     const unsigned sgrid = (unsigned)((V + bi::lmhead::kStrWarps * 32 - 1) / (bi::lmhead::kStrWarps * 32));
-    bi::lmhead::recompute_stream_kernel<1><<<sgrid, bi::lmhead::kStrThreads, bi::lmhead::stream_smem_bytes((int)K, 1), st>>>(
-        h, ldh, W, V, (int)K, (int)M, recomputed, out32, lay.arg_part, tokens, lay.ticket);
-    if (M > 1)
-      bi::lmhead::recompute_stream_kernel<8><<<sgrid, bi::lmhead::kStrThreads, bi::lmhead::stream_smem_bytes((int)K, 8),
-                                               st>>>(h, ldh, W, V, (int)K, (int)M, recomputed, out32, lay.arg_part,
-                                                     tokens, lay.ticket);
-    return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+    cudaError_t e = bi::launch_pdl(bi::lmhead::recompute_stream_kernel<1>, dim3(sgrid), dim3(bi::lmhead::kStrThreads),
+                                   (size_t)bi::lmhead::stream_smem_bytes((int)K, 1), st, h, ldh, W, V, (int)K, (int)M,
+                                   (const int32_t*)recomputed, out32, lay.arg_part, tokens, lay.ticket);
+    if (e == cudaSuccess && M > 1)
+      e = bi::launch_pdl(bi::lmhead::recompute_stream_kernel<8>, dim3(sgrid), dim3(bi::lmhead::kStrThreads),
+                         (size_t)bi::lmhead::stream_smem_bytes((int)K, 8), st, h, ldh, W, V, (int)K, (int)M,
+                         (const int32_t*)recomputed, out32, lay.arg_part, tokens, lay.ticket);
+    return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
   }
-  bi::lmhead::compact_kernel<<<1, 1024, 0, st>>>(recomputed, (int)M, lay.list);
+  cudaError_t e = bi::launch_pdl(bi::lmhead::compact_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)recomputed,
+                                 (int)M, lay.list);
   const dim3 rgrid((unsigned)((V + bi::lmhead::VB - 1) / bi::lmhead::VB),
                    (unsigned)((M + bi::lmhead::RB - 1) / bi::lmhead::RB));
-  bi::lmhead::recompute_kernel<<<rgrid, bi::lmhead::kRecThreads, 0, st>>>(h, ldh, W, V, (int)K, (int)M, lay.list, out32,
-                                                                         0);
-  bi::lmhead::argmax_kernel<<<(unsigned)(M * bi::lmhead::kParts), bi::lmhead::kThreads, 0, st>>>(out32, V, recomputed,
-                                                                                                tokens);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  if (e == cudaSuccess)
+    e = bi::launch_pdl(bi::lmhead::recompute_kernel, rgrid, dim3(bi::lmhead::kRecThreads), 0, st, h, ldh, W, V, (int)K,
+                       (int)M, (const int32_t*)lay.list, out32, 0);
+  if (e == cudaSuccess)
+    e = bi::launch_pdl(bi::lmhead::argmax_kernel, dim3((unsigned)(M * bi::lmhead::kParts)), dim3(bi::lmhead::kThreads),
+                       0, st, (const float*)out32, V, (const int32_t*)recomputed, tokens);
+  return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
 }
 
 bi_status bi_gather_rows(const bi_bf16* src, int64_t ld_src, int64_t nrows_src, const int32_t* idx, int64_t M,
@@ -459,9 +470,10 @@ bi_status bi_gather_rows(const bi_bf16* src, int64_t ld_src, int64_t nrows_src, 
     return BI_ERR_SHAPE;
   if (!aligned16(src) || !aligned16(dst) || ld_src % 8 || ld_dst % 8) return BI_ERR_ALIGN;
   if (M == 0) return BI_OK;
-  bi::glue::gather_rows_kernel<<<(unsigned)((M + 7) / 8), 256, 0, as_stream(stream)>>>(src, ld_src, nrows_src, idx,
-                                                                                        (int)M, width, dst, ld_dst);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  return bi::launch_pdl(bi::glue::gather_rows_kernel, dim3((unsigned)((M + 7) / 8)), dim3(256), 0, as_stream(stream),
+                        src, ld_src, nrows_src, idx, (int)M, width, dst, ld_dst) == cudaSuccess
+             ? BI_OK
+             : BI_ERR_CUDA;
 }
 
 bi_status bi_rope(bi_bf16* x, int64_t ldx, int64_t T, int H, int D, const int32_t* pos, const float* cos_sin,
@@ -472,9 +484,10 @@ bi_status bi_rope(bi_bf16* x, int64_t ldx, int64_t T, int H, int D, const int32_
   if (T == 0) return BI_OK;
   const int64_t n = T * H * (D / 2);
   if ((n + 255) / 256 > INT_MAX) return BI_ERR_SHAPE;
-  bi::glue::rope_kernel<<<(unsigned)((n + 255) / 256), 256, 0, as_stream(stream)>>>(
-      x, ldx, (int)T, H, D, pos, reinterpret_cast<const float2*>(cos_sin), max_pos);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  return bi::launch_pdl(bi::glue::rope_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, as_stream(stream), x,
+                        ldx, (int)T, H, D, pos, reinterpret_cast<const float2*>(cos_sin), max_pos) == cudaSuccess
+             ? BI_OK
+             : BI_ERR_CUDA;
 }
 
 bi_status bi_swiglu(const bi_bf16* gate_up, int64_t ld_gu, bi_bf16* out, int64_t ld_out, int64_t M, int64_t F,
@@ -485,9 +498,10 @@ bi_status bi_swiglu(const bi_bf16* gate_up, int64_t ld_gu, bi_bf16* out, int64_t
   if (M == 0) return BI_OK;
   const int64_t n = M * (F / 8);
   if ((n + 255) / 256 > INT_MAX || M > INT_MAX) return BI_ERR_SHAPE;
-  bi::glue::swiglu_kernel<<<(unsigned)((n + 255) / 256), 256, 0, as_stream(stream)>>>(gate_up, ld_gu, out, ld_out,
-                                                                                       (int)M, (int)F);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  return bi::launch_pdl(bi::glue::swiglu_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, as_stream(stream),
+                        gate_up, ld_gu, out, ld_out, (int)M, (int)F) == cudaSuccess
+             ? BI_OK
+             : BI_ERR_CUDA;
 }
 
 bi_status bi_add(const bi_bf16* a, const bi_bf16* b, bi_bf16* out, int64_t n, void* stream) {
@@ -497,8 +511,10 @@ bi_status bi_add(const bi_bf16* a, const bi_bf16* b, bi_bf16* out, int64_t n, vo
   if (n == 0) return BI_OK;
   const int64_t v = n / 8;
   if ((v + 255) / 256 > INT_MAX) return BI_ERR_SHAPE;
-  bi::glue::add_kernel<<<(unsigned)((v + 255) / 256), 256, 0, as_stream(stream)>>>(a, b, out, n);
-  return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+  return bi::launch_pdl(bi::glue::add_kernel, dim3((unsigned)((v + 255) / 256)), dim3(256), 0, as_stream(stream), a, b,
+                        out, n) == cudaSuccess
+             ? BI_OK
+             : BI_ERR_CUDA;
 }
 
 bi_status bi_selftest_wait_timeout(int limit_ms, void* stream) {

@@ -87,6 +87,8 @@ __device__ __forceinline__ Top2 block_top2(Top2 t, Top2* warp_best) {
 __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads)
     top2_kernel(const uint16_t* __restrict__ logits, int64_t V, float threshold, int32_t* __restrict__ tokens,
                 int32_t* __restrict__ flags, unsigned int* __restrict__ ticket) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   __shared__ Top2 warp_best[kThreads / 32];
   __shared__ Top2 part_best;
   const int64_t row = blockIdx.x / kParts;
@@ -122,6 +124,8 @@ __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads)
 // list[0..count) = indices of flagged rows, ascending; list[M] = count.
 __global__ void __launch_bounds__(1024) compact_kernel(const int32_t* __restrict__ flags, int M,
                                                        int32_t* __restrict__ list) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   __shared__ int32_t sums[1024];
   const int tid = threadIdx.x;
   const int per = (M + 1023) / 1024;
@@ -159,6 +163,8 @@ __global__ void __launch_bounds__(kRecThreads, 3) recompute_kernel(const uint16_
                                                                   const uint16_t* __restrict__ W, int64_t V, int K,
                                                                   int M, const int32_t* __restrict__ list,
                                                                   float* __restrict__ out, int skip_upto) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   __shared__ __align__(16) float2 hs[2][KB][RB];  // (h, h) per row
   __shared__ __align__(16) float ws[2][KB][VB];
   const int count = list[M];
@@ -272,6 +278,8 @@ __global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uin
                                                                       ArgBest* __restrict__ arg_part,
                                                                       int32_t* __restrict__ tokens,
                                                                       unsigned int* __restrict__ ticket) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_str[];
   float* hsm = reinterpret_cast<float*>(smem_str);                               // [K][NR]
   uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_str + (size_t)K * NR * 4);  // [warp][32][72]
@@ -426,6 +434,8 @@ __global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uin
 __global__ void __cluster_dims__(kParts, 1, 1) __launch_bounds__(kThreads)
     argmax_kernel(const float* __restrict__ logits, int64_t V, const int32_t* __restrict__ flags,
                   int32_t* __restrict__ tokens) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
   __shared__ float wv[kThreads / 32];
   __shared__ int wi[kThreads / 32];
   __shared__ float part_v;

@@ -48,6 +48,8 @@ __global__ void __launch_bounds__(kThreads) rmsnorm_kernel(const uint16_t* x,
   const uint4* wr = reinterpret_cast<const uint4*>(w);
   int64_t row = blockIdx.x;
   uint4 v[NV], vn[NV];
+  pdl_wait();  // the previous kernel on the stream has written x (or still reads y) until now
+  pdl_trigger();
   load_row<NV>(reinterpret_cast<const uint4*>(x + row * ldx), nvec, v);
   for (int it = 0; row < M; row += gridDim.x, ++it) {
     const int64_t next = row + gridDim.x;
@@ -111,8 +113,7 @@ inline cudaError_t launch_nv(const uint16_t* x, int64_t ldx, const uint16_t* w, 
   // the hardware schedules as CTAs retire (measured faster at M = 65536)
   const int64_t cap = (int64_t)sms * ctas_per_sm<NV>();
   const unsigned grid = (unsigned)(M <= 4 * cap ? (M < cap ? M : cap) : M);
-  rmsnorm_kernel<NV><<<grid, kThreads, 0, st>>>(x, ldx, w, y, ldy, M, K, eps);
-  return cudaGetLastError();
+  return launch_pdl(rmsnorm_kernel<NV>, dim3(grid), dim3(kThreads), 0, st, x, ldx, w, y, ldy, M, K, eps);
 }
 
 inline cudaError_t launch(const uint16_t* x, int64_t ldx, const uint16_t* w, uint16_t* y,
