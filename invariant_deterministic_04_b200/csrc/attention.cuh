@@ -319,16 +319,17 @@ struct RingState {
   uint32_t seq, issued, ph_bits;
 };
 
-// The split kernel's work loop for GW query heads per warp: items are (split slot f,
-// kv-head g, head part hp) with heads g*G + hp*GW .. +GW-1, dealt across CTAs first
-// (item = warp * gridDim.x + CTA) so that a launch with fewer items than warp slots
-// spreads them over every SM. Returns false if a copy never landed.
+// The split kernel's work loop for GW query heads per warp over the (split slot,
+// kv-head) items [begin, end): work units are (item, head part hp) with heads
+// g*G + hp*GW .. +GW-1, dealt across CTAs first (unit = begin * HP + warp * gridDim.x
+// + CTA + k * slots) so that fewer units than warp slots spread over every SM.
+// Returns false if a copy never landed.
 template <int D, int G, int GW>
 __device__ __forceinline__ bool split_items(const uint16_t* __restrict__ q, int64_t ldq, int Hq, int Hkv,
                                             const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc,
                                             int64_t num_pages, const int32_t* __restrict__ pt, const Rows& R,
                                             int nrows, const int32_t* __restrict__ off, float* __restrict__ po,
-                                            float2* __restrict__ pml, float c, int total, uint32_t ring,
+                                            float2* __restrict__ pml, float c, int begin, int end, uint32_t ring,
                                             uint32_t bars, RingState& rs) {
   using T = SplitLanes<D, G>;
   constexpr int DPL = T::DPL, LPT = T::LPT, PAGE_BYTES = T::PAGE_BYTES, STAGE_BYTES = T::STAGE_BYTES;
@@ -336,7 +337,7 @@ __device__ __forceinline__ bool split_items(const uint16_t* __restrict__ q, int6
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tg = lane / LPT, dl = lane % LPT;
   const int64_t kv_head_stride = (int64_t)PAGE * D;
-  for (int item = warp * gridDim.x + blockIdx.x; item < total * HP; item += gridDim.x * WARPS) {
+  for (int item = begin * HP + warp * gridDim.x + blockIdx.x; item < end * HP; item += gridDim.x * WARPS) {
     const int fg = item / HP, hp = item - (item / HP) * HP;
     const int f = fg / Hkv, g = fg - (fg / Hkv) * Hkv;
     const int h0 = g * G + hp * GW;
@@ -407,11 +408,14 @@ __device__ __forceinline__ bool split_items(const uint16_t* __restrict__ q, int6
 }
 
 // One warp per (row, kv-head g, split) -- or per (row, kv-head, split, half or quarter
-// of the G query heads) when the batch's items would fill at most half (a quarter) of
-// the warp slots: writes the split's (m, l) and unnormalised o[D] per query head into
-// the workspace. Each warp streams its split's pages through its own ring of NST
-// stages. How the heads are spread over warps is a launch shape: every head's
-// arithmetic is the same (see split_items).
+// of the G query heads) for the items of the last, partly filled round of warp slots
+// when 2 or 4 times as many units still fit in one round: writes the split's (m, l)
+// and unnormalised o[D] per query head into the workspace. Items that fill whole
+// rounds keep their G heads on one warp (the fewest instructions per byte); a tail of
+// fewer items than slots is cut finer so that it does not cost a full round. Each
+// warp streams its split's pages through its own ring of NST stages. How the heads
+// are spread over warps is a launch shape: every head's arithmetic is the same (see
+// split_items).
 template <int D, int G>
 __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
     attn_split_kernel(const uint16_t* __restrict__ q, int64_t ldq, int Hq, int Hkv, const uint16_t* __restrict__ kc,
@@ -438,17 +442,21 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
 
   const int total = off[nrows] * Hkv;  // (split slot, kv-head) items
   const int64_t slots = (int64_t)gridDim.x * WARPS;
+  const int full = (int)(total / slots * slots);  // items of the whole rounds
+  const int tail = total - full;
+  const int hs = (G >= 4 && tail > 0 && (int64_t)tail * 4 <= slots)   ? 4
+                 : (G >= 2 && tail > 0 && (int64_t)tail * 2 <= slots) ? 2
+                                                                      : 1;
+  const int whole = hs == 1 ? total : full;  // items reduced with G heads per warp
   RingState rs{0u, 0u, 0u};
-  bool ok;
-  if (G >= 4 && (int64_t)total * 4 <= slots)
+  bool ok = whole == 0 || split_items<D, G, G>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, off, po, pml, c, 0,
+                                               whole, ring, bars, rs);
+  if (ok && hs == 4)
     ok = split_items<D, G, (G >= 4 ? G / 4 : G)>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, off, po, pml, c,
-                                                 total, ring, bars, rs);
-  else if (G >= 2 && (int64_t)total * 2 <= slots)
+                                                 full, total, ring, bars, rs);
+  else if (ok && hs == 2)
     ok = split_items<D, G, (G >= 2 ? G / 2 : G)>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, off, po, pml, c,
-                                                 total, ring, bars, rs);
-  else
-    ok = split_items<D, G, G>(q, ldq, Hq, Hkv, kc, vc, num_pages, pt, R, nrows, off, po, pml, c, total, ring, bars,
-                              rs);
+                                                 full, total, ring, bars, rs);
   if (!ok) {  // a copy never landed: error recorded; let this warp's other copies land, then leave
     if (lane == 0) drain_copies(bars, 8, rs.issued, rs.ph_bits);
     __syncwarp();
