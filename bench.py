@@ -332,8 +332,18 @@ def cpu_baseline(budget_s: float = 10.0):
             flops += f
             t += dt
     what = f"{reps} whole steps of 2048 rows" if rows == 2048 else f"{rows} of the 2048 rows of one step"
-    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"fp64 numpy oracle: RMSNorm + matmuls (N=4096,6144,14336; K=4096), {what}, {t:.1f} s"}
+    out = {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+           "sample": f"fp64 numpy oracle: RMSNorm + matmuls (N=4096,6144,14336; K=4096), {what}, {t:.1f} s"}
+    # the same oracle on one core: a 32-row sample of the step (about two seconds)
+    try:
+        from threadpoolctl import threadpool_limits
+
+        with threadpool_limits(limits=1):
+            f1, t1 = oracle_step_sample(32, seed=3)
+        out["one_core"] = {"value": f1 / t1 / 1e12, "unit": "TFLOP/s", "sample": f"32 of the 2048 rows, {t1:.1f} s"}
+    except Exception as e:  # threadpoolctl missing or the BLAS not controllable
+        out["one_core"] = f"unavailable: {type(e).__name__}"
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -380,6 +390,8 @@ def _graph_us(fn, n=20, reps=10):
 def other_rows(bi, device, pk, only=None):
     out = {}
     want = (lambda name: only is None or only == name)
+    if want("chain"):
+        out.update(_row_chain(bi, device))
     # RMSNorm bandwidth at a size far above L2 (M = 65536, K = 4096: 1 GiB in + out)
     if want("rmsnorm"):
         out.update(_row_rmsnorm(bi, device, pk))
@@ -394,6 +406,38 @@ def other_rows(bi, device, pk, only=None):
     if want("config5"):
         out.update(_row_config5(bi, device, pk))
     return out
+
+
+def _row_chain(bi, device):
+    """Config 1: RMSNorm (K = 512) then the matmul 512 -> 1024 on 32 rows, x ~ N(0, 1),
+    w = 1 + N(0, 0.1), W ~ N(0, 0.02). Reported: microseconds per chain (two launches,
+    CUDA-graph replays, inputs warm: the whole chain is 1.3 MB), the same for F.rms_norm +
+    torch.matmul, and whether rows 0..m-1 and the last m rows recomputed as batches of
+    m = 1, 2, 7, 16 equal the 32-row batch bit for bit. Launch- and latency-bound: the
+    chain is 33.6 MFLOP and 1.1 MB."""
+    x, wn = synth.rmsnorm_inputs(32, 512, seed=0)
+    _, W = synth.matmul_inputs(32, 1024, 512, seed=2)
+    x, wn, W = x.to(device), wn.to(device), W.to(device)
+    y = torch.empty_like(x)
+    c = torch.empty((32, 1024), dtype=torch.bfloat16, device=device)
+
+    def chain():
+        bi.rmsnorm(x, wn, 1e-6, out=y)
+        bi.matmul(y, W, out=c)
+
+    us = _graph_per_call_us([chain] * 16)  # per closure: one RMSNorm and one matmul launch
+    full = bi.matmul(bi.rmsnorm(x, wn, 1e-6), W)
+    same = True
+    for m in (1, 2, 7, 16):
+        for start in (0, 32 - m):
+            part = bi.matmul(bi.rmsnorm(x[start:start + m].contiguous(), wn, 1e-6), W)
+            same = same and bool(torch.equal(part.view(torch.int16), full[start:start + m].view(torch.int16)))
+    def ref():
+        torch.matmul(torch.nn.functional.rms_norm(x, (512,), wn, 1e-6), W.t(), out=c)
+
+    ref_us = _graph_per_call_us([ref] * 16)
+    return {"chain_m32_k512_n1024": {"us": round(us, 2), "rows_bit_identical_m1_2_7_16": same,
+                                     "noninvariant_us": round(ref_us, 2), "slowdown": round(us / ref_us, 3)}}
 
 
 def _row_config5(bi, device, pk, repeats=3, base_repeats=2):
@@ -978,7 +1022,7 @@ def main():
                     help="add the matmul / RMSNorm / decode sweeps to the line (default on)")
     ap.add_argument("--no-sweeps", dest="sweeps", action="store_false")
     ap.add_argument("--sweep", action="store_true", help="only the sweeps, one JSON line per entry")
-    ap.add_argument("--row", choices=["rmsnorm", "decode", "prefill", "lmhead", "reduce", "config5"], default=None,
+    ap.add_argument("--row", choices=["chain", "rmsnorm", "decode", "prefill", "lmhead", "reduce", "config5"], default=None,
                     help="measure only this hot-path kernel (for profiling) and print its line")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--profile", choices=PROFILE_CASES, default=None,
