@@ -795,13 +795,13 @@ def run_sweep(bi, device, pk):
 # ---------------------------------------------------------------------------
 
 
-PROFILE_CASES = ("decode_b16", "decode_b1", "prefill_s4096", "rmsnorm", "lmhead_m4", "lmhead_m64", "matmul_small")
+PROFILE_CASES = ("decode_b16", "decode_b4", "decode_b1", "prefill_s4096", "rmsnorm", "lmhead_m4", "lmhead_m64", "matmul_small")
 
 
 def profile_case(bi, device, name):
     """A few plain launches of one kernel case, for an ncu capture (nothing timed):
-    decode_b16 = decode attention over the first 16 sequences of the decode sweep's
-    store (lengths ~ U[1, 32768], 1.1 GB of K/V); decode_b1 = decode attention over
+    decode_b16 / decode_b4 = decode attention over the first 16 / 4 sequences of the
+    decode sweep's lengths (~ U[1, 32768]; 1.1 GB of K/V for 16); decode_b1 = decode attention over
     one sequence of 16384 tokens (64 splits, 67 MB of K/V); prefill_s4096 = causal
     prefill of one 4096-token sequence on the CUDA cores; rmsnorm = RMSNorm at 65536 x 4096
     then 2048 x 4096; lmhead_m4 = the LM head at 4 rows, V = 32000, K = 2048, with no
@@ -809,12 +809,13 @@ def profile_case(bi, device, name):
     lmhead_m64 = the LM head at 64 rows, V = 32000, K = 2048, random N(0, 0.02) weights
     (53 rows flagged);
     matmul_small = bi_matmul at M = 1 and 128, K = N = 4096."""
-    if name == "decode_b16":
-        lens = synth.decode_lengths(16, 32768, seed=50)
+    if name in ("decode_b16", "decode_b4"):
+        nb = 16 if name == "decode_b16" else 4
+        lens = synth.decode_lengths(16, 32768, seed=50)[:nb]
         kv = synth.paged_kv_device(lens, 8, 128, seed=51, max_pages=2048, device=device)
-        q = synth.normal_bf16((16, 32, 128), 52).to(device)
+        q = synth.normal_bf16((nb, 32, 128), 52).to(device)
         o = torch.empty_like(q)
-        ws = torch.empty(bi.attention_workspace_size(16, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
+        ws = torch.empty(bi.attention_workspace_size(nb, 32, 128, kv.max_pages), dtype=torch.uint8, device=device)
         for _ in range(3):
             bi.attention_decode(q, kv.k_cache, kv.v_cache, kv.page_table, kv.seq_lens, out=o, workspace=ws)
     elif name == "decode_b1":

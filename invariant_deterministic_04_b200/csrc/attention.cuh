@@ -465,12 +465,14 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
 
 // Fold a row's splits in ascending order: one warp per (row, query head, group of
 // 32 * DPL output dims), DPL dims per lane. The maximum of the splits' running maxima
-// is taken lane-parallel (a maximum is exact in any order); lane j computes the weight
-// of split j of each group of 32 and the weights are broadcast, so that every output
-// dim and the normaliser are each one FMA chain in split order whatever DPL is. The
-// partial outputs of 32 / DPL splits are loaded before any of them is folded. DPL only
-// sets how many warps share a row: 1 when the batch gives few (row, head) pairs, D / 32
-// when it gives enough warps to fill the GPU.
+// is taken lane-parallel, 128 splits per round trip (a maximum is exact in any order);
+// lane j computes the weight of split j of each chunk of 32 and the weights are
+// broadcast, so that every output dim and the normaliser are each one FMA chain in
+// split order whatever DPL is. The splits are folded in groups of U = 32 / DPL whose
+// partial outputs are loaded one group ahead (two register buffers), and each chunk's
+// (m, l) one chunk ahead, so the fold waits for memory once per row rather than once
+// per group. DPL only sets how many warps share a row: 1 when the batch gives few
+// (row, head) pairs, D / 32 when it gives enough warps to fill the GPU.
 template <int D, int DPL>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ po,
                                                            const float2* __restrict__ pml,
@@ -479,7 +481,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   static_assert(DPL == 1 || DPL == 2 || DPL == 4, "dims per lane");
   static_assert(D % (32 * DPL) == 0, "a warp covers whole groups of dims");
   constexpr int NG = D / (32 * DPL);  // warps per (row, query head)
-  constexpr int U = 32 / DPL;         // splits whose partial outputs are loaded together
+  constexpr int U = 32 / DPL;         // splits per group
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   pdl_wait();  // the split partials are complete from here on
@@ -493,8 +495,16 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   const float* po_row = po + ((int64_t)f0 * Hq + h) * D + d0;    // split s at s * Hq * D
   const int64_t po_step = (int64_t)Hq * D;
   float M = -INFINITY;
-  for (int s0 = 0; s0 < n; s0 += 32)
-    if (s0 + lane < n) M = fmaxf(M, ml_row[(int64_t)(s0 + lane) * Hq].x);
+  for (int s0 = 0; s0 < n; s0 += 128) {
+    float mv[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int sp = s0 + c * 32 + lane;
+      mv[c] = sp < n ? ml_row[(int64_t)sp * Hq].x : -INFINITY;
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) M = fmaxf(M, mv[c]);
+  }
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float O[DPL];
@@ -502,38 +512,60 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   for (int d = 0; d < DPL; ++d) O[d] = 0.f;
   float L = 0.f;
   if (M != -INFINITY) {
-    for (int s0 = 0; s0 < n; s0 += 32) {
-      const int cnt = min(32, n - s0);
-      const float2 ml = lane < cnt ? ml_row[(int64_t)(s0 + lane) * Hq] : make_float2(-INFINITY, 0.f);
-      const float wl = lane < cnt ? exp2f(__fsub_rn(ml.x, M)) : 0.f;
+    // the partial outputs of group gi (splits gi*U .. gi*U+U-1; past n: split 0 again, unused)
+    auto load_group = [&](int gi, float (&v)[U][DPL]) {
 #pragma unroll
-      for (int u0 = 0; u0 < 32; u0 += U) {
-        if (u0 >= cnt) break;  // the same for every lane
-        float v[U][DPL];
-#pragma unroll
-        for (int j = 0; j < U; ++j) {
-          const float* src = po_row + (int64_t)(u0 + j < cnt ? s0 + u0 + j : s0) * po_step;
-          if constexpr (DPL == 4) {
-            const float4 q = *reinterpret_cast<const float4*>(src);
-            v[j][0] = q.x; v[j][1] = q.y; v[j][2] = q.z; v[j][3] = q.w;
-          } else if constexpr (DPL == 2) {
-            const float2 q = *reinterpret_cast<const float2*>(src);
-            v[j][0] = q.x; v[j][1] = q.y;
-          } else {
-            v[j][0] = *src;
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < U; ++j) {
-          const float wk = __shfl_sync(0xffffffffu, wl, u0 + j);
-          const float lk = __shfl_sync(0xffffffffu, ml.y, u0 + j);
-          if (u0 + j < cnt) {
-            L = __fmaf_rn(lk, wk, L);
-#pragma unroll
-            for (int d = 0; d < DPL; ++d) O[d] = __fmaf_rn(v[j][d], wk, O[d]);
-          }
+      for (int j = 0; j < U; ++j) {
+        const int sp = gi * U + j;
+        const float* src = po_row + (int64_t)(sp < n ? sp : 0) * po_step;
+        if constexpr (DPL == 4) {
+          const float4 q = *reinterpret_cast<const float4*>(src);
+          v[j][0] = q.x; v[j][1] = q.y; v[j][2] = q.z; v[j][3] = q.w;
+        } else if constexpr (DPL == 2) {
+          const float2 q = *reinterpret_cast<const float2*>(src);
+          v[j][0] = q.x; v[j][1] = q.y;
+        } else {
+          v[j][0] = *src;
         }
       }
+    };
+    auto load_ml = [&](int chunk) {
+      const int sp = chunk * 32 + lane;
+      return sp < n ? ml_row[(int64_t)sp * Hq] : make_float2(-INFINITY, 0.f);
+    };
+    float2 ml = load_ml(0), ml_next = load_ml(1);
+    float wl = lane < n ? exp2f(__fsub_rn(ml.x, M)) : 0.f;
+    // fold group gi from buffer v (its chunk's weights are in wl / ml.y)
+    auto fold_group = [&](int gi, const float (&v)[U][DPL]) {
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int sp = gi * U + j;
+        const float wk = __shfl_sync(0xffffffffu, wl, sp & 31);
+        const float lk = __shfl_sync(0xffffffffu, ml.y, sp & 31);
+        if (sp < n) {
+          L = __fmaf_rn(lk, wk, L);
+#pragma unroll
+          for (int d = 0; d < DPL; ++d) O[d] = __fmaf_rn(v[j][d], wk, O[d]);
+        }
+      }
+      // the next group starts a new chunk of 32 splits: take its weights
+      if (((gi + 1) * U) % 32 == 0) {
+        const int chunk = (gi + 1) * U / 32;
+        ml = ml_next;
+        ml_next = load_ml(chunk + 1);
+        const int sp = chunk * 32 + lane;
+        wl = sp < n ? exp2f(__fsub_rn(ml.x, M)) : 0.f;
+      }
+    };
+    const int ngroups = (n + U - 1) / U;
+    float va[U][DPL], vb[U][DPL];
+    load_group(0, va);
+    for (int gi = 0; gi < ngroups; gi += 2) {
+      if (gi + 1 < ngroups) load_group(gi + 1, vb);
+      fold_group(gi, va);
+      if (gi + 1 >= ngroups) break;
+      if (gi + 2 < ngroups) load_group(gi + 2, va);
+      fold_group(gi + 1, vb);
     }
   }
   float y[DPL];
