@@ -204,8 +204,9 @@ __device__ __forceinline__ void load_q(const uint16_t* __restrict__ q, int64_t l
 
 // Folds one page (K at kb, V at vb in shared memory, its first nvalid tokens
 // visible) into the running (m, l, o) of the lane's head: scores, the base-2
-// online-softmax rescale, then p * V.
-template <int D, int G, int GW>
+// online-softmax rescale, then p * V. FULL: all PAGE tokens are visible (the same
+// arithmetic without the visibility tests).
+template <int D, int G, int GW, bool FULL = false>
 __device__ __forceinline__ void fold_page(const float2 (&qf)[GW][SplitCfg<D, G>::DPL / 2], uint32_t kb, uint32_t vb,
                                           int nvalid, float c, int tg, int dl, float& m, float& l,
                                           float2 (&o)[GW][SplitCfg<D, G>::DPL / 2]) {
@@ -234,7 +235,7 @@ __device__ __forceinline__ void fold_page(const float2 (&qf)[GW][SplitCfg<D, G>:
 #pragma unroll
     for (int i = 0; i < GW; ++i) part[i] = __fadd_rn(acc[i].x, acc[i].y);
     const float dot = reduce_scatter<GW, LPT>(part, dl);
-    sc[u] = t < nvalid ? __fmul_rn(dot, c) : -INFINITY;
+    sc[u] = (FULL || t < nvalid) ? __fmul_rn(dot, c) : -INFINITY;
   }
   float pm = sc[0];
 #pragma unroll
@@ -258,7 +259,7 @@ __device__ __forceinline__ void fold_page(const float2 (&qf)[GW][SplitCfg<D, G>:
 #pragma unroll
   for (int u = 0; u < STEPS; ++u) {
     const int t = u * TPW + tg;
-    const bool valid = t < nvalid;
+    const bool valid = FULL || t < nvalid;
     const float p = valid ? exp2f(__fsub_rn(sc[u], m_new)) : 0.f;
     l = __fadd_rn(l, p);
     float pa[GW];
@@ -395,7 +396,13 @@ __device__ __forceinline__ bool split_items(const uint16_t* __restrict__ q, int6
       const int pg = prow[j];
       const int nvalid = (pg < 0 || pg >= num_pages) ? 0 : min(PAGE, t1 - t0 - j * PAGE);
       const uint32_t kb = ring + st * STAGE_BYTES;
-      fold_page<D, G, GW>(qf, kb, kb + PAGE_BYTES, nvalid, c, tg, dl, m, l, o);
+      // warps carrying part of a kv-head's query heads (batches that leave warp slots
+      // idle) have registers to spare for a second copy of the fold without the
+      // visibility tests; the all-heads path keeps one copy (a second one spills)
+      if (GW < G && nvalid == PAGE)
+        fold_page<D, G, GW, true>(qf, kb, kb + PAGE_BYTES, PAGE, c, tg, dl, m, l, o);
+      else
+        fold_page<D, G, GW, false>(qf, kb, kb + PAGE_BYTES, nvalid, c, tg, dl, m, l, o);
       __syncwarp();
       if (lane == 0 && j + NST < np) {
         fence_proxy_async_smem();
