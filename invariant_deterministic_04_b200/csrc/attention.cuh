@@ -475,13 +475,15 @@ __global__ void __launch_bounds__(SplitCfg<D, G>::WARPS * 32, 1)
 // is taken lane-parallel, 128 splits per round trip (a maximum is exact in any order);
 // lane j computes the weight of split j of each chunk of 32 and the weights are
 // broadcast, so that every output dim and the normaliser are each one FMA chain in
-// split order whatever DPL is. The splits are folded in groups of U = 32 / DPL whose
-// partial outputs are loaded one group ahead (two register buffers), and each chunk's
-// (m, l) one chunk ahead, so the fold waits for memory once per row rather than once
-// per group. DPL only sets how many warps share a row: 1 when the batch gives few
-// (row, head) pairs, D / 32 when it gives enough warps to fill the GPU.
+// split order whatever DPL is. The splits are folded in groups of U = 32 / DPL; with
+// one dim per lane (few rows) a group's partial outputs are loaded one group ahead
+// (two register buffers) and each chunk's (m, l) one chunk ahead, so the fold waits
+// for memory about once per row; with more dims per lane (many rows) one buffer keeps
+// the registers low and the occupancy high. DPL only sets how many warps share a row:
+// 1 when the batch gives few (row, head) pairs, D / 32 when it gives enough warps to
+// fill the GPU.
 template <int D, int DPL>
-__global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ po,
+__global__ void __launch_bounds__(256, DPL == 1 ? 1 : 4) attn_combine_kernel(const float* __restrict__ po,
                                                            const float2* __restrict__ pml,
                                                            const int32_t* __restrict__ off, int nrows,
                                                            int Hq, uint16_t* __restrict__ out) {
@@ -565,14 +567,25 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
       }
     };
     const int ngroups = (n + U - 1) / U;
-    float va[U][DPL], vb[U][DPL];
-    load_group(0, va);
-    for (int gi = 0; gi < ngroups; gi += 2) {
-      if (gi + 1 < ngroups) load_group(gi + 1, vb);
-      fold_group(gi, va);
-      if (gi + 1 >= ngroups) break;
-      if (gi + 2 < ngroups) load_group(gi + 2, va);
-      fold_group(gi + 1, vb);
+    if constexpr (DPL == 1) {
+      // one dim per lane (few rows): the next group's loads overlap this group's fold
+      float va[U][DPL], vb[U][DPL];
+      load_group(0, va);
+      for (int gi = 0; gi < ngroups; gi += 2) {
+        if (gi + 1 < ngroups) load_group(gi + 1, vb);
+        fold_group(gi, va);
+        if (gi + 1 >= ngroups) break;
+        if (gi + 2 < ngroups) load_group(gi + 2, va);
+        fold_group(gi + 1, vb);
+      }
+    } else {
+      // several dims per lane (many rows, e.g. prefill): one buffer, so that more warps
+      // stay resident; other warps cover the loads
+      float va[U][DPL];
+      for (int gi = 0; gi < ngroups; ++gi) {
+        load_group(gi, va);
+        fold_group(gi, va);
+      }
     }
   }
   float y[DPL];
