@@ -433,21 +433,15 @@ bi_status bi_lmhead_argmax(const bi_bf16* h, int64_t ldh, const bi_bf16* W, int6
     return BI_ERR_CUDA;
   float* out32 = logits_fp32 ? logits_fp32 : lay.logits32;
   if (small) {
-    static std::once_flag once1[64], once8[64];
-    static cudaError_t attr1[64], attr8[64];
-    if (bi::gemm::set_smem_once(bi::lmhead::recompute_stream_kernel<1>,
-                                bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK, 1), once1, attr1, dev) != cudaSuccess ||
-        bi::gemm::set_smem_once(bi::lmhead::recompute_stream_kernel<8>,
-                                bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK, 8), once8, attr8, dev) != cudaSuccess)
+    static std::once_flag once_str[64];
+    static cudaError_t attr_str[64];
+    if (bi::gemm::set_smem_once(bi::lmhead::recompute_stream_kernel, bi::lmhead::stream_smem_bytes(bi::lmhead::kStrMaxK),
+                                once_str, attr_str, dev) != cudaSuccess)
       return BI_ERR_CUDA;
     const unsigned sgrid = (unsigned)((V + bi::lmhead::kStrWarps * 32 - 1) / (bi::lmhead::kStrWarps * 32));
-    cudaError_t e = bi::launch_pdl(bi::lmhead::recompute_stream_kernel<1>, dim3(sgrid), dim3(bi::lmhead::kStrThreads),
-                                   (size_t)bi::lmhead::stream_smem_bytes((int)K, 1), st, h, ldh, W, V, (int)K, (int)M,
-                                   (const int32_t*)recomputed, out32, lay.arg_part, tokens, lay.ticket);
-    if (e == cudaSuccess && M > 1)
-      e = bi::launch_pdl(bi::lmhead::recompute_stream_kernel<8>, dim3(sgrid), dim3(bi::lmhead::kStrThreads),
-                         (size_t)bi::lmhead::stream_smem_bytes((int)K, 8), st, h, ldh, W, V, (int)K, (int)M,
-                         (const int32_t*)recomputed, out32, lay.arg_part, tokens, lay.ticket);
+    const cudaError_t e = bi::launch_pdl(bi::lmhead::recompute_stream_kernel, dim3(sgrid), dim3(bi::lmhead::kStrThreads),
+                                         (size_t)bi::lmhead::stream_smem_bytes((int)K), st, h, ldh, W, V, (int)K,
+                                         (int)M, (const int32_t*)recomputed, out32, lay.arg_part, tokens, lay.ticket);
     return e == cudaSuccess ? BI_OK : BI_ERR_CUDA;
   }
   cudaError_t e = bi::launch_pdl(bi::lmhead::compact_kernel, dim3(1), dim3(1024), 0, st, (const int32_t*)recomputed,

@@ -12,7 +12,7 @@
 //      never wins), margin = top1 - top2 in fp32, flag = margin < threshold;
 //      token = top-1 index.
 //   3. compact_kernel: ascending list of flagged rows.
-//   4. recompute_kernel, or recompute_stream_kernel<1 | 8> for few flagged rows: fp32
+//   4. recompute_kernel, or recompute_stream_kernel for few flagged rows: fp32
 //      logits of the flagged rows from bf16 operands widened to fp32, each logit one
 //      FMA chain over k = 0..K-1 (CUDA cores).
 //   5. argmax_kernel: token of each flagged row = argmax of its fp32 logits.
@@ -256,58 +256,76 @@ __global__ void __launch_bounds__(kRecThreads, 3) recompute_kernel(const uint16_
 // The same fp32 logits for batches of at most kStrMaxCount rows and hidden sizes up to
 // 4096, with W streamed once per NR flagged rows instead of once per 64-row tile
 // (identical FMA chains, so identical bits), and the flagged rows' tokens taken in the
-// same kernel. Both are launched; the on-device count of flagged rows picks the one
-// that works: recompute_stream_kernel<1> when exactly one row is flagged (the common
-// case of a trained model's rare near-tie), <8> for two or more.
+// same kernel. One launch; the on-device count of flagged rows picks the case:
+// stream_rows<1> when exactly one row is flagged (the common case of a trained model's
+// rare near-tie), stream_rows<8> for two or more.
 // Each warp owns 32 consecutive vocabulary entries (lane = entry) and walks K in tiles of
-// 64: the tile (32 rows x 128 bytes of W) is loaded coalesced (8 lanes per row) two tiles
-// ahead into registers, parked in the warp's shared-memory slot (rows padded to 144 bytes,
-// so each lane's 16-byte reads of its own row are conflict-free), and consumed by each lane
-// along its row. The CTA's NR current flagged rows of h sit in shared memory as fp32,
-// [k][row], read as broadcasts; packed f32x2 FMAs carry two rows each.
+// 64: a tile (32 rows x 128 bytes of W) is copied coalesced (8 lanes per row, cp.async)
+// into the warp's ring of shared-memory slots (rows padded to 144 bytes, so each lane's
+// 16-byte reads of its own row are conflict-free), three tiles ahead for one flagged row
+// and one ahead for groups of 8, and consumed by each lane along its row. The CTA's NR
+// current flagged rows of h sit in shared memory as fp32, [k][row], read as broadcasts;
+// packed f32x2 FMAs carry two rows each.
 constexpr int kStrWarps = 4, kStrThreads = 128, kStrTK = 64, kStrPad = 72, kStrMaxK = 4096;
 constexpr int kStrMaxCount = 24;
 
-inline int stream_smem_bytes(int K, int NR) { return K * NR * 4 + kStrWarps * 32 * kStrPad * 2; }
+// Tiles of W each warp has in flight: four for one flagged row (the h block is small,
+// so two CTAs per SM still fit), two for groups of 8 rows (their h block is 8x larger).
+__host__ __device__ constexpr int stream_ring(int NR) { return NR == 1 ? 4 : 2; }
 
+inline int stream_smem_bytes(int K, int NR) {
+  return K * NR * 4 + kStrWarps * stream_ring(NR) * 32 * kStrPad * 2;
+}
+// dynamic shared memory of recompute_stream_kernel (either case)
+inline int stream_smem_bytes(int K) {
+  const int a = stream_smem_bytes(K, 1), b = stream_smem_bytes(K, 8);
+  return a > b ? a : b;
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The rows of `list` (count of them, NR at a time): fp32 logits, per-CTA argmax partials,
+// and the last CTA's merge into tokens. smem_str: h of NR rows [K][NR], then the warps'
+// tile rings.
 template <int NR>
-__global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uint16_t* __restrict__ h, int64_t ldh,
-                                                                      const uint16_t* __restrict__ W, int64_t V,
-                                                                      int K, int M, const int32_t* __restrict__ flags,
-                                                                      float* __restrict__ out,
-                                                                      ArgBest* __restrict__ arg_part,
-                                                                      int32_t* __restrict__ tokens,
-                                                                      unsigned int* __restrict__ ticket) {
-  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
-  pdl_trigger();
-  extern __shared__ __align__(16) uint8_t smem_str[];
+__device__ __forceinline__ void stream_rows(const uint16_t* __restrict__ h, int64_t ldh, const uint16_t* __restrict__ W,
+                                            int64_t V, int K, float* __restrict__ out,
+                                            ArgBest* __restrict__ arg_part, int32_t* __restrict__ tokens,
+                                            unsigned int* __restrict__ ticket, uint8_t* smem_str, const int* list,
+                                            int count, ArgBest (&warp_arg)[kStrWarps][8], int& last) {
   float* hsm = reinterpret_cast<float*>(smem_str);                               // [K][NR]
-  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_str + (size_t)K * NR * 4);  // [warp][32][72]
-  __shared__ int list[kStrMaxCount + 1];  // flagged rows, ascending (M <= kStrMaxCount)
-  __shared__ ArgBest warp_arg[kStrWarps][NR];
-  __shared__ int last;
+  uint16_t* tiles = reinterpret_cast<uint16_t*>(smem_str + (size_t)K * NR * 4);  // [warp][ring][32][72]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp == 0) {  // the flagged rows in order: one ballot over M <= 24 rows
-    const bool f = lane < M && flags[lane] != 0;
-    const unsigned mask = __ballot_sync(kFullMask, f);
-    if (f) list[__popc(mask & ((1u << lane) - 1u))] = lane;
-    if (lane == 0) list[kStrMaxCount] = __popc(mask);
-  }
-  __syncthreads();
-  const int count = list[kStrMaxCount];
-  if (NR == 1 ? count != 1 : count < 2) return;
+  constexpr int RING = stream_ring(NR);
   const int64_t vbase = ((int64_t)blockIdx.x * kStrWarps + warp) * 32;
   const int64_t v = vbase + lane;
-  uint16_t* my = tiles + warp * 32 * kStrPad;
+  uint16_t* ring = tiles + warp * RING * 32 * kStrPad;  // this warp's RING tile slots
   const int ntile = K / kStrTK;
-  // tile t: instruction q loads rows 4q .. 4q+3, lane l the 16 bytes (l mod 8) of row 4q + l/8
-  auto load_tile = [&](int t, uint4 (&r)[8]) {
+  // tile t into slot t mod RING: copy q moves rows 4q .. 4q+3, lane l the 16 bytes
+  // (l mod 8) of row 4q + l/8 (coalesced); rows past V are zero-filled. One commit group
+  // per tile (an empty group past the last tile keeps the wait count uniform).
+  auto load_tile = [&](int t) {
+    if (t < ntile) {
+      uint16_t* slot = ring + (t % RING) * 32 * kStrPad;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int64_t vv = vbase + q * 4 + (lane >> 3);
-      r[q] = vv < V ? __ldg(reinterpret_cast<const uint4*>(W + vv * K + t * kStrTK + (lane & 7) * 8))
-                    : make_uint4(0, 0, 0, 0);
+      for (int q = 0; q < 8; ++q) {
+        const int row = q * 4 + (lane >> 3);
+        const int64_t vv = vbase + row;
+        uint16_t* dst = slot + row * kStrPad + (lane & 7) * 8;
+        if (vv < V)
+          cp_async16(dst, W + vv * K + t * kStrTK + (lane & 7) * 8);
+        else
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
     }
+    cp_async_commit();
   };
   for (int r0 = 0; r0 < count; r0 += NR) {
     const int nr = min(NR, count - r0);
@@ -328,17 +346,16 @@ __global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uin
     float acc[NR];
 #pragma unroll
     for (int j = 0; j < NR; ++j) acc[j] = 0.f;
-    // two tiles in flight in registers ahead of the one being consumed
-    uint4 b0[8], b1[8];
-    load_tile(0, b0);
-    if (ntile > 1) load_tile(1, b1);
-    auto step = [&](int t, uint4 (&buf)[8]) {
-      __syncwarp();  // every lane is done with the previous tile
+    // RING - 1 tiles in flight ahead of the one being consumed, copied straight into
+    // the warp's shared-memory slots
+    __syncwarp();  // the slots' previous contents (earlier rows) are no longer read
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<uint4*>(my + (q * 4 + (lane >> 3)) * kStrPad + (lane & 7) * 8) = buf[q];
-      __syncwarp();
-      if (t + 2 < ntile) load_tile(t + 2, buf);
+    for (int t = 0; t < RING - 1; ++t) load_tile(t);
+    auto step = [&](int t) {
+      load_tile(t + RING - 1);       // into the slot consumed at step t - 1
+      cp_async_wait<RING - 1>();     // this lane's copies of tile t have landed
+      __syncwarp();                  // and every lane's
+      const uint16_t* my = ring + (t % RING) * 32 * kStrPad;
 #pragma unroll
       for (int c = 0; c < kStrTK / 8; ++c) {
         float w[8];
@@ -365,10 +382,11 @@ __global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uin
         }
       }
     };
-    for (int t = 0; t < ntile; t += 2) {
-      step(t, b0);
-      if (t + 1 < ntile) step(t + 1, b1);
+    for (int t = 0; t < ntile; ++t) {
+      step(t);
+      __syncwarp();  // every lane is done with slot t mod RING before it is refilled
     }
+    cp_async_wait<0>();
     // fp32 logits out, and this CTA's argmax of each row over its 128 entries (lowest
     // index on ties, NaN never wins): lanes by an xor tree, then the warps in order
 #pragma unroll
@@ -426,6 +444,38 @@ __global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uin
       tokens[list[f]] = b.i;
     }
   }
+}
+
+// Both streaming cases in one launch: the flagged rows are listed with one ballot (M <=
+// kStrMaxCount), then exactly one flagged row reads W once with one fp32 chain per lane
+// (stream_rows<1>), two or more read it once per group of 8 (stream_rows<8>), and no
+// flagged row returns at once.
+__global__ void __launch_bounds__(kStrThreads) recompute_stream_kernel(const uint16_t* __restrict__ h, int64_t ldh,
+                                                                      const uint16_t* __restrict__ W, int64_t V,
+                                                                      int K, int M, const int32_t* __restrict__ flags,
+                                                                      float* __restrict__ out,
+                                                                      ArgBest* __restrict__ arg_part,
+                                                                      int32_t* __restrict__ tokens,
+                                                                      unsigned int* __restrict__ ticket) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are complete from here on
+  pdl_trigger();
+  extern __shared__ __align__(16) uint8_t smem_str[];
+  __shared__ int list[kStrMaxCount + 1];  // flagged rows, ascending (M <= kStrMaxCount)
+  __shared__ ArgBest warp_arg[kStrWarps][8];
+  __shared__ int last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {  // the flagged rows in order: one ballot over M <= 24 rows
+    const bool f = lane < M && flags[lane] != 0;
+    const unsigned mask = __ballot_sync(kFullMask, f);
+    if (f) list[__popc(mask & ((1u << lane) - 1u))] = lane;
+    if (lane == 0) list[kStrMaxCount] = __popc(mask);
+  }
+  __syncthreads();
+  const int count = list[kStrMaxCount];
+  if (count == 1)
+    stream_rows<1>(h, ldh, W, V, K, out, arg_part, tokens, ticket, smem_str, list, count, warp_arg, last);
+  else if (count >= 2)
+    stream_rows<8>(h, ldh, W, V, K, out, arg_part, tokens, ticket, smem_str, list, count, warp_arg, last);
 }
 
 // Token of each flagged row = argmax of its fp32 logits (lowest index on ties), a cluster
