@@ -269,7 +269,7 @@ def e2e_pipelined(bi, wl, xh, steps: int, warmup: int, world: int):
 def traffic_from_profile():
     """Per-launch DRAM bytes of the N=14336 matmul launch from the committed ncu
     summary, or None if gemm.cuh changed since it was captured."""
-    path = os.path.join(ROOT, "profiles", "gemm_bf16_kernel_traffic.txt")
+    path = os.path.join(ROOT, "profiles", "gemm_bf16_pair_kernel_traffic.txt")
     src = os.path.join(ROOT, "invariant_deterministic_04_b200", "csrc", "gemm.cuh")
     try:
         rec = {}
@@ -710,7 +710,7 @@ def sweep_matmul(bi, device, pk, clocks_mhz, ms_list=M_SWEEP, calls=12):
             cold = _graph_per_call_us([lambda w=Ws[i % R]: bi.matmul(a, w, out=c) for i in range(max(calls, R))]) / 1e3
             ref = _graph_per_call_us([lambda w=Ws[i % R]: torch.matmul(a, w.t(), out=c)
                                       for i in range(max(calls, R))]) / 1e3
-            out.append({"M": m, "N": n, "tile_n": tile_n,
+            out.append({"M": m, "N": n, "tile_m": bi.matmul_tile_m(m, n), "tile_n": tile_n,
                         "warm_us": round(warm * 1e3, 2), "warm_tflops": round(flops / warm / 1e9, 1),
                         "warm_frac_peak": round(flops / warm / 1e9 / pk["bf16_tflops"], 3),
                         "cold_us": round(cold * 1e3, 2), "cold_tflops": round(flops / cold / 1e9, 1),
@@ -964,7 +964,9 @@ def run_ours(args, rank, world, local):
     sm_max = (clocks or {}).get("sm_max_mhz") or pk["sm_max_mhz"]
     sustained = ms_total > 2000.0 or (sm_mhz is not None and sm_mhz < 0.95 * sm_max)
     peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
-    roof = {"bound": "tensor", "kernel": "gemm_bf16_kernel (tcgen05), M=2048 N=14336 K=4096 launch",
+    roof = {"bound": "tensor",
+            "kernel": ("gemm_bf16_pair_kernel<256> (tcgen05.mma.cta_group::2, 256 x 256 tiles on SM pairs), "
+                       "M=2048 N=14336 K=4096 launch"),
             "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 3),
             "peak_kind": (f"bf16 {'sustained' if sustained else 'burst'} ({pk['source']}); timed region "
@@ -976,7 +978,7 @@ def run_ours(args, rank, world, local):
             "kernel_share": round(gemm_ms / sum(kernel_ms), 3)}
     if roof["traffic"] is None:
         roof["traffic_note"] = ("gemm.cuh differs from the file the committed ncu counters "
-                                "(profiles/gemm_bf16_kernel_traffic.txt) were taken with")
+                                "(profiles/gemm_bf16_pair_kernel_traffic.txt) were taken with")
     rms_ms = kernel_ms[0] / args.steps
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,

@@ -72,7 +72,7 @@ int bi_version(void);
 /* Compile-time constants of the invariant schedule. */
 #define BI_PAGE_TOKENS 16   /* tokens per KV page */
 #define BI_KV_SPLIT 256     /* tokens per attention split (fixed size, not a fixed count) */
-#define BI_GEMM_BM 128      /* matmul tile rows (tcgen05 M) */
+#define BI_GEMM_BM 128      /* matmul tile rows per CTA (tcgen05 M); see bi_matmul_tile_m */
 #define BI_GEMM_BN_MAX 256  /* widest matmul tile (tcgen05 N); see bi_matmul_tile_n */
 #define BI_GEMM_BK 64       /* matmul K block; K is summed block by block in ascending order */
 
@@ -94,14 +94,15 @@ bi_status bi_rmsnorm(const bi_bf16* x, int64_t ldx, const bi_bf16* w, bi_bf16* y
  *   C[m, n] = bf16_rne( sum_k A[m, k] * W[n, k] ),  fp32 accumulation in TMEM
  * A: [M, K] bf16 row-major (K contiguous), stride lda. W: [N, K] bf16 row-major
  * (the nn.Linear weight layout), stride ldw. C: [M, N] bf16, stride ldc; must not
- * overlap A or W. Each C[m, n] is one chain of tcgen05.mma instructions (128 rows x
- * tile-width columns x 16 k, bf16 operands, fp32 accumulator in tensor memory)
- * over k = 0, 16, 32, ... in ascending order, then one bf16 rounding; no split-K.
- * That chain is the same for every M and every position of the row or column
- * inside its tile. The tile width (bi_matmul_tile_n) only decides how the columns
- * are dealt out to CTAs, and it does not enter an element's arithmetic: the GPU
+ * overlap A or W. Each C[m, n] is one chain of tcgen05.mma instructions (bf16
+ * operands, fp32 accumulator in tensor memory; 16 k each) over k = 0, 16, 32, ...
+ * in ascending order, then one bf16 rounding; no split-K. That chain is the same
+ * for every M and every position of the row or column inside its tile. The tile
+ * (bi_matmul_tile_m rows: 128 on one SM, or 256 on a pair of SMs issuing
+ * tcgen05.mma.cta_group::2; bi_matmul_tile_n columns) only decides how rows and
+ * columns are dealt out to SMs and does not enter an element's arithmetic: the GPU
  * tests check that every row of every M in 1..2048 equals the same row of the
- * 2048-row product, bit for bit, across the widths the sweep uses.
+ * 2048-row product, bit for bit, across the tiles the sweep uses.
  * M == 0 or N == 0 is a no-op. Requires K % 64 == 0, K >= 64, N % 8 == 0.
  */
 bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw, bi_bf16* C,
@@ -116,6 +117,15 @@ bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw
  * column, never how. Host only, launches nothing.
  */
 int bi_matmul_tile_n(int64_t M, int64_t N);
+
+/*
+ * Tile rows that bi_matmul uses for an M x N product on the current device: 128 (one
+ * CTA per tile) or 256 (a cluster of two CTAs per tile, from M = 256 on where the
+ * single-CTA tile would be 192 or 256 wide; each CTA loads half of the tile's A rows
+ * and half of its W rows, and one tcgen05.mma.cta_group::2 covers both). -1 if the
+ * device cannot be queried or M, N < 0. Host only, launches nothing.
+ */
+int bi_matmul_tile_m(int64_t M, int64_t N);
 
 /*
  * Workspace bytes for bi_attention_decode (rows = B) or bi_attention_prefill

@@ -6,7 +6,7 @@ memory and the current stream. There is no CPU or library fallback: if
 libbi.so is missing or fails to load, every call raises ``BIError``.
 
 Operations (see include/bi.h for the exact contracts):
-  rmsnorm, matmul, matmul_tile_n, attention_decode, attention_decode_static, attention_prefill,
+  rmsnorm, matmul, matmul_tile_n, matmul_tile_m, attention_decode, attention_decode_static, attention_prefill,
   kv_append, lmhead_argmax, gather_rows, rope, swiglu, add, log_softmax,
   token_logprob, row_mean, sampling_uniforms, sample, get_device_error.
 """
@@ -44,6 +44,7 @@ _SIGNATURES = {
     "bi_rmsnorm": ([_P, _I64, _P, _P, _I64, _I64, _I64, _F, _P], _I32),
     "bi_matmul": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _P], _I32),
     "bi_matmul_tile_n": ([_I64, _I64], _I32),
+    "bi_matmul_tile_m": ([_I64, _I64], _I32),
     "bi_attention_workspace_size": ([_I64, _I32, _I32, _I32], _SZ),
     "bi_attention_decode": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P, _SZ, _P], _I32),
     "bi_attention_decode_static": ([_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I32, _I32, _F, _P], _I32),
@@ -211,6 +212,15 @@ def matmul_tile_n(M: int, N: int) -> int:
     if w < 0:
         raise RuntimeError("bi_matmul_tile_n: device query failed")
     return w
+
+
+def matmul_tile_m(M: int, N: int) -> int:
+    """Tile rows bi_matmul uses for an M x N product on the current device: 128 (one
+    CTA per tile) or 256 (a pair of CTAs per tile); a scheduling choice like the width."""
+    r = int(lib().bi_matmul_tile_m(M, N))
+    if r < 0:
+        raise RuntimeError("bi_matmul_tile_m: device query failed")
+    return r
 
 
 def attention_workspace_size(rows: int, Hq: int, D: int, max_pages_per_seq: int) -> int:

@@ -42,6 +42,12 @@
 //     accumulators let the epilogue of one tile overlap the main loop of the next;
 //   * persistent grid of min(#tiles, #SMs) CTAs; tile t goes to CTA t mod grid,
 //     m-tiles of one W slice on neighbouring CTAs so the slice is read from HBM once;
+//   * from 256 rows on, where the single-CTA tile would be 192 or 256 wide, clusters
+//     of two CTAs compute 256 x 192 or 256 x 256 tiles with tcgen05.mma.cta_group::2
+//     (gemm_bf16_pair_kernel; pick_pair): each CTA loads half of the tile's A rows and
+//     half of its W rows, so a K block moves a third less into each SM's shared memory
+//     (M = 2048, N = 14336, K = 4096 on a B200: 164 us against 182 us for 128 x 256
+//     tiles, same bits);
 //   * launched as a programmatic dependent of the previous kernel on the stream: the
 //     barrier set-up, TMEM allocation and tensor-map prefetch overlap that kernel's
 //     tail, and the TMA thread waits for it (pdl_wait) before the first load;
@@ -324,6 +330,224 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// CTA-pair variant for large M: a cluster of two CTAs computes a 256 x PBN tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = PBN, 16 k): CTA r of the pair holds A rows
+// 128r .. 128r+127 and W rows (output columns) r*PBN/2 .. (r+1)*PBN/2-1 of the tile,
+// and its tensor memory receives output rows 128r .. 128r+127, all PBN columns. Each
+// element is still one chain of MMAs over k in ascending order (the pair instruction
+// sums the same 16-wide k slices of the same row and column), so the bits equal the
+// single-CTA kernel's. Per SM and K block the pair moves 16 KB of A and PBN/2 rows of
+// W into shared memory, where a 128 x 256 single-CTA tile moves 16 KB + 256 rows.
+//   * both CTAs' warp 0 loads its own halves into its own ring and counts the bytes on
+//     the leader's (rank 0) full barrier; the leader arms that barrier with both CTAs'
+//     bytes;
+//   * the leader's warp 1 issues the pair MMAs and commits each stage to both CTAs'
+//     empty barriers and each finished accumulator to both CTAs' tfull barriers;
+//   * both CTAs' warps 2-5 drain their own tensor memory and arrive on the leader's
+//     tempty barrier (256 arrivals);
+//   * the pair meets at cluster barriers after set-up and before tensor memory is freed,
+//     so neither CTA leaves while the other may still read its shared memory.
+template <int PBN>
+struct PairCfg {
+  static_assert(PBN % 32 == 0 && PBN >= 64 && PBN <= 256, "pair tile width");
+  static constexpr int W_ROWS = PBN / 2;                    // W rows one CTA loads per tile
+  static constexpr int STAGE = A_BYTES + W_ROWS * BK * 2;   // multiple of 1024: SW128 atoms stay aligned
+  static constexpr int STAGES = (kSmemBytes - 1024 - kBarBytes) / STAGE > 8 ? 8
+                                                                             : (kSmemBytes - 1024 - kBarBytes) / STAGE;
+  static constexpr int SMEM = 1024 + STAGES * STAGE + kBarBytes;
+  // kind::f16, bf16 x bf16 -> fp32, both K-major; N >> 3 at bit 17, M >> 4 at bit 24
+  static constexpr uint32_t IDESC =
+      (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PBN >> 3) << 17) | ((256u >> 4) << 24);
+  static_assert(STAGE % 1024 == 0, "stage alignment");
+  static_assert(STAGES >= 4 && SMEM <= kSmemBytes, "pair ring");
+};
+
+template <int PBN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          uint16_t* __restrict__ C, int64_t ldc, int M, int N, int K) {
+  using P = PairCfg<PBN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const Bars bars{base + (uint32_t)(P::STAGES * P::STAGE), P::STAGES};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + P::STAGES * P::STAGE + 8 * (2 * P::STAGES + 4));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = (int)blockIdx.x >> 1, npairs = (int)gridDim.x >> 1;
+  const int mt = (M + 255) / 256, nt = (N + PBN - 1) / PBN;
+  const int tiles = mt * nt;  // tile t: m-tile t % mt of W slice t / mt (one slice on neighbouring pairs)
+  const int nkb = K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P::STAGES; ++s) {
+      mbar_init(bars.full(s), 1);
+      mbar_init(bars.empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bars.tfull(a), 1);
+      mbar_init(bars.tempty(a), 2 * kEpiThreads);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_barrier();  // both CTAs' barriers are initialised and the pair's TMEM is allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) pdl_trigger();
+  uint32_t issued = 0, ph_bits = 0;  // the leader's armed stages and their parities
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();  // the previous kernel on the stream is done before the first load
+      int s = 0;
+      uint32_t ph = 0;
+      for (int t = pair; t < tiles && !*abort_flag; t += npairs) {
+        const int m0 = (t % mt) * 256 + (int)rank * 128, n0 = (t / mt) * PBN + (int)rank * P::W_ROWS;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(bars.empty(s), ph ^ 1u)) {
+            *abort_flag = 1;
+            break;
+          }
+          const uint32_t full_leader = map_to_rank(bars.full(s), 0);
+          if (leader) {
+            mbar_arrive_expect_tx(bars.full(s), 2u * (uint32_t)P::STAGE);
+            note_fill(issued, ph_bits, s, ph);
+          }
+          const uint32_t st = base + (uint32_t)s * P::STAGE;
+          tma_load_2d_pair(st, &tmA, kb * BK, m0, full_leader);
+          tma_load_2d_pair(st + A_BYTES, &tmB, kb * BK, n0, full_leader);
+          if (++s == P::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      for (int t = pair; t < tiles && !*abort_flag; t += npairs) {
+        if (!mbar_wait(bars.tempty(acc), aph ^ 1u)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * 256);
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(bars.full(s), ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = base + (uint32_t)s * P::STAGE, b = a + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16_pair(d, sw128_desc(a + kk * 32), sw128_desc(b + kk * 32), P::IDESC, (kb | kk) != 0 ? 1u : 0u);
+          tc_commit_pair_mc(bars.empty(s), (uint16_t)0x3);  // both CTAs' stage s is free once read
+          if (++s == P::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_commit_pair_mc(bars.tfull(acc), (uint16_t)0x3);  // both halves of the accumulator are complete
+        acc ^= 1;
+        if (acc == 0) aph ^= 1u;
+      }
+    }
+  } else {  // ---- epilogue: warps 2..5 of both CTAs; warp w reads TMEM lanes 32*(w%4) .. +31
+    const int quarter = warp & 3;
+    const uint32_t tempty_leader0 = map_to_rank(bars.tempty(0), 0), tempty_leader1 = map_to_rank(bars.tempty(1), 0);
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int t = pair; t < tiles; t += npairs) {
+      const int m0 = (t % mt) * 256 + (int)rank * 128, n0 = (t / mt) * PBN;
+      const bool ok = __all_sync(kFullMask, mbar_wait(bars.tfull(acc), aph));
+      if (!ok || *abort_flag) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int row = m0 + quarter * 32 + lane;
+      uint16_t* crow = C + (int64_t)row * ldc;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * 256);
+#pragma unroll 1
+      for (int c = 0; c < PBN / 32; ++c) {
+        uint32_t r[32];
+        __syncwarp();  // tcgen05.ld is .sync.aligned: the warp must be converged
+        tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
+        tmem_wait_ld();
+        const int col = n0 + c * 32;
+        if (row < M && col < N) {
+          if (col + 32 <= N) {
+            uint4* dst = reinterpret_cast<uint4*>(crow + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              dst[v] = o;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (col + e < N) crow[col + e] = to_bf16_bits(__uint_as_float(r[e]));
+          }
+        }
+      }
+      tc_fence_before();
+      if (leader)
+        mbar_arrive(bars.tempty(acc));
+      else
+        mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && warp == 0 && lane == 0) {
+    if (leader) {
+      drain_copies(bars.bar0, 8, issued, ph_bits);  // the armed stages count both CTAs' copies
+    } else {
+      // this CTA's copies are counted on the leader's barriers: give any still in flight
+      // a bounded time to land before the pair is released
+      const uint64_t t0 = global_timer_ns();
+      while (global_timer_ns() - t0 < 200000ull) {
+      }
+    }
+  }
+  __syncthreads();
+  cluster_barrier();  // neither CTA leaves while the other's MMAs or copies may use its shared memory
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -412,6 +636,21 @@ inline int pick_bn(int64_t M, int64_t N, int sms) {
   return best;
 }
 
+// Width of the CTA-pair tile (256 rows x 256 or 192 columns) for an M x N product, or
+// 0 for the single-CTA kernel. Pairs from 256 rows on, where the single-CTA choice is a
+// wide tile (192 or 256): a pair moves a third less into each SM's shared memory per
+// K block. Of the two pair widths, the one with the lower cost of whole rounds of tiles
+// over the pairs (sms / 2 clusters), a 256 x 192 tile costing 8/9 of a 256 x 256 one
+// (as measured on a B200: the time of a tile falls more slowly than its width).
+inline int pick_pair(int64_t M, int64_t N, int sms) {
+  if (M < 256 || pick_bn(M, N, sms) < 192) return 0;
+  const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
+  const int64_t mt = (M + 255) / 256;
+  const int64_t r256 = (mt * ((N + 255) / 256) + pairs - 1) / pairs;
+  const int64_t r192 = (mt * ((N + 191) / 192) + pairs - 1) / pairs;
+  return 8 * r192 < 9 * r256 ? 192 : 256;
+}
+
 // The stage ring for an M-row product with tile width bn. From 65 rows of A on: full
 // 128-row A slots in 198 KB, two K blocks per stage where that leaves three stages
 // (tile widths up to 128), else one (width 256: four stages). Up to 64 rows: the A
@@ -462,6 +701,30 @@ inline bi_status launch_kps(const uint16_t* A, int64_t lda, const uint16_t* W, i
              : BI_ERR_CUDA;
 }
 
+// The CTA-pair kernel with tile width PBN: one cluster of two CTAs per 256 x PBN tile
+// at a time, as many clusters as can be resident at once (queried once per device: a
+// cluster's two CTAs share a GPC, so odd SM counts per GPC can leave an SM out).
+template <int PBN>
+inline int pair_clusters(int dev) {
+  using P = PairCfg<PBN>;
+  static std::once_flag once[64];
+  static int clusters[64];
+  if (dev < 0 || dev >= 64) return 0;
+  std::call_once(once[dev], [&] {
+    int n = 0;
+    if (cudaFuncSetAttribute(gemm_bf16_pair_kernel<PBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM) ==
+        cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = P::SMEM;
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_pair_kernel<PBN>, &cfg) != cudaSuccess) n = 0;
+    }
+    clusters[dev] = n > 0 ? n : 0;
+  });
+  return clusters[dev];
+}
+
 template <int BN>
 inline bi_status launch_bn(const uint16_t* A, int64_t lda, const uint16_t* W, int64_t ldw, uint16_t* C,
                            int64_t ldc, int64_t M, int64_t N, int64_t K, int dev, int sms, cudaStream_t st) {
@@ -475,6 +738,26 @@ inline bi_status launch_bn(const uint16_t* A, int64_t lda, const uint16_t* W, in
   return launch_kps<BN, 1, true>(A, lda, W, ldw, C, ldc, M, N, K, L, dev, sms, st);
 }
 
+// An M x N product on CTA pairs with tile width PBN: one cluster of two CTAs per
+// 256 x PBN tile at a time, as many clusters as can be resident at once. Tiles of the
+// last round (fewer than the pairs) are not cut up: a dependent pair MMA takes about as
+// long at any width (narrower tiles for that round, or handing its tiles to the
+// single-CTA kernel in a second launch, measured no faster on a B200).
+template <int PBN>
+inline bi_status launch_pair(const uint16_t* A, int64_t lda, const uint16_t* W, int64_t ldw, uint16_t* C,
+                             int64_t ldc, int64_t M, int64_t N, int64_t K, int dev, cudaStream_t st) {
+  const int clusters = pair_clusters<PBN>(dev);
+  if (clusters <= 0) return BI_ERR_CUDA;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, lda, 128) || !make_map(&tb, W, N, K, ldw, PBN / 2)) return BI_ERR_CUDA;
+  const int64_t tiles = ((M + 255) / 256) * ((N + PBN - 1) / PBN);
+  const int pairs = (int)(tiles < clusters ? tiles : clusters);
+  return launch_pdl(gemm_bf16_pair_kernel<PBN>, dim3(2 * pairs), dim3(kThreads), (size_t)PairCfg<PBN>::SMEM, st,
+                    ta, tb, C, ldc, (int)M, (int)N, (int)K) == cudaSuccess
+             ? BI_OK
+             : BI_ERR_CUDA;
+}
+
 // bn: tile width (0 = pick_bn's choice for this device).
 inline bi_status launch(const uint16_t* A, int64_t lda, const uint16_t* W, int64_t ldw, uint16_t* C,
                         int64_t ldc, int64_t M, int64_t N, int64_t K, cudaStream_t st, int bn = 0) {
@@ -482,7 +765,14 @@ inline bi_status launch(const uint16_t* A, int64_t lda, const uint16_t* W, int64
   if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
   const int sms = device_sms(dev);
   if (sms <= 0) return BI_ERR_CUDA;
-  if (bn == 0) bn = pick_bn(M, N, sms);
+  if (bn == 0) {
+    // large products: CTA pairs on 256-row tiles (the same element chains)
+    switch (pick_pair(M, N, sms)) {
+      case 256: return launch_pair<256>(A, lda, W, ldw, C, ldc, M, N, K, dev, st);
+      case 192: return launch_pair<192>(A, lda, W, ldw, C, ldc, M, N, K, dev, st);
+      default: bn = pick_bn(M, N, sms);
+    }
+  }
   switch (bn) {
     case 32: return launch_bn<32>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
     case 64: return launch_bn<64>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);

@@ -276,7 +276,18 @@ int bi_matmul_tile_n(int64_t M, int64_t N) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
   const int sms = bi::gemm::device_sms(dev);
-  return sms > 0 ? bi::gemm::pick_bn(M, N, sms) : -1;
+  if (sms <= 0) return -1;
+  const int pair = bi::gemm::pick_pair(M, N, sms);
+  return pair ? pair : bi::gemm::pick_bn(M, N, sms);
+}
+
+int bi_matmul_tile_m(int64_t M, int64_t N) {
+  if (M < 0 || N < 0) return -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  const int sms = bi::gemm::device_sms(dev);
+  if (sms <= 0) return -1;
+  return bi::gemm::pick_pair(M, N, sms) ? 256 : 128;
 }
 
 size_t bi_attention_workspace_size(int64_t rows, int Hq, int D, int max_pages_per_seq) {

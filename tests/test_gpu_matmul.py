@@ -1,6 +1,7 @@
 """bi_matmul on the GPU (tcgen05 + TMA): parity with the fp64 oracle, exact
 small-integer products (pins the shared-memory layout and descriptors),
-row-position independence inside a 128-row tile, bit-invariance across the M
+row-position independence inside a 128-row tile, ragged products on CTA-pair
+(256-row) tiles, bit-invariance across the M
 sweep at K=4096, N in {4096, 6144, 14336}, run-to-run bit-exactness, and the
 RMSNorm -> matmul chain of the 32 x 512 -> 1024 configuration."""
 import numpy as np
@@ -24,6 +25,23 @@ def test_matmul_matches_oracle(M, N, K):
     a, w = synth.matmul_inputs(M, N, K, seed=M * 7 + N + K)
     c = bi.matmul(a.to(dev()), w.to(dev()))
     assert max_rel(c, oracle.matmul(synth.to_f64(a), synth.to_f64(w))) <= TOL_BF16
+
+
+# Ragged products on CTA pairs (256-row tiles; on a 148-SM B200 (1100, 4000), (1000,
+# 5992) and (513, 6152) take 192-wide tiles, the others 256-wide): a last pair tile whose
+# second CTA holds no valid row (M = 1100, 1000), a last tile whose W half lies past N, a
+# 32-column chunk cut by N (N = 5992, 4104, 6152), odd M, and last rounds with a few
+# tiles (M = 1024, 2047 at N = 14336) or a partial W slice (M = 513, N = 6152).
+@pytest.mark.parametrize("M,N,K", [(1100, 4000, 512), (1000, 5992, 320), (2047, 4104, 256), (600, 6000, 1024),
+                                   (1024, 14336, 128), (2047, 14336, 64), (513, 6152, 256)])
+def test_matmul_pair_tiles_match_oracle(M, N, K):
+    assert bi.matmul_tile_m(M, N) == 256
+    a, w = synth.matmul_inputs(M, N, K, seed=M + N + K)
+    c = bi.matmul(a.to(dev()), w.to(dev()))
+    assert max_rel(c, oracle.matmul(synth.to_f64(a), synth.to_f64(w))) <= TOL_BF16
+    # the same rows on single-CTA tiles (fewer than 256 rows) give the same bits
+    for r0 in (0, M - 7):
+        assert same_bits(bi.matmul(a[r0:r0 + 7].to(dev()), w.to(dev())), c[r0:r0 + 7]), r0
 
 
 def test_matmul_small_integers_exact():
@@ -70,7 +88,9 @@ def test_matmul_batch_invariant_over_m_sweep(N):
     for m in M_SWEEP:
         assert same_bits(bi.matmul(a[:m].contiguous(), w), full[:m]), m
     # the sweep crosses tile widths (on a 148-SM B200: 32/64/128/256, and 192 at N = 6144)
+    # and both tile heights: 128-row tiles on one CTA, 256-row tiles on a CTA pair
     assert len({bi.matmul_tile_n(m, N) for m in M_SWEEP + [2048]}) >= 2
+    assert {bi.matmul_tile_m(m, N) for m in M_SWEEP + [2048]} == {128, 256}
     # rows in a permuted batch and a batch taken from the middle
     perm = synth.permutation(2048, 25).to(dev())
     assert same_bits(bi.matmul(a[perm].contiguous(), w), full[perm])
