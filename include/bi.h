@@ -120,7 +120,7 @@ int bi_matmul_tile_n(int64_t M, int64_t N);
 
 /*
  * Tile rows that bi_matmul uses for an M x N product on the current device: 128 (one
- * CTA per tile) or 256 (a cluster of two CTAs per tile, from M = 256 on where the
+ * CTA per tile) or 256 (a cluster of two CTAs per tile, from M = 129 on where the
  * single-CTA tile would be 192 or 256 wide; each CTA loads half of the tile's A rows
  * and half of its W rows, and one tcgen05.mma.cta_group::2 covers both). -1 if the
  * device cannot be queried or M, N < 0. Host only, launches nothing.

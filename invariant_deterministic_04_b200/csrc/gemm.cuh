@@ -42,7 +42,7 @@
 //     accumulators let the epilogue of one tile overlap the main loop of the next;
 //   * persistent grid of min(#tiles, #SMs) CTAs; tile t goes to CTA t mod grid,
 //     m-tiles of one W slice on neighbouring CTAs so the slice is read from HBM once;
-//   * from 256 rows on, where the single-CTA tile would be 192 or 256 wide, clusters
+//   * from 129 rows on, where the single-CTA tile would be 192 or 256 wide, clusters
 //     of two CTAs compute 256 x 192 or 256 x 256 tiles with tcgen05.mma.cta_group::2
 //     (gemm_bf16_pair_kernel; pick_pair): each CTA loads half of the tile's A rows and
 //     half of its W rows, so a K block moves a third less into each SM's shared memory
@@ -637,13 +637,13 @@ inline int pick_bn(int64_t M, int64_t N, int sms) {
 }
 
 // Width of the CTA-pair tile (256 rows x 256 or 192 columns) for an M x N product, or
-// 0 for the single-CTA kernel. Pairs from 256 rows on, where the single-CTA choice is a
-// wide tile (192 or 256): a pair moves a third less into each SM's shared memory per
-// K block. Of the two pair widths, the one with the lower cost of whole rounds of tiles
+// 0 for the single-CTA kernel. Pairs from 129 rows on (two 128-row m-tiles become one
+// pair tile on as many SMs), where the single-CTA choice is a wide tile (192 or 256): a
+// pair moves a third less into each SM's shared memory per K block. Of the two pair widths, the one with the lower cost of whole rounds of tiles
 // over the pairs (sms / 2 clusters), a 256 x 192 tile costing 8/9 of a 256 x 256 one
 // (as measured on a B200: the time of a tile falls more slowly than its width).
 inline int pick_pair(int64_t M, int64_t N, int sms) {
-  if (M < 256 || pick_bn(M, N, sms) < 192) return 0;
+  if (M <= 128 || pick_bn(M, N, sms) < 192) return 0;
   const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
   const int64_t mt = (M + 255) / 256;
   const int64_t r256 = (mt * ((N + 255) / 256) + pairs - 1) / pairs;

@@ -29,11 +29,12 @@ def test_matmul_matches_oracle(M, N, K):
 
 # Ragged products on CTA pairs (256-row tiles; on a 148-SM B200 (1100, 4000), (1000,
 # 5992) and (513, 6152) take 192-wide tiles, the others 256-wide): a last pair tile whose
-# second CTA holds no valid row (M = 1100, 1000), a last tile whose W half lies past N, a
-# 32-column chunk cut by N (N = 5992, 4104, 6152), odd M, and last rounds with a few
-# tiles (M = 1024, 2047 at N = 14336) or a partial W slice (M = 513, N = 6152).
+# second CTA holds no valid row (M = 1100, 1000) or part of one (M = 200), a last tile
+# whose W half lies past N, a 32-column chunk cut by N (N = 5992, 4104, 6152), odd M, and
+# last rounds with a few tiles (M = 1024, 2047 at N = 14336) or a partial W slice
+# (M = 513, N = 6152).
 @pytest.mark.parametrize("M,N,K", [(1100, 4000, 512), (1000, 5992, 320), (2047, 4104, 256), (600, 6000, 1024),
-                                   (1024, 14336, 128), (2047, 14336, 64), (513, 6152, 256)])
+                                   (1024, 14336, 128), (2047, 14336, 64), (513, 6152, 256), (200, 14336, 64)])
 def test_matmul_pair_tiles_match_oracle(M, N, K):
     assert bi.matmul_tile_m(M, N) == 256
     a, w = synth.matmul_inputs(M, N, K, seed=M + N + K)
