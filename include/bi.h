@@ -109,6 +109,22 @@ bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw
                     int64_t ldc, int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
+ * Several products with the same A in one call: C_g = A * W_g^T for g = 0 .. count-1,
+ * each exactly as bi_matmul would compute it (bit for bit: the same MMA chain per
+ * element). A, M, K, lda as for bi_matmul; W, ldw, C, ldc, N: host arrays of count
+ * entries (read before the call returns), each entry with bi_matmul's requirements;
+ * no C_g may overlap A, any W_h or another C_h. 1 <= count <= BI_MATMUL_MULTI_MAX.
+ * When every product would run on CTA-pair tiles alone (bi_matmul_tile_m == 256), one
+ * launch takes the tiles of all of them in one list, so the SMs run whole rounds over
+ * the joint list instead of a short last round per product; otherwise the products
+ * are launched one after another. M == 0 is a no-op; a product with N == 0 is skipped.
+ */
+#define BI_MATMUL_MULTI_MAX 3
+bi_status bi_matmul_multi(const bi_bf16* A, int64_t lda, int count, const bi_bf16* const* W, const int64_t* ldw,
+                          bi_bf16* const* C, const int64_t* ldc, const int64_t* N, int64_t M, int64_t K,
+                          void* stream);
+
+/*
  * Tile width (32, 64, 128, 192 or 256 columns) that bi_matmul uses for an M x N
  * product on the current device; -1 if the device cannot be queried or M, N < 0.
  * Narrow tiles spread a small-M product over more SMs (each streams a thin slice

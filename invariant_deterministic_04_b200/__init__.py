@@ -6,7 +6,7 @@ memory and the current stream. There is no CPU or library fallback: if
 libbi.so is missing or fails to load, every call raises ``BIError``.
 
 Operations (see include/bi.h for the exact contracts):
-  rmsnorm, matmul, matmul_tile_n, matmul_tile_m, attention_decode, attention_decode_static, attention_prefill,
+  rmsnorm, matmul, matmul_multi, matmul_tile_n, matmul_tile_m, attention_decode, attention_decode_static, attention_prefill,
   kv_append, lmhead_argmax, gather_rows, rope, swiglu, add, log_softmax,
   token_logprob, row_mean, sampling_uniforms, sample, get_device_error.
 """
@@ -43,6 +43,7 @@ _SIGNATURES = {
     "bi_version": ([], _I32),
     "bi_rmsnorm": ([_P, _I64, _P, _P, _I64, _I64, _I64, _F, _P], _I32),
     "bi_matmul": ([_P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _P], _I32),
+    "bi_matmul_multi": ([_P, _I64, _I32, _P, _P, _P, _P, _P, _I64, _I64, _P], _I32),
     "bi_matmul_tile_n": ([_I64, _I64], _I32),
     "bi_matmul_tile_m": ([_I64, _I64], _I32),
     "bi_attention_workspace_size": ([_I64, _I32, _I32, _I32], _SZ),
@@ -203,6 +204,45 @@ def matmul(a: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, st
         _check("bi_matmul", lib().bi_matmul(_ptr(a), a.stride(0), _ptr(w), w.stride(0), _ptr(c), c.stride(0), M, N,
                                            K, _stream()))
     return c
+
+
+MATMUL_MULTI_MAX = 3
+
+
+def matmul_multi(a: torch.Tensor, ws, outs=None, stream=None):
+    """[A W_g^T for each W_g in ws] in one call (at most MATMUL_MULTI_MAX products), each
+    bit-identical to matmul(a, W_g); one launch when every product runs on CTA-pair tiles."""
+    ws = list(ws)
+    if not 1 <= len(ws) <= MATMUL_MULTI_MAX:
+        raise ValueError(f"between 1 and {MATMUL_MULTI_MAX} weight matrices, got {len(ws)}")
+    _req(a, torch.bfloat16, "a", 2)
+    if a.stride(1) != 1:
+        raise ValueError("a rows must be contiguous")
+    M, K = a.shape
+    for g, w in enumerate(ws):
+        _req(w, torch.bfloat16, f"ws[{g}]", 2)
+        if w.stride(1) != 1:
+            raise ValueError(f"ws[{g}] rows must be contiguous")
+        if w.shape[1] != K:
+            raise ValueError(f"inner dimensions differ: {tuple(a.shape)} x {tuple(w.shape)}^T")
+    if outs is not None:
+        outs = list(outs)
+        if len(outs) != len(ws):
+            raise ValueError(f"{len(ws)} weight matrices but {len(outs)} outputs")
+        for g, (w, c) in enumerate(zip(ws, outs)):
+            _out(c, torch.bfloat16, (M, w.shape[0]), f"outs[{g}]", strided_rows=True)
+    device = _same_device(a, *ws, *(outs or []))
+    n = len(ws)
+    with _on(device, stream):
+        cs = [torch.empty((M, w.shape[0]), dtype=torch.bfloat16, device=device) for w in ws] if outs is None else outs
+        wp = (ctypes.c_void_p * n)(*[w.data_ptr() for w in ws])
+        cp = (ctypes.c_void_p * n)(*[c.data_ptr() for c in cs])
+        ldw = (ctypes.c_int64 * n)(*[w.stride(0) for w in ws])
+        ldc = (ctypes.c_int64 * n)(*[c.stride(0) for c in cs])
+        ns = (ctypes.c_int64 * n)(*[w.shape[0] for w in ws])
+        _check("bi_matmul_multi", lib().bi_matmul_multi(_ptr(a), a.stride(0), n, wp, ldw, cp, ldc, ns, M, K,
+                                                         _stream()))
+    return cs
 
 
 def matmul_tile_n(M: int, N: int) -> int:

@@ -55,6 +55,7 @@
 //     BI_ERR_DEVICE_TIMEOUT, all roles leave their loops, TMEM is freed.
 #pragma once
 
+#include <climits>
 #include <mutex>
 
 #include "device.cuh"
@@ -362,10 +363,26 @@ struct PairCfg {
   static_assert(STAGES >= 4 && SMEM <= kSmemBytes, "pair ring");
 };
 
+// Up to three products C_g = A W_g^T with the same A (M x K) in one launch of the pair
+// kernel: their tiles form one list (product 0's, then 1's, then 2's), so the pairs run
+// whole rounds over all of them instead of a short last round per product. Fields are
+// picked by g with selects, not indexed, so the parameter block stays in constant memory.
+struct PairProblems {
+  uint16_t* C0;
+  uint16_t* C1;
+  uint16_t* C2;
+  int64_t ldc0, ldc1, ldc2;
+  int N0, N1, N2;
+  int start1, start2, total;  // first tile of products 1 and 2; tiles in all
+  int count;
+};
+constexpr int kMaxProblems = 3;
+
 template <int PBN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                          uint16_t* __restrict__ C, int64_t ldc, int M, int N, int K) {
+    gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                          const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+                          const PairProblems pp, int M, int K) {
   using P = PairCfg<PBN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -379,8 +396,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
   const int pair = (int)blockIdx.x >> 1, npairs = (int)gridDim.x >> 1;
-  const int mt = (M + 255) / 256, nt = (N + PBN - 1) / PBN;
-  const int tiles = mt * nt;  // tile t: m-tile t % mt of W slice t / mt (one slice on neighbouring pairs)
+  const int mt = (M + 255) / 256;
+  const int tiles = pp.total;
+  // tile t: product g (the last whose first tile is <= t); within it, local tile u is
+  // m-tile u % mt of W slice u / mt (the m-tiles of one slice on neighbouring pairs)
+  auto product_of = [&](int t, int& u) -> int {
+    const int g = (pp.count > 2 && t >= pp.start2) ? 2 : ((pp.count > 1 && t >= pp.start1) ? 1 : 0);
+    u = t - (g == 2 ? pp.start2 : (g == 1 ? pp.start1 : 0));
+    return g;
+  };
   const int nkb = K / BK;
 
   if (threadIdx.x == 0) {
@@ -396,7 +420,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     fence_proxy_async_smem();
     prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmB0);
+    if (pp.count > 1) prefetch_tensormap(&tmB1);
+    if (pp.count > 2) prefetch_tensormap(&tmB2);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), 512);
@@ -416,7 +442,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       for (int t = pair; t < tiles && !*abort_flag; t += npairs) {
-        const int m0 = (t % mt) * 256 + (int)rank * 128, n0 = (t / mt) * PBN + (int)rank * P::W_ROWS;
+        int u;
+        const int g = product_of(t, u);
+        const CUtensorMap* tmB = g == 0 ? &tmB0 : (g == 1 ? &tmB1 : &tmB2);
+        const int m0 = (u % mt) * 256 + (int)rank * 128, n0 = (u / mt) * PBN + (int)rank * P::W_ROWS;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(bars.empty(s), ph ^ 1u)) {
             *abort_flag = 1;
@@ -429,7 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           const uint32_t st = base + (uint32_t)s * P::STAGE;
           tma_load_2d_pair(st, &tmA, kb * BK, m0, full_leader);
-          tma_load_2d_pair(st + A_BYTES, &tmB, kb * BK, n0, full_leader);
+          tma_load_2d_pair(st + A_BYTES, tmB, kb * BK, n0, full_leader);
           if (++s == P::STAGES) {
             s = 0;
             ph ^= 1u;
@@ -480,7 +509,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t aph = 0;
     for (int t = pair; t < tiles; t += npairs) {
-      const int m0 = (t % mt) * 256 + (int)rank * 128, n0 = (t / mt) * PBN;
+      int u;
+      const int g = product_of(t, u);
+      uint16_t* const C = g == 0 ? pp.C0 : (g == 1 ? pp.C1 : pp.C2);
+      const int64_t ldc = g == 0 ? pp.ldc0 : (g == 1 ? pp.ldc1 : pp.ldc2);
+      const int N = g == 0 ? pp.N0 : (g == 1 ? pp.N1 : pp.N2);
+      const int m0 = (u % mt) * 256 + (int)rank * 128, n0 = (u / mt) * PBN;
       const bool ok = __all_sync(kFullMask, mbar_wait(bars.tfull(acc), aph));
       if (!ok || *abort_flag) {
         *abort_flag = 1;
@@ -743,17 +777,53 @@ inline bi_status launch_bn(const uint16_t* A, int64_t lda, const uint16_t* W, in
 // last round (fewer than the pairs) are not cut up: a dependent pair MMA takes about as
 // long at any width (narrower tiles for that round, or handing its tiles to the
 // single-CTA kernel in a second launch, measured no faster on a B200).
+// One product of a multi-product launch: C = A W^T, W [N, K] with row stride ldw.
+struct Product {
+  const uint16_t* W;
+  int64_t ldw;
+  uint16_t* C;
+  int64_t ldc;
+  int64_t N;
+};
+
 template <int PBN>
-inline bi_status launch_pair(const uint16_t* A, int64_t lda, const uint16_t* W, int64_t ldw, uint16_t* C,
-                             int64_t ldc, int64_t M, int64_t N, int64_t K, int dev, cudaStream_t st) {
+inline bi_status launch_pair(const uint16_t* A, int64_t lda, const Product* prods, int count, int64_t M, int64_t K,
+                             int dev, cudaStream_t st) {
   const int clusters = pair_clusters<PBN>(dev);
   if (clusters <= 0) return BI_ERR_CUDA;
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K, lda, 128) || !make_map(&tb, W, N, K, ldw, PBN / 2)) return BI_ERR_CUDA;
-  const int64_t tiles = ((M + 255) / 256) * ((N + PBN - 1) / PBN);
-  const int pairs = (int)(tiles < clusters ? tiles : clusters);
+  if (count < 1 || count > kMaxProblems) return BI_ERR_SHAPE;
+  CUtensorMap ta, tb[kMaxProblems];
+  if (!make_map(&ta, A, M, K, lda, 128)) return BI_ERR_CUDA;
+  const int64_t mt = (M + 255) / 256;
+  int64_t start[kMaxProblems + 1] = {0, 0, 0, 0};
+  for (int g = 0; g < count; ++g) {
+    if (!make_map(&tb[g], prods[g].W, prods[g].N, K, prods[g].ldw, PBN / 2)) return BI_ERR_CUDA;
+    start[g + 1] = start[g] + mt * ((prods[g].N + PBN - 1) / PBN);
+  }
+  for (int g = count; g < kMaxProblems; ++g) {
+    tb[g] = tb[0];
+    start[g + 1] = start[g];
+  }
+  if (start[count] > INT_MAX / 2) return BI_ERR_SHAPE;
+  const Product& p1 = prods[count > 1 ? 1 : 0];
+  const Product& p2 = prods[count > 2 ? 2 : 0];
+  PairProblems pp{};
+  pp.C0 = prods[0].C;
+  pp.C1 = p1.C;
+  pp.C2 = p2.C;
+  pp.ldc0 = prods[0].ldc;
+  pp.ldc1 = p1.ldc;
+  pp.ldc2 = p2.ldc;
+  pp.N0 = (int)prods[0].N;
+  pp.N1 = (int)p1.N;
+  pp.N2 = (int)p2.N;
+  pp.start1 = (int)start[1];
+  pp.start2 = (int)start[2];
+  pp.total = (int)start[count];
+  pp.count = count;
+  const int pairs = (int)(pp.total < clusters ? pp.total : clusters);
   return launch_pdl(gemm_bf16_pair_kernel<PBN>, dim3(2 * pairs), dim3(kThreads), (size_t)PairCfg<PBN>::SMEM, st,
-                    ta, tb, C, ldc, (int)M, (int)N, (int)K) == cudaSuccess
+                    ta, tb[0], tb[1], tb[2], pp, (int)M, (int)K) == cudaSuccess
              ? BI_OK
              : BI_ERR_CUDA;
 }
@@ -768,8 +838,14 @@ inline bi_status launch(const uint16_t* A, int64_t lda, const uint16_t* W, int64
   if (bn == 0) {
     // large products: CTA pairs on 256-row tiles (the same element chains)
     switch (pick_pair(M, N, sms)) {
-      case 256: return launch_pair<256>(A, lda, W, ldw, C, ldc, M, N, K, dev, st);
-      case 192: return launch_pair<192>(A, lda, W, ldw, C, ldc, M, N, K, dev, st);
+      case 256: {
+        const Product p{W, ldw, C, ldc, N};
+        return launch_pair<256>(A, lda, &p, 1, M, K, dev, st);
+      }
+      case 192: {
+        const Product p{W, ldw, C, ldc, N};
+        return launch_pair<192>(A, lda, &p, 1, M, K, dev, st);
+      }
       default: bn = pick_bn(M, N, sms);
     }
   }
@@ -781,6 +857,37 @@ inline bi_status launch(const uint16_t* A, int64_t lda, const uint16_t* W, int64
     case 256: return launch_bn<256>(A, lda, W, ldw, C, ldc, M, N, K, dev, sms, st);
     default: return BI_ERR_UNSUPPORTED;
   }
+}
+
+// Several products with the same A: C_g = A W_g^T, g < count (at most kMaxProblems).
+// When every product would run on CTA pairs alone (pick_pair), one launch of the pair
+// kernel takes all their tiles in one list, with the tile width chosen the way
+// pick_pair chooses it, from the joint tile counts; otherwise each product is its own
+// launch. Either way each element is the same MMA chain as in a bi_matmul call alone.
+inline bi_status launch_multi(const uint16_t* A, int64_t lda, const Product* prods, int count, int64_t M, int64_t K,
+                              cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
+  const int sms = device_sms(dev);
+  if (sms <= 0) return BI_ERR_CUDA;
+  bool joint = count > 1;
+  for (int g = 0; g < count && joint; ++g) joint = pick_pair(M, prods[g].N, sms) != 0;
+  if (joint) {
+    const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1, mt = (M + 255) / 256;
+    int64_t t256 = 0, t192 = 0;
+    for (int g = 0; g < count; ++g) {
+      t256 += mt * ((prods[g].N + 255) / 256);
+      t192 += mt * ((prods[g].N + 191) / 192);
+    }
+    const int64_t r256 = (t256 + pairs - 1) / pairs, r192 = (t192 + pairs - 1) / pairs;
+    return 8 * r192 < 9 * r256 ? launch_pair<192>(A, lda, prods, count, M, K, dev, st)
+                               : launch_pair<256>(A, lda, prods, count, M, K, dev, st);
+  }
+  for (int g = 0; g < count; ++g) {
+    const bi_status r = launch(A, lda, prods[g].W, prods[g].ldw, prods[g].C, prods[g].ldc, M, prods[g].N, K, st);
+    if (r != BI_OK) return r;
+  }
+  return BI_OK;
 }
 
 }  // namespace gemm

@@ -31,6 +31,26 @@ size_t span_bytes(int64_t rows, int64_t cols, int64_t ld, size_t elem) {
   return rows <= 0 ? 0 : (size_t)((rows - 1) * ld + cols) * elem;
 }
 
+// Whether two M-row blocks of 2-byte elements (rows of na / nb elements, lda / ldb
+// elements apart, na <= lda, nb <= ldb) share an element. Exact for equal row strides,
+// where column ranges of one wider matrix are disjoint: elements a + i*ld + j and
+// b + i'*ld + j' coincide iff (i - i')*ld + (j - j') = (b - a), and with both widths at
+// most ld only k = i - i' = floor((b - a) / ld) and k + 1 can give j - j' in (-nb, na).
+// Otherwise by the blocks' address spans.
+bool blocks_overlap(const void* a, int64_t lda, int64_t na, const void* b, int64_t ldb, int64_t nb, int64_t M) {
+  if (M <= 0 || na <= 0 || nb <= 0) return false;
+  const int64_t db = (int64_t)(reinterpret_cast<intptr_t>(b) - reinterpret_cast<intptr_t>(a));
+  if (lda != ldb || db % 2 != 0) return ranges_overlap(a, span_bytes(M, na, lda, 2), b, span_bytes(M, nb, ldb, 2));
+  const int64_t d = db / 2;
+  const int64_t k0 = d >= 0 ? d / lda : -((-d + lda - 1) / lda);
+  for (int64_t k = k0; k <= k0 + 1; ++k) {
+    if (k <= -M || k >= M) continue;
+    const int64_t r = d - k * lda;
+    if (r > -nb && r < na) return true;
+  }
+  return false;
+}
+
 int device_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -269,6 +289,35 @@ bi_status bi_matmul(const bi_bf16* A, int64_t lda, const bi_bf16* W, int64_t ldw
   if (ranges_overlap(C, cb, A, span_bytes(M, K, lda, 2)) || ranges_overlap(C, cb, W, span_bytes(N, K, ldw, 2)))
     return BI_ERR_SHAPE;
   return bi::gemm::launch(A, lda, W, ldw, C, ldc, M, N, K, as_stream(stream));
+}
+
+bi_status bi_matmul_multi(const bi_bf16* A, int64_t lda, int count, const bi_bf16* const* W, const int64_t* ldw,
+                          bi_bf16* const* C, const int64_t* ldc, const int64_t* N, int64_t M, int64_t K,
+                          void* stream) {
+  if (!A || !W || !ldw || !C || !ldc || !N) return BI_ERR_NULL;
+  if (count < 1 || count > BI_MATMUL_MULTI_MAX) return BI_ERR_SHAPE;
+  if (M < 0 || K < 64 || K % 64 != 0 || M > INT_MAX || K > INT_MAX || lda < K) return BI_ERR_SHAPE;
+  if (!aligned16(A) || lda % 8) return BI_ERR_ALIGN;
+  const size_t abytes = span_bytes(M, K, lda, 2);
+  bi::gemm::Product prods[BI_MATMUL_MULTI_MAX];
+  int live = 0;
+  for (int g = 0; g < count; ++g) {
+    if (!W[g] || !C[g]) return BI_ERR_NULL;
+    if (N[g] < 0 || N[g] % 8 != 0 || N[g] > INT_MAX || ldw[g] < K || ldc[g] < N[g]) return BI_ERR_SHAPE;
+    if (!aligned16(W[g]) || !aligned16(C[g]) || ldw[g] % 8 || ldc[g] % 8) return BI_ERR_ALIGN;
+  }
+  for (int g = 0; g < count; ++g) {
+    if (M == 0 || N[g] == 0) continue;
+    const size_t cb = span_bytes(M, N[g], ldc[g], 2);
+    if (ranges_overlap(C[g], cb, A, abytes)) return BI_ERR_SHAPE;
+    for (int h = 0; h < count; ++h) {
+      if (N[h] > 0 && ranges_overlap(C[g], cb, W[h], span_bytes(N[h], K, ldw[h], 2))) return BI_ERR_SHAPE;
+      if (h != g && blocks_overlap(C[g], ldc[g], N[g], C[h], ldc[h], N[h], M)) return BI_ERR_SHAPE;
+    }
+    prods[live++] = bi::gemm::Product{W[g], ldw[g], C[g], ldc[g], N[g]};
+  }
+  if (live == 0) return BI_OK;
+  return bi::gemm::launch_multi(A, lda, prods, live, M, K, as_stream(stream));
 }
 
 int bi_matmul_tile_n(int64_t M, int64_t N) {

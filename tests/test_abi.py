@@ -80,6 +80,40 @@ def test_matmul_validation(L):
     assert f(P, 512, P + 0x1000000, 512, P + 64, 64, 4, 64, 512, None) == SHAPE
 
 
+def test_matmul_multi_validation(L):
+    f = L.bi_matmul_multi
+    f.restype = ctypes.c_int
+    P = ctypes.c_void_p
+    f.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, P, P, P, P, ctypes.c_int64, ctypes.c_int64, P]
+
+    def arrays(ws, ldws, cs, ldcs, ns):
+        n = len(ws)
+        return ((P * n)(*ws), (ctypes.c_int64 * n)(*ldws), (P * n)(*cs), (ctypes.c_int64 * n)(*ldcs),
+                (ctypes.c_int64 * n)(*ns))
+
+    a, w0, w1, c0, c1 = 0x10000, 0x200000, 0x400000, 0x600000, 0x800000
+    ok = arrays([w0, w1], [64, 64], [c0, c1], [128, 256], [128, 256])
+    assert f(None, 64, 2, *ok, 4, 64, None) == 1                      # null A
+    assert f(a, 64, 2, None, ok[1], ok[2], ok[3], ok[4], 4, 64, None) == 1  # null array
+    assert f(a, 64, 2, *arrays([w0, 0], [64, 64], [c0, c1], [128, 256], [128, 256]), 4, 64, None) == 1
+    assert f(a, 64, 0, *ok, 4, 64, None) == 2                         # count 0
+    assert f(a, 64, 4, *arrays([w0] * 4, [64] * 4, [c0] * 4, [128] * 4, [128] * 4), 4, 64, None) == 2
+    assert f(a, 96, 2, *ok, 4, 96, None) == 2                         # K % 64
+    assert f(a, 64, 2, *arrays([w0, w1], [64, 64], [c0, c1], [128, 256], [128, 12]), 4, 64, None) == 2  # N % 8
+    assert f(a, 64, 2, *arrays([w0, w1], [64, 64], [c0, c1], [128, 100], [128, 256]), 4, 64, None) == 2  # ldc < N
+    assert f(a + 8, 64, 2, *ok, 4, 64, None) == 3                     # A not 16-byte aligned
+    assert f(a, 64, 2, *arrays([w0, w1 + 2], [64, 64], [c0, c1], [128, 256], [128, 256]), 4, 64, None) == 3
+    # outputs overlapping A, a weight, or each other
+    assert f(a, 64, 2, *arrays([w0, w1], [64, 64], [a, c1], [128, 256], [128, 256]), 4, 64, None) == 2
+    assert f(a, 64, 2, *arrays([w0, w1], [64, 64], [c0, w1], [128, 256], [128, 256]), 4, 64, None) == 2
+    assert f(a, 64, 2, *arrays([w0, w1], [64, 64], [c0, c0 + 64], [128, 256], [128, 256]), 4, 64, None) == 2
+    # column ranges of one wider output (row stride 256) that share columns 120..127
+    assert f(a, 64, 2, *arrays([w0, w1], [64, 64], [c0, c0 + 2 * 120], [256, 256], [128, 128]), 4, 64, None) == 2
+    # M == 0, or every N == 0: nothing to launch (no device needed)
+    assert f(a, 64, 2, *ok, 0, 64, None) == 0
+    assert f(a, 64, 2, *arrays([w0, w1], [64, 64], [c0, c1], [128, 256], [0, 0]), 4, 64, None) == 0
+
+
 def test_attention_workspace_size(L):
     s = L.bi_attention_workspace_size
     assert s(0, 32, 128, 2048) > 0

@@ -132,3 +132,43 @@ def test_rmsnorm_matmul_chain_32x512x1024():
     # the chain in double, no bf16 intermediate
     ref = oracle.matmul(oracle.rmsnorm(synth.to_f64(x), synth.to_f64(wn), 1e-6), synth.to_f64(W))
     assert max_rel(c, ref) <= TOL_BF16
+
+
+def _multi_inputs(M, Ns, K, seed):
+    a = synth.normal_bf16((M, K), seed)
+    ws = [synth.normal_bf16((n, K), seed + 1 + j, std=0.02) for j, n in enumerate(Ns)]
+    return a.to(dev()), [w.to(dev()) for w in ws]
+
+
+# Several products with one A in one call: each output equals bi_matmul's, bit for bit,
+# whether the call runs them as one joint launch on CTA pairs (every product on pair
+# tiles: M >= 129 here, and at N = 4096 from M = 600 on) or as separate launches.
+@pytest.mark.parametrize("M", [1, 64, 128, 129, 255, 256, 300, 512, 1023, 2048])
+def test_matmul_multi_equals_separate_calls(M):
+    a, ws = _multi_inputs(M, [4096, 6144, 14336], 4096, seed=60 + M)
+    cs = bi.matmul_multi(a, ws)
+    for w, c in zip(ws, cs):
+        assert same_bits(c, bi.matmul(a, w)), (M, w.shape[0])
+
+
+def test_matmul_multi_ragged_two_and_one_products_and_strided_outputs():
+    # ragged N and M; on a 148-SM B200 the first call runs as one joint launch on
+    # 256-wide pair tiles (485 tiles; alone, N = 4000 would take 192-wide ones)
+    a, ws = _multi_inputs(1100, [4000, 6152, 14336], 512, seed=70)
+    cs = bi.matmul_multi(a, ws)
+    for w, c in zip(ws, cs):
+        assert same_bits(c, bi.matmul(a, w))
+    ref = oracle.matmul(synth.to_f64(a[::97].cpu()), synth.to_f64(ws[1].cpu()))
+    assert max_rel(cs[1][::97], ref) <= TOL_BF16
+    # two products, written into column ranges of one wider output
+    big = torch.full((1100, 4000 + 6152 + 8), float("nan"), dtype=torch.bfloat16, device=dev())
+    outs = [big[:, :4000], big[:, 4000:4000 + 6152]]
+    bi.matmul_multi(a, ws[:2], outs=outs)
+    assert same_bits(outs[0], cs[0]) and same_bits(outs[1], cs[1])
+    assert torch.isnan(big[:, -8:].float()).all()  # columns past the outputs untouched
+    # one product: the same as bi_matmul
+    assert same_bits(bi.matmul_multi(a, ws[2:])[0], cs[2])
+    # a mix where one product alone would not use pair tiles (narrow N): separate launches
+    a2, ws2 = _multi_inputs(300, [264, 14336], 256, seed=71)
+    for w, c in zip(ws2, bi.matmul_multi(a2, ws2)):
+        assert same_bits(c, bi.matmul(a2, w))
