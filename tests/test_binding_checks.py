@@ -105,6 +105,10 @@ def test_every_wrapper_accepts_the_call_patterns_in_use(fake):
     a, W = _bf(5, 128), _bf(512, 128)
     bi.matmul(a, W)
     bi.matmul(a, W, out=_bf(8, 1024)[:5, 256:768])                  # strided output
+    outs = bi.matmul_multi(a, [W, _bf(256, 128), _bf(64, 128)])
+    assert [tuple(c.shape) for c in outs] == [(5, 512), (5, 256), (5, 64)]
+    wide = _bf(5, 768)
+    bi.matmul_multi(a, [W, _bf(256, 128)], outs=[wide[:, :512], wide[:, 512:]])  # column ranges of one output
     q, kc = _bf(3, 32, 128), _bf(10, 8, 16, 128)
     pt, lens = _i32(3, 4), _i32(3)
     bi.attention_decode(q, kc, kc, pt, lens)
@@ -139,7 +143,7 @@ def test_every_wrapper_accepts_the_call_patterns_in_use(fake):
     bi.sampling_uniforms(seeds, steps, 1000)
     bi.sample(lg, seeds, steps, 0.8, out=_i32(64))
     names = set(fake.calls)
-    for n in ("bi_rmsnorm", "bi_matmul", "bi_attention_decode", "bi_attention_decode_static", "bi_attention_prefill",
+    for n in ("bi_rmsnorm", "bi_matmul", "bi_matmul_multi", "bi_attention_decode", "bi_attention_decode_static", "bi_attention_prefill",
               "bi_attention_prefill_tc", "bi_kv_append", "bi_rope", "bi_gather_rows", "bi_swiglu", "bi_add",
               "bi_lmhead_argmax", "bi_log_softmax", "bi_token_logprob", "bi_row_mean", "bi_sampling_uniforms",
               "bi_sample"):
@@ -154,6 +158,12 @@ def test_wrong_outputs_and_index_tensors_are_refused_before_the_c_call(fake):
         (ValueError, lambda: bi.matmul(_bf(5, 128), _bf(512, 128), out=_bf(5, 256))),
         (TypeError, lambda: bi.matmul(_bf(5, 128), _bf(512, 128), out=_c(torch.zeros((5, 512))))),
         (ValueError, lambda: bi.matmul(_bf(5, 128), _bf(512, 128), out=_bf(512, 5).t())),  # columns strided
+        (ValueError, lambda: bi.matmul_multi(_bf(5, 128), [])),                            # no product
+        (ValueError, lambda: bi.matmul_multi(_bf(5, 128), [_bf(64, 128)] * 4)),            # more than three
+        (ValueError, lambda: bi.matmul_multi(_bf(5, 128), [_bf(64, 128), _bf(64, 256)])),  # inner dims differ
+        (ValueError, lambda: bi.matmul_multi(_bf(5, 128), [_bf(64, 128)], outs=[])),       # outs count
+        (ValueError, lambda: bi.matmul_multi(_bf(5, 128), [_bf(64, 128)], outs=[_bf(5, 32)])),  # out shape
+        (ValueError, lambda: bi.matmul_multi(_bf(5, 128), [_bf(128, 64).t()])),             # W rows strided
         (ValueError, lambda: bi.attention_decode(_bf(3, 32, 128), _bf(10, 8, 16, 128), _bf(10, 8, 16, 128),
                                                  _i32(3, 4), _i32(3), out=_bf(2, 32, 128))),
         (ValueError, lambda: bi.attention_prefill_tc(_bf(7, 32, 128), 0, 0, _bf(10, 8, 16, 128), _bf(10, 8, 16, 128),
