@@ -868,7 +868,7 @@ def profile_case(bi, device, name):
 
 def ours_config(M, world):
     """The workload description both arms print (the same dict, so the two lines compare)."""
-    return {"workload": WORKLOAD, "M": M, "K": K_HIDDEN, "N": list(NS), "step": "bi_rmsnorm + 3 x bi_matmul",
+    return {"workload": WORKLOAD, "M": M, "K": K_HIDDEN, "N": list(NS), "step": "bi_rmsnorm + bi_matmul_multi (the three products, one launch)",
             "parallelism": f"replicas x{world}",
             "l2": "working set > L2 (201 MB of weights per step; two activation buffers rotate)"}
 
